@@ -1,0 +1,154 @@
+"""Seeded synthetic inputs and the workload table.
+
+This module only makes inputs: byte streams shaped like the byte-level text
+the method is evaluated on, and N(0, 1) query/key/value/gradient tensors.  It
+holds none of the method's arithmetic; both the CUDA path's tests and the
+oracle draw their inputs from here.
+
+Byte streams (stand-ins for raw UTF-8 book/wiki text, which is not available):
+a sample is a run of 32-byte segments.  With probability f a segment is
+high-entropy — 32 bytes drawn uniformly from printable ASCII 32..126 —
+otherwise it repeats a phrase of 1–3 words (from a 16-word vocabulary of
+2–5 lowercase letters drawn per sample), words joined and followed by a
+space, to fill the 32 bytes.  The long-context workload instead repeats one
+16-byte phrase per sample, so that every untouched 64-byte block compresses
+the same and only about sqrt(N) blocks rise above the mean.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+SEGMENT = 32
+LOCAL, LITERAL, HYBRID = 0, 1, 2
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    S: int                 # batch (samples)
+    L: int                 # bytes (= tokens) per sample
+    b: int                 # block size in bytes
+    w: int                 # local window in blocks
+    H: int                 # heads
+    d: int                 # head dimension
+    dtype: str             # "f32" or "bf16"
+    backward: bool
+    entropy: tuple         # ("fixed", f) | ("uniform", lo, hi) | ("period16", f)
+    salt: int
+
+    @property
+    def N(self) -> int:
+        return self.L // self.b
+
+    def head_classes(self) -> np.ndarray:
+        """Half local, a quarter literal, a quarter hybrid, in that order."""
+        h = np.empty(self.H, dtype=np.uint8)
+        h[: self.H // 2] = LOCAL
+        h[self.H // 2: 3 * self.H // 4] = LITERAL
+        h[3 * self.H // 4:] = HYBRID
+        return h
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", S=1, L=256, b=16, w=1, H=4, d=32, dtype="f32",
+                          backward=False, entropy=("fixed", 0.5), salt=1),
+    "b8_4k": Workload("b8_4k", S=8, L=4096, b=64, w=2, H=12, d=64, dtype="bf16",
+                      backward=False, entropy=("uniform", 0.2, 0.6), salt=2),
+    "b8_8k": Workload("b8_8k", S=8, L=8192, b=64, w=2, H=12, d=64, dtype="bf16",
+                      backward=True, entropy=("uniform", 0.2, 0.6), salt=3),
+    "b1_64k": Workload("b1_64k", S=1, L=65536, b=64, w=4, H=16, d=128, dtype="bf16",
+                       backward=True, entropy=("period16", 0.015), salt=4),
+}
+
+
+def mask_sweep(b: int, f: float) -> Workload:
+    """Mask-stage sweep point: 256 samples of 8192 bytes, window 2."""
+    return Workload(f"mask_b{b}_f{f}", S=256, L=8192, b=b, w=2, H=12, d=64, dtype="bf16",
+                    backward=False, entropy=("fixed", f), salt=5 + b * 1000 + int(round(f * 100)))
+
+
+MASK_SWEEP = [(b, f) for b in (32, 64, 128) for f in (0.05, 0.3, 0.7)]
+
+
+def _rng(seed: int, salt: int, s: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, salt, s])))
+
+
+def _vocab(rng, n=16):
+    words = []
+    for _ in range(n):
+        ln = int(rng.integers(2, 6))
+        words.append(bytes(rng.integers(ord("a"), ord("z") + 1, size=ln).astype(np.uint8)))
+    return words
+
+
+def _phrase_segment(rng, vocab) -> bytes:
+    k = int(rng.integers(1, 4))
+    idx = rng.integers(0, len(vocab), size=k)
+    phrase = b" ".join(vocab[i] for i in idx) + b" "
+    return (phrase * (SEGMENT // len(phrase) + 1))[:SEGMENT]
+
+
+def _noise_segment(rng) -> bytes:
+    return bytes(rng.integers(32, 127, size=SEGMENT).astype(np.uint8))
+
+
+def sample_bytes(L: int, entropy: tuple, seed: int, salt: int, s: int) -> np.ndarray:
+    """One sample of L bytes (L a multiple of 32)."""
+    if L % SEGMENT:
+        raise ValueError("L must be a multiple of 32")
+    rng = _rng(seed, salt, s)
+    vocab = _vocab(rng)
+    kind = entropy[0]
+    if kind == "fixed":
+        f = float(entropy[1])
+    elif kind == "uniform":
+        f = float(rng.uniform(entropy[1], entropy[2]))
+    elif kind == "period16":
+        f = float(entropy[1])
+    else:
+        raise ValueError(kind)
+    if kind == "period16":
+        words = b" ".join(vocab) + b" "
+        period = (words * 2)[:16]
+        fill = period * (SEGMENT // 16)
+    out = bytearray()
+    for _ in range(L // SEGMENT):
+        if rng.random() < f:
+            out += _noise_segment(rng)
+        elif kind == "period16":
+            out += fill
+        else:
+            out += _phrase_segment(rng, vocab)
+    return np.frombuffer(bytes(out), dtype=np.uint8)
+
+
+def batch_bytes(wl: Workload, seed: int = 0) -> np.ndarray:
+    """uint8 [S, L] byte streams of a workload."""
+    return np.stack([sample_bytes(wl.L, wl.entropy, seed, wl.salt, s) for s in range(wl.S)])
+
+
+def custom_bytes(S: int, L: int, entropy: tuple, seed: int = 0, salt: int = 99) -> np.ndarray:
+    return np.stack([sample_bytes(L, entropy, seed, salt, s) for s in range(S)])
+
+
+def qkv(wl: Workload, seed: int = 0, device="cpu", grad: bool = False):
+    """Q, K, V (and dO when grad) ~ N(0, 1), [S, H, L, d], in the workload's
+    dtype, from a seeded torch generator on the given device."""
+    import torch
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    g = torch.Generator(device=device)
+    g.manual_seed(1_000_003 * seed + wl.salt)
+    shape = (wl.S, wl.H, wl.L, wl.d)
+    out = [torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt) for _ in range(4 if grad else 3)]
+    return tuple(out)
+
+
+def random_tensors(shape, n, dtype, seed, device="cpu"):
+    """n tensors ~ N(0, 1) of a shape, seeded."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return tuple(torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dtype) for _ in range(n))
