@@ -1,0 +1,267 @@
+"""Gzip-guided sparse attention hot path on B200 — Python binding of libgsa.
+
+Thin ctypes marshalling over the C ABI in include/gsa.h: every function here
+checks tensor placement/dtype/shape, builds the C argument structs and calls
+the library function of the same name.  All arithmetic runs in the CUDA
+kernels of libgsa.so; there is no CPU fallback.  PyTorch only provides the
+device memory and the stream.
+
+Pipeline (Gzip-guided Sparse Attention, daiwk.github.io, "核心公式"):
+    lengths = gsa_block_lengths(bytes, b)            # |gzip(block)| per block
+    flags   = gsa_literal_flags(lengths)             # l_i = 1[r_i > mean r]
+    csr     = gsa_build_block_csr(flags, w)          # mask lists per head class
+    o, lse  = gsa_attn_fwd(q, k, v, csr, head_classes, b)
+    dq, dk, dv = gsa_attn_bwd(q, k, v, o, lse, do, csr, head_classes, b)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GsaError", "BlockCsr", "HEAD_LOCAL", "HEAD_LITERAL", "HEAD_HYBRID",
+    "gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_csr_capacity",
+    "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_device_error",
+    "gsa_status_string", "library", "library_path",
+]
+
+HEAD_LOCAL, HEAD_LITERAL, HEAD_HYBRID = 0, 1, 2
+GSA_F32, GSA_BF16 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "lib", "libgsa.so")
+_lib = None
+
+
+class GsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {gsa_status_string(status)} (status {status})")
+        self.status = status
+
+
+class _Csr(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("nblk", ctypes.c_int32), ("w", ctypes.c_int32),
+        ("reserved", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+        ("col_ptr", ctypes.c_void_p), ("row_idx", ctypes.c_void_p),
+        ("q_order", ctypes.c_void_p), ("k_order", ctypes.c_void_p),
+    ]
+
+
+class _AttnDesc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int64),
+        ("d", ctypes.c_int32), ("b", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("head_classes", ctypes.c_void_p),
+    ]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library():
+    """Load libgsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libgsa.so is not built ({_LIB_PATH}); run "
+                               "`python -m content_adaptive_block_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        lib.gsa_block_lengths.argtypes = [vp, i32, i64, i32, vp, vp]
+        lib.gsa_literal_flags.argtypes = [vp, i32, i32, vp, vp]
+        lib.gsa_build_block_csr.argtypes = [vp, i32, ctypes.POINTER(_Csr), vp]
+        lib.gsa_csr_capacity.argtypes = [i32]
+        lib.gsa_csr_capacity.restype = i64
+        lib.gsa_attn_fwd.argtypes = [vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc), vp, vp, vp]
+        lib.gsa_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc),
+                                     vp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.gsa_attn_bwd_workspace.argtypes = [ctypes.POINTER(_AttnDesc)]
+        lib.gsa_attn_bwd_workspace.restype = ctypes.c_size_t
+        lib.gsa_device_error.argtypes = [ctypes.POINTER(i32), i32]
+        lib.gsa_status_string.argtypes = [ctypes.c_int]
+        lib.gsa_status_string.restype = ctypes.c_char_p
+        for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd",
+                   "gsa_attn_bwd", "gsa_device_error"):
+            getattr(lib, fn).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def gsa_status_string(status: int) -> str:
+    return library().gsa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise GsaError(fn, status)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+# ------------------------------------------------------------------ mask stage
+
+def gsa_block_lengths(data: torch.Tensor, b: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """|gzip level 1| of every b-byte block of data (uint8 [B, L]) -> int32 [B, L/b]."""
+    _need(data, "data", torch.uint8, 2)
+    B, L = data.shape
+    if out is None:
+        out = torch.empty((B, L // b if b > 0 else 0), dtype=torch.int32, device=data.device)
+    _need(out, "out", torch.int32)
+    _check("gsa_block_lengths",
+           library().gsa_block_lengths(_ptr(data), B, L, int(b), _ptr(out), _stream(stream)))
+    return out
+
+
+def gsa_literal_flags(lengths: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Literal flags (uint8 [B, nblk]) from per-block lengths (int32 [B, nblk])."""
+    _need(lengths, "lengths", torch.int32, 2)
+    B, n = lengths.shape
+    if out is None:
+        out = torch.empty((B, n), dtype=torch.uint8, device=lengths.device)
+    _need(out, "out", torch.uint8)
+    _check("gsa_literal_flags", library().gsa_literal_flags(_ptr(lengths), B, n, _ptr(out), _stream(stream)))
+    return out
+
+
+def gsa_csr_capacity(nblk: int) -> int:
+    return int(library().gsa_csr_capacity(int(nblk)))
+
+
+class BlockCsr:
+    """Device buffers of the per-(sample, class) block lists (gsa_block_csr)."""
+
+    def __init__(self, B: int, nblk: int, device, capacity: int | None = None):
+        cap = gsa_csr_capacity(nblk) if capacity is None else int(capacity)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.B, self.nblk, self.capacity, self.w = B, nblk, cap, -1
+        self.row_ptr = torch.empty((B, 3, nblk + 1), **i32)
+        self.col_idx = torch.empty((B, 3, cap), **i32)
+        self.col_ptr = torch.empty((B, 3, nblk + 1), **i32)
+        self.row_idx = torch.empty((B, 3, cap), **i32)
+        self.q_order = torch.empty((B, 3, nblk), **i32)
+        self.k_order = torch.empty((B, 3, nblk), **i32)
+
+    def struct(self) -> _Csr:
+        return _Csr(self.B, self.nblk, self.w, 0, self.capacity,
+                    self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_ptr.data_ptr(),
+                    self.row_idx.data_ptr(), self.q_order.data_ptr(), self.k_order.data_ptr())
+
+    def rows(self, s: int, c: int) -> list:
+        """Key-block list of every query block of (sample s, class c), on the host."""
+        rp = self.row_ptr[s, c].cpu().tolist()
+        ci = self.col_idx[s, c, : rp[-1]].cpu().tolist()
+        return [ci[rp[i]: rp[i + 1]] for i in range(self.nblk)]
+
+    def cols(self, s: int, c: int) -> list:
+        cp = self.col_ptr[s, c].cpu().tolist()
+        ri = self.row_idx[s, c, : cp[-1]].cpu().tolist()
+        return [ri[cp[j]: cp[j + 1]] for j in range(self.nblk)]
+
+
+def gsa_build_block_csr(flags: torch.Tensor, w: int, csr: BlockCsr | None = None, stream=None) -> BlockCsr:
+    """Block lists of the mask for all three head classes from literal flags."""
+    _need(flags, "flags", torch.uint8, 2)
+    B, n = flags.shape
+    if csr is None:
+        csr = BlockCsr(B, n, flags.device)
+    st = csr.struct()
+    _check("gsa_build_block_csr", library().gsa_build_block_csr(_ptr(flags), int(w), ctypes.byref(st),
+                                                                 _stream(stream)))
+    csr.w = st.w
+    return csr
+
+
+# ------------------------------------------------------------------ attention
+
+def _desc(q: torch.Tensor, b: int, head_classes, scale: float):
+    B, H, L, d = q.shape
+    hc = (ctypes.c_uint8 * H)(*[int(c) for c in head_classes])
+    dtype = GSA_F32 if q.dtype == torch.float32 else GSA_BF16
+    return _AttnDesc(B, H, L, d, int(b), dtype, float(scale), ctypes.cast(hc, ctypes.c_void_p)), hc
+
+
+def gsa_attn_fwd(q, k, v, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,
+                 o: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Block-sparse causal attention forward; q, k, v [B, H, L, d] (bf16 or
+    float32).  Returns (o, lse) with lse float32 [B, H, L]."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k and v must have the same shape")
+    if len(head_classes) != q.shape[1]:
+        raise ValueError("one head class per head")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    _need(o, "o", q.dtype)
+    _need(lse, "lse", torch.float32)
+    desc, keep = _desc(q, b, head_classes, scale)
+    st = csr.struct()
+    _check("gsa_attn_fwd", library().gsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(st), ctypes.byref(desc),
+                                                  _ptr(o), _ptr(lse), _stream(stream)))
+    del keep
+    return o, lse
+
+
+def gsa_attn_bwd_workspace(q: torch.Tensor, b: int, head_classes) -> int:
+    desc, keep = _desc(q, b, head_classes, 0.0)
+    return int(library().gsa_attn_bwd_workspace(ctypes.byref(desc)))
+
+
+def gsa_attn_bwd(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,
+                 dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None):
+    """Gradients (dq, dk, dv) of gsa_attn_fwd for upstream gradient do."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, name, q.dtype, 4)
+    _need(lse, "lse", torch.float32, 3)
+    if len(head_classes) != q.shape[1]:
+        raise ValueError("one head class per head")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    desc, keep = _desc(q, b, head_classes, scale)
+    need = int(library().gsa_attn_bwd_workspace(ctypes.byref(desc)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    st = csr.struct()
+    _check("gsa_attn_bwd", library().gsa_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), ctypes.byref(st), ctypes.byref(desc),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    del keep
+    return dq, dk, dv
+
+
+def gsa_device_error(clear: bool = True) -> int:
+    """The library's device error word (0 = no kernel gave up a wait)."""
+    code = ctypes.c_int32(0)
+    library().gsa_device_error(ctypes.byref(code), 1 if clear else 0)
+    return int(code.value)

@@ -1,0 +1,287 @@
+// libgsa: the C ABI of include/gsa.h.  Host-side argument checks, TMA
+// descriptor set-up and kernel launches; all arithmetic of the path runs in
+// the kernels included below.  One translation unit, so the device error
+// word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "gsa.h"
+
+#include "common.cuh"
+#include "deflate_len.cuh"
+#include "flags_csr.cuh"
+#include "attn_fwd_f32.cuh"
+#include "attn_fwd_bf16.cuh"
+#include "attn_bwd_bf16.cuh"
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+gsa_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+// ---- TMA descriptor encoding through the driver entry point (no -lcuda)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A bf16 [rows][cols] row-major matrix, 64 x 64 boxes, 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool csr_ok(const gsa_block_csr* c) {
+    return c && c->B >= 1 && c->nblk >= 1 && c->row_ptr && c->col_idx && c->col_ptr && c->row_idx && c->q_order &&
+           c->k_order && c->capacity >= gsa_csr_capacity(c->nblk);
+}
+
+// Common checks of an attention call; fills the class table.
+gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
+    if (!d || !csr || !d->head_classes) return GSA_ERR_INVALID_ARGUMENT;
+    if (!csr_ok(csr)) return csr && csr->capacity < gsa_csr_capacity(csr->nblk) ? GSA_ERR_CAPACITY
+                                                                              : GSA_ERR_INVALID_ARGUMENT;
+    if (d->B < 1 || d->H < 1 || d->L < 1 || d->b < 1 || d->d < 1) return GSA_ERR_INVALID_ARGUMENT;
+    if (d->H > GSA_MAX_HEADS) return GSA_ERR_UNSUPPORTED;
+    if (d->B != csr->B || d->L != static_cast<int64_t>(csr->nblk) * d->b) return GSA_ERR_INVALID_ARGUMENT;
+    if (!(d->scale >= 0.f) || !std::isfinite(d->scale)) return GSA_ERR_INVALID_ARGUMENT;
+    for (int h = 0; h < d->H; ++h) {
+        if (d->head_classes[h] > 2) return GSA_ERR_INVALID_ARGUMENT;
+        cls[h] = d->head_classes[h];
+    }
+    if (d->dtype != GSA_F32 && d->dtype != GSA_BF16) return GSA_ERR_INVALID_ARGUMENT;
+    return GSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t gsa_csr_capacity(int32_t nblk) {
+    if (nblk < 0) return 0;
+    return static_cast<int64_t>(nblk) * (nblk + 1) / 2;
+}
+
+gsa_status gsa_block_lengths(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t* lengths, void* stream) {
+    if (!bytes || !lengths || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES || L < b || L % b != 0)
+        return GSA_ERR_INVALID_ARGUMENT;
+    using namespace gsa::deflate;
+    const int64_t total = static_cast<int64_t>(B) * (L / b);
+    const int64_t grid = (total + kWarps - 1) / kWarps;
+    if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(block_lengths_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    });
+    block_lengths_kernel<<<static_cast<unsigned>(grid), 32 * kWarps, kSmemBytes, as_stream(stream)>>>(
+        bytes, L, b, total, lengths);
+    return launch_status();
+}
+
+gsa_status gsa_literal_flags(const int32_t* lengths, int32_t B, int32_t nblk, uint8_t* flags, void* stream) {
+    if (!lengths || !flags || B < 1 || nblk < 1) return GSA_ERR_INVALID_ARGUMENT;
+    gsa::mask::literal_flags_kernel<<<B, 256, 0, as_stream(stream)>>>(lengths, nblk, flags);
+    return launch_status();
+}
+
+gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* csr, void* stream) {
+    if (!flags || !csr || w < 0) return GSA_ERR_INVALID_ARGUMENT;
+    if (csr->B < 1 || csr->nblk < 1 || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
+        !csr->q_order || !csr->k_order)
+        return GSA_ERR_INVALID_ARGUMENT;
+    if (csr->nblk > gsa::mask::kMaxBlocksCsr) return GSA_ERR_UNSUPPORTED;
+    if (csr->capacity < gsa_csr_capacity(csr->nblk)) return GSA_ERR_CAPACITY;
+    csr->w = w;
+    gsa::mask::CsrArgs a;
+    a.flags = flags;
+    a.nblk = csr->nblk;
+    a.w = w;
+    a.cap = csr->capacity;
+    a.row_ptr = csr->row_ptr;
+    a.col_idx = csr->col_idx;
+    a.col_ptr = csr->col_ptr;
+    a.row_idx = csr->row_idx;
+    a.q_order = csr->q_order;
+    a.k_order = csr->k_order;
+    const size_t smem = gsa::mask::csr_smem_bytes(csr->nblk);
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(gsa::mask::build_csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gsa::mask::csr_smem_bytes(gsa::mask::kMaxBlocksCsr)));
+    });
+    dim3 grid(3, csr->B);
+    gsa::mask::build_csr_kernel<<<grid, gsa::mask::kThreads, smem, as_stream(stream)>>>(a);
+    return launch_status();
+}
+
+gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_block_csr* csr,
+                        const gsa_attn_desc* desc, void* o, float* lse, void* stream) {
+    if (!q || !k || !v || !o) return GSA_ERR_INVALID_ARGUMENT;
+    uint8_t cls[GSA_MAX_HEADS];
+    gsa_status st = check_attn(desc, csr, cls);
+    if (st != GSA_OK) return st;
+    const float scale = desc->scale > 0.f ? desc->scale : 1.f / std::sqrt(static_cast<float>(desc->d));
+    const cudaStream_t cs = as_stream(stream);
+
+    if (desc->dtype == GSA_F32) {
+        if (desc->b > 128 || !(desc->d == 16 || desc->d == 32 || desc->d == 64 || desc->d == 128))
+            return GSA_ERR_UNSUPPORTED;
+        gsa::f32::Params p;
+        p.q = static_cast<const float*>(q);
+        p.k = static_cast<const float*>(k);
+        p.v = static_cast<const float*>(v);
+        p.o = static_cast<float*>(o);
+        p.lse = lse;
+        p.row_ptr = csr->row_ptr;
+        p.col_idx = csr->col_idx;
+        p.cap = csr->capacity;
+        p.S = desc->B;
+        p.H = desc->H;
+        p.nblk = csr->nblk;
+        p.b = desc->b;
+        p.L = desc->L;
+        p.scale = scale;
+        std::memcpy(p.cls, cls, desc->H);
+        dim3 grid(csr->nblk, desc->H, desc->B);
+        const size_t smem = 3u * desc->b * desc->d * sizeof(float);
+        static std::once_flag once;
+        std::call_once(once, [] {
+            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 3 * 128 * 16 * 4);
+            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 3 * 128 * 32 * 4);
+            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 3 * 128 * 64 * 4);
+            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 3 * 128 * 128 * 4);
+        });
+        switch (desc->d) {
+            case 16: gsa::f32::attn_fwd_f32_kernel<16><<<grid, 128, smem, cs>>>(p); break;
+            case 32: gsa::f32::attn_fwd_f32_kernel<32><<<grid, 128, smem, cs>>>(p); break;
+            case 64: gsa::f32::attn_fwd_f32_kernel<64><<<grid, 128, smem, cs>>>(p); break;
+            default: gsa::f32::attn_fwd_f32_kernel<128><<<grid, 128, smem, cs>>>(p); break;
+        }
+        return launch_status();
+    }
+
+    // bf16 tensor-core path
+    if (desc->b != gsa::bf16::kBlk || !(desc->d == 64 || desc->d == 128) || csr->nblk > GSA_MAX_BLOCKS_BF16)
+        return GSA_ERR_UNSUPPORTED;
+    if (!lse) return GSA_ERR_INVALID_ARGUMENT;
+    const uint64_t rows = static_cast<uint64_t>(desc->B) * desc->H * desc->L;
+    if (rows >= (1ull << 31)) return GSA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_bf16(&tq, q, rows, desc->d) || !make_tmap_bf16(&tk, k, rows, desc->d) ||
+        !make_tmap_bf16(&tv, v, rows, desc->d))
+        return GSA_ERR_CUDA;
+    gsa::bf16::FwdParams p;
+    p.row_ptr = csr->row_ptr;
+    p.col_idx = csr->col_idx;
+    p.q_order = csr->q_order;
+    p.cap = csr->capacity;
+    p.S = desc->B;
+    p.H = desc->H;
+    p.nblk = csr->nblk;
+    p.L = desc->L;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    std::memcpy(p.cls, cls, desc->H);
+    dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
+    if (desc->d == 64) {
+        using C = gsa::bf16::FwdCfg<64>;
+        static std::once_flag once;
+        std::call_once(once, [] {
+            cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
+        });
+        gsa::bf16::attn_fwd_bf16_kernel<64><<<grid, 192, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+    } else {
+        using C = gsa::bf16::FwdCfg<128>;
+        static std::once_flag once;
+        std::call_once(once, [] {
+            cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        });
+        gsa::bf16::attn_fwd_bf16_kernel<128><<<grid, 192, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+    }
+    return launch_status();
+}
+
+size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc) {
+    if (!desc || desc->B < 1 || desc->H < 1 || desc->L < 1) return 0;
+    return sizeof(float) * static_cast<size_t>(desc->B) * desc->H * desc->L;
+}
+
+gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                        const gsa_block_csr* csr, const gsa_attn_desc* desc, void* dq, void* dk, void* dv,
+                        void* workspace, size_t ws_bytes, void* stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return GSA_ERR_INVALID_ARGUMENT;
+    uint8_t cls[GSA_MAX_HEADS];
+    gsa_status st = check_attn(desc, csr, cls);
+    if (st != GSA_OK) return st;
+    if (ws_bytes < gsa_attn_bwd_workspace(desc)) return GSA_ERR_CAPACITY;
+    if (desc->dtype != GSA_BF16) return GSA_ERR_UNSUPPORTED;
+    if (desc->b != gsa::bf16::kBlk || !(desc->d == 64 || desc->d == 128) || csr->nblk > GSA_MAX_BLOCKS_BF16)
+        return GSA_ERR_UNSUPPORTED;
+    const uint64_t rows = static_cast<uint64_t>(desc->B) * desc->H * desc->L;
+    if (rows >= (1ull << 31)) return GSA_ERR_UNSUPPORTED;
+    const float scale = desc->scale > 0.f ? desc->scale : 1.f / std::sqrt(static_cast<float>(desc->d));
+    return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, static_cast<float*>(workspace),
+                            as_stream(stream));
+}
+
+gsa_status gsa_device_error(int32_t* code, int32_t clear) {
+    if (!code) return GSA_ERR_INVALID_ARGUMENT;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GSA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, gsa::g_device_error, sizeof(int)) != cudaSuccess) return GSA_ERR_CUDA;
+    if (clear && v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(gsa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return GSA_ERR_CUDA;
+    }
+    *code = v;
+    return v ? GSA_ERR_TIMEOUT : GSA_OK;
+}
+
+const char* gsa_status_string(gsa_status s) {
+    switch (s) {
+        case GSA_OK: return "ok";
+        case GSA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case GSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GSA_ERR_CAPACITY: return "buffer too small";
+        case GSA_ERR_CUDA: return "CUDA error";
+        case GSA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,144 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+function include/gsa.h declares, and rejects bad arguments before launching
+anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import content_adaptive_block_b200 as gsa
+from content_adaptive_block_b200 import build as gsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gsa_build.build()
+    return gsa.library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_path(lib):
+    names = _declared()
+    for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd",
+               "gsa_attn_bwd", "gsa_csr_capacity", "gsa_attn_bwd_workspace", "gsa_device_error",
+               "gsa_status_string"):
+        assert fn in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for fn in _declared():
+        assert hasattr(lib, fn), fn
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert gsa.gsa_status_string(code)
+    assert gsa.gsa_status_string(99) == "unknown status"
+
+
+def test_csr_capacity(lib):
+    assert gsa.gsa_csr_capacity(1) == 1
+    assert gsa.gsa_csr_capacity(128) == 128 * 129 // 2
+    assert gsa.gsa_csr_capacity(0) == 0
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(0x1000)   # never dereferenced: every call below fails its host checks
+
+
+def test_block_lengths_rejects_bad_arguments(lib):
+    f = lib.gsa_block_lengths
+    assert f(NULL, 1, 64, 64, FAKE, NULL) == 1
+    assert f(FAKE, 1, 64, 64, NULL, NULL) == 1
+    assert f(FAKE, 0, 64, 64, FAKE, NULL) == 1     # no samples
+    assert f(FAKE, 1, 100, 64, FAKE, NULL) == 1    # L not a multiple of b
+    assert f(FAKE, 1, 64, 0, FAKE, NULL) == 1      # b = 0
+    assert f(FAKE, 1, 512, 256, FAKE, NULL) == 1   # b above the maximum
+    assert f(FAKE, 1, 32, 64, FAKE, NULL) == 1     # L < b
+
+
+def test_literal_flags_rejects_bad_arguments(lib):
+    f = lib.gsa_literal_flags
+    assert f(NULL, 1, 4, FAKE, NULL) == 1
+    assert f(FAKE, 1, 4, NULL, NULL) == 1
+    assert f(FAKE, 0, 4, FAKE, NULL) == 1
+    assert f(FAKE, 1, 0, FAKE, NULL) == 1
+
+
+def _csr(B=1, n=4, cap=None):
+    p = 0x1000
+    return gsa._Csr(B, n, 0, 0, gsa.gsa_csr_capacity(n) if cap is None else cap, p, p, p, p, p, p)
+
+
+def test_build_csr_rejects_bad_arguments(lib):
+    f = lib.gsa_build_block_csr
+    c = _csr()
+    assert f(NULL, 1, ctypes.byref(c), NULL) == 1
+    assert f(FAKE, -1, ctypes.byref(c), NULL) == 1          # negative window
+    c0 = _csr(B=0)
+    assert f(FAKE, 1, ctypes.byref(c0), NULL) == 1
+    small = _csr(n=8, cap=10)
+    assert f(FAKE, 1, ctypes.byref(small), NULL) == 3       # capacity
+    nul = _csr()
+    nul.q_order = None
+    assert f(FAKE, 1, ctypes.byref(nul), NULL) == 1
+
+
+def _desc(B=1, H=4, L=256, d=64, b=64, dtype=1, classes=(0, 0, 1, 2), scale=0.0):
+    hc = (ctypes.c_uint8 * len(classes))(*classes)
+    return gsa._AttnDesc(B, H, L, d, b, dtype, scale, ctypes.cast(hc, ctypes.c_void_p)), hc
+
+
+def test_attn_fwd_rejects_bad_arguments(lib):
+    f = lib.gsa_attn_fwd
+    c = _csr(n=4)
+    d, keep = _desc()
+    assert f(NULL, FAKE, FAKE, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, NULL) == 1
+    bad_l, k1 = _desc(L=200)                                 # L != nblk * b
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(bad_l), FAKE, FAKE, NULL) == 1
+    bad_c, k2 = _desc(classes=(0, 0, 1, 3))                  # class outside 0..2
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(bad_c), FAKE, FAKE, NULL) == 1
+    bad_b, k3 = _desc(B=2)                                   # batch disagrees with the lists
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(bad_b), FAKE, FAKE, NULL) == 1
+    c32 = _csr(n=8)
+    d32, k4 = _desc(L=256, b=32)                             # bf16 path needs b = 64
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c32), ctypes.byref(d32), FAKE, FAKE, NULL) == 2
+    dd, k5 = _desc(d=96)                                     # head dim not implemented
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(dd), FAKE, FAKE, NULL) == 2
+    small = _csr(n=4, cap=3)
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(small), ctypes.byref(d), FAKE, FAKE, NULL) == 3
+    neg, k6 = _desc(scale=-1.0)
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(neg), FAKE, FAKE, NULL) == 1
+
+
+def test_attn_bwd_rejects_bad_arguments(lib):
+    f = lib.gsa_attn_bwd
+    c = _csr(n=4)
+    d, keep = _desc()
+    ws = lib.gsa_attn_bwd_workspace(ctypes.byref(d))
+    assert ws == 4 * 1 * 4 * 256
+    args = [FAKE] * 6
+    assert f(*args[:5], NULL, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws, NULL) == 1
+    assert f(*args, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws - 4, NULL) == 3
+    d32, k2 = _desc(dtype=0, d=32)
+    assert f(*args, ctypes.byref(c), ctypes.byref(d32), FAKE, FAKE, FAKE, FAKE, 1 << 20, NULL) == 2
+
+
+def test_device_error_rejects_null(lib):
+    assert lib.gsa_device_error(None, 0) == 1
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        gsa.gsa_block_lengths(torch.zeros((1, 64), dtype=torch.uint8), 64)
+    with pytest.raises(ValueError):
+        gsa.gsa_literal_flags(torch.zeros((1, 4), dtype=torch.int32))
