@@ -1,0 +1,469 @@
+"""Benchmark of the gzip-guided sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole path over one synthetic batch of the 8K-byte
+workload (8 samples x 8192 bytes, 64-byte blocks -> 128 blocks, window 2,
+12 heads split 6 local / 3 literal / 3 hybrid, head dim 64, bf16):
+    gsa_block_lengths -> gsa_literal_flags -> gsa_build_block_csr
+    -> gsa_attn_fwd -> gsa_attn_bwd
+all through the C ABI (libgsa.so).  The headline value is live-block
+attention TFLOP/s (forward 4*d and backward 8*d FLOPs per live
+(query token, key token) pair, the S recompute not counted) of the whole
+step, inputs resident in HBM.  The L2 is flushed between steps (a 256 MiB
+write, outside the timed events).  Rank 0 prints one JSON line.
+
+Under torchrun each rank runs its own batch (data-parallel, no collective on
+the data path); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "live-block attn TFLOP/s fwd+bwd @8K bytes; gzip-mask GB/s of input bytes"
+UNIT = "TFLOP/s"
+WORKLOAD = "b8_8k"
+MASK_POINT = (64, 0.3)
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def workload_desc(wl):
+    return (f"{wl.name}: batch {wl.S} x {wl.L} bytes, b={wl.b} ({wl.N} blocks), w={wl.w}, "
+            f"{wl.H} heads (6 local/3 literal/3 hybrid), d={wl.d}, {wl.dtype}, fwd+bwd")
+
+
+def live_token_pairs_from_counts(nnz_sc, n, b, head_classes):
+    """Live (query token, key token) pairs summed over heads of one sample,
+    from the per-class live block-pair counts (diagonal blocks are causal)."""
+    total = 0
+    for c in head_classes:
+        nnz = int(nnz_sc[int(c)])
+        total += (nnz - n) * b * b + n * b * (b + 1) // 2
+    return total
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        self.device = device_index
+
+    def start(self):
+        try:
+            import torch
+            bus = getattr(torch.cuda.get_device_properties(self.device), "pci_bus_id", None)
+        except Exception:
+            bus = None
+        fd, self.path = tempfile.mkstemp(prefix="gsa_clocks_", suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if bus is not None:
+            cmd += ["-i", str(bus)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        for r in rows:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [x for x in sm if x > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline)
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(wl, x, q, k, v, do, hc, head):
+    """One bounded sample of the workload on the oracle: the mask stage of
+    sample 0 and the forward + backward of one head of it.  Returns the
+    algorithmic FLOPs of that head."""
+    from oracle import attention as oatt, deflate1, flags as oflags, mask as omask
+    ln = deflate1.block_lengths(x[:1], wl.b, nthreads=1)
+    fl = oflags.literal_flags(ln, wl.b)
+    m = omask.block_mask(fl[0], wl.w, int(hc[head]))
+    oatt.forward(q[0, head], k[0, head], v[0, head], m, wl.b)
+    oatt.backward(q[0, head], k[0, head], v[0, head], do[0, head], m, wl.b)
+    return 12 * wl.d * omask.live_token_pairs(m, wl.b)
+
+
+def oracle_inputs(wl, seed):
+    import torch
+    x = W.batch_bytes(wl, seed=seed)
+    g = torch.Generator().manual_seed(seed)
+    shape = (1, wl.H, wl.L, wl.d)
+    q, k, v, do = (torch.randn(shape, generator=g).to(torch.bfloat16).to(torch.float64).numpy() for _ in range(4))
+    return x, q, k, v, do
+
+
+def cpu_baseline(wl, budget_s=12.0, seed=0):
+    x, q, k, v, do = oracle_inputs(wl, seed)
+    hc = wl.head_classes()
+    order = [0, wl.H // 2, 3 * wl.H // 4]          # one head of each class, then the rest
+    order += [h for h in range(wl.H) if h not in order]
+    flops, t0, heads = 0, time.perf_counter(), 0
+    while heads < 3 or (time.perf_counter() - t0 < budget_s and heads < len(order)):
+        flops += oracle_sample_step(wl, x, q, k, v, do, hc, order[heads % len(order)])
+        heads += 1
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"sample 0 of {wl.S}: gzip lengths, flags and mask, then forward + backward of "
+                      f"{heads} of {wl.H} heads (one per class first), float64 numpy; {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    wl = W.WORKLOADS[WORKLOAD]
+    if rank != 0:
+        return 0
+    x, q, k, v, do = oracle_inputs(wl, 0)
+    hc = wl.head_classes()
+    order = [0, wl.H // 2, 3 * wl.H // 4]
+    for i in range(args.warmup):
+        oracle_sample_step(wl, x, q, k, v, do, hc, order[i % 3])
+    times, flops = [], 0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        flops += oracle_sample_step(wl, x, q, k, v, do, hc, order[i % 3])
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    val = flops / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(wl)},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                             "sample": "each step: gzip lengths, flags and mask of sample 0 and forward + "
+                                       "backward of one head (classes in turn), float64 numpy"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ ours
+
+def _traffic_record(kernel):
+    """dram bytes per launch from a committed ncu capture, if the kernel's
+    source is unchanged since (else None)."""
+    try:
+        import hashlib
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+        if not rec:
+            return None
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return rec["bytes_per_launch"] if h.hexdigest() == rec["sha256"] else None
+    except Exception:
+        return None
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import content_adaptive_block_b200 as gsa
+    from content_adaptive_block_b200 import build
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    wl = W.WORKLOADS[WORKLOAD]
+    peaks = _peaks()
+    hc = [int(c) for c in wl.head_classes()]
+
+    # ---- inputs (per-rank seed), resident in HBM
+    x_host = W.batch_bytes(wl, seed=rank)
+    x = torch.from_numpy(x_host).to(dev)
+    q, k, v, do = W.qkv(wl, seed=rank, device=dev, grad=True)
+    lengths = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
+    flags = torch.empty((wl.S, wl.N), dtype=torch.uint8, device=dev)
+    csr = gsa.BlockCsr(wl.S, wl.N, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.S, wl.H, wl.L), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(gsa.gsa_attn_bwd_workspace(q, wl.b, hc), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd", "gsa_attn_bwd")
+    launches_per_step = 1 + 1 + 1 + 1 + 3
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        gsa.gsa_block_lengths(x, wl.b, out=lengths)
+        if ev:
+            ev[1].record(stream)
+        gsa.gsa_literal_flags(lengths, out=flags)
+        if ev:
+            ev[2].record(stream)
+        gsa.gsa_build_block_csr(flags, wl.w, csr)
+        if ev:
+            ev[3].record(stream)
+        gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse)
+        if ev:
+            ev[4].record(stream)
+        gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b, dq=dq, dk=dk, dv=dv, workspace=ws)
+        if ev:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0, "a kernel gave up a bounded wait"
+
+    # algorithmic work of this rank's batch
+    nnz = csr.row_ptr[:, :, -1].cpu().numpy()
+    pairs = sum(live_token_pairs_from_counts(nnz[s], wl.N, wl.b, hc) for s in range(wl.S))
+    fwd_flops, bwd_flops = 4 * wl.d * pairs, 8 * wl.d * pairs
+    step_flops = fwd_flops + bwd_flops
+    dense_pairs = wl.S * wl.H * wl.L * (wl.L + 1) // 2
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+
+    per_call = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(args.steps)])
+    step_ms = per_call.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the API with host buffers
+    x_pin = torch.from_numpy(x_host).pin_memory()
+    q_pin, k_pin, v_pin, do_pin = (t.cpu().pin_memory() for t in (q, k, v, do))
+    dq_pin, dk_pin, dv_pin = (torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv))
+    h2d = x_pin.numel() + sum(t.numel() * t.element_size() for t in (q_pin, k_pin, v_pin, do_pin))
+    d2h = sum(t.numel() * t.element_size() for t in (dq_pin, dk_pin, dv_pin))
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        x.copy_(x_pin, non_blocking=True)
+        for dst, src in ((q, q_pin), (k, k_pin), (v, v_pin), (do, do_pin)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in ((dq_pin, dq), (dk_pin, dk), (dv_pin, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+
+    # ---- mask-stage sweep (secondary metric), rank 0
+    mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
+
+    if rank != 0:
+        return 0
+    call_ms = {n: float(per_call[:, j].mean()) for j, n in enumerate(names)}
+    bwd_ms, fwd_ms = call_ms["gsa_attn_bwd"], call_ms["gsa_attn_fwd"]
+    peak_t = peaks["bf16_tflops_sustained"]
+    bwd_ach = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    fwd_ach = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(wl),
+                   "l2": "flushed between steps (256 MiB write outside the timed events); "
+                         "q/k/v/dO alone are 403 MB",
+                   "live_token_pairs": pairs, "dense_causal_pairs": dense_pairs,
+                   "live_fraction": pairs / dense_pairs, "step_gflop": step_flops / 1e9},
+        "roofline": {"kernel": "gsa_attn_bwd (dot + dq + dk/dv launches)", "bound": "tensor",
+                     "achieved": bwd_ach, "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_ach / peak_t,
+                     "peak_kind": f"bf16 sustained, {peaks['source']}",
+                     "frac_of_burst": bwd_ach / peaks["bf16_tflops"],
+                     "traffic": _traffic_record("gsa_attn_bwd")},
+        "roofline_fwd": {"kernel": "gsa_attn_fwd", "bound": "tensor", "achieved": fwd_ach, "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": fwd_ach / peak_t, "traffic": _traffic_record("gsa_attn_fwd")},
+        "call_ms": call_ms,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms},
+        "clocks": clocks,
+    }
+    if mask:
+        line["mask_stage"] = mask
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line))
+    return 0
+
+
+def mask_stage(gsa, dev):
+    """gzip-mask GB/s of input bytes: lengths + flags + block lists over 256
+    samples x 8192 bytes.  Input batches rotate over > 320 MiB so the bytes
+    come from HBM, not L2."""
+    import torch
+    out = {"metric": "gzip-mask GB/s of input bytes", "unit": "GB/s", "points": {}}
+    n_rot = 160
+    for b, f in W.MASK_SWEEP:
+        wl = W.mask_sweep(b, f)
+        base = torch.from_numpy(W.batch_bytes(wl, seed=0)).to(dev)
+        # distinct copies: rotated rows keep the statistics, change the addresses
+        batches = [torch.roll(base, shifts=i, dims=0).contiguous() for i in range(n_rot)]
+        lengths = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
+        flags = torch.empty((wl.S, wl.N), dtype=torch.uint8, device=dev)
+        csr = gsa.BlockCsr(wl.S, wl.N, dev)
+
+        def one(xb):
+            gsa.gsa_block_lengths(xb, wl.b, out=lengths)
+            gsa.gsa_literal_flags(lengths, out=flags)
+            gsa.gsa_build_block_csr(flags, wl.w, csr)
+
+        for i in range(3):
+            one(batches[i])
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        for i in range(n_rot):
+            gsa.gsa_block_lengths(batches[i], wl.b, out=lengths)
+        e[1].record()
+        for i in range(n_rot):
+            one(batches[i])
+        e[2].record()
+        torch.cuda.synchronize()
+        len_ms = e[0].elapsed_time(e[1]) / n_rot
+        all_ms = e[1].elapsed_time(e[2]) / n_rot
+        nbytes = wl.S * wl.L
+        nnz = int(csr.row_ptr[:, :, -1].sum().item())
+        # what the stage must write: lengths (int32) and flags (uint8) per
+        # block; CSR and CSC pointers, entries and pairing orders (int32)
+        out_bytes = (wl.S * wl.N * (4 + 1)
+                     + 4 * (2 * wl.S * 3 * (wl.N + 1) + 2 * nnz + 2 * wl.S * 3 * wl.N))
+        out["points"][f"b{b}_f{f}"] = {
+            "gbs": nbytes / (all_ms * 1e-3) / 1e9, "lengths_gbs": nbytes / (len_ms * 1e-3) / 1e9,
+            "ms": all_ms, "lengths_ms": len_ms, "bytes_in": nbytes, "bytes_out": out_bytes,
+            "hbm_frac": (nbytes + out_bytes) / (all_ms * 1e-3) / 1e9 / _peaks()["hbm_gbs"]}
+    key = f"b{MASK_POINT[0]}_f{MASK_POINT[1]}"
+    out["value"] = out["points"][key]["gbs"]
+    out["workload"] = f"{key}: 256 x 8192 bytes, w=2"
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-mask-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,15 +1,657 @@
-// Block-sparse causal attention backward (placeholder until the kernels land).
+// Block-sparse causal attention backward, bf16 in / fp32 accumulate, on
+// tcgen05 tensor cores (sm_100a).
+//
+// The pages train the model with this mask (Gzip-guided Sparse Attention,
+// daiwk.github.io, "论文离线与线上效果": 20K steps), so the gradient of the
+// masked softmax attention is part of the path.  With P = softmax (from the
+// forward's LSE), D_t = Σ_e dO_te O_te:
+//   dS = P ∘ (dO V^T − D),  dQ = scale · dS K,  dK = scale · dS^T Q,  dV = P^T dO,
+// over live pairs only.  Three launches, no atomics (deterministic):
+//   1. dot_kernel   D_t for every query row (read O and dO once);
+//   2. dq_kernel    one CTA per query tile (two query blocks from the class's
+//                   pairing order); walks the union of their CSR rows:
+//                     S = Q K^T, dP = dO V^T  -> TMEM (double-buffered)
+//                     dS (bf16, shared)       <- softmax warps
+//                     dQ += dS K              (TMEM accumulator)
+//   3. dkdv_kernel  one CTA per key tile (two key blocks from the class's key
+//                   pairing order); walks the union of their CSC columns:
+//                     S^T = K Q^T, dP^T = V dO^T -> TMEM (double-buffered)
+//                     P^T, dS^T (bf16, shared)   <- elementwise warps
+//                     dV += P^T dO, dK += dS^T Q (TMEM accumulators)
+// Warp roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner and
+// MMA issuer, warps 2-5 the elementwise work with one thread per TMEM lane.
 #pragma once
 
 #include "common.cuh"
+#include "tiles.cuh"
 
 namespace gsa {
 namespace bwd {
 
-inline gsa_status launch(const void*, const void*, const void*, const void*, const float*, const void*,
-                         const gsa_block_csr*, const gsa_attn_desc*, const uint8_t*, float, void*, void*, void*,
-                         float*, cudaStream_t) {
-    return GSA_ERR_UNSUPPORTED;
+constexpr int kBlk = 64;
+constexpr int kMaxHeads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct Params {
+    const int32_t* ptr;     // CSR row_ptr (dq) or CSC col_ptr (dkdv)
+    const int32_t* idx;     // col_idx or row_idx
+    const int32_t* order;   // q_order or k_order
+    int64_t cap;
+    int S, H, nblk;
+    int64_t L;
+    const float* lse;
+    const float* dvec;      // D_t
+    __nv_bfloat16* out0;    // dq (dq_kernel) or dv (dkdv_kernel)
+    __nv_bfloat16* out1;    // dk (dkdv_kernel)
+    float scale;
+    float scale_log2;
+    uint8_t cls[kMaxHeads];
+};
+
+// ------------------------------------------------------------ D_t = dO·O
+
+template <int D>
+__global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
+                                                  const __nv_bfloat16* __restrict__ dO, float* __restrict__ dvec,
+                                                  int64_t rows) {
+    constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
+    constexpr int kRowsPerCta = 256 / kTpr;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
+    const int part = threadIdx.x % kTpr;
+    float acc = 0.f;
+    if (row < rows) {
+        const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+        const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+        const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(ah[e]);
+            const float2 fb = __bfloat1622float2(bh[e]);
+            acc = fmaf(fa.x, fb.x, acc);
+            acc = fmaf(fa.y, fb.y, acc);
+        }
+    }
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) dvec[row] = acc;
+}
+
+// ------------------------------------------------------------ dQ
+
+template <int D>
+struct DqCfg {
+    static constexpr int kAtoms = D / 64;
+    static constexpr int kStages = D == 64 ? 4 : 3;
+    static constexpr int kTileBytes = 128 * D * 2;      // Q or dO tile (128 rows)
+    static constexpr int kKVBytes = kBlk * D * 2;       // one key block of K or V
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffDO = kOffQ + kTileBytes;
+    static constexpr int kOffK = kOffDO + kTileBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffDS = kOffV + kStages * kKVBytes;
+    static constexpr int kOffBar = kOffDS + 128 * 128;
+    // full[st], empty[st], q_full, s_full[2], s_free[2], ds_full, ds_free
+    static constexpr int kNumBars = 2 * kStages + 7;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kOffList = kOffMisc + 16;
+    static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
+    static constexpr int kOffBits = kOffLive + kListMaxBlocks;
+    static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
+    static constexpr int kSmemBytes = kEnd + 1024;
+    static constexpr int kTmemCols = 512;
+    // S[b] at 128 * b, dP[b] at 128 * b + 64, dQ at 256
+    static constexpr int kTmemDQ = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
+    using C = DqCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sQ = smem + C::kOffQ;
+    uint8_t* sDO = smem + C::kOffDO;
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
+    uint8_t* sDS = smem + C::kOffDS;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + C::kStages;
+    uint64_t* q_full = bars + 2 * C::kStages;
+    uint64_t* s_full = q_full + 1;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* ds_full = s_free + 2;
+    uint64_t* ds_free = ds_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    TileList tl;
+    tl.count = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
+    tl.list = reinterpret_cast<int16_t*>(smem + C::kOffList);
+    tl.live = smem + C::kOffLive;
+    tl.bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
+    tl.bitsB = tl.bitsA + kListMaxBlocks / 32;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sh = blockIdx.x;
+    const int s = sh / p.H, h = sh % p.H;
+    const int tile = blockIdx.y;
+    const int c = p.cls[h];
+    const int nblk = p.nblk;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int qa = p.order[g * nblk + 2 * tile];
+    const int qb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < C::kStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(&s_free[0], 128);
+        mbar_init(&s_free[1], 128);
+        mbar_init(ds_full, 128);
+        mbar_init(ds_free, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, qa, qb, nblk);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int T = *tl.count;
+    const uint32_t tmem = *tmem_slot;
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, (qb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
+            for (int half = 0; half < 2; ++half) {
+                const int blk = half ? qb : qa;
+                if (blk < 0) continue;
+                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
+                    tma_load_2d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, row);
+                }
+            }
+            for (int n = 0; n < T; ++n) {
+                const int st = n % C::kStages;
+                if (n >= C::kStages &&
+                    !mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer))
+                    break;
+                mbar_arrive_expect_tx(&full[st], 2 * C::kKVBytes);
+                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(tl.list[n]) * kBlk);
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    tma_load_2d(sK + st * C::kKVBytes + at * (kBlk * 128), &tmK, &full[st], at * 64, row);
+                    tma_load_2d(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, row);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
+            constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1);
+            const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV),
+                           aDS = smem_u32(sDS);
+            bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
+            auto issue_dq = [&](int m) -> bool {
+                if (!mbar_wait(ds_full, m & 1, abort_flag, kErrTimeoutMma)) return false;
+                tc_fence_after();
+                const int st = m % C::kStages;
+#pragma unroll
+                for (int kk = 0; kk < kBlk / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(aDS + kk * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                    umma_bf16(tmem + C::kTmemDQ, ad, bd, idesc_dq, (m > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(ds_free);
+                umma_commit(&empty[st]);
+                return true;
+            };
+            for (int n = 0; ok && n < T; ++n) {
+                const int st = n % C::kStages;
+                const int buf = n & 1;
+                if (!mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                if (n >= 2 && !mbar_wait(&s_free[buf], ((n - 2) >> 1) & 1, abort_flag, kErrTimeoutMma)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int at = kk >> 2, ko = (kk & 3) * 32;
+                    const uint64_t aq = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                    const uint64_t bk = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                    umma_bf16(tmem + buf * 128, aq, bk, idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int at = kk >> 2, ko = (kk & 3) * 32;
+                    const uint64_t ado = sdesc_sw128(aDO + at * (128 * 128) + ko, 16, 1024);
+                    const uint64_t bv = sdesc_sw128(aV + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                    umma_bf16(tmem + buf * 128 + 64, ado, bv, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[buf]);
+                if (n >= 1 && !issue_dq(n - 1)) { ok = false; break; }
+            }
+            if (ok && T > 0) issue_dq(T - 1);
+        }
+        __syncwarp();
+    } else {
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int half = r >> 6;
+        const int my_blk = half ? qb : qa;
+        const int rr = r & 63;
+        const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + rr;
+        const float lse2 = my_blk >= 0 ? p.lse[tok] * kLog2e : 0.f;
+        const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
+        bool ok = true;
+        for (int n = 0; n < T; ++n) {
+            const int buf = n & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[kBlk], dp[kBlk];
+            tmem_ld32(tlane + buf * 128, sv);
+            tmem_ld32(tlane + buf * 128 + 32, sv + 32);
+            tmem_ld32(tlane + buf * 128 + 64, dp);
+            tmem_ld32(tlane + buf * 128 + 96, dp + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_free[buf]);
+            const int j = tl.list[n];
+            const bool is_live = (tl.live[n] >> half) & 1;
+            const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);
+#pragma unroll
+            for (int cc = 0; cc < kBlk; ++cc) {
+                const float pr = cc <= last ? ex2(fmaf(sv[cc], p.scale_log2, -lse2)) : 0.f;
+                sv[cc] = pr * (dp[cc] - dt);
+            }
+            if (n >= 1 &&
+                !__all_sync(0xffffffffu, mbar_wait(ds_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
+            }
+            store_row_sw128(sDS, r, sv);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        if (ok && T > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(ds_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            tc_fence_after();
+            __nv_bfloat16* orow = p.out0 + tok * D;
+#pragma unroll
+            for (int cb = 0; cb < D; cb += 32) {
+                float ov[32];
+                tmem_ld32(tlane + C::kTmemDQ + cb, ov);
+                tmem_wait_ld();
+                if (my_blk >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(ov[e + 0] * p.scale, ov[e + 1] * p.scale);
+                        pk.y = pack_bf16x2(ov[e + 2] * p.scale, ov[e + 3] * p.scale);
+                        pk.z = pack_bf16x2(ov[e + 4] * p.scale, ov[e + 5] * p.scale);
+                        pk.w = pack_bf16x2(ov[e + 6] * p.scale, ov[e + 7] * p.scale);
+                        *reinterpret_cast<uint4*>(orow + cb + e) = pk;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------ dK, dV
+
+template <int D>
+struct DkvCfg {
+    static constexpr int kAtoms = D / 64;
+    static constexpr int kStages = 3;
+    static constexpr int kTileBytes = 128 * D * 2;      // K or V tile (128 key rows)
+    static constexpr int kQBytes = kBlk * D * 2;        // one query block of Q or dO
+    static constexpr int kVecBytes = kBlk * 4;          // LSE or D of one query block
+    static constexpr int kStageBytes = 2 * kQBytes;          // stage: Q, dO (TMA, 1024-aligned)
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kTileBytes;
+    static constexpr int kOffStage = kOffV + kTileBytes;
+    static constexpr int kOffPT = kOffStage + kStages * kStageBytes;
+    static constexpr int kOffDST = kOffPT + 128 * 128;
+    static constexpr int kOffVec = kOffDST + 128 * 128;      // per stage: LSE[64], D[64]
+    static constexpr int kOffBar = kOffVec + kStages * 2 * kVecBytes;
+    // full[st], empty[st], kv_full, s_full[2], s_free[2], p_full, p_free
+    static constexpr int kNumBars = 2 * kStages + 7;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kOffList = kOffMisc + 16;
+    static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
+    static constexpr int kOffBits = kOffLive + kListMaxBlocks;
+    static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
+    static constexpr int kSmemBytes = kEnd + 1024;
+    static constexpr int kTmemCols = 512;
+    // S^T[b] at 128 * b, dP^T[b] at 128 * b + 64, dV at 256, dK at 256 + D
+    static constexpr int kTmemDV = 256;
+    static constexpr int kTmemDK = 256 + D;
+    static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
+    using C = DkvCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
+    uint8_t* sStage = smem + C::kOffStage;
+    uint8_t* sPT = smem + C::kOffPT;
+    uint8_t* sDST = smem + C::kOffDST;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + C::kStages;
+    uint64_t* kv_full = bars + 2 * C::kStages;
+    uint64_t* s_full = kv_full + 1;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* p_full = s_free + 2;
+    uint64_t* p_free = p_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    TileList tl;
+    tl.count = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
+    tl.list = reinterpret_cast<int16_t*>(smem + C::kOffList);
+    tl.live = smem + C::kOffLive;
+    tl.bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
+    tl.bitsB = tl.bitsA + kListMaxBlocks / 32;
+    auto stage_q = [&](int st) { return sStage + st * C::kStageBytes; };
+    auto stage_do = [&](int st) { return sStage + st * C::kStageBytes + C::kQBytes; };
+    auto stage_lse = [&](int st) { return reinterpret_cast<float*>(smem + C::kOffVec + st * 2 * C::kVecBytes); };
+    auto stage_d = [&](int st) {
+        return reinterpret_cast<float*>(smem + C::kOffVec + st * 2 * C::kVecBytes + C::kVecBytes);
+    };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sh = blockIdx.x;
+    const int s = sh / p.H, h = sh % p.H;
+    const int tile = blockIdx.y;
+    const int c = p.cls[h];
+    const int nblk = p.nblk;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int ka = p.order[g * nblk + 2 * tile];
+    const int kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < C::kStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        mbar_init(kv_full, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(&s_free[0], 128);
+        mbar_init(&s_free[1], 128);
+        mbar_init(p_full, 128);
+        mbar_init(p_free, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, ka, kb, nblk);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int T = *tl.count;
+    const uint32_t tmem = *tmem_slot;
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
+            for (int half = 0; half < 2; ++half) {
+                const int blk = half ? kb : ka;
+                if (blk < 0) continue;
+                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    tma_load_2d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, row);
+                    tma_load_2d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, row);
+                }
+            }
+            for (int n = 0; n < T; ++n) {
+                const int st = n % C::kStages;
+                if (n >= C::kStages &&
+                    !mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer))
+                    break;
+                mbar_arrive_expect_tx(&full[st], C::kStageBytes + 2 * C::kVecBytes);
+                const int64_t row64 = head_row0 + static_cast<int64_t>(tl.list[n]) * kBlk;
+                const int row = static_cast<int>(row64);
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    tma_load_2d(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, row);
+                    tma_load_2d(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, row);
+                }
+                bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
+                bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
+            constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), aDST = smem_u32(sDST);
+            bool ok = mbar_wait(kv_full, 0, abort_flag, kErrTimeoutMma);
+            auto issue_acc = [&](int m) -> bool {
+                if (!mbar_wait(p_full, m & 1, abort_flag, kErrTimeoutMma)) return false;
+                tc_fence_after();
+                const int st = m % C::kStages;
+                const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+#pragma unroll
+                for (int kk = 0; kk < kBlk / 16; ++kk) {
+                    const uint64_t ap = sdesc_sw128(aPT + kk * 32, 16, 1024);
+                    const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
+                    umma_bf16(tmem + C::kTmemDV, ap, bdo, idesc_acc, (m > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kBlk / 16; ++kk) {
+                    const uint64_t ads = sdesc_sw128(aDST + kk * 32, 16, 1024);
+                    const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
+                    umma_bf16(tmem + C::kTmemDK, ads, bq, idesc_acc, (m > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(p_free);
+                umma_commit(&empty[st]);
+                return true;
+            };
+            for (int n = 0; ok && n < T; ++n) {
+                const int st = n % C::kStages;
+                const int buf = n & 1;
+                if (!mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                if (n >= 2 && !mbar_wait(&s_free[buf], ((n - 2) >> 1) & 1, abort_flag, kErrTimeoutMma)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int at = kk >> 2, ko = (kk & 3) * 32;
+                    const uint64_t ak = sdesc_sw128(aK + at * (128 * 128) + ko, 16, 1024);
+                    const uint64_t bq = sdesc_sw128(aQs + at * (kBlk * 128) + ko, 16, 1024);
+                    umma_bf16(tmem + buf * 128, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int at = kk >> 2, ko = (kk & 3) * 32;
+                    const uint64_t av = sdesc_sw128(aV + at * (128 * 128) + ko, 16, 1024);
+                    const uint64_t bdo = sdesc_sw128(aDOs + at * (kBlk * 128) + ko, 16, 1024);
+                    umma_bf16(tmem + buf * 128 + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[buf]);
+                if (n >= 1 && !issue_acc(n - 1)) { ok = false; break; }
+            }
+            if (ok && T > 0) issue_acc(T - 1);
+        }
+        __syncwarp();
+    } else {
+        const int quad = warp & 3;
+        const int u = quad * 32 + lane;          // key row of the tile = TMEM lane
+        const int half = u >> 6;
+        const int my_blk = half ? kb : ka;
+        const int uu = u & 63;
+        const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        bool ok = true;
+        for (int n = 0; n < T; ++n) {
+            const int buf = n & 1;
+            const int st = n % C::kStages;
+            bool w_ok = mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax);
+            // the stage's LSE and D came in by TMA: observe its barrier too
+            w_ok = w_ok && mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
+            if (!__all_sync(0xffffffffu, w_ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[kBlk], dp[kBlk];
+            tmem_ld32(tlane + buf * 128, sv);
+            tmem_ld32(tlane + buf * 128 + 32, sv + 32);
+            tmem_ld32(tlane + buf * 128 + 64, dp);
+            tmem_ld32(tlane + buf * 128 + 96, dp + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_free[buf]);
+            const int i = tl.list[n];
+            const bool is_live = (tl.live[n] >> half) & 1;
+            // query columns cc allowed: live block, and in the diagonal block t >= u
+            const int first = !is_live ? kBlk : (i == my_blk ? uu : 0);
+            const float* lse = stage_lse(st);
+            const float* dv = stage_d(st);
+#pragma unroll
+            for (int cc = 0; cc < kBlk; ++cc) {
+                const float pr = cc >= first ? ex2(fmaf(sv[cc], p.scale_log2, -lse[cc] * kLog2e)) : 0.f;
+                sv[cc] = pr;
+                dp[cc] = pr * (dp[cc] - dv[cc]);
+            }
+            if (n >= 1 &&
+                !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
+            }
+            store_row_sw128(sPT, u, sv);
+            store_row_sw128(sDST, u, dp);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (ok && T > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            tc_fence_after();
+            const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
+                const float mul = which == 0 ? 1.f : p.scale;
+                const uint32_t col = which == 0 ? C::kTmemDV : C::kTmemDK;
+#pragma unroll
+                for (int cb = 0; cb < D; cb += 32) {
+                    float ov[32];
+                    tmem_ld32(tlane + col + cb, ov);
+                    tmem_wait_ld();
+                    if (my_blk >= 0) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(ov[e + 0] * mul, ov[e + 1] * mul);
+                            pk.y = pack_bf16x2(ov[e + 2] * mul, ov[e + 3] * mul);
+                            pk.z = pack_bf16x2(ov[e + 4] * mul, ov[e + 5] * mul);
+                            pk.w = pack_bf16x2(ov[e + 6] * mul, ov[e + 7] * mul);
+                            *reinterpret_cast<uint4*>(orow + cb + e) = pk;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------ launch
+
+template <int D>
+gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                    const __nv_bfloat16* o, const __nv_bfloat16* dO, Params pq, Params pkv, int64_t rows, int S,
+                    int H, int nblk, cudaStream_t st) {
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemBytes);
+        cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvCfg<D>::kSmemBytes);
+    });
+    constexpr int kRowsPerCta = 256 / (D / 8);
+    dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
+        o, dO, const_cast<float*>(pq.dvec), rows);
+    dim3 grid(S * H, (nblk + 1) / 2);
+    dq_kernel<D><<<grid, 192, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+    dkdv_kernel<D><<<grid, 192, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+    return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+inline gsa_status launch(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                         const gsa_block_csr* csr, const gsa_attn_desc* desc, const uint8_t* cls, float scale,
+                         void* dq, void* dk, void* dv, float* work, cudaStream_t st) {
+    if ((reinterpret_cast<uintptr_t>(lse) & 15u) || (reinterpret_cast<uintptr_t>(work) & 15u))
+        return GSA_ERR_INVALID_ARGUMENT;
+    const int64_t rows = static_cast<int64_t>(desc->B) * desc->H * desc->L;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_tmap_bf16(&tq, q, rows, desc->d) || !make_tmap_bf16(&tk, k, rows, desc->d) ||
+        !make_tmap_bf16(&tv, v, rows, desc->d) || !make_tmap_bf16(&tdo, dO, rows, desc->d))
+        return GSA_ERR_CUDA;
+    Params base{};
+    base.cap = csr->capacity;
+    base.S = desc->B;
+    base.H = desc->H;
+    base.nblk = csr->nblk;
+    base.L = desc->L;
+    base.lse = lse;
+    base.dvec = work;
+    base.scale = scale;
+    base.scale_log2 = scale * kLog2e;
+    for (int h = 0; h < desc->H; ++h) base.cls[h] = cls[h];
+    Params pq = base, pkv = base;
+    pq.ptr = csr->row_ptr;
+    pq.idx = csr->col_idx;
+    pq.order = csr->q_order;
+    pq.out0 = static_cast<__nv_bfloat16*>(dq);
+    pq.out1 = nullptr;
+    pkv.ptr = csr->col_ptr;
+    pkv.idx = csr->row_idx;
+    pkv.order = csr->k_order;
+    pkv.out0 = static_cast<__nv_bfloat16*>(dv);
+    pkv.out1 = static_cast<__nv_bfloat16*>(dk);
+    const auto* ob = static_cast<const __nv_bfloat16*>(o);
+    const auto* dob = static_cast<const __nv_bfloat16*>(dO);
+    if (desc->d == 64) return launch_d<64>(tq, tk, tv, tdo, ob, dob, pq, pkv, rows, desc->B, desc->H, csr->nblk, st);
+    return launch_d<128>(tq, tk, tv, tdo, ob, dob, pq, pkv, rows, desc->B, desc->H, csr->nblk, st);
 }
 
 }  // namespace bwd

@@ -4,7 +4,6 @@
 // word is a single symbol.
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstring>
@@ -26,36 +25,6 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 gsa_status launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
-}
-
-// ---- TMA descriptor encoding through the driver entry point (no -lcuda)
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// A bf16 [rows][cols] row-major matrix, 64 x 64 boxes, 128-byte swizzle.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 bool csr_ok(const gsa_block_csr* c) {
@@ -199,8 +168,8 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     const uint64_t rows = static_cast<uint64_t>(desc->B) * desc->H * desc->L;
     if (rows >= (1ull << 31)) return GSA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
-    if (!make_tmap_bf16(&tq, q, rows, desc->d) || !make_tmap_bf16(&tk, k, rows, desc->d) ||
-        !make_tmap_bf16(&tv, v, rows, desc->d))
+    if (!gsa::make_tmap_bf16(&tq, q, rows, desc->d) || !gsa::make_tmap_bf16(&tk, k, rows, desc->d) ||
+        !gsa::make_tmap_bf16(&tv, v, rows, desc->d))
         return GSA_ERR_CUDA;
     gsa::bf16::FwdParams p;
     p.row_ptr = csr->row_ptr;

@@ -1,0 +1,93 @@
+// The tile list of one attention CTA: the union of two block lists (two CSR
+// rows for a query tile, two CSC columns for a key tile), ascending, with a
+// two-bit mark per entry telling which of the two halves it is live for.
+#pragma once
+
+#include "common.cuh"
+
+namespace gsa {
+
+constexpr int kListMaxBlocks = 2048;
+
+struct TileList {
+    int16_t* list;    // [kListMaxBlocks] block index per tile
+    uint8_t* live;    // [kListMaxBlocks] bit 0: live for half 0, bit 1: for half 1
+    uint32_t* bitsA;  // [kListMaxBlocks / 32]
+    uint32_t* bitsB;  // [kListMaxBlocks / 32]
+    int* count;       // number of entries
+};
+
+// Whole CTA.  ptr/idx: CSR (or CSC) arrays of this (sample, class), a and b:
+// the two rows (b < 0: none).  Ends with __syncthreads().
+__device__ __forceinline__ void build_tile_list(const TileList& t, const int32_t* ptr, const int32_t* idx, int a,
+                                                int b, int nblk) {
+    const int nwords = (nblk + 31) >> 5;
+    for (int k = threadIdx.x; k < nwords; k += blockDim.x) {
+        t.bitsA[k] = 0u;
+        t.bitsB[k] = 0u;
+    }
+    __syncthreads();
+    for (int e = ptr[a] + threadIdx.x; e < ptr[a + 1]; e += blockDim.x) {
+        const int j = idx[e];
+        atomicOr(&t.bitsA[j >> 5], 1u << (j & 31));
+    }
+    if (b >= 0) {
+        for (int e = ptr[b] + threadIdx.x; e < ptr[b + 1]; e += blockDim.x) {
+            const int j = idx[e];
+            atomicOr(&t.bitsB[j >> 5], 1u << (j & 31));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (nwords + 31) >> 5;
+        const int w0 = lane * per, w1 = min(nwords, w0 + per);
+        int cnt = 0;
+        for (int k = w0; k < w1; ++k) cnt += __popc(t.bitsA[k] | t.bitsB[k]);
+        int incl = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int pos = incl - cnt;
+        for (int k = w0; k < w1; ++k) {
+            const uint32_t ua = t.bitsA[k], ub = t.bitsB[k];
+            uint32_t u = ua | ub;
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                u &= u - 1;
+                t.list[pos] = static_cast<int16_t>(32 * k + bit);
+                t.live[pos] = static_cast<uint8_t>(((ua >> bit) & 1u) | (((ub >> bit) & 1u) << 1));
+                ++pos;
+            }
+        }
+        if (lane == 31) *t.count = incl;
+    }
+    __syncthreads();
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing `bar`'s transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Store 64 fp32 values of one row as bf16 into a 128-byte-swizzled K-major
+// tile (row r at r * 128 bytes, 16-byte chunk c at (c ^ (r % 8)) * 16).
+__device__ __forceinline__ void store_row_sw128(uint8_t* tile, int r, const float* v) {
+    uint8_t* row = tile + r * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]);
+        pk.y = pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]);
+        pk.z = pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]);
+        pk.w = pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]);
+        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = pk;
+    }
+}
+
+}  // namespace gsa
