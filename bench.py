@@ -82,17 +82,28 @@ class ClockSampler:
         self.path = None
         self.device = device_index
 
-    def start(self):
+    def _select(self):
+        """nvidia-smi -i argument for the CUDA device (its UUID), if known."""
         try:
             import torch
-            bus = getattr(torch.cuda.get_device_properties(self.device), "pci_bus_id", None)
+            u = getattr(torch.cuda.get_device_properties(self.device), "uuid", None)
+            if u is not None:
+                u = str(u)
+                return u if u.startswith("GPU-") else "GPU-" + u
         except Exception:
-            bus = None
+            pass
+        return None
+
+    def start(self):
+        sel = self._select()
         fd, self.path = tempfile.mkstemp(prefix="gsa_clocks_", suffix=".csv")
         os.close(fd)
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
-        if bus is not None:
-            cmd += ["-i", str(bus)]
+        if sel is not None:
+            probe = subprocess.run(["nvidia-smi", "-i", sel, "--query-gpu=index", "--format=csv,noheader"],
+                                   capture_output=True, text=True)
+            if probe.returncode == 0 and probe.stdout.strip():
+                cmd += ["-i", sel]
         try:
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
@@ -162,18 +173,21 @@ def oracle_inputs(wl, seed):
 
 
 def cpu_baseline(wl, budget_s=12.0, seed=0):
+    """The oracle on the host cores over a bounded sample of the workload:
+    (sample, head) units, one head of each class first, until budget_s."""
     x, q, k, v, do = oracle_inputs(wl, seed)
     hc = wl.head_classes()
-    order = [0, wl.H // 2, 3 * wl.H // 4]          # one head of each class, then the rest
+    order = [0, wl.H // 2, 3 * wl.H // 4]
     order += [h for h in range(wl.H) if h not in order]
-    flops, t0, heads = 0, time.perf_counter(), 0
-    while heads < 3 or (time.perf_counter() - t0 < budget_s and heads < len(order)):
-        flops += oracle_sample_step(wl, x, q, k, v, do, hc, order[heads % len(order)])
-        heads += 1
+    flops, t0, units = 0, time.perf_counter(), 0
+    while units < 3 or time.perf_counter() - t0 < budget_s:
+        flops += oracle_sample_step(wl, x, q, k, v, do, hc, order[units % len(order)])
+        units += 1
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"sample 0 of {wl.S}: gzip lengths, flags and mask, then forward + backward of "
-                      f"{heads} of {wl.H} heads (one per class first), float64 numpy; {dt:.1f} s"}
+            "sample": f"{units} (sample, head) units of the {wl.S}x{wl.H} workload: each the gzip lengths, "
+                      f"flags and mask of a sample and the forward + backward of one head (classes in "
+                      f"turn), float64 numpy; {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -311,6 +325,21 @@ def run_ours(args, rank, world, local_rank):
     value = world * step_flops / (ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the API with host buffers
+    e2e = None if args.no_e2e else e2e_timing(args, gsa, step, x_host, x, q, k, v, do, dq, dk, dv, stream,
+                                                 world, dev, step_flops)
+
+    # ---- mask-stage sweep (secondary metric), rank 0
+    mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
+
+    if rank != 0:
+        return 0
+    return report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops,
+                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask)
+
+
+def e2e_timing(args, gsa, step, x_host, x, q, k, v, do, dq, dk, dv, stream, world, dev, step_flops):
+    import torch
+    import torch.distributed as dist
     x_pin = torch.from_numpy(x_host).pin_memory()
     q_pin, k_pin, v_pin, do_pin = (t.cpu().pin_memory() for t in (q, k, v, do))
     dq_pin, dk_pin, dv_pin = (torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv))
@@ -342,12 +371,12 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": e2e_ms}
 
-    # ---- mask-stage sweep (secondary metric), rank 0
-    mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
 
-    if rank != 0:
-        return 0
+def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops, pairs,
+           dense_pairs, launches_per_step, e2e, clocks, mask):
     call_ms = {n: float(per_call[:, j].mean()) for j, n in enumerate(names)}
     bwd_ms, fwd_ms = call_ms["gsa_attn_bwd"], call_ms["gsa_attn_fwd"]
     peak_t = peaks["bf16_tflops_sustained"]
@@ -371,8 +400,7 @@ def run_ours(args, rank, world, local_rank):
                          "unit": "TFLOP/s", "frac": fwd_ach / peak_t, "traffic": _traffic_record("gsa_attn_fwd")},
         "call_ms": call_ms,
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": e2e_ms},
+        "e2e": e2e,
         "clocks": clocks,
     }
     if mask:
@@ -442,6 +470,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-mask-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
