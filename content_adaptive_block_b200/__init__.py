@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "GsaError", "BlockCsr", "HEAD_LOCAL", "HEAD_LITERAL", "HEAD_HYBRID",
     "gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_csr_capacity",
-    "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_device_error",
+    "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_attn_bwd_noalloc", "gsa_device_error",
     "gsa_status_string", "library", "library_path",
 ]
 
@@ -256,6 +256,32 @@ def gsa_attn_bwd(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), ctypes.byref(st), ctypes.byref(desc),
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+    del keep
+    return dq, dk, dv
+
+
+def gsa_attn_bwd_noalloc(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,
+                         dq=None, dk=None, dv=None, stream=None):
+    """gsa_attn_bwd without a workspace argument: the library's built-in
+    scratch array is used and nothing is allocated by the library (for
+    callers that cannot allocate device memory).  Calls that overlap on the
+    GPU race on that array; the first call on a device must precede any
+    stream capture."""
+    lib = library()
+    fn = lib.gsa_attn_bwd_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc), vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, name, q.dtype, 4)
+    _need(lse, "lse", torch.float32, 3)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    desc, keep = _desc(q, b, head_classes, scale)
+    st = csr.struct()
+    _check("gsa_attn_bwd_noalloc", fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), ctypes.byref(st),
+                                      ctypes.byref(desc), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))
     del keep
     return dq, dk, dv
 

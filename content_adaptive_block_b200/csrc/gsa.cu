@@ -27,6 +27,40 @@ gsa_status launch_status() {
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
+// ---- scratch of gsa_attn_bwd_noalloc
+//
+// Some callers cannot allocate device memory themselves (a host framework
+// that owns every byte through its own pool, or a latency-bound loop that
+// cannot afford cudaMalloc's implicit synchronisation).  For them the
+// backward's per-row scratch (D_t = dO_t · O_t, float32) lives in this
+// fixed array, which every GPU that loads the library holds until exit.
+constexpr int64_t kNoAllocRows = int64_t(1) << 21;   // query rows (B*H*L); 8 MiB
+static __device__ __align__(256) float g_bwd_noalloc_scratch[kNoAllocRows];
+constexpr int kMaxDevices = 64;
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the symbol itself as an address).
+float* noalloc_scratch(gsa_status* st) {
+    static std::mutex mu;
+    static float* addr[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = GSA_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch) != cudaSuccess || !p) {
+            *st = GSA_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = static_cast<float*>(p);
+    }
+    *st = GSA_OK;
+    return addr[dev];
+}
+
 bool csr_ok(const gsa_block_csr* c) {
     return c && c->B >= 1 && c->nblk >= 1 && c->row_ptr && c->col_idx && c->col_ptr && c->row_idx && c->q_order &&
            c->k_order && c->capacity >= gsa_csr_capacity(c->nblk);
@@ -227,6 +261,26 @@ gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void*
     return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, static_cast<float*>(workspace),
                             as_stream(stream));
 }
+
+gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dO, const gsa_block_csr* csr, const gsa_attn_desc* desc, void* dq,
+                                void* dk, void* dv, void* stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GSA_ERR_INVALID_ARGUMENT;
+    uint8_t cls[GSA_MAX_HEADS];
+    gsa_status st = check_attn(desc, csr, cls);
+    if (st != GSA_OK) return st;
+    if (desc->dtype != GSA_BF16) return GSA_ERR_UNSUPPORTED;
+    if (desc->b != gsa::bf16::kBlk || !(desc->d == 64 || desc->d == 128) || csr->nblk > GSA_MAX_BLOCKS_BF16)
+        return GSA_ERR_UNSUPPORTED;
+    const int64_t rows = static_cast<int64_t>(desc->B) * desc->H * desc->L;
+    if (rows > kNoAllocRows) return GSA_ERR_CAPACITY;
+    float* scratch = noalloc_scratch(&st);
+    if (st != GSA_OK) return st;
+    const float scale = desc->scale > 0.f ? desc->scale : 1.f / std::sqrt(static_cast<float>(desc->d));
+    return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, scratch, as_stream(stream));
+}
+
+int64_t gsa_attn_bwd_noalloc_max_rows(void) { return kNoAllocRows; }
 
 gsa_status gsa_device_error(int32_t* code, int32_t clear) {
     if (!code) return GSA_ERR_INVALID_ARGUMENT;

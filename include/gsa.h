@@ -204,6 +204,35 @@ gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void*
 size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc);
 
 /*
+ * gsa_attn_bwd_noalloc — gsa_attn_bwd for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a deployment
+ * variant.  Some callers own no allocator of their own (a host framework
+ * that hands out every device byte from its pool and forbids other
+ * allocations) or cannot afford cudaMalloc's implicit device
+ * synchronisation in their loop.  This call needs no workspace argument: its
+ * float32 scratch (D_t, one value per query row) is a fixed array compiled
+ * into the library, at most gsa_attn_bwd_noalloc_max_rows() rows
+ * (2^21 = B*H*L; 8 MiB, held on every GPU that loads the library until the
+ * process exits).  The caller still passes all inputs and outputs, exactly as
+ * for gsa_attn_bwd; results are identical.
+ *   - Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (every call overwrites the rows it uses before reading them, so nothing
+ *     needs clearing).  Calls that overlap on the GPU (other streams, other
+ *     threads) race on it: serialise them.
+ * Errors: as gsa_attn_bwd; GSA_ERR_CAPACITY when B*H*L exceeds the maximum.
+ */
+gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dO, const gsa_block_csr* csr,
+                                const gsa_attn_desc* desc, void* dq, void* dk, void* dv, void* stream);
+
+/* Rows (B*H*L) gsa_attn_bwd_noalloc can take. */
+int64_t gsa_attn_bwd_noalloc_max_rows(void);
+
+/*
  * gsa_device_error — read (and optionally clear) the library's device error
  * word.  Kernels that give up a bounded wait record a nonzero code there
  * instead of hanging.  Synchronises the device.  *code receives the word
