@@ -98,7 +98,7 @@ class ClockSampler:
         sel = self._select()
         fd, self.path = tempfile.mkstemp(prefix="gsa_clocks_", suffix=".csv")
         os.close(fd)
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if sel is not None:
             probe = subprocess.run(["nvidia-smi", "-i", sel, "--query-gpu=index", "--format=csv,noheader"],
                                    capture_output=True, text=True)
@@ -465,7 +465,7 @@ def mask_stage(gsa, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-mask-sweep", action="store_true")

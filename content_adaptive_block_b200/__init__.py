@@ -31,7 +31,8 @@ HEAD_LOCAL, HEAD_LITERAL, HEAD_HYBRID = 0, 1, 2
 GSA_F32, GSA_BF16 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "lib", "libgsa.so")
+# GSA_LIBRARY_PATH may point at another build of the same library (tuning).
+_LIB_PATH = os.environ.get("GSA_LIBRARY_PATH") or os.path.join(_HERE, "lib", "libgsa.so")
 _lib = None
 
 

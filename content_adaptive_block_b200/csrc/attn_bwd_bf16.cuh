@@ -31,6 +31,13 @@ namespace bwd {
 constexpr int kBlk = 64;
 constexpr int kMaxHeads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
+// Elementwise warpgroups: each TMEM lane (tile row) is shared by kEwGroups
+// threads, one per group, each owning kCw of the tile's 64 columns.
+constexpr int kEwGroups = 2;
+constexpr int kCw = kBlk / kEwGroups;
+constexpr int kEwThreads = 128 * kEwGroups;
+constexpr int kThreads = 64 + kEwThreads;
+static_assert(kCw == 32, "one 32-column TMEM load per operand");
 
 struct Params {
     const int32_t* ptr;     // CSR row_ptr (dq) or CSC col_ptr (dkdv)
@@ -79,10 +86,24 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
 
 // ------------------------------------------------------------ dQ
 
+// Ring depths: a stage is released after the last MMA that reads it.
+#ifndef GSA_DQ64_STAGES
+#define GSA_DQ64_STAGES 4
+#endif
+#ifndef GSA_DQ128_STAGES
+#define GSA_DQ128_STAGES 3
+#endif
+#ifndef GSA_DKV64_STAGES
+#define GSA_DKV64_STAGES 3
+#endif
+#ifndef GSA_DKV128_STAGES
+#define GSA_DKV128_STAGES 3
+#endif
+
 template <int D>
 struct DqCfg {
     static constexpr int kAtoms = D / 64;
-    static constexpr int kStages = D == 64 ? 4 : 3;
+    static constexpr int kStages = D == 64 ? GSA_DQ64_STAGES : GSA_DQ128_STAGES;
     static constexpr int kTileBytes = 128 * D * 2;      // Q or dO tile (128 rows)
     static constexpr int kKVBytes = kBlk * D * 2;       // one key block of K or V
     static constexpr int kOffQ = 0;
@@ -99,13 +120,14 @@ struct DqCfg {
     static constexpr int kOffBits = kOffLive + kListMaxBlocks;
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr int kTmemCols = 512;
     // S[b] at 128 * b, dP[b] at 128 * b + 64, dQ at 256
     static constexpr int kTmemDQ = 256;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
     using C = DqCfg<D>;
@@ -151,9 +173,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
-        mbar_init(ds_full, 128);
+        mbar_init(&s_free[0], kEwThreads);
+        mbar_init(&s_free[1], kEwThreads);
+        mbar_init(ds_full, kEwThreads);
         mbar_init(ds_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -246,7 +268,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         __syncwarp();
     } else {
-        const int quad = warp & 3;
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int grp = (warp - 2) >> 2;        // column group
+        const int c0 = grp * kCw;               // first key column of this thread
         const int r = quad * 32 + lane;
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
@@ -263,28 +287,34 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 break;
             }
             tc_fence_after();
-            float sv[kBlk], dp[kBlk];
-            tmem_ld32(tlane + buf * 128, sv);
-            tmem_ld32(tlane + buf * 128 + 32, sv + 32);
-            tmem_ld32(tlane + buf * 128 + 64, dp);
-            tmem_ld32(tlane + buf * 128 + 96, dp + 32);
+            float sv[kCw], dp[kCw];
+            tmem_ld32(tlane + buf * 128 + c0, sv);
+            tmem_ld32(tlane + buf * 128 + 64 + c0, dp);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free[buf]);
             const int j = tl.list[n];
             const bool is_live = (tl.live[n] >> half) & 1;
-            const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);
+            const int last = (!is_live ? -1 : (j == my_blk ? rr : kBlk - 1)) - c0;
+            if (last >= kCw - 1) {
 #pragma unroll
-            for (int cc = 0; cc < kBlk; ++cc) {
-                const float pr = cc <= last ? ex2(fmaf(sv[cc], p.scale_log2, -lse2)) : 0.f;
-                sv[cc] = pr * (dp[cc] - dt);
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -lse2)) * (dp[cc] - dt);
+            } else if (last < 0) {
+#pragma unroll
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = 0.f;
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < kCw; ++cc) {
+                    const float pr = cc <= last ? ex2(fmaf(sv[cc], p.scale_log2, -lse2)) : 0.f;
+                    sv[cc] = pr * (dp[cc] - dt);
+                }
             }
             if (n >= 1 &&
                 !__all_sync(0xffffffffu, mbar_wait(ds_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
-            store_row_sw128(sDS, r, sv);
+            store_cols_sw128(sDS, r, sv, c0 / 8, kCw / 8);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(ds_full);
@@ -293,22 +323,13 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             __all_sync(0xffffffffu, mbar_wait(ds_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             __nv_bfloat16* orow = p.out0 + tok * D;
+            constexpr int kOc = D / kEwGroups;   // output columns per thread
 #pragma unroll
-            for (int cb = 0; cb < D; cb += 32) {
+            for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
                 float ov[32];
                 tmem_ld32(tlane + C::kTmemDQ + cb, ov);
                 tmem_wait_ld();
-                if (my_blk >= 0) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(ov[e + 0] * p.scale, ov[e + 1] * p.scale);
-                        pk.y = pack_bf16x2(ov[e + 2] * p.scale, ov[e + 3] * p.scale);
-                        pk.z = pack_bf16x2(ov[e + 4] * p.scale, ov[e + 5] * p.scale);
-                        pk.w = pack_bf16x2(ov[e + 6] * p.scale, ov[e + 7] * p.scale);
-                        *reinterpret_cast<uint4*>(orow + cb + e) = pk;
-                    }
-                }
+                if (my_blk >= 0) store_scaled_bf16(orow + cb, ov, p.scale);
             }
         }
     }
@@ -325,7 +346,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 template <int D>
 struct DkvCfg {
     static constexpr int kAtoms = D / 64;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = D == 64 ? GSA_DKV64_STAGES : GSA_DKV128_STAGES;
     static constexpr int kTileBytes = 128 * D * 2;      // K or V tile (128 key rows)
     static constexpr int kQBytes = kBlk * D * 2;        // one query block of Q or dO
     static constexpr int kVecBytes = kBlk * 4;          // LSE or D of one query block
@@ -345,6 +366,7 @@ struct DkvCfg {
     static constexpr int kOffBits = kOffLive + kListMaxBlocks;
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr int kTmemCols = 512;
     // S^T[b] at 128 * b, dP^T[b] at 128 * b + 64, dV at 256, dK at 256 + D
     static constexpr int kTmemDV = 256;
@@ -353,7 +375,7 @@ struct DkvCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
     using C = DkvCfg<D>;
@@ -405,9 +427,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(kv_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
-        mbar_init(p_full, 128);
+        mbar_init(&s_free[0], kEwThreads);
+        mbar_init(&s_free[1], kEwThreads);
+        mbar_init(p_full, kEwThreads);
         mbar_init(p_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -511,6 +533,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         __syncwarp();
     } else {
         const int quad = warp & 3;
+        const int grp = (warp - 2) >> 2;
+        const int c0 = grp * kCw;                // first query column of this thread
         const int u = quad * 32 + lane;          // key row of the tile = TMEM lane
         const int half = u >> 6;
         const int my_blk = half ? kb : ka;
@@ -528,33 +552,45 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 break;
             }
             tc_fence_after();
-            float sv[kBlk], dp[kBlk];
-            tmem_ld32(tlane + buf * 128, sv);
-            tmem_ld32(tlane + buf * 128 + 32, sv + 32);
-            tmem_ld32(tlane + buf * 128 + 64, dp);
-            tmem_ld32(tlane + buf * 128 + 96, dp + 32);
+            float sv[kCw], dp[kCw];
+            tmem_ld32(tlane + buf * 128 + c0, sv);
+            tmem_ld32(tlane + buf * 128 + 64 + c0, dp);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free[buf]);
             const int i = tl.list[n];
             const bool is_live = (tl.live[n] >> half) & 1;
-            // query columns cc allowed: live block, and in the diagonal block t >= u
-            const int first = !is_live ? kBlk : (i == my_blk ? uu : 0);
-            const float* lse = stage_lse(st);
-            const float* dv = stage_d(st);
+            // query columns allowed: live block, and in the diagonal block t >= u
+            const int first = (!is_live ? kBlk : (i == my_blk ? uu : 0)) - c0;
+            const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st) + c0);
+            const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st) + c0);
+            if (first >= kCw) {
 #pragma unroll
-            for (int cc = 0; cc < kBlk; ++cc) {
-                const float pr = cc >= first ? ex2(fmaf(sv[cc], p.scale_log2, -lse[cc] * kLog2e)) : 0.f;
-                sv[cc] = pr;
-                dp[cc] = pr * (dp[cc] - dv[cc]);
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = dp[cc] = 0.f;
+            } else {
+#pragma unroll
+                for (int c4 = 0; c4 < kCw / 4; ++c4) {
+                    const float4 l4 = lse4[c4];
+                    const float4 d4 = dv4[c4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int cc = 4 * c4 + e;
+                        float pr = ex2(fmaf(sv[cc], p.scale_log2, -lv[e] * kLog2e));
+                        if (first > 0) pr = cc >= first ? pr : 0.f;
+                        sv[cc] = pr;
+                        dp[cc] = pr * (dp[cc] - dd[e]);
+                    }
+                }
             }
             if (n >= 1 &&
                 !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
-            store_row_sw128(sPT, u, sv);
-            store_row_sw128(sDST, u, dp);
+            store_cols_sw128(sPT, u, sv, c0 / 8, kCw / 8);
+            store_cols_sw128(sDST, u, dp, c0 / 8, kCw / 8);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
@@ -563,27 +599,18 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
+            constexpr int kOc = D / kEwGroups;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
                 const float mul = which == 0 ? 1.f : p.scale;
                 const uint32_t col = which == 0 ? C::kTmemDV : C::kTmemDK;
 #pragma unroll
-                for (int cb = 0; cb < D; cb += 32) {
+                for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
                     float ov[32];
                     tmem_ld32(tlane + col + cb, ov);
                     tmem_wait_ld();
-                    if (my_blk >= 0) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 pk;
-                            pk.x = pack_bf16x2(ov[e + 0] * mul, ov[e + 1] * mul);
-                            pk.y = pack_bf16x2(ov[e + 2] * mul, ov[e + 3] * mul);
-                            pk.z = pack_bf16x2(ov[e + 4] * mul, ov[e + 5] * mul);
-                            pk.w = pack_bf16x2(ov[e + 6] * mul, ov[e + 7] * mul);
-                            *reinterpret_cast<uint4*>(orow + cb + e) = pk;
-                        }
-                    }
+                    if (my_blk >= 0) store_scaled_bf16(orow + cb, ov, mul);
                 }
             }
         }
@@ -611,8 +638,8 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
         o, dO, const_cast<float*>(pq.dvec), rows);
     dim3 grid(S * H, (nblk + 1) / 2);
-    dq_kernel<D><<<grid, 192, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
-    dkdv_kernel<D><<<grid, 192, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+    dq_kernel<D><<<grid, kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+    dkdv_kernel<D><<<grid, kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 

@@ -34,6 +34,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tiles.cuh"
 
 namespace gsa {
 namespace bf16 {
@@ -42,6 +43,22 @@ constexpr int kMaxHeads = 256;
 constexpr int kMaxBlocks = 2048;
 constexpr int kBlk = 64;   // block size in tokens
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// Softmax warpgroups: the two threads of a row (one per group) own 32 of the
+// tile's 64 key columns each and exchange their partial row maxima.
+constexpr int kSmGroups = 2;
+constexpr int kCw = kBlk / kSmGroups;
+constexpr int kSmThreads = 128 * kSmGroups;
+constexpr int kFwdThreads = 64 + kSmThreads;
+
+// Named barrier (ids 1..4) joining the two warps that share a TMEM lane quadrant.
+__device__ __forceinline__ void pair_barrier(int quad) {
+    switch (quad) {
+        case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+        case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+        case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+        default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+    }
+}
 
 struct FwdParams {
     const int32_t* row_ptr;
@@ -56,10 +73,22 @@ struct FwdParams {
     uint8_t cls[kMaxHeads];
 };
 
+// K/V ring depth (one stage = one 64-key block of K and of V), and CTAs per
+// SM for d = 64 (two CTAs overlap each other's hand-offs).
+#ifndef GSA_FWD64_STAGES
+#define GSA_FWD64_STAGES 4
+#endif
+#ifndef GSA_FWD128_STAGES
+#define GSA_FWD128_STAGES 3
+#endif
+#ifndef GSA_FWD64_CTAS_PER_SM
+#define GSA_FWD64_CTAS_PER_SM 2
+#endif
+
 template <int D>
 struct FwdCfg {
     static constexpr int kAtoms = D / 64;
-    static constexpr int kStages = D == 64 ? 4 : 3;
+    static constexpr int kStages = D == 64 ? GSA_FWD64_STAGES : GSA_FWD128_STAGES;
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = kBlk * D * 2;   // one block of K (or V)
     static constexpr int kPBytes = 128 * kBlk * 2;
@@ -74,15 +103,19 @@ struct FwdCfg {
     static constexpr int kOffList = kOffMisc + 16;            // int16 key block per tile
     static constexpr int kOffLive = kOffList + kMaxBlocks * 2;
     static constexpr int kOffBits = kOffLive + kMaxBlocks;    // two bitmaps
-    static constexpr int kEnd = kOffBits + 2 * (kMaxBlocks / 32) * 4;
+    static constexpr int kOffRed = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [2 parity][2 group][128] partial maxima
+    static constexpr int kOffOk = kOffRed + 2 * 2 * 128 * 4;               // [2 parity][2 group][4 quad] flags
+    static constexpr int kOffLsum = kOffOk + 2 * 2 * 4 * 4;                // [2 group][128] partial sums
+    static constexpr int kEnd = kOffLsum + 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;            // + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr int kTmemCols = 256;
     static constexpr int kTmemS = 0;       // S buffers at columns 0 and 64
     static constexpr int kTmemO = 128;     // O at columns 128 .. 128 + D
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kFwdThreads, D == 64 ? GSA_FWD64_CTAS_PER_SM : 1)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdCfg<D>;
@@ -128,9 +161,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
-        mbar_init(p_full, 128);
+        mbar_init(&s_free[0], kSmThreads);
+        mbar_init(&s_free[1], kSmThreads);
+        mbar_init(p_full, kSmThreads);
         mbar_init(p_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -268,41 +301,56 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         __syncwarp();
     } else {
-        // ================= softmax warpgroup (warps 2..5)
+        // ================= softmax warpgroups (warps 2..9)
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int grp = (warp - 2) >> 2;        // column group
+        const int c0 = grp * kCw;               // first key column of this thread
         const int r = quad * 32 + lane;         // query row in the tile = TMEM lane
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
         const int rr = r & 63;
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        float m = -INFINITY, l = 0.f;
+        float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+        volatile int* okf = reinterpret_cast<volatile int*>(smem + C::kOffOk);
+        float* lsum = reinterpret_cast<float*>(smem + C::kOffLsum);
+        float m = -INFINITY, l = 0.f;           // l: this thread's share of the row sum
         bool ok = true;
-        uint8_t* prow = sP + r * 128;
         for (int n = 0; n < T; ++n) {
             const int buf = n & 1;
-            // waits are made warp-uniform: the tcgen05 loads below are warp-collective
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            // waits are warp-uniform (the tcgen05 loads are warp-collective); the
+            // two warps of a row pair leave the loop together, after their barrier
+            const bool w = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag,
+                                                                   kErrTimeoutSoftmax));
+            float sv[kCw];
+            if (w) {
+                tc_fence_after();
+                tmem_ld32(tl + C::kTmemS + buf * kBlk + c0, sv);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&s_free[buf]);
+            }
+            const int j = list[n];
+            const bool is_live = (live[n] >> half) & 1;
+            const int last = (!is_live ? -1 : (j == my_blk ? rr : kBlk - 1)) - c0;
+            // raw-score maximum of this thread's columns (the scale is positive);
+            // masked columns become -inf, so their exponentials below are 0
+            float mt;
+            if (last >= kCw - 1) {
+                mt = max_reduce<kCw>(sv);
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = cc <= last ? sv[cc] : -INFINITY;
+                mt = max_reduce<kCw>(sv);
+            }
+            mt *= p.scale_log2;
+            red[(buf * 2 + grp) * 128 + r] = mt;
+            if (lane == 0) okf[(buf * 2 + grp) * 4 + quad] = w ? 1 : 0;
+            pair_barrier(quad);
+            if (!(okf[(buf * 2 + 0) * 4 + quad] && okf[(buf * 2 + 1) * 4 + quad])) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            float sv[kBlk];
-            tmem_ld32(tl + C::kTmemS + buf * kBlk, sv);
-            tmem_ld32(tl + C::kTmemS + buf * kBlk + 32, sv + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_free[buf]);
-
-            const int j = list[n];
-            const bool is_live = (live[n] >> half) & 1;
-            const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);
-            float mt = -INFINITY;
-#pragma unroll
-            for (int cc = 0; cc < kBlk; ++cc) {
-                const float x = cc <= last ? sv[cc] * p.scale_log2 : -INFINITY;
-                sv[cc] = x;
-                mt = fmaxf(mt, x);
-            }
+            mt = fmaxf(mt, red[(buf * 2 + (grp ^ 1)) * 128 + r]);
             const float m_new = fmaxf(m, mt);
             float alpha = 1.f;
             bool rescale = false;
@@ -315,25 +363,29 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 rescale = true;
             }
             const float msafe = m_use == -INFINITY ? 0.f : m_use;
-            float sum = 0.f;
+            // p = 2^(s * scale * log2 e - m): one FFMA and one MUFU.EX2 per score
+            float sum;
+            if (last < 0) {
 #pragma unroll
-            for (int cc = 0; cc < kBlk; ++cc) {
-                const float pv = ex2(sv[cc] - msafe);
-                sv[cc] = pv;
-                sum += pv;
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = 0.f;
+                sum = 0.f;
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < kCw; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -msafe));
+                sum = sum_reduce<kCw>(sv);
             }
             l = l * alpha + sum;
             m = m_use;
 
             if (n >= 1 &&
                 !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
-                ok = false;
-                break;
+                ok = false;   // reported to the partner warp at the next barrier
+                continue;
             }
             tc_fence_after();
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                for (int cb = 0; cb < D; cb += 32) {
+                for (int cb = grp * (D / kSmGroups); cb < (grp + 1) * (D / kSmGroups); cb += 32) {
                     float ov[32];
                     tmem_ld32(tl + C::kTmemO + cb, ov);
                     tmem_wait_ld();
@@ -343,45 +395,29 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 tmem_wait_st();
             }
-            // P row: 64 bf16 = 8 chunks of 16 bytes, chunk index xor (row % 8)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint4 pk;
-                pk.x = pack_bf16x2(sv[8 * ch + 0], sv[8 * ch + 1]);
-                pk.y = pack_bf16x2(sv[8 * ch + 2], sv[8 * ch + 3]);
-                pk.z = pack_bf16x2(sv[8 * ch + 4], sv[8 * ch + 5]);
-                pk.w = pack_bf16x2(sv[8 * ch + 6], sv[8 * ch + 7]);
-                *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = pk;
-            }
+            store_cols_sw128(sP, r, sv, c0 / 8, kCw / 8);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
         }
+        lsum[grp * 128 + r] = l;
+        pair_barrier(quad);
+        l = lsum[r] + lsum[128 + r];
         if (ok && T > 0 &&
             __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             const float inv = 1.f / l;
             const bool store = my_blk >= 0;
-            const int64_t tok = head_row0 + static_cast<int64_t>(my_blk) * kBlk + rr;
+            const int64_t tok = head_row0 + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
             __nv_bfloat16* orow = p.o + tok * D;
 #pragma unroll
-            for (int cb = 0; cb < D; cb += 32) {
+            for (int cb = grp * (D / kSmGroups); cb < (grp + 1) * (D / kSmGroups); cb += 32) {
                 float ov[32];
                 tmem_ld32(tl + C::kTmemO + cb, ov);
                 tmem_wait_ld();
-                if (store) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(ov[e + 0] * inv, ov[e + 1] * inv);
-                        pk.y = pack_bf16x2(ov[e + 2] * inv, ov[e + 3] * inv);
-                        pk.z = pack_bf16x2(ov[e + 4] * inv, ov[e + 5] * inv);
-                        pk.w = pack_bf16x2(ov[e + 6] * inv, ov[e + 7] * inv);
-                        *reinterpret_cast<uint4*>(orow + cb + e) = pk;
-                    }
-                }
+                if (store) store_scaled_bf16(orow + cb, ov, inv);
             }
-            if (store && p.lse) p.lse[tok] = (m + log2f(l)) * 0.69314718055994531f;
+            if (store && grp == 0 && p.lse) p.lse[tok] = (m + log2f(l)) * 0.69314718055994531f;
         }
     }
 

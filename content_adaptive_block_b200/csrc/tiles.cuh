@@ -90,4 +90,58 @@ __device__ __forceinline__ void store_row_sw128(uint8_t* tile, int r, const floa
     }
 }
 
+// Store 8 * nch fp32 values as bf16 into 16-byte chunks ch0 .. ch0+nch-1 of
+// row r of a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ void store_cols_sw128(uint8_t* tile, int r, const float* v, int ch0, int nch) {
+    uint8_t* row = tile + r * 128;
+#pragma unroll
+    for (int k = 0; k < nch; ++k) {
+        const int ch = ch0 + k;
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+        pk.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+        pk.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+        pk.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = pk;
+    }
+}
+
+// Pairwise reductions (log-depth dependency chains instead of linear ones).
+template <int N>
+__device__ __forceinline__ float max_reduce(const float* v) {
+    float t[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) t[i] = fmaxf(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+    for (int w = N / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) t[i] = fmaxf(t[2 * i], t[2 * i + 1]);
+    return t[0];
+}
+
+template <int N>
+__device__ __forceinline__ float sum_reduce(const float* v) {
+    float t[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) t[i] = v[2 * i] + v[2 * i + 1];
+#pragma unroll
+    for (int w = N / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) t[i] = t[2 * i] + t[2 * i + 1];
+    return t[0];
+}
+
+// 32 fp32 values times `mul` as bf16 to global memory (16-byte stores).
+__device__ __forceinline__ void store_scaled_bf16(__nv_bfloat16* dst, const float* v, float mul) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[e + 0] * mul, v[e + 1] * mul);
+        pk.y = pack_bf16x2(v[e + 2] * mul, v[e + 3] * mul);
+        pk.z = pack_bf16x2(v[e + 4] * mul, v[e + 5] * mul);
+        pk.w = pack_bf16x2(v[e + 6] * mul, v[e + 7] * mul);
+        *reinterpret_cast<uint4*>(dst + e) = pk;
+    }
+}
+
 }  // namespace gsa
