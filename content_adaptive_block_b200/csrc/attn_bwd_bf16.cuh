@@ -31,13 +31,12 @@ namespace bwd {
 constexpr int kBlk = 64;
 constexpr int kMaxHeads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
-// Elementwise warpgroups: each TMEM lane (tile row) is shared by kEwGroups
-// threads, one per group, each owning kCw of the tile's 64 columns.
+// Elementwise warpgroups: group g takes the tiles n with n % 2 == g, one
+// thread per tile row (TMEM lane), all 64 columns, so the two groups run
+// independently and their MUFU and ALU phases overlap.
 constexpr int kEwGroups = 2;
-constexpr int kCw = kBlk / kEwGroups;
 constexpr int kEwThreads = 128 * kEwGroups;
 constexpr int kThreads = 64 + kEwThreads;
-static_assert(kCw == 32, "one 32-column TMEM load per operand");
 
 struct Params {
     const int32_t* ptr;     // CSR row_ptr (dq) or CSC col_ptr (dkdv)
@@ -88,16 +87,16 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
 
 // Ring depths: a stage is released after the last MMA that reads it.
 #ifndef GSA_DQ64_STAGES
-#define GSA_DQ64_STAGES 4
+#define GSA_DQ64_STAGES 6
 #endif
 #ifndef GSA_DQ128_STAGES
 #define GSA_DQ128_STAGES 3
 #endif
 #ifndef GSA_DKV64_STAGES
-#define GSA_DKV64_STAGES 3
+#define GSA_DKV64_STAGES 5
 #endif
 #ifndef GSA_DKV128_STAGES
-#define GSA_DKV128_STAGES 3
+#define GSA_DKV128_STAGES 2
 #endif
 
 template <int D>
@@ -111,9 +110,9 @@ struct DqCfg {
     static constexpr int kOffK = kOffDO + kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
     static constexpr int kOffDS = kOffV + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffDS + 128 * 128;
-    // full[st], empty[st], q_full, s_full[2], s_free[2], ds_full, ds_free
-    static constexpr int kNumBars = 2 * kStages + 7;
+    static constexpr int kOffBar = kOffDS + 2 * 128 * 128;    // dS double-buffered
+    // full[st], empty[st], q_full, s_full[2], s_free[2], ds_full[2], ds_free[2], done
+    static constexpr int kNumBars = 2 * kStages + 10;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -145,7 +144,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     uint64_t* s_full = q_full + 1;
     uint64_t* s_free = s_full + 2;
     uint64_t* ds_full = s_free + 2;
-    uint64_t* ds_free = ds_full + 1;
+    uint64_t* ds_free = ds_full + 2;
+    uint64_t* done = ds_free + 2;   // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -173,10 +173,13 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], kEwThreads);
-        mbar_init(&s_free[1], kEwThreads);
-        mbar_init(ds_full, kEwThreads);
-        mbar_init(ds_free, 1);
+        mbar_init(&s_free[0], 128);
+        mbar_init(&s_free[1], 128);
+        mbar_init(&ds_full[0], 128);
+        mbar_init(&ds_full[1], 128);
+        mbar_init(&ds_free[0], 1);
+        mbar_init(&ds_free[1], 1);
+        mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -224,53 +227,64 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV),
                            aDS = smem_u32(sDS);
             bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
-            auto issue_dq = [&](int m) -> bool {
-                if (!mbar_wait(ds_full, m & 1, abort_flag, kErrTimeoutMma)) return false;
-                tc_fence_after();
-                const int st = m % C::kStages;
+            // Event-driven issue (see the forward): S and dP of tile ns, dQ of tile na.
+            int ns = 0, na = 0;
+            PollGuard guard;
+            while (ok && na < T) {
+                bool moved = false;
+                if (ns < T) {
+                    const int st = ns % C::kStages, buf = ns & 1;
+                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
+                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(aDS + kk * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                    umma_bf16(tmem + C::kTmemDQ, ad, bd, idesc_dq, (m > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(ds_free);
-                umma_commit(&empty[st]);
-                return true;
-            };
-            for (int n = 0; ok && n < T; ++n) {
-                const int st = n % C::kStages;
-                const int buf = n & 1;
-                if (!mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                if (n >= 2 && !mbar_wait(&s_free[buf], ((n - 2) >> 1) & 1, abort_flag, kErrTimeoutMma)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t aq = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bk =
+                                sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + buf * 128, aq, bk, idesc_s, kk > 0 ? 1u : 0u);
+                        }
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int at = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t aq = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
-                    const uint64_t bk = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + buf * 128, aq, bk, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ado = sdesc_sw128(aDO + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bv =
+                                sdesc_sw128(aV + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + buf * 128 + 64, ado, bv, idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&s_full[buf]);
+                        ++ns;
+                        moved = true;
+                    }
                 }
+                if (na < ns) {
+                    const int db = na & 1;
+                    if (mbar_test(&ds_full[db], (na >> 1) & 1)) {
+                        tc_fence_after();
+                        const int st = na % C::kStages;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int at = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t ado = sdesc_sw128(aDO + at * (128 * 128) + ko, 16, 1024);
-                    const uint64_t bv = sdesc_sw128(aV + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + buf * 128 + 64, ado, bv, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(aDS + db * (128 * 128) + kk * 32, 16, 1024);
+                            const uint64_t bd =
+                                sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                            umma_bf16(tmem + C::kTmemDQ, ad, bd, idesc_dq, (na > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&ds_free[db]);
+                        umma_commit(&empty[st]);
+                        ++na;
+                        moved = true;
+                    }
                 }
-                umma_commit(&s_full[buf]);
-                if (n >= 1 && !issue_dq(n - 1)) { ok = false; break; }
+                if (moved) guard.progress();
+                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
             }
-            if (ok && T > 0) issue_dq(T - 1);
+            if (ok && T > 0) umma_commit(done);
         }
         __syncwarp();
     } else {
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int grp = (warp - 2) >> 2;        // column group
-        const int c0 = grp * kCw;               // first key column of this thread
+        const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
         const int r = quad * 32 + lane;
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
@@ -280,50 +294,54 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const float lse2 = my_blk >= 0 ? p.lse[tok] * kLog2e : 0.f;
         const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
         bool ok = true;
-        for (int n = 0; n < T; ++n) {
-            const int buf = n & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+        for (int n = grp; n < T; n += 2) {
+            const int ph = (n >> 1) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float sv[kCw], dp[kCw];
-            tmem_ld32(tlane + buf * 128 + c0, sv);
-            tmem_ld32(tlane + buf * 128 + 64 + c0, dp);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_free[buf]);
             const int j = tl.list[n];
             const bool is_live = (tl.live[n] >> half) & 1;
-            const int last = (!is_live ? -1 : (j == my_blk ? rr : kBlk - 1)) - c0;
-            if (last >= kCw - 1) {
+            const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);   // visible key columns 0..last
+            uint32_t pk[32];
+            if (last < 0) {
 #pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -lse2)) * (dp[cc] - dt);
-            } else if (last < 0) {
-#pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = 0.f;
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             } else {
 #pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) {
-                    const float pr = cc <= last ? ex2(fmaf(sv[cc], p.scale_log2, -lse2)) : 0.f;
-                    sv[cc] = pr * (dp[cc] - dt);
+                for (int ch = 0; ch < 2; ++ch) {
+                    float sv[32], dp[32];
+                    tmem_ld32(tlane + grp * 128 + 32 * ch, sv);
+                    tmem_ld32(tlane + grp * 128 + 64 + 32 * ch, dp);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -lse2)) * (dp[cc] - dt);
+                    if (last < 32 * ch + 31) {
+#pragma unroll
+                        for (int cc = 0; cc < 32; ++cc) sv[cc] = 32 * ch + cc <= last ? sv[cc] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(sv[2 * e], sv[2 * e + 1]);
                 }
             }
-            if (n >= 1 &&
-                !__all_sync(0xffffffffu, mbar_wait(ds_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            tc_fence_before();
+            mbar_arrive(&s_free[grp]);
+            // dS[grp] was last read by the dQ product of tile n - 2
+            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&ds_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
-            store_cols_sw128(sDS, r, sv, c0 / 8, kCw / 8);
+            store_packed_row_sw128(sDS + grp * (128 * 128), r, pk);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(ds_full);
+            mbar_arrive(&ds_full[grp]);
         }
         if (ok && T > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(ds_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             __nv_bfloat16* orow = p.out0 + tok * D;
-            constexpr int kOc = D / kEwGroups;   // output columns per thread
+            constexpr int kOc = D / kEwGroups;   // output columns per thread (split between the groups)
 #pragma unroll
             for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
                 float ov[32];
@@ -354,12 +372,12 @@ struct DkvCfg {
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kTileBytes;
     static constexpr int kOffStage = kOffV + kTileBytes;
-    static constexpr int kOffPT = kOffStage + kStages * kStageBytes;
-    static constexpr int kOffDST = kOffPT + 128 * 128;
-    static constexpr int kOffVec = kOffDST + 128 * 128;      // per stage: LSE[64], D[64]
+    static constexpr int kOffPT = kOffStage + kStages * kStageBytes;   // P^T, double-buffered
+    static constexpr int kOffDST = kOffPT + 2 * 128 * 128;             // dS^T, double-buffered
+    static constexpr int kOffVec = kOffDST + 2 * 128 * 128;            // per stage: LSE[64], D[64]
     static constexpr int kOffBar = kOffVec + kStages * 2 * kVecBytes;
-    // full[st], empty[st], kv_full, s_full[2], s_free[2], p_full, p_free
-    static constexpr int kNumBars = 2 * kStages + 7;
+    // full[st], empty[st], kv_full, s_full[2], s_free[2], p_full[2], p_free[2], done
+    static constexpr int kNumBars = 2 * kStages + 10;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -393,7 +411,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* s_full = kv_full + 1;
     uint64_t* s_free = s_full + 2;
     uint64_t* p_full = s_free + 2;
-    uint64_t* p_free = p_full + 1;
+    uint64_t* p_free = p_full + 2;
+    uint64_t* done = p_free + 2;    // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -427,10 +446,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(kv_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], kEwThreads);
-        mbar_init(&s_free[1], kEwThreads);
-        mbar_init(p_full, kEwThreads);
-        mbar_init(p_free, 1);
+        mbar_init(&s_free[0], 128);
+        mbar_init(&s_free[1], 128);
+        mbar_init(&p_full[0], 128);
+        mbar_init(&p_full[1], 128);
+        mbar_init(&p_free[0], 1);
+        mbar_init(&p_free[1], 1);
+        mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -480,71 +502,80 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), aDST = smem_u32(sDST);
             bool ok = mbar_wait(kv_full, 0, abort_flag, kErrTimeoutMma);
-            auto issue_acc = [&](int m) -> bool {
-                if (!mbar_wait(p_full, m & 1, abort_flag, kErrTimeoutMma)) return false;
-                tc_fence_after();
-                const int st = m % C::kStages;
-                const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+            // Event-driven issue (see the forward): S^T and dP^T of tile ns,
+            // dV and dK of tile na.
+            int ns = 0, na = 0;
+            PollGuard guard;
+            while (ok && na < T) {
+                bool moved = false;
+                if (ns < T) {
+                    const int st = ns % C::kStages, buf = ns & 1;
+                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
+                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t ap = sdesc_sw128(aPT + kk * 32, 16, 1024);
-                    const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
-                    umma_bf16(tmem + C::kTmemDV, ap, bdo, idesc_acc, (m > 0 || kk > 0) ? 1u : 0u);
-                }
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ak = sdesc_sw128(aK + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bq = sdesc_sw128(aQs + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + buf * 128, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
+                        }
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t ads = sdesc_sw128(aDST + kk * 32, 16, 1024);
-                    const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
-                    umma_bf16(tmem + C::kTmemDK, ads, bq, idesc_acc, (m > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t av = sdesc_sw128(aV + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bdo = sdesc_sw128(aDOs + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + buf * 128 + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&s_full[buf]);
+                        ++ns;
+                        moved = true;
+                    }
                 }
-                umma_commit(p_free);
-                umma_commit(&empty[st]);
-                return true;
-            };
-            for (int n = 0; ok && n < T; ++n) {
-                const int st = n % C::kStages;
-                const int buf = n & 1;
-                if (!mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                if (n >= 2 && !mbar_wait(&s_free[buf], ((n - 2) >> 1) & 1, abort_flag, kErrTimeoutMma)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+                if (na < ns) {
+                    const int pb = na & 1;
+                    if (mbar_test(&p_full[pb], (na >> 1) & 1)) {
+                        tc_fence_after();
+                        const int st = na % C::kStages;
+                        const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int at = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t ak = sdesc_sw128(aK + at * (128 * 128) + ko, 16, 1024);
-                    const uint64_t bq = sdesc_sw128(aQs + at * (kBlk * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + buf * 128, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
-                }
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const uint64_t ap = sdesc_sw128(aPT + pb * (128 * 128) + kk * 32, 16, 1024);
+                            const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
+                            umma_bf16(tmem + C::kTmemDV, ap, bdo, idesc_acc, (na > 0 || kk > 0) ? 1u : 0u);
+                        }
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int at = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t av = sdesc_sw128(aV + at * (128 * 128) + ko, 16, 1024);
-                    const uint64_t bdo = sdesc_sw128(aDOs + at * (kBlk * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + buf * 128 + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const uint64_t ads = sdesc_sw128(aDST + pb * (128 * 128) + kk * 32, 16, 1024);
+                            const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
+                            umma_bf16(tmem + C::kTmemDK, ads, bq, idesc_acc, (na > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&p_free[pb]);
+                        umma_commit(&empty[st]);
+                        ++na;
+                        moved = true;
+                    }
                 }
-                umma_commit(&s_full[buf]);
-                if (n >= 1 && !issue_acc(n - 1)) { ok = false; break; }
+                if (moved) guard.progress();
+                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
             }
-            if (ok && T > 0) issue_acc(T - 1);
+            if (ok && T > 0) umma_commit(done);
         }
         __syncwarp();
     } else {
         const int quad = warp & 3;
-        const int grp = (warp - 2) >> 2;
-        const int c0 = grp * kCw;                // first query column of this thread
+        const int grp = (warp - 2) >> 2;         // this group takes the tiles n % 2 == grp
         const int u = quad * 32 + lane;          // key row of the tile = TMEM lane
         const int half = u >> 6;
         const int my_blk = half ? kb : ka;
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         bool ok = true;
-        for (int n = 0; n < T; ++n) {
-            const int buf = n & 1;
+        for (int n = grp; n < T; n += 2) {
             const int st = n % C::kStages;
-            bool w_ok = mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax);
+            const int ph = (n >> 1) & 1;
+            bool w_ok = mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax);
             // the stage's LSE and D came in by TMA: observe its barrier too
             w_ok = w_ok && mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
             if (!__all_sync(0xffffffffu, w_ok)) {
@@ -552,51 +583,60 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 break;
             }
             tc_fence_after();
-            float sv[kCw], dp[kCw];
-            tmem_ld32(tlane + buf * 128 + c0, sv);
-            tmem_ld32(tlane + buf * 128 + 64 + c0, dp);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_free[buf]);
             const int i = tl.list[n];
             const bool is_live = (tl.live[n] >> half) & 1;
             // query columns allowed: live block, and in the diagonal block t >= u
-            const int first = (!is_live ? kBlk : (i == my_blk ? uu : 0)) - c0;
-            const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st) + c0);
-            const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st) + c0);
-            if (first >= kCw) {
+            const int first = !is_live ? kBlk : (i == my_blk ? uu : 0);
+            uint32_t pp[32], pd[32];
+            if (first >= kBlk) {
 #pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = dp[cc] = 0.f;
+                for (int e = 0; e < 32; ++e) pp[e] = pd[e] = 0u;
             } else {
+                const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st));
+                const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st));
 #pragma unroll
-                for (int c4 = 0; c4 < kCw / 4; ++c4) {
-                    const float4 l4 = lse4[c4];
-                    const float4 d4 = dv4[c4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                for (int ch = 0; ch < 2; ++ch) {
+                    float sv[32], dp[32];
+                    tmem_ld32(tlane + grp * 128 + 32 * ch, sv);
+                    tmem_ld32(tlane + grp * 128 + 64 + 32 * ch, dp);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int cc = 4 * c4 + e;
-                        float pr = ex2(fmaf(sv[cc], p.scale_log2, -lv[e] * kLog2e));
-                        if (first > 0) pr = cc >= first ? pr : 0.f;
-                        sv[cc] = pr;
-                        dp[cc] = pr * (dp[cc] - dd[e]);
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 l4 = lse4[8 * ch + c4];
+                        const float4 d4 = dv4[8 * ch + c4];
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int cc = 4 * c4 + e;
+                            float pr = ex2(fmaf(sv[cc], p.scale_log2, -lv[e] * kLog2e));
+                            if (first > 32 * ch) pr = 32 * ch + cc >= first ? pr : 0.f;
+                            sv[cc] = pr;
+                            dp[cc] = pr * (dp[cc] - dd[e]);
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        pp[16 * ch + e] = pack_bf16x2(sv[2 * e], sv[2 * e + 1]);
+                        pd[16 * ch + e] = pack_bf16x2(dp[2 * e], dp[2 * e + 1]);
                     }
                 }
             }
-            if (n >= 1 &&
-                !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            tc_fence_before();
+            mbar_arrive(&s_free[grp]);
+            // P^T[grp] and dS^T[grp] were last read by the dV/dK products of tile n - 2
+            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
-            store_cols_sw128(sPT, u, sv, c0 / 8, kCw / 8);
-            store_cols_sw128(sDST, u, dp, c0 / 8, kCw / 8);
+            store_packed_row_sw128(sPT + grp * (128 * 128), u, pp);
+            store_packed_row_sw128(sDST + grp * (128 * 128), u, pd);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[grp]);
         }
         if (ok && T > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+            __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
             constexpr int kOc = D / kEwGroups;

@@ -18,19 +18,23 @@
 //   warp 1  allocates TMEM; one thread issues the MMAs:
 //             S[buf] = Q K^T       (M=128, N=64,  K=d;   double-buffered S)
 //             O     += P V         (M=128, N=d,   K=64;  O accumulates in TMEM)
-//   warps 2-5  softmax: thread = query row = TMEM lane; reads S, applies the
-//           mask and scale, keeps the running max m and sum l, writes P
-//           (bf16, 128-byte swizzled, the MMA's A layout) to shared memory,
-//           and rescales O in TMEM when m grows by more than 2^8 (the
-//           result is exact for any reference max; the threshold only bounds
-//           P <= 256).  At the end O / l and the LSE are written out.
+//   warps 2-9  softmax, two warpgroups; group g takes the tiles n with
+//           n % 2 == g, one thread per query row (TMEM lane), all 64 key
+//           columns.  Each group keeps its own running max m_g, row sum l_g
+//           and accumulator O_g = Σ P V over its tiles (split-key online
+//           softmax), so the groups run independently and their exp2 (MUFU)
+//           and ALU phases overlap.  O_g is rescaled in TMEM only when m_g
+//           grows by more than 8 (log2 units): exact for any reference max,
+//           the threshold bounds P <= 256.  P goes out as bf16 in the MMA's
+//           128-byte-swizzled A layout.  At the end the two halves combine:
+//           m = max(m_0, m_1), O = Σ_g O_g 2^(m_g - m) / Σ_g l_g 2^(m_g - m).
 // The QK^T of tile n+1 overlaps the softmax of tile n.
 //
 // Shared memory (128-byte swizzle, 1024-byte aligned):
 //   Q  [d/64 column atoms][128 rows][128 B]
 //   K  stage [d/64 atoms][64 rows][128 B]          (B operand, K-major)
 //   V  stage [d/64 atoms][64 rows][128 B]          (B operand, MN-major)
-//   P  [128 rows][128 B]                           (A operand, K-major)
+//   P  [2][128 rows][128 B]                        (A operand, K-major; P[n % 2])
 #pragma once
 
 #include "common.cuh"
@@ -43,10 +47,8 @@ constexpr int kMaxHeads = 256;
 constexpr int kMaxBlocks = 2048;
 constexpr int kBlk = 64;   // block size in tokens
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// Softmax warpgroups: the two threads of a row (one per group) own 32 of the
-// tile's 64 key columns each and exchange their partial row maxima.
+// Softmax warpgroups: group g owns the tiles n with n % 2 == g.
 constexpr int kSmGroups = 2;
-constexpr int kCw = kBlk / kSmGroups;
 constexpr int kSmThreads = 128 * kSmGroups;
 constexpr int kFwdThreads = 64 + kSmThreads;
 
@@ -76,7 +78,7 @@ struct FwdParams {
 // K/V ring depth (one stage = one 64-key block of K and of V), and CTAs per
 // SM for d = 64 (two CTAs overlap each other's hand-offs).
 #ifndef GSA_FWD64_STAGES
-#define GSA_FWD64_STAGES 4
+#define GSA_FWD64_STAGES 3
 #endif
 #ifndef GSA_FWD128_STAGES
 #define GSA_FWD128_STAGES 3
@@ -91,27 +93,26 @@ struct FwdCfg {
     static constexpr int kStages = D == 64 ? GSA_FWD64_STAGES : GSA_FWD128_STAGES;
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = kBlk * D * 2;   // one block of K (or V)
-    static constexpr int kPBytes = 128 * kBlk * 2;
+    static constexpr int kPBytes = 128 * kBlk * 2;   // one P buffer (two are kept)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
     static constexpr int kOffP = kOffV + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    // barriers: full[st], empty[st], q_full, s_full[2], s_free[2], p_full, p_free
-    static constexpr int kNumBars = 2 * kStages + 7;
+    static constexpr int kOffBar = kOffP + 2 * kPBytes;
+    // barriers: full[st], empty[st], q_full, s_full[2], s_free[2], p_full[2], p_free[2], done
+    static constexpr int kNumBars = 2 * kStages + 10;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, ntiles
     static constexpr int kOffList = kOffMisc + 16;            // int16 key block per tile
     static constexpr int kOffLive = kOffList + kMaxBlocks * 2;
     static constexpr int kOffBits = kOffLive + kMaxBlocks;    // two bitmaps
-    static constexpr int kOffRed = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [2 parity][2 group][128] partial maxima
-    static constexpr int kOffOk = kOffRed + 2 * 2 * 128 * 4;               // [2 parity][2 group][4 quad] flags
-    static constexpr int kOffLsum = kOffOk + 2 * 2 * 4 * 4;                // [2 group][128] partial sums
-    static constexpr int kEnd = kOffLsum + 2 * 128 * 4;
+    static constexpr int kOffMl = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [2 group][2][128]: m_g, l_g
+    static constexpr int kEnd = kOffMl + 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;            // + alignment slack
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static constexpr int kTmemCols = 256;
-    static constexpr int kTmemS = 0;       // S buffers at columns 0 and 64
-    static constexpr int kTmemO = 128;     // O at columns 128 .. 128 + D
+    static_assert(D != 64 || GSA_FWD64_CTAS_PER_SM == 1 || kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
+    static constexpr int kTmemCols = (128 + 2 * D) <= 256 ? 256 : 512;
+    static constexpr int kTmemS = 0;       // S[g] at columns 64 g
+    static constexpr int kTmemO = 128;     // O_g at columns 128 + g D
 };
 
 template <int D>
@@ -132,7 +133,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     uint64_t* s_full = q_full + 1;
     uint64_t* s_free = s_full + 2;
     uint64_t* p_full = s_free + 2;
-    uint64_t* p_free = p_full + 1;
+    uint64_t* p_free = p_full + 2;
+    uint64_t* done = p_free + 2;    // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     int* ntiles_slot = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -161,10 +163,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], kSmThreads);
-        mbar_init(&s_free[1], kSmThreads);
-        mbar_init(p_full, kSmThreads);
-        mbar_init(p_free, 1);
+        mbar_init(&s_free[0], 128);
+        mbar_init(&s_free[1], 128);
+        mbar_init(&p_full[0], 128);
+        mbar_init(&p_full[1], 128);
+        mbar_init(&p_free[0], 1);
+        mbar_init(&p_free[1], 1);
+        mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -264,93 +269,95 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
             bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
-            auto issue_pv = [&](int m) -> bool {
-                if (!mbar_wait(p_full, m & 1, abort_flag, kErrTimeoutMma)) return false;
-                tc_fence_after();
-                const int st = m % C::kStages;
+            // Event-driven issue: QK^T of tile ns as soon as its K/V stage is
+            // loaded and its S buffer was read (tile ns - 2), P V of tile na as
+            // soon as its P is written.  Both streams advance in tile order.
+            int ns = 0, na = 0;
+            PollGuard guard;
+            while (ok && na < T) {
+                bool moved = false;
+                if (ns < T) {
+                    const int st = ns % C::kStages, buf = ns & 1;
+                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
+                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
+                        tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(aP + kk * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                    umma_bf16(tmem + C::kTmemO, ad, bd, idesc_pv, (m > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bd =
+                                sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + C::kTmemS + buf * kBlk, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&s_full[buf]);
+                        ++ns;
+                        moved = true;
+                    }
                 }
-                umma_commit(p_free);
-                umma_commit(&empty[st]);
-                return true;
-            };
-            for (int n = 0; ok && n < T; ++n) {
-                const int st = n % C::kStages;
-                const int buf = n & 1;
-                if (!mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                if (n >= 2 && !mbar_wait(&s_free[buf], ((n - 2) >> 1) & 1, abort_flag, kErrTimeoutMma)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+                if (na < ns) {
+                    const int pb = na & 1;   // P[pb] -> O_pb
+                    if (mbar_test(&p_full[pb], (na >> 1) & 1)) {
+                        tc_fence_after();
+                        const int st = na % C::kStages;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int at = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + C::kTmemS + buf * kBlk, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(aP + pb * C::kPBytes + kk * 32, 16, 1024);
+                            const uint64_t bd =
+                                sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                            umma_bf16(tmem + C::kTmemO + pb * D, ad, bd, idesc_pv, (na >= 2 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&p_free[pb]);
+                        umma_commit(&empty[st]);
+                        ++na;
+                        moved = true;
+                    }
                 }
-                umma_commit(&s_full[buf]);
-                if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
+                if (moved) guard.progress();
+                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
             }
-            if (ok && T > 0) issue_pv(T - 1);
+            if (ok && T > 0) umma_commit(done);
         }
         __syncwarp();
     } else {
         // ================= softmax warpgroups (warps 2..9)
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int grp = (warp - 2) >> 2;        // column group
-        const int c0 = grp * kCw;               // first key column of this thread
+        const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
         const int r = quad * 32 + lane;         // query row in the tile = TMEM lane
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
         const int rr = r & 63;
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        float* red = reinterpret_cast<float*>(smem + C::kOffRed);
-        volatile int* okf = reinterpret_cast<volatile int*>(smem + C::kOffOk);
-        float* lsum = reinterpret_cast<float*>(smem + C::kOffLsum);
-        float m = -INFINITY, l = 0.f;           // l: this thread's share of the row sum
+        const uint32_t tS = tl + C::kTmemS + grp * kBlk;
+        const uint32_t tO = tl + C::kTmemO + grp * D;
+        uint8_t* sPg = sP + grp * C::kPBytes;
+        float m = -INFINITY, l = 0.f;           // this group's running max and sum
         bool ok = true;
-        for (int n = 0; n < T; ++n) {
-            const int buf = n & 1;
-            // waits are warp-uniform (the tcgen05 loads are warp-collective); the
-            // two warps of a row pair leave the loop together, after their barrier
-            const bool w = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, abort_flag,
-                                                                   kErrTimeoutSoftmax));
-            float sv[kCw];
-            if (w) {
-                tc_fence_after();
-                tmem_ld32(tl + C::kTmemS + buf * kBlk + c0, sv);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&s_free[buf]);
-            }
-            const int j = list[n];
-            const bool is_live = (live[n] >> half) & 1;
-            const int last = (!is_live ? -1 : (j == my_blk ? rr : kBlk - 1)) - c0;
-            // raw-score maximum of this thread's columns (the scale is positive);
-            // masked columns become -inf, so their exponentials below are 0
-            float mt;
-            if (last >= kCw - 1) {
-                mt = max_reduce<kCw>(sv);
-            } else {
-#pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = cc <= last ? sv[cc] : -INFINITY;
-                mt = max_reduce<kCw>(sv);
-            }
-            mt *= p.scale_log2;
-            red[(buf * 2 + grp) * 128 + r] = mt;
-            if (lane == 0) okf[(buf * 2 + grp) * 4 + quad] = w ? 1 : 0;
-            pair_barrier(quad);
-            if (!(okf[(buf * 2 + 0) * 4 + quad] && okf[(buf * 2 + 1) * 4 + quad])) {
+        for (int n = grp; n < T; n += 2) {
+            const int ph = (n >> 1) & 1;        // phase of this group's barriers
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
-            mt = fmaxf(mt, red[(buf * 2 + (grp ^ 1)) * 128 + r]);
+            tc_fence_after();
+            const int j = list[n];
+            const bool is_live = (live[n] >> half) & 1;
+            const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);   // visible columns 0..last
+            // pass 1: raw-score maximum (the scale is positive)
+            float mt = -INFINITY;
+            if (last >= 0) {
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    float v[32];
+                    tmem_ld32(tS + 32 * ch, v);
+                    tmem_wait_ld();
+                    if (last < 32 * ch + 31) {
+#pragma unroll
+                        for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : -INFINITY;
+                    }
+                    mt = fmaxf(mt, max_reduce<32>(v));
+                }
+            }
+            mt *= p.scale_log2;
             const float m_new = fmaxf(m, mt);
             float alpha = 1.f;
             bool rescale = false;
@@ -363,61 +370,101 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 rescale = true;
             }
             const float msafe = m_use == -INFINITY ? 0.f : m_use;
-            // p = 2^(s * scale * log2 e - m): one FFMA and one MUFU.EX2 per score
-            float sum;
+            // pass 2: p = 2^(s * scale * log2 e - m), packed to bf16
+            uint32_t pk[32];
+            float sum = 0.f;
             if (last < 0) {
 #pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = 0.f;
-                sum = 0.f;
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             } else {
 #pragma unroll
-                for (int cc = 0; cc < kCw; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -msafe));
-                sum = sum_reduce<kCw>(sv);
+                for (int ch = 0; ch < 2; ++ch) {
+                    float v[32];
+                    tmem_ld32(tS + 32 * ch, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 32; ++cc) v[cc] = ex2(fmaf(v[cc], p.scale_log2, -msafe));
+                    if (last < 32 * ch + 31) {
+#pragma unroll
+                        for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : 0.f;
+                    }
+                    sum += sum_reduce<32>(v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                }
             }
+            tc_fence_before();
+            mbar_arrive(&s_free[grp]);
             l = l * alpha + sum;
             m = m_use;
 
-            if (n >= 1 &&
-                !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
-                ok = false;   // reported to the partner warp at the next barrier
-                continue;
+            // P[grp] and O_grp were last used by the P V product of tile n - 2
+            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
             }
             tc_fence_after();
+            uint8_t* prow = sPg + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                for (int cb = grp * (D / kSmGroups); cb < (grp + 1) * (D / kSmGroups); cb += 32) {
+                for (int cb = 0; cb < D; cb += 32) {
                     float ov[32];
-                    tmem_ld32(tl + C::kTmemO + cb, ov);
+                    tmem_ld32(tO + cb, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-                    tmem_st32(tl + C::kTmemO + cb, ov);
+                    tmem_st32(tO + cb, ov);
                 }
                 tmem_wait_st();
             }
-            store_cols_sw128(sP, r, sv, c0 / 8, kCw / 8);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[grp]);
         }
-        lsum[grp * 128 + r] = l;
+        // combine the two groups: exchange (m_g, l_g) through shared memory
+        float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
+        ml[(grp * 2 + 0) * 128 + r] = m;
+        ml[(grp * 2 + 1) * 128 + r] = l;
         pair_barrier(quad);
-        l = lsum[r] + lsum[128 + r];
-        if (ok && T > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(p_free, (T - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+        const float m0 = ml[0 * 128 + r], l0 = ml[1 * 128 + r];
+        const float m1 = ml[2 * 128 + r], l1 = ml[3 * 128 + r];
+        // every product of the CTA completed (a single-phase barrier: the other
+        // group's buffer barriers may be more than one phase behind)
+        if (ok && T > 0 && __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
-            const float inv = 1.f / l;
+            const bool has1 = T >= 2;           // O_1 holds products only if group 1 had a tile
+            const float mm = fmaxf(m0, has1 ? m1 : -INFINITY);
+            const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+            const float w1 = (!has1 || m1 == -INFINITY) ? 0.f : ex2(m1 - mm);
+            const float lt = l0 * w0 + l1 * w1;
+            const float inv = 1.f / lt;
             const bool store = my_blk >= 0;
             const int64_t tok = head_row0 + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
             __nv_bfloat16* orow = p.o + tok * D;
 #pragma unroll
-            for (int cb = grp * (D / kSmGroups); cb < (grp + 1) * (D / kSmGroups); cb += 32) {
-                float ov[32];
-                tmem_ld32(tl + C::kTmemO + cb, ov);
+            for (int cb = grp * (D / 2); cb < (grp + 1) * (D / 2); cb += 32) {
+                float a[32];
+                tmem_ld32(tl + C::kTmemO + cb, a);
                 tmem_wait_ld();
-                if (store) store_scaled_bf16(orow + cb, ov, inv);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) a[e] *= w0;
+                if (has1) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float b2[16];
+                        tmem_ld16(tl + C::kTmemO + D + cb + 16 * hh, b2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) a[16 * hh + e] = fmaf(b2[e], w1, a[16 * hh + e]);
+                    }
+                }
+                if (store) store_scaled_bf16(orow + cb, a, inv);
             }
-            if (store && grp == 0 && p.lse) p.lse[tok] = (m + log2f(l)) * 0.69314718055994531f;
+            if (store && grp == 0 && p.lse) p.lse[tok] = (mm + log2f(lt)) * 0.69314718055994531f;
         }
     }
 

@@ -72,6 +72,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of a phase's completion.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Spin bookkeeping for a loop that polls several barriers with mbar_test:
+// call stalled() whenever a pass made no progress; it returns true (and
+// records `code`, raises *abort) once kWaitLimitNs passed without progress,
+// or when another role raised *abort.  progress() resets the clock.
+struct PollGuard {
+    unsigned long long t0 = 0;
+    uint32_t spins = 0;
+    __device__ __forceinline__ void progress() { spins = 0; }
+    __device__ __forceinline__ bool stalled(volatile int* abort, int code) {
+        if (spins++ == 0) t0 = globaltimer_ns();
+        if ((spins & 63u) == 0) {
+            if (*abort) return true;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_error(code);
+                *abort = 1;
+                return true;
+            }
+        }
+        return false;
+    }
+};
+
 // Wait for the phase with the given parity to complete.  Gives up (returns
 // false) when *abort becomes nonzero or after kWaitLimitNs; on a timeout it
 // records `code` in the device error word and raises *abort so the other
@@ -189,6 +224,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         : "r"(taddr));
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {

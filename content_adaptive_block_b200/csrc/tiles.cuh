@@ -106,6 +106,16 @@ __device__ __forceinline__ void store_cols_sw128(uint8_t* tile, int r, const flo
     }
 }
 
+// Store a row of 64 bf16 already packed in pairs (32 words) into a
+// 128-byte-swizzled K-major tile.
+__device__ __forceinline__ void store_packed_row_sw128(uint8_t* tile, int r, const uint32_t* pk) {
+    uint8_t* row = tile + r * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+}
+
 // Pairwise reductions (log-depth dependency chains instead of linear ones).
 template <int N>
 __device__ __forceinline__ float max_reduce(const float* v) {
