@@ -11,15 +11,19 @@
 //   2. dq_kernel    one CTA per query tile (two query blocks from the class's
 //                   pairing order); walks the union of their CSR rows:
 //                     S = Q K^T, dP = dO V^T  -> TMEM (double-buffered)
-//                     dS (bf16, shared)       <- softmax warps
-//                     dQ += dS K              (TMEM accumulator)
+//                     dS (bf16, back to TMEM) <- elementwise warps
+//                     dQ += dS K              (A from TMEM; TMEM accumulator)
 //   3. dkdv_kernel  one CTA per key tile (two key blocks from the class's key
 //                   pairing order); walks the union of their CSC columns:
 //                     S^T = K Q^T, dP^T = V dO^T -> TMEM (double-buffered)
-//                     P^T, dS^T (bf16, shared)   <- elementwise warps
-//                     dV += P^T dO, dK += dS^T Q (TMEM accumulators)
-// Warp roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner and
-// MMA issuer, warps 2-5 the elementwise work with one thread per TMEM lane.
+//                     P^T, dS^T (bf16, back to TMEM) <- elementwise warps
+//                     dV += P^T dO, dK += dS^T Q (A from TMEM; TMEM accumulators)
+// Warp roles as in the forward: warp 0 TMA producer, warp 1 TMEM owner,
+// warps 2-9 two elementwise groups with one thread per TMEM lane; one thread
+// of each group issues that group's MMAs right after its rows are in TMEM.
+// The bf16 operands written by the elementwise warps stay in TMEM as packed
+// pairs (lane = row, column c = elements 2c, 2c+1), the layout of an M=128
+// A operand, so they never pass through shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -87,16 +91,16 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
 
 // Ring depths: a stage is released after the last MMA that reads it.
 #ifndef GSA_DQ64_STAGES
-#define GSA_DQ64_STAGES 6
+#define GSA_DQ64_STAGES 8
 #endif
 #ifndef GSA_DQ128_STAGES
-#define GSA_DQ128_STAGES 3
+#define GSA_DQ128_STAGES 4
 #endif
 #ifndef GSA_DKV64_STAGES
-#define GSA_DKV64_STAGES 5
+#define GSA_DKV64_STAGES 8
 #endif
 #ifndef GSA_DKV128_STAGES
-#define GSA_DKV128_STAGES 2
+#define GSA_DKV128_STAGES 4
 #endif
 
 template <int D>
@@ -109,10 +113,9 @@ struct DqCfg {
     static constexpr int kOffDO = kOffQ + kTileBytes;
     static constexpr int kOffK = kOffDO + kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffDS = kOffV + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffDS + 2 * 128 * 128;    // dS double-buffered
-    // full[st], empty[st], q_full, s_full[2], s_free[2], ds_full[2], ds_free[2], done
-    static constexpr int kNumBars = 2 * kStages + 10;
+    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+    // full[st], empty[st], q_full, s_full[2], ds_full[2], done
+    static constexpr int kNumBars = 2 * kStages + 6;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -121,7 +124,8 @@ struct DqCfg {
     static constexpr int kSmemBytes = kEnd + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr int kTmemCols = 512;
-    // S[b] at 128 * b, dP[b] at 128 * b + 64, dQ at 256
+    // S[g] at 128 g (dS over its first 32 columns), dP[g] at 128 g + 64,
+    // dQ_g (group g's share of the sum) at 256 + g D
     static constexpr int kTmemDQ = 256;
 };
 
@@ -136,16 +140,13 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     uint8_t* sDO = smem + C::kOffDO;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
-    uint8_t* sDS = smem + C::kOffDS;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
     uint64_t* empty = bars + C::kStages;
     uint64_t* q_full = bars + 2 * C::kStages;
     uint64_t* s_full = q_full + 1;
-    uint64_t* s_free = s_full + 2;
-    uint64_t* ds_full = s_free + 2;
-    uint64_t* ds_free = ds_full + 2;
-    uint64_t* done = ds_free + 2;   // one phase: every product of the CTA completed
+    uint64_t* ds_full = s_full + 2;
+    uint64_t* done = ds_full + 2;   // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -164,6 +165,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int64_t g = static_cast<int64_t>(s) * 3 + c;
     const int qa = p.order[g * nblk + 2 * tile];
     const int qb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < C::kStages; ++st) {
@@ -173,40 +175,41 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
         mbar_init(&ds_full[0], 128);
         mbar_init(&ds_full[1], 128);
-        mbar_init(&ds_free[0], 1);
-        mbar_init(&ds_free[1], 1);
-        mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        // Q and dO of the tile load while the key lists merge
+        mbar_arrive_expect_tx(q_full, (qb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
+        for (int half = 0; half < 2; ++half) {
+            const int blk = half ? qb : qa;
+            if (blk < 0) continue;
+            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+            for (int at = 0; at < C::kAtoms; ++at) {
+                tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
+                tma_load_2d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, row);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, qa, qb, nblk);
+    if (threadIdx.x == 0) {
+        mbar_init(done, *tl.count >= 2 ? 2 : 1);   // one arrival per group that has tiles
+        fence_mbar_init();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const int T = *tl.count;
     const uint32_t tmem = *tmem_slot;
-    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, (qb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
-            for (int half = 0; half < 2; ++half) {
-                const int blk = half ? qb : qa;
-                if (blk < 0) continue;
-                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
-                    tma_load_2d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, row);
-                }
-            }
             for (int n = 0; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages &&
@@ -220,69 +223,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 }
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
-            constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1);
-            const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV),
-                           aDS = smem_u32(sDS);
-            bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
-            // Event-driven issue (see the forward): S and dP of tile ns, dQ of tile na.
-            int ns = 0, na = 0;
-            PollGuard guard;
-            while (ok && na < T) {
-                bool moved = false;
-                if (ns < T) {
-                    const int st = ns % C::kStages, buf = ns & 1;
-                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
-                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int at = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t aq = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
-                            const uint64_t bk =
-                                sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                            umma_bf16(tmem + buf * 128, aq, bk, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int at = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ado = sdesc_sw128(aDO + at * (128 * 128) + ko, 16, 1024);
-                            const uint64_t bv =
-                                sdesc_sw128(aV + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                            umma_bf16(tmem + buf * 128 + 64, ado, bv, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&s_full[buf]);
-                        ++ns;
-                        moved = true;
-                    }
-                }
-                if (na < ns) {
-                    const int db = na & 1;
-                    if (mbar_test(&ds_full[db], (na >> 1) & 1)) {
-                        tc_fence_after();
-                        const int st = na % C::kStages;
-#pragma unroll
-                        for (int kk = 0; kk < kBlk / 16; ++kk) {
-                            const uint64_t ad = sdesc_sw128(aDS + db * (128 * 128) + kk * 32, 16, 1024);
-                            const uint64_t bd =
-                                sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                            umma_bf16(tmem + C::kTmemDQ, ad, bd, idesc_dq, (na > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&ds_free[db]);
-                        umma_commit(&empty[st]);
-                        ++na;
-                        moved = true;
-                    }
-                }
-                if (moved) guard.progress();
-                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
-            }
-            if (ok && T > 0) umma_commit(done);
-        }
-        __syncwarp();
-    } else {
+    } else if (warp >= 2) {
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
         const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
         const int r = quad * 32 + lane;
@@ -293,6 +234,38 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + rr;
         const float lse2 = my_blk >= 0 ? p.lse[tok] * kLog2e : 0.f;
         const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
+        // the group's MMA issuer: lane 0 of its first warp
+        const bool issuer_warp = ((warp - 2) & 3) == 0;
+        constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
+        constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1);
+        const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
+        auto issue_s = [&](int t) {   // S[grp] = Q K_t^T, dP[grp] = dO V_t^T, then s_full[grp]
+            const int st = t % C::kStages;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int at = kk >> 2, ko = (kk & 3) * 32;
+                const uint64_t aq = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                const uint64_t bk = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                umma_bf16(tmem + grp * 128, aq, bk, idesc_s, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int at = kk >> 2, ko = (kk & 3) * 32;
+                const uint64_t ado = sdesc_sw128(aDO + at * (128 * 128) + ko, 16, 1024);
+                const uint64_t bv = sdesc_sw128(aV + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                umma_bf16(tmem + grp * 128 + 64, ado, bv, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[grp]);
+        };
+        if (issuer_warp) {
+            if (lane == 0 && grp < T &&
+                mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma) &&
+                mbar_wait(&full[grp % C::kStages], (grp / C::kStages) & 1, abort_flag, kErrTimeoutMma)) {
+                tc_fence_after();
+                issue_s(grp);
+            }
+            __syncwarp();
+        }
         bool ok = true;
         for (int n = grp; n < T; n += 2) {
             const int ph = (n >> 1) & 1;
@@ -325,21 +298,40 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(sv[2 * e], sv[2 * e + 1]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[grp]);
-            // dS[grp] was last read by the dQ product of tile n - 2
-            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&ds_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
-                ok = false;
-                break;
-            }
-            store_packed_row_sw128(sDS + grp * (128 * 128), r, pk);
-            fence_proxy_async_smem();
+            // dS over the first 32 columns of S[grp] (both chunks were read above)
+            tmem_st32u(tlane + grp * 128, pk);
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&ds_full[grp]);
+            if (issuer_warp) {
+                if (lane == 0 && mbar_wait(&ds_full[grp], ph, abort_flag, kErrTimeoutMma)) {
+                    // dQ_grp += dS K (dS read from TMEM), then S and dP of the group's next tile
+                    tc_fence_after();
+                    const int st = n % C::kStages;
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                        umma_bf16_ts(tmem + C::kTmemDQ + grp * D, tmem + grp * 128 + kk * 8, bd, idesc_dq,
+                                     (n >= 2 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[st]);
+                    if (n + 2 < T) {
+                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                                      kErrTimeoutMma)) {
+                            tc_fence_after();
+                            issue_s(n + 2);
+                        }
+                    } else {
+                        umma_commit(done);
+                    }
+                }
+                __syncwarp();
+            }
         }
         if (ok && T > 0 &&
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
+            const bool has1 = T >= 2;            // dQ_1 holds products only if group 1 had a tile
             __nv_bfloat16* orow = p.out0 + tok * D;
             constexpr int kOc = D / kEwGroups;   // output columns per thread (split between the groups)
 #pragma unroll
@@ -347,6 +339,16 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 float ov[32];
                 tmem_ld32(tlane + C::kTmemDQ + cb, ov);
                 tmem_wait_ld();
+                if (has1) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float o2[16];
+                        tmem_ld16(tlane + C::kTmemDQ + D + cb + 16 * hh, o2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) ov[16 * hh + e] += o2[e];
+                    }
+                }
                 if (my_blk >= 0) store_scaled_bf16(orow + cb, ov, p.scale);
             }
         }
@@ -372,12 +374,10 @@ struct DkvCfg {
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kTileBytes;
     static constexpr int kOffStage = kOffV + kTileBytes;
-    static constexpr int kOffPT = kOffStage + kStages * kStageBytes;   // P^T, double-buffered
-    static constexpr int kOffDST = kOffPT + 2 * 128 * 128;             // dS^T, double-buffered
-    static constexpr int kOffVec = kOffDST + 2 * 128 * 128;            // per stage: LSE[64], D[64]
+    static constexpr int kOffVec = kOffStage + kStages * kStageBytes;   // per stage: LSE[64], D[64]
     static constexpr int kOffBar = kOffVec + kStages * 2 * kVecBytes;
-    // full[st], empty[st], kv_full, s_full[2], s_free[2], p_full[2], p_free[2], done
-    static constexpr int kNumBars = 2 * kStages + 10;
+    // full[st], empty[st], kv_full, s_full[2], p_full[2], acc[2], done
+    static constexpr int kNumBars = 2 * kStages + 8;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -385,11 +385,16 @@ struct DkvCfg {
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static constexpr int kTmemCols = 512;
-    // S^T[b] at 128 * b, dP^T[b] at 128 * b + 64, dV at 256, dK at 256 + D
-    static constexpr int kTmemDV = 256;
-    static constexpr int kTmemDK = 256 + D;
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+    static constexpr int kTmemCols = 512;
+    // S^T[g] at 128 g (P^T over its first 32 columns), dP^T[g] at 128 g + 64
+    // (dS^T over its first 32).  d = 64: each group keeps its own dV_g, dK_g
+    // (at 256 + 128 g and 256 + 128 g + 64) and the epilogue adds them; d =
+    // 128 has room for one dV and one dK (256, 256 + D), which the two
+    // groups' products take in turn (the acc barriers order them).
+    static constexpr bool kSplit = D == 64;
+    __host__ __device__ static constexpr uint32_t dv_col(int grp) { return kSplit ? 256 + 128 * grp : 256; }
+    __host__ __device__ static constexpr uint32_t dk_col(int grp) { return kSplit ? 256 + 128 * grp + 64 : 256 + D; }
 };
 
 template <int D>
@@ -402,17 +407,14 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
     uint8_t* sStage = smem + C::kOffStage;
-    uint8_t* sPT = smem + C::kOffPT;
-    uint8_t* sDST = smem + C::kOffDST;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
     uint64_t* empty = bars + C::kStages;
     uint64_t* kv_full = bars + 2 * C::kStages;
     uint64_t* s_full = kv_full + 1;
-    uint64_t* s_free = s_full + 2;
-    uint64_t* p_full = s_free + 2;
-    uint64_t* p_free = p_full + 2;
-    uint64_t* done = p_free + 2;    // one phase: every product of the CTA completed
+    uint64_t* p_full = s_full + 2;
+    uint64_t* acc = p_full + 2;     // d = 128: group g's dV/dK products of its latest tile completed
+    uint64_t* done = acc + 2;       // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -437,6 +439,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int64_t g = static_cast<int64_t>(s) * 3 + c;
     const int ka = p.order[g * nblk + 2 * tile];
     const int kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < C::kStages; ++st) {
@@ -446,40 +449,43 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(kv_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
         mbar_init(&p_full[0], 128);
         mbar_init(&p_full[1], 128);
-        mbar_init(&p_free[0], 1);
-        mbar_init(&p_free[1], 1);
-        mbar_init(done, 1);
+        mbar_init(&acc[0], 1);
+        mbar_init(&acc[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmDO);
+        // K and V of the tile load while the query lists merge
+        mbar_arrive_expect_tx(kv_full, (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
+        for (int half = 0; half < 2; ++half) {
+            const int blk = half ? kb : ka;
+            if (blk < 0) continue;
+            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+            for (int at = 0; at < C::kAtoms; ++at) {
+                tma_load_2d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, row);
+                tma_load_2d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, row);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, ka, kb, nblk);
+    if (threadIdx.x == 0) {
+        mbar_init(done, *tl.count >= 2 ? 2 : 1);   // one arrival per group that has tiles
+        fence_mbar_init();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const int T = *tl.count;
     const uint32_t tmem = *tmem_slot;
-    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
-            for (int half = 0; half < 2; ++half) {
-                const int blk = half ? kb : ka;
-                if (blk < 0) continue;
-                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_2d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, row);
-                    tma_load_2d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, row);
-                }
-            }
             for (int n = 0; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages &&
@@ -496,74 +502,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
-            constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
-            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPT = smem_u32(sPT), aDST = smem_u32(sDST);
-            bool ok = mbar_wait(kv_full, 0, abort_flag, kErrTimeoutMma);
-            // Event-driven issue (see the forward): S^T and dP^T of tile ns,
-            // dV and dK of tile na.
-            int ns = 0, na = 0;
-            PollGuard guard;
-            while (ok && na < T) {
-                bool moved = false;
-                if (ns < T) {
-                    const int st = ns % C::kStages, buf = ns & 1;
-                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
-                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int at = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ak = sdesc_sw128(aK + at * (128 * 128) + ko, 16, 1024);
-                            const uint64_t bq = sdesc_sw128(aQs + at * (kBlk * 128) + ko, 16, 1024);
-                            umma_bf16(tmem + buf * 128, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int at = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t av = sdesc_sw128(aV + at * (128 * 128) + ko, 16, 1024);
-                            const uint64_t bdo = sdesc_sw128(aDOs + at * (kBlk * 128) + ko, 16, 1024);
-                            umma_bf16(tmem + buf * 128 + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&s_full[buf]);
-                        ++ns;
-                        moved = true;
-                    }
-                }
-                if (na < ns) {
-                    const int pb = na & 1;
-                    if (mbar_test(&p_full[pb], (na >> 1) & 1)) {
-                        tc_fence_after();
-                        const int st = na % C::kStages;
-                        const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
-#pragma unroll
-                        for (int kk = 0; kk < kBlk / 16; ++kk) {
-                            const uint64_t ap = sdesc_sw128(aPT + pb * (128 * 128) + kk * 32, 16, 1024);
-                            const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
-                            umma_bf16(tmem + C::kTmemDV, ap, bdo, idesc_acc, (na > 0 || kk > 0) ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < kBlk / 16; ++kk) {
-                            const uint64_t ads = sdesc_sw128(aDST + pb * (128 * 128) + kk * 32, 16, 1024);
-                            const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
-                            umma_bf16(tmem + C::kTmemDK, ads, bq, idesc_acc, (na > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&p_free[pb]);
-                        umma_commit(&empty[st]);
-                        ++na;
-                        moved = true;
-                    }
-                }
-                if (moved) guard.progress();
-                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
-            }
-            if (ok && T > 0) umma_commit(done);
-        }
-        __syncwarp();
-    } else {
+    } else if (warp >= 2) {
         const int quad = warp & 3;
         const int grp = (warp - 2) >> 2;         // this group takes the tiles n % 2 == grp
         const int u = quad * 32 + lane;          // key row of the tile = TMEM lane
@@ -571,6 +510,39 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int my_blk = half ? kb : ka;
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        // the group's MMA issuer: lane 0 of its first warp
+        const bool issuer_warp = ((warp - 2) & 3) == 0;
+        constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
+        constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
+        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+        auto issue_s = [&](int t) {   // S^T[grp] = K Q_t^T, dP^T[grp] = V dO_t^T, then s_full[grp]
+            const int st = t % C::kStages;
+            const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int at = kk >> 2, ko = (kk & 3) * 32;
+                const uint64_t ak = sdesc_sw128(aK + at * (128 * 128) + ko, 16, 1024);
+                const uint64_t bq = sdesc_sw128(aQs + at * (kBlk * 128) + ko, 16, 1024);
+                umma_bf16(tmem + grp * 128, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int at = kk >> 2, ko = (kk & 3) * 32;
+                const uint64_t av = sdesc_sw128(aV + at * (128 * 128) + ko, 16, 1024);
+                const uint64_t bdo = sdesc_sw128(aDOs + at * (kBlk * 128) + ko, 16, 1024);
+                umma_bf16(tmem + grp * 128 + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[grp]);
+        };
+        if (issuer_warp) {
+            if (lane == 0 && grp < T &&
+                mbar_wait(kv_full, 0, abort_flag, kErrTimeoutMma) &&
+                mbar_wait(&full[grp % C::kStages], (grp / C::kStages) & 1, abort_flag, kErrTimeoutMma)) {
+                tc_fence_after();
+                issue_s(grp);
+            }
+            __syncwarp();
+        }
         bool ok = true;
         for (int n = grp; n < T; n += 2) {
             const int st = n % C::kStages;
@@ -622,34 +594,76 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[grp]);
-            // P^T[grp] and dS^T[grp] were last read by the dV/dK products of tile n - 2
-            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
-                ok = false;
-                break;
-            }
-            store_packed_row_sw128(sPT + grp * (128 * 128), u, pp);
-            store_packed_row_sw128(sDST + grp * (128 * 128), u, pd);
-            fence_proxy_async_smem();
+            // P^T over the first 32 columns of S^T[grp], dS^T over those of dP^T[grp]
+            tmem_st32u(tlane + grp * 128, pp);
+            tmem_st32u(tlane + grp * 128 + 64, pd);
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[grp]);
+            if (issuer_warp) {
+                bool go = lane == 0 && mbar_wait(&p_full[grp], ph, abort_flag, kErrTimeoutMma);
+                // shared accumulators: the other group's products of tile n - 1 completed first
+                if (!C::kSplit && go && n >= 1)
+                    go = mbar_wait(&acc[grp ^ 1], ((n - 1) >> 1) & 1, abort_flag, kErrTimeoutMma);
+                if (go) {
+                    // dV += P^T dO, dK += dS^T Q (A from TMEM), then the group's next S^T, dP^T
+                    tc_fence_after();
+                    const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
+                    const bool first_prod = C::kSplit ? n < 2 : n < 1;
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
+                        umma_bf16_ts(tmem + C::dv_col(grp), tmem + grp * 128 + kk * 8, bdo, idesc_acc,
+                                     (!first_prod || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
+                        umma_bf16_ts(tmem + C::dk_col(grp), tmem + grp * 128 + 64 + kk * 8, bq, idesc_acc,
+                                     (!first_prod || kk > 0) ? 1u : 0u);
+                    }
+                    if (!C::kSplit) umma_commit(&acc[grp]);
+                    umma_commit(&empty[st]);
+                    if (n + 2 < T) {
+                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                                      kErrTimeoutMma)) {
+                            tc_fence_after();
+                            issue_s(n + 2);
+                        }
+                    } else {
+                        umma_commit(done);
+                    }
+                }
+                __syncwarp();
+            }
         }
         if (ok && T > 0 &&
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
+            const bool has1 = C::kSplit && T >= 2;   // the group-1 accumulators hold products
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
             constexpr int kOc = D / kEwGroups;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
                 const float mul = which == 0 ? 1.f : p.scale;
-                const uint32_t col = which == 0 ? C::kTmemDV : C::kTmemDK;
+                const uint32_t col0 = which == 0 ? C::dv_col(0) : C::dk_col(0);
+                const uint32_t col1 = which == 0 ? C::dv_col(1) : C::dk_col(1);
 #pragma unroll
                 for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
                     float ov[32];
-                    tmem_ld32(tlane + col + cb, ov);
+                    tmem_ld32(tlane + col0 + cb, ov);
                     tmem_wait_ld();
+                    if (has1) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float o2[16];
+                            tmem_ld16(tlane + col1 + cb + 16 * hh, o2);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) ov[16 * hh + e] += o2[e];
+                        }
+                    }
                     if (my_blk >= 0) store_scaled_bf16(orow + cb, ov, mul);
                 }
             }

@@ -12,12 +12,12 @@
 // one key block of 64 tokens.  Rows of a half whose block is not live for a
 // key tile are masked out of it; the diagonal block gets the token causal cut.
 //
-// Roles (192 threads):
-//   warp 0  one thread issues TMA loads: Q (once), then K and V of each key
-//           tile into a ring of shared-memory stages;
-//   warp 1  allocates TMEM; one thread issues the MMAs:
-//             S[buf] = Q K^T       (M=128, N=64,  K=d;   double-buffered S)
-//             O     += P V         (M=128, N=d,   K=64;  O accumulates in TMEM)
+// Roles (320 threads):
+//   thread 0 issues the TMA load of Q as soon as the barriers exist, so it
+//           overlaps the merge of the key lists;
+//   warp 0  one thread issues the TMA loads of K and V of each key tile
+//           into a ring of shared-memory stages;
+//   warp 1  allocates TMEM;
 //   warps 2-9  softmax, two warpgroups; group g takes the tiles n with
 //           n % 2 == g, one thread per query row (TMEM lane), all 64 key
 //           columns.  Each group keeps its own running max m_g, row sum l_g
@@ -25,8 +25,19 @@
 //           softmax), so the groups run independently and their exp2 (MUFU)
 //           and ALU phases overlap.  O_g is rescaled in TMEM only when m_g
 //           grows by more than 8 (log2 units): exact for any reference max,
-//           the threshold bounds P <= 256.  P goes out as bf16 in the MMA's
-//           128-byte-swizzled A layout.  At the end the two halves combine:
+//           the threshold bounds P <= 256.  P goes back to TMEM as packed
+//           bf16 pairs over the first 32 columns of S[g] (lane = query row,
+//           column c = key columns 2c, 2c+1: the layout of an M=128 A operand
+//           in TMEM), so it never passes through shared memory.  The
+//           tensor pipe runs one thread's MMAs in issue order, so the QK^T of
+//           tile n+2 may overwrite S[g] once the P V of tile n is issued.
+//           One thread of each group issues that group's MMAs,
+//             S[g]  = Q K^T   (M=128, N=64, K=d;  A and B from shared memory)
+//             O_g  += P V     (M=128, N=d,  K=64; A = P from TMEM, B = V),
+//           right after the group's 128 rows of P are in TMEM: two
+//           independent MMA streams per CTA, and every product a group's
+//           rows read was issued (so ordered and tracked) by one thread.
+//           At the end the two halves combine:
 //           m = max(m_0, m_1), O = Σ_g O_g 2^(m_g - m) / Σ_g l_g 2^(m_g - m).
 // The QK^T of tile n+1 overlaps the softmax of tile n.
 //
@@ -34,7 +45,8 @@
 //   Q  [d/64 column atoms][128 rows][128 B]
 //   K  stage [d/64 atoms][64 rows][128 B]          (B operand, K-major)
 //   V  stage [d/64 atoms][64 rows][128 B]          (B operand, MN-major)
-//   P  [2][128 rows][128 B]                        (A operand, K-major; P[n % 2])
+// TMEM (lanes = query rows): S[0], S[1] at columns 0 and 64 (P over their
+// first 32 columns), O_0 and O_1 at columns 128 and 128 + d.
 #pragma once
 
 #include "common.cuh"
@@ -78,10 +90,10 @@ struct FwdParams {
 // K/V ring depth (one stage = one 64-key block of K and of V), and CTAs per
 // SM for d = 64 (two CTAs overlap each other's hand-offs).
 #ifndef GSA_FWD64_STAGES
-#define GSA_FWD64_STAGES 3
+#define GSA_FWD64_STAGES 5
 #endif
 #ifndef GSA_FWD128_STAGES
-#define GSA_FWD128_STAGES 3
+#define GSA_FWD128_STAGES 5
 #endif
 #ifndef GSA_FWD64_CTAS_PER_SM
 #define GSA_FWD64_CTAS_PER_SM 2
@@ -93,14 +105,12 @@ struct FwdCfg {
     static constexpr int kStages = D == 64 ? GSA_FWD64_STAGES : GSA_FWD128_STAGES;
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = kBlk * D * 2;   // one block of K (or V)
-    static constexpr int kPBytes = 128 * kBlk * 2;   // one P buffer (two are kept)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffP + 2 * kPBytes;
-    // barriers: full[st], empty[st], q_full, s_full[2], s_free[2], p_full[2], p_free[2], done
-    static constexpr int kNumBars = 2 * kStages + 10;
+    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+    // barriers: full[st], empty[st], q_full, s_full[2], p_full[2], done
+    static constexpr int kNumBars = 2 * kStages + 6;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, ntiles
     static constexpr int kOffList = kOffMisc + 16;            // int16 key block per tile
     static constexpr int kOffLive = kOffList + kMaxBlocks * 2;
@@ -125,16 +135,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
-    uint8_t* sP = smem + C::kOffP;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
     uint64_t* empty = bars + C::kStages;
     uint64_t* q_full = bars + 2 * C::kStages;
     uint64_t* s_full = q_full + 1;
-    uint64_t* s_free = s_full + 2;
-    uint64_t* p_full = s_free + 2;
-    uint64_t* p_free = p_full + 2;
-    uint64_t* done = p_free + 2;    // one phase: every product of the CTA completed
+    uint64_t* p_full = s_full + 2;
+    uint64_t* done = p_full + 2;    // one phase: every product of the CTA completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     int* ntiles_slot = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -163,20 +170,22 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&s_free[0], 128);
-        mbar_init(&s_free[1], 128);
         mbar_init(&p_full[0], 128);
         mbar_init(&p_full[1], 128);
-        mbar_init(&p_free[0], 1);
-        mbar_init(&p_free[1], 1);
-        mbar_init(done, 1);
         *abort_flag = 0;
         fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        // Q of the tile: needs only qa and qb, so it loads while the key lists merge
+        const int64_t row0 = static_cast<int64_t>(sh) * p.L;
+        mbar_arrive_expect_tx(q_full, (qb >= 0 ? 2 : 1) * kBlk * D * 2);
+        for (int half = 0; half < 2; ++half) {
+            const int blk = half ? qb : qa;
+            if (blk < 0) continue;
+            const int row = static_cast<int>(row0 + static_cast<int64_t>(blk) * kBlk);
+            for (int at = 0; at < C::kAtoms; ++at)
+                tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -226,7 +235,11 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 ++pos;
             }
         }
-        if (lane == 31) *ntiles_slot = incl;
+        if (lane == 31) {
+            *ntiles_slot = incl;
+            mbar_init(done, incl >= 2 ? 2 : 1);   // one arrival per group that has tiles
+            fence_mbar_init();
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -238,15 +251,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     if (warp == 0) {
         // ================= TMA producer
         if (lane == 0) {
-            const uint32_t qbytes = (qb >= 0 ? 2 : 1) * kBlk * D * 2;
-            mbar_arrive_expect_tx(q_full, qbytes);
-            for (int half = 0; half < 2; ++half) {
-                const int blk = half ? qb : qa;
-                if (blk < 0) continue;
-                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
-                for (int at = 0; at < C::kAtoms; ++at)
-                    tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
-            }
             for (int n = 0; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages) {
@@ -262,63 +266,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
             }
         }
-    } else if (warp == 1) {
-        // ================= MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-            bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
-            // Event-driven issue: QK^T of tile ns as soon as its K/V stage is
-            // loaded and its S buffer was read (tile ns - 2), P V of tile na as
-            // soon as its P is written.  Both streams advance in tile order.
-            int ns = 0, na = 0;
-            PollGuard guard;
-            while (ok && na < T) {
-                bool moved = false;
-                if (ns < T) {
-                    const int st = ns % C::kStages, buf = ns & 1;
-                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
-                        (ns < 2 || mbar_test(&s_free[buf], ((ns - 2) >> 1) & 1))) {
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int at = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
-                            const uint64_t bd =
-                                sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                            umma_bf16(tmem + C::kTmemS + buf * kBlk, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&s_full[buf]);
-                        ++ns;
-                        moved = true;
-                    }
-                }
-                if (na < ns) {
-                    const int pb = na & 1;   // P[pb] -> O_pb
-                    if (mbar_test(&p_full[pb], (na >> 1) & 1)) {
-                        tc_fence_after();
-                        const int st = na % C::kStages;
-#pragma unroll
-                        for (int kk = 0; kk < kBlk / 16; ++kk) {
-                            const uint64_t ad = sdesc_sw128(aP + pb * C::kPBytes + kk * 32, 16, 1024);
-                            const uint64_t bd =
-                                sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                            umma_bf16(tmem + C::kTmemO + pb * D, ad, bd, idesc_pv, (na >= 2 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&p_free[pb]);
-                        umma_commit(&empty[st]);
-                        ++na;
-                        moved = true;
-                    }
-                }
-                if (moved) guard.progress();
-                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
-            }
-            if (ok && T > 0) umma_commit(done);
-        }
-        __syncwarp();
-    } else {
+    } else if (warp >= 2) {
         // ================= softmax warpgroups (warps 2..9)
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
         const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
@@ -329,9 +277,35 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t tS = tl + C::kTmemS + grp * kBlk;
         const uint32_t tO = tl + C::kTmemO + grp * D;
-        uint8_t* sPg = sP + grp * C::kPBytes;
         float m = -INFINITY, l = 0.f;           // this group's running max and sum
         bool ok = true;
+        // the group's MMA issuer: lane 0 of its first warp
+        const bool issuer_warp = ((warp - 2) & 3) == 0;
+        constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        auto issue_qk = [&](int t) {   // S[grp] = Q K_t^T, then arrive on s_full[grp]
+            const int st = t % C::kStages;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int at = kk >> 2, ko = (kk & 3) * 32;
+                const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                umma_bf16(tmem + C::kTmemS + grp * kBlk, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[grp]);
+        };
+        if (issuer_warp) {
+            if (lane == 0 && grp < T) {
+                const int st = grp % C::kStages;
+                if (mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma) &&
+                    mbar_wait(&full[st], (grp / C::kStages) & 1, abort_flag, kErrTimeoutMma)) {
+                    tc_fence_after();
+                    issue_qk(grp);
+                }
+            }
+            __syncwarp();
+        }
         for (int n = grp; n < T; n += 2) {
             const int ph = (n >> 1) & 1;        // phase of this group's barriers
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
@@ -393,22 +367,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[grp]);
             l = l * alpha + sum;
             m = m_use;
 
-            // P[grp] and O_grp were last used by the P V product of tile n - 2
-            if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[grp], ph ^ 1, abort_flag, kErrTimeoutSoftmax))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint8_t* prow = sPg + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            // P over the first 32 columns of S[grp] (both score chunks were
+            // loaded and waited for above).  O_grp is free to rescale: the
+            // QK^T of this tile completed, and with it every earlier product.
+            tmem_st32u(tS, pk);
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                 for (int cb = 0; cb < D; cb += 32) {
@@ -419,11 +384,34 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     for (int e = 0; e < 32; ++e) ov[e] *= alpha;
                     tmem_st32(tO + cb, ov);
                 }
-                tmem_wait_st();
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[grp]);
+            if (issuer_warp) {
+                if (lane == 0 && mbar_wait(&p_full[grp], ph, abort_flag, kErrTimeoutMma)) {
+                    // O_grp += P V (P read from S[grp]), then the next QK^T into S[grp]
+                    tc_fence_after();
+                    const int st = n % C::kStages;
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t bd = sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                        umma_bf16_ts(tmem + C::kTmemO + grp * D, tmem + C::kTmemS + grp * kBlk + kk * 8, bd,
+                                     idesc_pv, (n >= 2 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[st]);
+                    if (n + 2 < T) {
+                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                                      kErrTimeoutMma)) {
+                            tc_fence_after();
+                            issue_qk(n + 2);
+                        }
+                    } else {
+                        umma_commit(done);
+                    }
+                }
+                __syncwarp();
+            }
         }
         // combine the two groups: exchange (m_g, l_g) through shared memory
         float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
