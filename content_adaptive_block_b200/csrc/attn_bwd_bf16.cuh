@@ -35,12 +35,20 @@ namespace bwd {
 constexpr int kBlk = 64;
 constexpr int kMaxHeads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
-// Elementwise warpgroups: group g takes the tiles n with n % 2 == g, one
-// thread per tile row (TMEM lane), all 64 columns, so the two groups run
-// independently and their MUFU and ALU phases overlap.
-constexpr int kEwGroups = 2;
-constexpr int kEwThreads = 128 * kEwGroups;
-constexpr int kThreads = 64 + kEwThreads;
+// Elementwise warpgroups: group g takes the tiles n with n % G == g, one
+// thread per tile row (TMEM lane), all 64 columns.  d = 64 runs one group
+// per CTA and two CTAs per SM (a CTA then fits in 256 TMEM columns and half
+// the shared memory), so one CTA's set-up and epilogue overlap the other's
+// tiles; d = 128 runs two groups in one CTA per SM.
+#ifndef GSA_BWD64_GROUPS
+#define GSA_BWD64_GROUPS 1
+#endif
+template <int D>
+struct Shape {
+    static constexpr int kGroups = D == 64 ? GSA_BWD64_GROUPS : 2;
+    static constexpr int kThreads = 64 + 128 * kGroups;
+    static constexpr int kCtasPerSm = kGroups == 1 ? 2 : 1;
+};
 
 struct Params {
     const int32_t* ptr;     // CSR row_ptr (dq) or CSC col_ptr (dkdv)
@@ -91,13 +99,13 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
 
 // Ring depths: a stage is released after the last MMA that reads it.
 #ifndef GSA_DQ64_STAGES
-#define GSA_DQ64_STAGES 8
+#define GSA_DQ64_STAGES (GSA_BWD64_GROUPS == 1 ? 4 : 8)
 #endif
 #ifndef GSA_DQ128_STAGES
 #define GSA_DQ128_STAGES 4
 #endif
 #ifndef GSA_DKV64_STAGES
-#define GSA_DKV64_STAGES 8
+#define GSA_DKV64_STAGES (GSA_BWD64_GROUPS == 1 ? 4 : 8)
 #endif
 #ifndef GSA_DKV128_STAGES
 #define GSA_DKV128_STAGES 4
@@ -105,6 +113,7 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
 
 template <int D>
 struct DqCfg {
+    static constexpr int G = Shape<D>::kGroups;
     static constexpr int kAtoms = D / 64;
     static constexpr int kStages = D == 64 ? GSA_DQ64_STAGES : GSA_DQ128_STAGES;
     static constexpr int kTileBytes = 128 * D * 2;      // Q or dO tile (128 rows)
@@ -122,15 +131,16 @@ struct DqCfg {
     static constexpr int kOffBits = kOffLive + kListMaxBlocks;
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
-    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static constexpr int kTmemCols = 512;
+    static_assert(kSmemBytes <= 232448 / Shape<D>::kCtasPerSm - 1024, "shared memory per CTA");
     // S[g] at 128 g (dS over its first 32 columns), dP[g] at 128 g + 64,
-    // dQ_g (group g's share of the sum) at 256 + g D
-    static constexpr int kTmemDQ = 256;
+    // dQ_g (group g's share of the sum) at 128 G + g D
+    static constexpr int kTmemDQ = 128 * G;
+    static constexpr int kTmemCols = kTmemDQ + G * D <= 256 ? 256 : 512;
+    static_assert(kTmemCols * Shape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Shape<D>::kThreads, Shape<D>::kCtasPerSm)
 dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
     using C = DqCfg<D>;
@@ -199,7 +209,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
     build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, qa, qb, nblk);
     if (threadIdx.x == 0) {
-        mbar_init(done, *tl.count >= 2 ? 2 : 1);   // one arrival per group that has tiles
+        mbar_init(done, *tl.count >= C::G ? C::G : 1);   // one arrival per group that has tiles
         fence_mbar_init();
     }
     tc_fence_before();
@@ -267,8 +277,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             __syncwarp();
         }
         bool ok = true;
-        for (int n = grp; n < T; n += 2) {
-            const int ph = (n >> 1) & 1;
+        for (int n = grp; n < T; n += C::G) {
+            const int ph = (n / C::G) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
@@ -312,14 +322,14 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
                         const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
                         umma_bf16_ts(tmem + C::kTmemDQ + grp * D, tmem + grp * 128 + kk * 8, bd, idesc_dq,
-                                     (n >= 2 || kk > 0) ? 1u : 0u);
+                                     (n >= C::G || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[st]);
-                    if (n + 2 < T) {
-                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                    if (n + C::G < T) {
+                        if (mbar_wait(&full[(n + C::G) % C::kStages], ((n + C::G) / C::kStages) & 1, abort_flag,
                                       kErrTimeoutMma)) {
                             tc_fence_after();
-                            issue_s(n + 2);
+                            issue_s(n + C::G);
                         }
                     } else {
                         umma_commit(done);
@@ -331,9 +341,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (ok && T > 0 &&
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
-            const bool has1 = T >= 2;            // dQ_1 holds products only if group 1 had a tile
+            const bool has1 = C::G == 2 && T >= 2;   // dQ_1 holds products only if group 1 had a tile
             __nv_bfloat16* orow = p.out0 + tok * D;
-            constexpr int kOc = D / kEwGroups;   // output columns per thread (split between the groups)
+            constexpr int kOc = D / C::G;        // output columns per thread (split between the groups)
 #pragma unroll
             for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
                 float ov[32];
@@ -365,6 +375,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 
 template <int D>
 struct DkvCfg {
+    static constexpr int G = Shape<D>::kGroups;
     static constexpr int kAtoms = D / 64;
     static constexpr int kStages = D == 64 ? GSA_DKV64_STAGES : GSA_DKV128_STAGES;
     static constexpr int kTileBytes = 128 * D * 2;      // K or V tile (128 key rows)
@@ -384,21 +395,26 @@ struct DkvCfg {
     static constexpr int kOffBits = kOffLive + kListMaxBlocks;
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
-    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kSmemBytes <= 232448 / Shape<D>::kCtasPerSm - 1024, "shared memory per CTA");
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
-    static constexpr int kTmemCols = 512;
     // S^T[g] at 128 g (P^T over its first 32 columns), dP^T[g] at 128 g + 64
-    // (dS^T over its first 32).  d = 64: each group keeps its own dV_g, dK_g
-    // (at 256 + 128 g and 256 + 128 g + 64) and the epilogue adds them; d =
-    // 128 has room for one dV and one dK (256, 256 + D), which the two
-    // groups' products take in turn (the acc barriers order them).
-    static constexpr bool kSplit = D == 64;
-    __host__ __device__ static constexpr uint32_t dv_col(int grp) { return kSplit ? 256 + 128 * grp : 256; }
-    __host__ __device__ static constexpr uint32_t dk_col(int grp) { return kSplit ? 256 + 128 * grp + 64 : 256 + D; }
+    // (dS^T over its first 32), accumulators from 128 G.  With two groups at
+    // d = 64 each group keeps its own dV_g, dK_g (at 128 G + 2 D g and
+    // 128 G + 2 D g + D) and the epilogue adds them; two groups at d = 128
+    // leave room for one dV and one dK, which the groups' products take in
+    // turn (the acc barriers order them).
+    static constexpr bool kSplit = G == 1 || D == 64;
+    static constexpr uint32_t kAcc = 128 * G;
+    __host__ __device__ static constexpr uint32_t dv_col(int grp) { return kSplit ? kAcc + 2 * D * grp : kAcc; }
+    __host__ __device__ static constexpr uint32_t dk_col(int grp) {
+        return kSplit ? kAcc + 2 * D * grp + D : kAcc + D;
+    }
+    static constexpr int kTmemCols = kAcc + (kSplit ? G : 1) * 2 * D <= 256 ? 256 : 512;
+    static_assert(kTmemCols * Shape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Shape<D>::kThreads, Shape<D>::kCtasPerSm)
 dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
     using C = DkvCfg<D>;
@@ -475,7 +491,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
     build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, ka, kb, nblk);
     if (threadIdx.x == 0) {
-        mbar_init(done, *tl.count >= 2 ? 2 : 1);   // one arrival per group that has tiles
+        mbar_init(done, *tl.count >= C::G ? C::G : 1);   // one arrival per group that has tiles
         fence_mbar_init();
     }
     tc_fence_before();
@@ -544,9 +560,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             __syncwarp();
         }
         bool ok = true;
-        for (int n = grp; n < T; n += 2) {
+        for (int n = grp; n < T; n += C::G) {
             const int st = n % C::kStages;
-            const int ph = (n >> 1) & 1;
+            const int ph = (n / C::G) & 1;
             bool w_ok = mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax);
             // the stage's LSE and D came in by TMA: observe its barrier too
             w_ok = w_ok && mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
@@ -609,7 +625,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     // dV += P^T dO, dK += dS^T Q (A from TMEM), then the group's next S^T, dP^T
                     tc_fence_after();
                     const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
-                    const bool first_prod = C::kSplit ? n < 2 : n < 1;
+                    const bool first_prod = C::kSplit ? n < C::G : n < 1;
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
                         const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
@@ -624,11 +640,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     }
                     if (!C::kSplit) umma_commit(&acc[grp]);
                     umma_commit(&empty[st]);
-                    if (n + 2 < T) {
-                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                    if (n + C::G < T) {
+                        if (mbar_wait(&full[(n + C::G) % C::kStages], ((n + C::G) / C::kStages) & 1, abort_flag,
                                       kErrTimeoutMma)) {
                             tc_fence_after();
-                            issue_s(n + 2);
+                            issue_s(n + C::G);
                         }
                     } else {
                         umma_commit(done);
@@ -640,9 +656,9 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (ok && T > 0 &&
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
-            const bool has1 = C::kSplit && T >= 2;   // the group-1 accumulators hold products
+            const bool has1 = C::G == 2 && C::kSplit && T >= 2;   // the group-1 accumulators hold products
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
-            constexpr int kOc = D / kEwGroups;
+            constexpr int kOc = D / C::G;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
@@ -692,8 +708,8 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
         o, dO, const_cast<float*>(pq.dvec), rows);
     dim3 grid(S * H, (nblk + 1) / 2);
-    dq_kernel<D><<<grid, kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
-    dkdv_kernel<D><<<grid, kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+    dq_kernel<D><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+    dkdv_kernel<D><<<grid, Shape<D>::kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
