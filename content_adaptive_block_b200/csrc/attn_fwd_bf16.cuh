@@ -59,10 +59,22 @@ constexpr int kMaxHeads = 256;
 constexpr int kMaxBlocks = 2048;
 constexpr int kBlk = 64;   // block size in tokens
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// Softmax warpgroups: group g owns the tiles n with n % 2 == g.
-constexpr int kSmGroups = 2;
-constexpr int kSmThreads = 128 * kSmGroups;
-constexpr int kFwdThreads = 64 + kSmThreads;
+// Softmax warpgroups: group g owns the tiles n with n % G == g.  d = 64
+// runs one group per CTA and three CTAs per SM (128 TMEM columns each), so
+// CTAs overlap each other's set-up and epilogue; d = 128 runs two groups in
+// one CTA per SM.
+#ifndef GSA_FWD64_GROUPS
+#define GSA_FWD64_GROUPS 1
+#endif
+#ifndef GSA_FWD64_CTAS_PER_SM
+#define GSA_FWD64_CTAS_PER_SM (GSA_FWD64_GROUPS == 1 ? 3 : 2)
+#endif
+template <int D>
+struct FwdShape {
+    static constexpr int kGroups = D == 64 ? GSA_FWD64_GROUPS : 2;
+    static constexpr int kThreads = 64 + 128 * kGroups;
+    static constexpr int kCtasPerSm = D == 64 ? GSA_FWD64_CTAS_PER_SM : 1;
+};
 
 // Named barrier (ids 1..4) joining the two warps that share a TMEM lane quadrant.
 __device__ __forceinline__ void pair_barrier(int quad) {
@@ -87,20 +99,17 @@ struct FwdParams {
     uint8_t cls[kMaxHeads];
 };
 
-// K/V ring depth (one stage = one 64-key block of K and of V), and CTAs per
-// SM for d = 64 (two CTAs overlap each other's hand-offs).
+// K/V ring depth (one stage = one 64-key block of K and of V).
 #ifndef GSA_FWD64_STAGES
-#define GSA_FWD64_STAGES 5
+#define GSA_FWD64_STAGES (GSA_FWD64_GROUPS == 1 ? 3 : 5)
 #endif
 #ifndef GSA_FWD128_STAGES
 #define GSA_FWD128_STAGES 5
 #endif
-#ifndef GSA_FWD64_CTAS_PER_SM
-#define GSA_FWD64_CTAS_PER_SM 2
-#endif
 
 template <int D>
 struct FwdCfg {
+    static constexpr int G = FwdShape<D>::kGroups;
     static constexpr int kAtoms = D / 64;
     static constexpr int kStages = D == 64 ? GSA_FWD64_STAGES : GSA_FWD128_STAGES;
     static constexpr int kQBytes = 128 * D * 2;
@@ -115,18 +124,20 @@ struct FwdCfg {
     static constexpr int kOffList = kOffMisc + 16;            // int16 key block per tile
     static constexpr int kOffLive = kOffList + kMaxBlocks * 2;
     static constexpr int kOffBits = kOffLive + kMaxBlocks;    // two bitmaps
-    static constexpr int kOffMl = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [2 group][2][128]: m_g, l_g
-    static constexpr int kEnd = kOffMl + 2 * 2 * 128 * 4;
+    static constexpr int kOffMl = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [G group][2][128]: m_g, l_g
+    static constexpr int kEnd = kOffMl + G * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;            // + alignment slack
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static_assert(D != 64 || GSA_FWD64_CTAS_PER_SM == 1 || kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
-    static constexpr int kTmemCols = (128 + 2 * D) <= 256 ? 256 : 512;
+    static_assert(kSmemBytes <= 232448 / FwdShape<D>::kCtasPerSm - 1024, "shared memory per SM");
     static constexpr int kTmemS = 0;       // S[g] at columns 64 g
-    static constexpr int kTmemO = 128;     // O_g at columns 128 + g D
+    static constexpr int kTmemO = 64 * G;  // O_g at columns 64 G + g D
+    static constexpr int kTmemNeed = kTmemO + G * D;
+    static constexpr int kTmemCols = kTmemNeed <= 128 ? 128 : (kTmemNeed <= 256 ? 256 : 512);
+    static_assert(kTmemCols * FwdShape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, D == 64 ? GSA_FWD64_CTAS_PER_SM : 1)
+__global__ void __launch_bounds__(FwdShape<D>::kThreads, FwdShape<D>::kCtasPerSm)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdCfg<D>;
@@ -237,7 +248,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
         if (lane == 31) {
             *ntiles_slot = incl;
-            mbar_init(done, incl >= 2 ? 2 : 1);   // one arrival per group that has tiles
+            mbar_init(done, incl >= C::G ? C::G : 1);   // one arrival per group that has tiles
             fence_mbar_init();
         }
     }
@@ -306,8 +317,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
             __syncwarp();
         }
-        for (int n = grp; n < T; n += 2) {
-            const int ph = (n >> 1) & 1;        // phase of this group's barriers
+        for (int n = grp; n < T; n += C::G) {
+            const int ph = (n / C::G) & 1;      // phase of this group's barriers
             if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
@@ -397,14 +408,14 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
                         const uint64_t bd = sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
                         umma_bf16_ts(tmem + C::kTmemO + grp * D, tmem + C::kTmemS + grp * kBlk + kk * 8, bd,
-                                     idesc_pv, (n >= 2 || kk > 0) ? 1u : 0u);
+                                     idesc_pv, (n >= C::G || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[st]);
-                    if (n + 2 < T) {
-                        if (mbar_wait(&full[(n + 2) % C::kStages], ((n + 2) / C::kStages) & 1, abort_flag,
+                    if (n + C::G < T) {
+                        if (mbar_wait(&full[(n + C::G) % C::kStages], ((n + C::G) / C::kStages) & 1, abort_flag,
                                       kErrTimeoutMma)) {
                             tc_fence_after();
-                            issue_qk(n + 2);
+                            issue_qk(n + C::G);
                         }
                     } else {
                         umma_commit(done);
@@ -413,18 +424,23 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 __syncwarp();
             }
         }
-        // combine the two groups: exchange (m_g, l_g) through shared memory
-        float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
-        ml[(grp * 2 + 0) * 128 + r] = m;
-        ml[(grp * 2 + 1) * 128 + r] = l;
-        pair_barrier(quad);
-        const float m0 = ml[0 * 128 + r], l0 = ml[1 * 128 + r];
-        const float m1 = ml[2 * 128 + r], l1 = ml[3 * 128 + r];
+        // combine the groups: exchange (m_g, l_g) through shared memory
+        float m0 = m, l0 = l, m1 = -INFINITY, l1 = 0.f;
+        if constexpr (C::G == 2) {
+            float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
+            ml[(grp * 2 + 0) * 128 + r] = m;
+            ml[(grp * 2 + 1) * 128 + r] = l;
+            pair_barrier(quad);
+            m0 = ml[0 * 128 + r];
+            l0 = ml[1 * 128 + r];
+            m1 = ml[2 * 128 + r];
+            l1 = ml[3 * 128 + r];
+        }
         // every product of the CTA completed (a single-phase barrier: the other
         // group's buffer barriers may be more than one phase behind)
         if (ok && T > 0 && __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
-            const bool has1 = T >= 2;           // O_1 holds products only if group 1 had a tile
+            const bool has1 = C::G == 2 && T >= 2;   // O_1 holds products only if group 1 had a tile
             const float mm = fmaxf(m0, has1 ? m1 : -INFINITY);
             const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
             const float w1 = (!has1 || m1 == -INFINITY) ? 0.f : ex2(m1 - mm);
@@ -434,7 +450,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const int64_t tok = head_row0 + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
             __nv_bfloat16* orow = p.o + tok * D;
 #pragma unroll
-            for (int cb = grp * (D / 2); cb < (grp + 1) * (D / 2); cb += 32) {
+            for (int cb = grp * (D / C::G); cb < (grp + 1) * (D / C::G); cb += 32) {
                 float a[32];
                 tmem_ld32(tl + C::kTmemO + cb, a);
                 tmem_wait_ld();

@@ -226,7 +226,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
             cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
         });
-        gsa::bf16::attn_fwd_bf16_kernel<64><<<grid, gsa::bf16::kFwdThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+        gsa::bf16::attn_fwd_bf16_kernel<64><<<grid, gsa::bf16::FwdShape<64>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
     } else {
         using C = gsa::bf16::FwdCfg<128>;
         static std::once_flag once;
@@ -234,7 +234,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
             cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         });
-        gsa::bf16::attn_fwd_bf16_kernel<128><<<grid, gsa::bf16::kFwdThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+        gsa::bf16::attn_fwd_bf16_kernel<128><<<grid, gsa::bf16::FwdShape<128>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
     }
     return launch_status();
 }
