@@ -12,41 +12,38 @@
 // one key block of 64 tokens.  Rows of a half whose block is not live for a
 // key tile are masked out of it; the diagonal block gets the token causal cut.
 //
-// Roles (320 threads):
+// Roles (64 + 128 G threads):
 //   thread 0 issues the TMA load of Q as soon as the barriers exist, so it
 //           overlaps the merge of the key lists;
 //   warp 0  one thread issues the TMA loads of K and V of each key tile
 //           into a ring of shared-memory stages;
-//   warp 1  allocates TMEM;
-//   warps 2-9  softmax, two warpgroups; group g takes the tiles n with
-//           n % 2 == g, one thread per query row (TMEM lane), all 64 key
+//   warp 1  allocates TMEM; one thread issues every MMA of the CTA, in tile
+//           order, as soon as its operands are ready:
+//             S[g][b] = Q K^T   (M=128, N=64, K=d;  A and B from shared memory)
+//             O_g    += P_g V   (M=128, N=d,  K=64; A = P from TMEM, B = V)
+//           The QK^T of a tile needs its K/V stage and a free S buffer of its
+//           group; with two S buffers per group it runs while the group's
+//           softmax works on the previous tile.
+//   warps 2..  softmax, G warpgroups; group g takes the tiles n with
+//           n % G == g, one thread per query row (TMEM lane), all 64 key
 //           columns.  Each group keeps its own running max m_g, row sum l_g
 //           and accumulator O_g = Σ P V over its tiles (split-key online
-//           softmax), so the groups run independently and their exp2 (MUFU)
-//           and ALU phases overlap.  O_g is rescaled in TMEM only when m_g
-//           grows by more than 8 (log2 units): exact for any reference max,
-//           the threshold bounds P <= 256.  P goes back to TMEM as packed
-//           bf16 pairs over the first 32 columns of S[g] (lane = query row,
-//           column c = key columns 2c, 2c+1: the layout of an M=128 A operand
-//           in TMEM), so it never passes through shared memory.  The
-//           tensor pipe runs one thread's MMAs in issue order, so the QK^T of
-//           tile n+2 may overwrite S[g] once the P V of tile n is issued.
-//           One thread of each group issues that group's MMAs,
-//             S[g]  = Q K^T   (M=128, N=64, K=d;  A and B from shared memory)
-//             O_g  += P V     (M=128, N=d,  K=64; A = P from TMEM, B = V),
-//           right after the group's 128 rows of P are in TMEM: two
-//           independent MMA streams per CTA, and every product a group's
-//           rows read was issued (so ordered and tracked) by one thread.
-//           At the end the two halves combine:
+//           softmax).  O_g is rescaled in TMEM only when m_g grows by more
+//           than 8 (log2 units): exact for any reference max, the threshold
+//           bounds P <= 256.  P goes to TMEM as packed bf16 pairs (lane =
+//           query row, column c = key columns 2c, 2c+1: the layout of an
+//           M=128 A operand in TMEM), so it never passes through shared
+//           memory.  With G = 2 the halves combine at the end:
 //           m = max(m_0, m_1), O = Σ_g O_g 2^(m_g - m) / Σ_g l_g 2^(m_g - m).
-// The QK^T of tile n+1 overlaps the softmax of tile n.
+// d = 64 runs one softmax group per CTA with two S buffers and two CTAs per
+// SM; d = 128 runs two groups with one S buffer each in one CTA per SM.
 //
 // Shared memory (128-byte swizzle, 1024-byte aligned):
 //   Q  [d/64 column atoms][128 rows][128 B]
 //   K  stage [d/64 atoms][64 rows][128 B]          (B operand, K-major)
 //   V  stage [d/64 atoms][64 rows][128 B]          (B operand, MN-major)
-// TMEM (lanes = query rows): S[0], S[1] at columns 0 and 64 (P over their
-// first 32 columns), O_0 and O_1 at columns 128 and 128 + d.
+// TMEM (lanes = query rows): S[g][b] at columns 64 (g NS + b), O_g at
+// 64 G NS + g d, P_g (32 columns) after the O accumulators.
 #pragma once
 
 #include "common.cuh"
@@ -59,19 +56,28 @@ constexpr int kMaxHeads = 256;
 constexpr int kMaxBlocks = 2048;
 constexpr int kBlk = 64;   // block size in tokens
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// Softmax warpgroups: group g owns the tiles n with n % G == g.  d = 64
-// runs one group per CTA and three CTAs per SM (128 TMEM columns each), so
-// CTAs overlap each other's set-up and epilogue; d = 128 runs two groups in
-// one CTA per SM.
+
 #ifndef GSA_FWD64_GROUPS
 #define GSA_FWD64_GROUPS 1
 #endif
-#ifndef GSA_FWD64_CTAS_PER_SM
-#define GSA_FWD64_CTAS_PER_SM (GSA_FWD64_GROUPS == 1 ? 3 : 2)
+#ifndef GSA_FWD64_SBUF
+#define GSA_FWD64_SBUF 2
 #endif
+#ifndef GSA_FWD64_CTAS_PER_SM
+#define GSA_FWD64_CTAS_PER_SM 2
+#endif
+// K/V ring depth (one stage = one 64-key block of K and of V).
+#ifndef GSA_FWD64_STAGES
+#define GSA_FWD64_STAGES 5
+#endif
+#ifndef GSA_FWD128_STAGES
+#define GSA_FWD128_STAGES 5
+#endif
+
 template <int D>
 struct FwdShape {
     static constexpr int kGroups = D == 64 ? GSA_FWD64_GROUPS : 2;
+    static constexpr int kSBuf = D == 64 ? GSA_FWD64_SBUF : 1;   // S buffers per group
     static constexpr int kThreads = 64 + 128 * kGroups;
     static constexpr int kCtasPerSm = D == 64 ? GSA_FWD64_CTAS_PER_SM : 1;
 };
@@ -99,17 +105,10 @@ struct FwdParams {
     uint8_t cls[kMaxHeads];
 };
 
-// K/V ring depth (one stage = one 64-key block of K and of V).
-#ifndef GSA_FWD64_STAGES
-#define GSA_FWD64_STAGES (GSA_FWD64_GROUPS == 1 ? 3 : 5)
-#endif
-#ifndef GSA_FWD128_STAGES
-#define GSA_FWD128_STAGES 5
-#endif
-
 template <int D>
 struct FwdCfg {
     static constexpr int G = FwdShape<D>::kGroups;
+    static constexpr int NS = FwdShape<D>::kSBuf;
     static constexpr int kAtoms = D / 64;
     static constexpr int kStages = D == 64 ? GSA_FWD64_STAGES : GSA_FWD128_STAGES;
     static constexpr int kQBytes = 128 * D * 2;
@@ -118,8 +117,8 @@ struct FwdCfg {
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
     static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-    // barriers: full[st], empty[st], q_full, s_full[2], p_full[2], done
-    static constexpr int kNumBars = 2 * kStages + 6;
+    // barriers: full[st], empty[st], q_full, done, s_full[G][NS], s_free[G][NS], p_full[G], p_free[G]
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 * G * NS + 2 * G;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, ntiles
     static constexpr int kOffList = kOffMisc + 16;            // int16 key block per tile
     static constexpr int kOffLive = kOffList + kMaxBlocks * 2;
@@ -127,11 +126,11 @@ struct FwdCfg {
     static constexpr int kOffMl = kOffBits + 2 * (kMaxBlocks / 32) * 4;   // [G group][2][128]: m_g, l_g
     static constexpr int kEnd = kOffMl + G * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;            // + alignment slack
-    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes <= 232448 / FwdShape<D>::kCtasPerSm - 1024, "shared memory per SM");
-    static constexpr int kTmemS = 0;       // S[g] at columns 64 g
-    static constexpr int kTmemO = 64 * G;  // O_g at columns 64 G + g D
-    static constexpr int kTmemNeed = kTmemO + G * D;
+    static constexpr int kTmemS = 0;                  // S[g][b] at 64 (g NS + b)
+    static constexpr int kTmemO = 64 * G * NS;        // O_g at kTmemO + g D
+    static constexpr int kTmemP = kTmemO + G * D;     // P_g at kTmemP + 32 g
+    static constexpr int kTmemNeed = kTmemP + 32 * G;
     static constexpr int kTmemCols = kTmemNeed <= 128 ? 128 : (kTmemNeed <= 256 ? 256 : 512);
     static_assert(kTmemCols * FwdShape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
@@ -141,6 +140,7 @@ __global__ void __launch_bounds__(FwdShape<D>::kThreads, FwdShape<D>::kCtasPerSm
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdCfg<D>;
+    constexpr int G = C::G, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sQ = smem + C::kOffQ;
@@ -150,9 +150,11 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     uint64_t* full = bars;
     uint64_t* empty = bars + C::kStages;
     uint64_t* q_full = bars + 2 * C::kStages;
-    uint64_t* s_full = q_full + 1;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* done = p_full + 2;    // one phase: every product of the CTA completed
+    uint64_t* done = q_full + 1;        // one phase: every product of the CTA completed
+    uint64_t* s_full = done + 1;        // [G][NS] QK^T landed in S[g][b]
+    uint64_t* s_free = s_full + G * NS; // [G][NS] the group read S[g][b]
+    uint64_t* p_full = s_free + G * NS; // [G] the group's P is in TMEM
+    uint64_t* p_free = p_full + G;      // [G] the group's P V completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     int* ntiles_slot = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
@@ -171,6 +173,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int qa = p.q_order[g * nblk + 2 * tile];
     const int qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
     const int nwords = (nblk + 31) >> 5;
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;   // first row of this (s, h) in the 2-D views
 
     // ---- set-up: barriers, TMEM, merged key list
     if (threadIdx.x == 0) {
@@ -179,21 +182,25 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_init(&empty[st], 1);
         }
         mbar_init(q_full, 1);
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
-        mbar_init(&p_full[0], 128);
-        mbar_init(&p_full[1], 128);
+        mbar_init(done, 1);
+        for (int i = 0; i < G * NS; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 128);
+        }
+        for (int i = 0; i < G; ++i) {
+            mbar_init(&p_full[i], 128);
+            mbar_init(&p_free[i], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         // Q of the tile: needs only qa and qb, so it loads while the key lists merge
-        const int64_t row0 = static_cast<int64_t>(sh) * p.L;
         mbar_arrive_expect_tx(q_full, (qb >= 0 ? 2 : 1) * kBlk * D * 2);
         for (int half = 0; half < 2; ++half) {
             const int blk = half ? qb : qa;
             if (blk < 0) continue;
-            const int row = static_cast<int>(row0 + static_cast<int64_t>(blk) * kBlk);
+            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
             for (int at = 0; at < C::kAtoms; ++at)
                 tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
         }
@@ -246,18 +253,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 ++pos;
             }
         }
-        if (lane == 31) {
-            *ntiles_slot = incl;
-            mbar_init(done, incl >= C::G ? C::G : 1);   // one arrival per group that has tiles
-            fence_mbar_init();
-        }
+        if (lane == 31) *ntiles_slot = incl;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const int T = *ntiles_slot;
     const uint32_t tmem = *tmem_slot;
-    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;   // first row of this (s, h) in the 2-D views
 
     if (warp == 0) {
         // ================= TMA producer
@@ -277,49 +279,82 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
             }
         }
-    } else if (warp >= 2) {
-        // ================= softmax warpgroups (warps 2..9)
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            // Q is waited for even without tiles: no load may be in flight at exit
+            bool ok = mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma);
+            // Both streams advance in tile order: QK^T of tile ns (group ns % G,
+            // its k-th, S buffer k % NS) once its K/V stage is loaded and the
+            // group has read that buffer's previous scores; P V of tile na once
+            // the group's P is in TMEM.
+            int ns = 0, na = 0;
+            PollGuard guard;
+            while (ok && na < T) {
+                bool moved = false;
+                if (ns < T) {
+                    const int st = ns % C::kStages;
+                    const int gq = ns % G, kq = ns / G, sb = gq * NS + kq % NS;
+                    if (mbar_test(&full[st], (ns / C::kStages) & 1) &&
+                        (kq < NS || mbar_test(&s_free[sb], ((kq - NS) / NS) & 1))) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int at = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
+                            const uint64_t bd =
+                                sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
+                            umma_bf16(tmem + C::kTmemS + 64 * sb, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&s_full[sb]);
+                        ++ns;
+                        moved = true;
+                    }
+                }
+                if (na < ns) {
+                    const int st = na % C::kStages;
+                    const int gp = na % G, kp = na / G;
+                    if (mbar_test(&p_full[gp], kp & 1)) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const uint64_t bd =
+                                sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
+                            umma_bf16_ts(tmem + C::kTmemO + gp * D, tmem + C::kTmemP + 32 * gp + kk * 8, bd,
+                                         idesc_pv, (kp > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&p_free[gp]);
+                        umma_commit(&empty[st]);
+                        ++na;
+                        moved = true;
+                    }
+                }
+                if (moved) guard.progress();
+                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
+            }
+            if (ok && T > 0) umma_commit(done);
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax warpgroups (warps 2..)
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
+        const int grp = (warp - 2) >> 2;        // this group takes the tiles n % G == grp
         const int r = quad * 32 + lane;         // query row in the tile = TMEM lane
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
         const int rr = r & 63;
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const uint32_t tS = tl + C::kTmemS + grp * kBlk;
         const uint32_t tO = tl + C::kTmemO + grp * D;
+        const uint32_t tP = tl + C::kTmemP + 32 * grp;
         float m = -INFINITY, l = 0.f;           // this group's running max and sum
         bool ok = true;
-        // the group's MMA issuer: lane 0 of its first warp
-        const bool issuer_warp = ((warp - 2) & 3) == 0;
-        constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
-        constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-        auto issue_qk = [&](int t) {   // S[grp] = Q K_t^T, then arrive on s_full[grp]
-            const int st = t % C::kStages;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int at = kk >> 2, ko = (kk & 3) * 32;
-                const uint64_t ad = sdesc_sw128(aQ + at * (128 * 128) + ko, 16, 1024);
-                const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + at * (kBlk * 128) + ko, 16, 1024);
-                umma_bf16(tmem + C::kTmemS + grp * kBlk, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&s_full[grp]);
-        };
-        if (issuer_warp) {
-            if (lane == 0 && grp < T) {
-                const int st = grp % C::kStages;
-                if (mbar_wait(q_full, 0, abort_flag, kErrTimeoutMma) &&
-                    mbar_wait(&full[st], (grp / C::kStages) & 1, abort_flag, kErrTimeoutMma)) {
-                    tc_fence_after();
-                    issue_qk(grp);
-                }
-            }
-            __syncwarp();
-        }
-        for (int n = grp; n < T; n += C::G) {
-            const int ph = (n / C::G) & 1;      // phase of this group's barriers
-            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[grp], ph, abort_flag, kErrTimeoutSoftmax))) {
+        for (int n = grp, k = 0; n < T; n += G, ++k) {
+            const int sb = grp * NS + k % NS;
+            const uint32_t tS = tl + C::kTmemS + 64 * sb;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (k / NS) & 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
@@ -380,11 +415,19 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
             l = l * alpha + sum;
             m = m_use;
+            // the scores are in registers: S[grp][b] may take the group's next QK^T
+            tc_fence_before();
+            mbar_arrive(&s_free[sb]);
 
-            // P over the first 32 columns of S[grp] (both score chunks were
-            // loaded and waited for above).  O_grp is free to rescale: the
-            // QK^T of this tile completed, and with it every earlier product.
-            tmem_st32u(tS, pk);
+            // P_grp and O_grp were last used by the P V product of the group's
+            // previous tile
+            if (k >= 1 &&
+                !__all_sync(0xffffffffu, mbar_wait(&p_free[grp], (k - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_st32u(tP, pk);
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                 for (int cb = 0; cb < D; cb += 32) {
@@ -399,30 +442,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[grp]);
-            if (issuer_warp) {
-                if (lane == 0 && mbar_wait(&p_full[grp], ph, abort_flag, kErrTimeoutMma)) {
-                    // O_grp += P V (P read from S[grp]), then the next QK^T into S[grp]
-                    tc_fence_after();
-                    const int st = n % C::kStages;
-#pragma unroll
-                    for (int kk = 0; kk < kBlk / 16; ++kk) {
-                        const uint64_t bd = sdesc_sw128(aV + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                        umma_bf16_ts(tmem + C::kTmemO + grp * D, tmem + C::kTmemS + grp * kBlk + kk * 8, bd,
-                                     idesc_pv, (n >= C::G || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&empty[st]);
-                    if (n + C::G < T) {
-                        if (mbar_wait(&full[(n + C::G) % C::kStages], ((n + C::G) / C::kStages) & 1, abort_flag,
-                                      kErrTimeoutMma)) {
-                            tc_fence_after();
-                            issue_qk(n + C::G);
-                        }
-                    } else {
-                        umma_commit(done);
-                    }
-                }
-                __syncwarp();
-            }
         }
         // combine the groups: exchange (m_g, l_g) through shared memory
         float m0 = m, l0 = l, m1 = -INFINITY, l1 = 0.f;
