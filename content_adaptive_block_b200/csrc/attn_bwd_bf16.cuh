@@ -292,20 +292,28 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = 0u;
             } else {
+                // 16-column chunks; the next chunk's TMEM loads are in flight
+                // while this one is computed
+                float sv[2][16], dp[2][16];
+                tmem_ld16(tlane + grp * 128, sv[0]);
+                tmem_ld16(tlane + grp * 128 + 64, dp[0]);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    float sv[32], dp[32];
-                    tmem_ld32(tlane + grp * 128 + 32 * ch, sv);
-                    tmem_ld32(tlane + grp * 128 + 64 + 32 * ch, dp);
+                for (int ch = 0; ch < 4; ++ch) {
                     tmem_wait_ld();
+                    if (ch < 3) {
+                        tmem_ld16(tlane + grp * 128 + 16 * (ch + 1), sv[(ch + 1) & 1]);
+                        tmem_ld16(tlane + grp * 128 + 64 + 16 * (ch + 1), dp[(ch + 1) & 1]);
+                    }
+                    float* s_ = sv[ch & 1];
+                    const float* d_ = dp[ch & 1];
 #pragma unroll
-                    for (int cc = 0; cc < 32; ++cc) sv[cc] = ex2(fmaf(sv[cc], p.scale_log2, -lse2)) * (dp[cc] - dt);
-                    if (last < 32 * ch + 31) {
+                    for (int cc = 0; cc < 16; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, -lse2)) * (d_[cc] - dt);
+                    if (last < 16 * ch + 15) {
 #pragma unroll
-                        for (int cc = 0; cc < 32; ++cc) sv[cc] = 32 * ch + cc <= last ? sv[cc] : 0.f;
+                        for (int cc = 0; cc < 16; ++cc) s_[cc] = 16 * ch + cc <= last ? s_[cc] : 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(sv[2 * e], sv[2 * e + 1]);
+                    for (int e = 0; e < 8; ++e) pk[8 * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
                 }
             }
             // dS over the first 32 columns of S[grp] (both chunks were read above)
@@ -582,31 +590,39 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             } else {
                 const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st));
                 const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st));
+                // 16-column chunks; the next chunk's TMEM loads are in flight
+                // while this one is computed
+                float sv[2][16], dp[2][16];
+                tmem_ld16(tlane + grp * 128, sv[0]);
+                tmem_ld16(tlane + grp * 128 + 64, dp[0]);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    float sv[32], dp[32];
-                    tmem_ld32(tlane + grp * 128 + 32 * ch, sv);
-                    tmem_ld32(tlane + grp * 128 + 64 + 32 * ch, dp);
+                for (int ch = 0; ch < 4; ++ch) {
                     tmem_wait_ld();
+                    if (ch < 3) {
+                        tmem_ld16(tlane + grp * 128 + 16 * (ch + 1), sv[(ch + 1) & 1]);
+                        tmem_ld16(tlane + grp * 128 + 64 + 16 * (ch + 1), dp[(ch + 1) & 1]);
+                    }
+                    float* s_ = sv[ch & 1];
+                    float* d_ = dp[ch & 1];
 #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 l4 = lse4[8 * ch + c4];
-                        const float4 d4 = dv4[8 * ch + c4];
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float4 l4 = lse4[4 * ch + c4];
+                        const float4 d4 = dv4[4 * ch + c4];
                         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                         const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int cc = 4 * c4 + e;
-                            float pr = ex2(fmaf(sv[cc], p.scale_log2, -lv[e] * kLog2e));
-                            if (first > 32 * ch) pr = 32 * ch + cc >= first ? pr : 0.f;
-                            sv[cc] = pr;
-                            dp[cc] = pr * (dp[cc] - dd[e]);
+                            float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e] * kLog2e));
+                            if (first > 16 * ch) pr = 16 * ch + cc >= first ? pr : 0.f;
+                            s_[cc] = pr;
+                            d_[cc] = pr * (d_[cc] - dd[e]);
                         }
                     }
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        pp[16 * ch + e] = pack_bf16x2(sv[2 * e], sv[2 * e + 1]);
-                        pd[16 * ch + e] = pack_bf16x2(dp[2 * e], dp[2 * e + 1]);
+                    for (int e = 0; e < 8; ++e) {
+                        pp[8 * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
+                        pd[8 * ch + e] = pack_bf16x2(d_[2 * e], d_[2 * e + 1]);
                     }
                 }
             }
