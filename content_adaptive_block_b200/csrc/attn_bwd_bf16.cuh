@@ -43,10 +43,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 #ifndef GSA_BWD64_GROUPS
 #define GSA_BWD64_GROUPS 1
 #endif
+// With one group, each tile's 64 columns are split between two warpgroups
+// (32 columns per thread), so eight elementwise warps share a tile.
+#ifndef GSA_BWD64_HALVES
+#define GSA_BWD64_HALVES 2
+#endif
 template <int D>
 struct Shape {
     static constexpr int kGroups = D == 64 ? GSA_BWD64_GROUPS : 2;
-    static constexpr int kThreads = 64 + 128 * kGroups;
+    static constexpr int kHalves = kGroups == 1 ? GSA_BWD64_HALVES : 1;
+    static constexpr int kThreads = 64 + 128 * kGroups * kHalves;
     static constexpr int kCtasPerSm = kGroups == 1 ? 2 : 1;
 };
 
@@ -185,8 +191,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(q_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&ds_full[0], 128);
-        mbar_init(&ds_full[1], 128);
+        mbar_init(&ds_full[0], 128 * Shape<D>::kHalves);
+        mbar_init(&ds_full[1], 128 * Shape<D>::kHalves);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
@@ -234,8 +240,15 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
         }
     } else if (warp >= 2) {
+        // warp e = warp - 2: group (e / 4) % G, column half (e / 4) / G
+        constexpr int H = Shape<D>::kHalves;
+        constexpr int kCols = kBlk / H;         // key columns per thread
+        constexpr int kW = 16 / H;              // chunk width (four chunks)
+        const int e4 = (warp - 2) >> 2;
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int grp = (warp - 2) >> 2;        // this group takes the tiles n % 2 == grp
+        const int grp = e4 % C::G;              // this group takes the tiles n % G == grp
+        const int hc = e4 / C::G;               // key columns [kCols hc, kCols (hc + 1))
+        const int c0 = kCols * hc;
         const int r = quad * 32 + lane;
         const int half = r >> 6;
         const int my_blk = half ? qb : qa;
@@ -245,7 +258,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const float lse2 = my_blk >= 0 ? p.lse[tok] * kLog2e : 0.f;
         const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
         // the group's MMA issuer: lane 0 of its first warp
-        const bool issuer_warp = ((warp - 2) & 3) == 0;
+        const bool issuer_warp = ((warp - 2) & 3) == 0 && hc == 0;
         constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
         constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1);
         const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
@@ -287,37 +300,40 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const int j = tl.list[n];
             const bool is_live = (tl.live[n] >> half) & 1;
             const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);   // visible key columns 0..last
-            uint32_t pk[32];
-            if (last < 0) {
+            uint32_t pk[kCols / 2];
+            if (last < c0) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pk[e] = 0u;
+                for (int e = 0; e < kCols / 2; ++e) pk[e] = 0u;
             } else {
-                // 16-column chunks; the next chunk's TMEM loads are in flight
-                // while this one is computed
-                float sv[2][16], dp[2][16];
-                tmem_ld16(tlane + grp * 128, sv[0]);
-                tmem_ld16(tlane + grp * 128 + 64, dp[0]);
+                // four chunks of kW columns; the next chunk's TMEM loads are in
+                // flight while one is computed
+                float sv[2][kW], dp[2][kW];
+                tmem_ldw<kW>(tlane + grp * 128 + c0, sv[0]);
+                tmem_ldw<kW>(tlane + grp * 128 + 64 + c0, dp[0]);
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     tmem_wait_ld();
                     if (ch < 3) {
-                        tmem_ld16(tlane + grp * 128 + 16 * (ch + 1), sv[(ch + 1) & 1]);
-                        tmem_ld16(tlane + grp * 128 + 64 + 16 * (ch + 1), dp[(ch + 1) & 1]);
+                        tmem_ldw<kW>(tlane + grp * 128 + c0 + kW * (ch + 1), sv[(ch + 1) & 1]);
+                        tmem_ldw<kW>(tlane + grp * 128 + 64 + c0 + kW * (ch + 1), dp[(ch + 1) & 1]);
                     }
                     float* s_ = sv[ch & 1];
                     const float* d_ = dp[ch & 1];
+                    const int cb = c0 + kW * ch;   // first key column of the chunk
 #pragma unroll
-                    for (int cc = 0; cc < 16; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, -lse2)) * (d_[cc] - dt);
-                    if (last < 16 * ch + 15) {
+                    for (int cc = 0; cc < kW; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, -lse2)) * (d_[cc] - dt);
+                    if (last < cb + kW - 1) {
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc) s_[cc] = 16 * ch + cc <= last ? s_[cc] : 0.f;
+                        for (int cc = 0; cc < kW; ++cc) s_[cc] = cb + cc <= last ? s_[cc] : 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) pk[8 * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
+                    for (int e = 0; e < kW / 2; ++e) pk[(kW / 2) * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
                 }
             }
-            // dS over the first 32 columns of S[grp] (both chunks were read above)
-            tmem_st32u(tlane + grp * 128, pk);
+            // this thread's dS, packed, over the first kCols / 2 of its own S
+            // columns (all read above): key pairs of columns [c0, c0 + kCols)
+            // sit at S[grp] columns c0 .. c0 + kCols / 2 - 1
+            tmem_stn<kCols / 2>(tlane + grp * 128 + c0, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&ds_full[grp]);
@@ -328,8 +344,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int st = n % C::kStages;
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const int h_ = (16 * kk) / kCols;   // the half holding keys 16 kk ..
+                        const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
                         const uint64_t bd = sdesc_sw128(aK + st * C::kKVBytes + kk * (16 * 128), kBlk * 128, 1024);
-                        umma_bf16_ts(tmem + C::kTmemDQ + grp * D, tmem + grp * 128 + kk * 8, bd, idesc_dq,
+                        umma_bf16_ts(tmem + C::kTmemDQ + grp * D, tmem + grp * 128 + acol, bd, idesc_dq,
                                      (n >= C::G || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[st]);
@@ -351,9 +369,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             tc_fence_after();
             const bool has1 = C::G == 2 && T >= 2;   // dQ_1 holds products only if group 1 had a tile
             __nv_bfloat16* orow = p.out0 + tok * D;
-            constexpr int kOc = D / C::G;        // output columns per thread (split between the groups)
+            constexpr int kOc = D / (C::G * H);   // output columns per thread (split among a row's threads)
+            const int slot = grp * H + hc;
 #pragma unroll
-            for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
+            for (int cb = slot * kOc; cb < (slot + 1) * kOc; cb += 32) {
                 float ov[32];
                 tmem_ld32(tlane + C::kTmemDQ + cb, ov);
                 tmem_wait_ld();
@@ -473,8 +492,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(kv_full, 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(&p_full[0], 128);
-        mbar_init(&p_full[1], 128);
+        mbar_init(&p_full[0], 128 * Shape<D>::kHalves);
+        mbar_init(&p_full[1], 128 * Shape<D>::kHalves);
         mbar_init(&acc[0], 1);
         mbar_init(&acc[1], 1);
         *abort_flag = 0;
@@ -527,15 +546,22 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             }
         }
     } else if (warp >= 2) {
+        // warp e = warp - 2: group (e / 4) % G, column half (e / 4) / G
+        constexpr int H = Shape<D>::kHalves;
+        constexpr int kCols = kBlk / H;          // query columns per thread
+        constexpr int kW = 16 / H;               // chunk width (four chunks)
+        const int e4 = (warp - 2) >> 2;
         const int quad = warp & 3;
-        const int grp = (warp - 2) >> 2;         // this group takes the tiles n % 2 == grp
+        const int grp = e4 % C::G;               // this group takes the tiles n % G == grp
+        const int hc = e4 / C::G;                // query columns [kCols hc, kCols (hc + 1))
+        const int c0 = kCols * hc;
         const int u = quad * 32 + lane;          // key row of the tile = TMEM lane
         const int half = u >> 6;
         const int my_blk = half ? kb : ka;
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         // the group's MMA issuer: lane 0 of its first warp
-        const bool issuer_warp = ((warp - 2) & 3) == 0;
+        const bool issuer_warp = ((warp - 2) & 3) == 0 && hc == 0;
         constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
         constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
         const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
@@ -583,52 +609,54 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const bool is_live = (tl.live[n] >> half) & 1;
             // query columns allowed: live block, and in the diagonal block t >= u
             const int first = !is_live ? kBlk : (i == my_blk ? uu : 0);
-            uint32_t pp[32], pd[32];
-            if (first >= kBlk) {
+            uint32_t pp[kCols / 2], pd[kCols / 2];
+            if (first >= c0 + kCols) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pp[e] = pd[e] = 0u;
+                for (int e = 0; e < kCols / 2; ++e) pp[e] = pd[e] = 0u;
             } else {
                 const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st));
                 const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st));
-                // 16-column chunks; the next chunk's TMEM loads are in flight
-                // while this one is computed
-                float sv[2][16], dp[2][16];
-                tmem_ld16(tlane + grp * 128, sv[0]);
-                tmem_ld16(tlane + grp * 128 + 64, dp[0]);
+                // four chunks of kW columns; the next chunk's TMEM loads are in
+                // flight while one is computed
+                float sv[2][kW], dp[2][kW];
+                tmem_ldw<kW>(tlane + grp * 128 + c0, sv[0]);
+                tmem_ldw<kW>(tlane + grp * 128 + 64 + c0, dp[0]);
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     tmem_wait_ld();
                     if (ch < 3) {
-                        tmem_ld16(tlane + grp * 128 + 16 * (ch + 1), sv[(ch + 1) & 1]);
-                        tmem_ld16(tlane + grp * 128 + 64 + 16 * (ch + 1), dp[(ch + 1) & 1]);
+                        tmem_ldw<kW>(tlane + grp * 128 + c0 + kW * (ch + 1), sv[(ch + 1) & 1]);
+                        tmem_ldw<kW>(tlane + grp * 128 + 64 + c0 + kW * (ch + 1), dp[(ch + 1) & 1]);
                     }
                     float* s_ = sv[ch & 1];
                     float* d_ = dp[ch & 1];
+                    const int cb = c0 + kW * ch;   // first query column of the chunk
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const float4 l4 = lse4[4 * ch + c4];
-                        const float4 d4 = dv4[4 * ch + c4];
+                    for (int c4 = 0; c4 < kW / 4; ++c4) {
+                        const float4 l4 = lse4[cb / 4 + c4];
+                        const float4 d4 = dv4[cb / 4 + c4];
                         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                         const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int cc = 4 * c4 + e;
                             float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e] * kLog2e));
-                            if (first > 16 * ch) pr = 16 * ch + cc >= first ? pr : 0.f;
+                            if (first > cb) pr = cb + cc >= first ? pr : 0.f;
                             s_[cc] = pr;
                             d_[cc] = pr * (d_[cc] - dd[e]);
                         }
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        pp[8 * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
-                        pd[8 * ch + e] = pack_bf16x2(d_[2 * e], d_[2 * e + 1]);
+                    for (int e = 0; e < kW / 2; ++e) {
+                        pp[(kW / 2) * ch + e] = pack_bf16x2(s_[2 * e], s_[2 * e + 1]);
+                        pd[(kW / 2) * ch + e] = pack_bf16x2(d_[2 * e], d_[2 * e + 1]);
                     }
                 }
             }
-            // P^T over the first 32 columns of S^T[grp], dS^T over those of dP^T[grp]
-            tmem_st32u(tlane + grp * 128, pp);
-            tmem_st32u(tlane + grp * 128 + 64, pd);
+            // this thread's P^T and dS^T, packed, over the first kCols / 2 of its
+            // own S^T and dP^T columns (all read above)
+            tmem_stn<kCols / 2>(tlane + grp * 128 + c0, pp);
+            tmem_stn<kCols / 2>(tlane + grp * 128 + 64 + c0, pd);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[grp]);
@@ -644,14 +672,18 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     const bool first_prod = C::kSplit ? n < C::G : n < 1;
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const int h_ = (16 * kk) / kCols;   // the half holding queries 16 kk ..
+                        const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
                         const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
-                        umma_bf16_ts(tmem + C::dv_col(grp), tmem + grp * 128 + kk * 8, bdo, idesc_acc,
+                        umma_bf16_ts(tmem + C::dv_col(grp), tmem + grp * 128 + acol, bdo, idesc_acc,
                                      (!first_prod || kk > 0) ? 1u : 0u);
                     }
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const int h_ = (16 * kk) / kCols;
+                        const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
                         const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
-                        umma_bf16_ts(tmem + C::dk_col(grp), tmem + grp * 128 + 64 + kk * 8, bq, idesc_acc,
+                        umma_bf16_ts(tmem + C::dk_col(grp), tmem + grp * 128 + 64 + acol, bq, idesc_acc,
                                      (!first_prod || kk > 0) ? 1u : 0u);
                     }
                     if (!C::kSplit) umma_commit(&acc[grp]);
@@ -674,7 +706,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             tc_fence_after();
             const bool has1 = C::G == 2 && C::kSplit && T >= 2;   // the group-1 accumulators hold products
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + uu;
-            constexpr int kOc = D / C::G;
+            constexpr int kOc = D / (C::G * H);   // output columns per thread (split among a row's threads)
+            const int slot = grp * H + hc;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
@@ -682,7 +715,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const uint32_t col0 = which == 0 ? C::dv_col(0) : C::dk_col(0);
                 const uint32_t col1 = which == 0 ? C::dv_col(1) : C::dk_col(1);
 #pragma unroll
-                for (int cb = grp * kOc; cb < (grp + 1) * kOc; cb += 32) {
+                for (int cb = slot * kOc; cb < (slot + 1) * kOc; cb += 32) {
                     float ov[32];
                     tmem_ld32(tlane + col0 + cb, ov);
                     tmem_wait_ld();
