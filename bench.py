@@ -220,6 +220,57 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ ours
 
+# The kernels behind each timed call, and the sources whose hash ties a
+# recorded traffic figure to the code that produced it.
+_TRAFFIC_CALLS = {
+    "gsa_attn_fwd": (["attn_fwd_bf16_kernel<64>"],
+                     ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh"]),
+    "gsa_attn_bwd": (["dot_kernel<64>", "dq_kernel<64>", "dkdv_kernel<64>"],
+                     ["content_adaptive_block_b200/csrc/attn_bwd_bf16.cuh"]),
+}
+_TRAFFIC_COMMON = ["content_adaptive_block_b200/csrc/common.cuh", "content_adaptive_block_b200/csrc/tiles.cuh",
+                   "content_adaptive_block_b200/csrc/gsa.cu"]
+
+
+def record_traffic(csv_path, capture):
+    """Write profiles/traffic.json from an ncu raw-page CSV export (one
+    launch per kernel): dram read + write bytes per call, summed over the
+    call's kernels, with the hash of the sources they were built from."""
+    import csv
+    import hashlib
+    rows = list(csv.reader(open(csv_path)))
+    hdr, units, data = rows[0], rows[1], rows[2:]
+    col = {h: i for i, h in enumerate(hdr)}
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+
+    def dram(row):
+        tot = 0.0
+        for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            tot += float(row[col[m]].replace(",", "")) * scale[units[col[m]]]
+        return tot
+
+    out = {}
+    for call, (kernels, srcs) in _TRAFFIC_CALLS.items():
+        found = {}
+        for row in data:
+            name = row[col["Kernel Name"]]
+            for k in kernels:
+                if k in name and k not in found:
+                    found[k] = dram(row)
+        if len(found) != len(kernels):
+            continue
+        sources = srcs + _TRAFFIC_COMMON
+        h = hashlib.sha256()
+        for s in sources:
+            with open(os.path.join(ROOT, s), "rb") as fh:
+                h.update(fh.read())
+        out[call] = {"bytes_per_launch": int(sum(found.values())), "per_kernel": {k: int(v) for k, v in found.items()},
+                     "sources": sources, "sha256": h.hexdigest(), "capture": capture}
+    with open(os.path.join(ROOT, "profiles", "traffic.json"), "w") as fh:
+        json.dump(out, fh, indent=1)
+    print(json.dumps(out))
+
+
 def _traffic_record(kernel):
     """dram bytes per launch from a committed ncu capture, if the kernel's
     source is unchanged since (else None)."""
@@ -471,7 +522,13 @@ def main():
     ap.add_argument("--no-mask-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
+                    help="write profiles/traffic.json from an ncu raw-page CSV export and exit")
+    ap.add_argument("--capture", default="", help="the ncu command recorded with --record-traffic")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.capture)
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
