@@ -72,6 +72,17 @@ def mask_sweep(b: int, f: float) -> Workload:
 MASK_SWEEP = [(b, f) for b in (32, 64, 128) for f in (0.05, 0.3, 0.7)]
 
 
+def seq_sweep(L: int) -> Workload:
+    """Sequence-length sweep point: the 8x8K configuration (b=64, w=2, 12
+    heads 6/3/3, d=64, bf16, forward and backward, entropy U[0.2, 0.6]) at
+    length L with the batch shrunk so that S * L = 65536 bytes per step."""
+    return Workload(f"seq_{L // 1024}k", S=max(1, 65536 // L), L=L, b=64, w=2, H=12, d=64, dtype="bf16",
+                    backward=True, entropy=("uniform", 0.2, 0.6), salt=7 + L)
+
+
+SEQ_SWEEP = [4096, 8192, 16384, 32768, 65536]
+
+
 def _rng(seed: int, salt: int, s: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, salt, s])))
 
