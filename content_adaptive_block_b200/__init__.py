@@ -76,6 +76,7 @@ def library():
         lib.gsa_block_lengths.argtypes = [vp, i32, i64, i32, vp, vp]
         lib.gsa_literal_flags.argtypes = [vp, i32, i32, vp, vp]
         lib.gsa_build_block_csr.argtypes = [vp, i32, ctypes.POINTER(_Csr), vp]
+        lib.gsa_mask_pipeline.argtypes = [vp, i32, i64, i32, i32, vp, vp, ctypes.POINTER(_Csr), vp, vp]
         lib.gsa_csr_capacity.argtypes = [i32]
         lib.gsa_csr_capacity.restype = i64
         lib.gsa_attn_fwd.argtypes = [vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc), vp, vp, vp]
@@ -196,6 +197,34 @@ def gsa_build_block_csr(flags: torch.Tensor, w: int, csr: BlockCsr | None = None
                                                                  _stream(stream)))
     csr.w = st.w
     return csr
+
+
+def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None = None,
+                      lengths: torch.Tensor | None = None, flags: torch.Tensor | None = None,
+                      counters: torch.Tensor | None = None, stream=None):
+    """lengths -> flags -> block lists in one launch; returns (lengths, flags, csr).
+    counters (int32 [B], zero, left zero by each call) may be passed to avoid
+    allocating one per call."""
+    _need(data, "data", torch.uint8, 2)
+    B, L = data.shape
+    n = L // b if b > 0 else 0
+    if lengths is None:
+        lengths = torch.empty((B, n), dtype=torch.int32, device=data.device)
+    if flags is None:
+        flags = torch.empty((B, n), dtype=torch.uint8, device=data.device)
+    if csr is None:
+        csr = BlockCsr(B, n, data.device)
+    if counters is None:
+        counters = torch.zeros(B, dtype=torch.int32, device=data.device)
+    _need(lengths, "lengths", torch.int32)
+    _need(flags, "flags", torch.uint8)
+    _need(counters, "counters", torch.int32)
+    st = csr.struct()
+    _check("gsa_mask_pipeline", library().gsa_mask_pipeline(_ptr(data), B, L, int(b), int(w), _ptr(lengths),
+                                                             _ptr(flags), ctypes.byref(st), _ptr(counters),
+                                                             _stream(stream)))
+    csr.w = st.w
+    return lengths, flags, csr
 
 
 # ------------------------------------------------------------------ attention

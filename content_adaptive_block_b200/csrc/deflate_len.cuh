@@ -413,17 +413,9 @@ __device__ __forceinline__ int warp_sum(int v) {
 
 // ------------------------------------------------ the kernel
 
-__global__ void __launch_bounds__(32 * kWarps)
-block_lengths_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_t nblocks_total,
-                     int32_t* __restrict__ lengths) {
-    extern __shared__ __align__(16) uint8_t dsmem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpSmem& ws = reinterpret_cast<WarpSmem*>(dsmem)[warp];
-    const int64_t task = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-    if (task >= nblocks_total) return;   // warp-uniform
-    const int64_t nblk = L / b;
-    const int64_t s = task / nblk, i = task % nblk;
-    const uint8_t* src = bytes + s * L + i * b;
+// gzip length (18 + raw DEFLATE bytes) of the b bytes at src; the whole
+// warp calls it, the result is valid on every lane.
+__device__ int block_length_warp(WarpSmem& ws, const uint8_t* __restrict__ src, int b, int lane) {
     for (int k = lane; k < b + 16; k += 32) ws.x[k] = k < b ? src[k] : 0;
     __syncwarp();
 
@@ -472,13 +464,25 @@ block_lengths_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_
     if (hclen < 4) hclen = 4;
     dyn += blbits + 5 + 5 + 4 + 3 * hclen;
 
-    if (lane == 0) {
-        int opt = (dyn + 3 + 7) >> 3;
-        const int stat = (fix + 3 + 7) >> 3;
-        if (stat <= opt) opt = stat;
-        const int raw = (n + 4 <= opt) ? n + 5 : opt;
-        lengths[task] = raw + 18;
-    }
+    int opt = (dyn + 3 + 7) >> 3;
+    const int stat = (fix + 3 + 7) >> 3;
+    if (stat <= opt) opt = stat;
+    const int raw = (n + 4 <= opt) ? n + 5 : opt;
+    return raw + 18;
+}
+
+__global__ void __launch_bounds__(32 * kWarps)
+block_lengths_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_t nblocks_total,
+                     int32_t* __restrict__ lengths) {
+    extern __shared__ __align__(16) uint8_t dsmem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WarpSmem& ws = reinterpret_cast<WarpSmem*>(dsmem)[warp];
+    const int64_t task = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    if (task >= nblocks_total) return;   // warp-uniform
+    const int64_t nblk = L / b;
+    const int64_t s = task / nblk, i = task % nblk;
+    const int len = block_length_warp(ws, bytes + s * L + i * b, b, lane);
+    if (lane == 0) lengths[task] = len;
 }
 
 constexpr size_t kSmemBytes = sizeof(WarpSmem) * kWarps;

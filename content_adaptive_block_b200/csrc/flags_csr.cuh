@@ -88,8 +88,10 @@ struct CsrArgs {
 __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
 __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
 
-__global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
-    extern __shared__ __align__(16) uint8_t dsm[];
+// Lists of class c for sample s, by the whole CTA (any multiple of 32
+// threads up to 1024); dsm holds csr_smem_bytes(nblk).  Reads the flags from
+// a.flags, so a CTA that wrote them must synchronise first.
+__device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm) {
     const int n = a.nblk;
     uint8_t* fl = dsm;                                              // [n]
     int* pre = reinterpret_cast<int*>(dsm + ((n + 15) & ~15));      // [n] inclusive literal count
@@ -98,8 +100,6 @@ __global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
     int* cptr = rptr + n + 1;                                       // [n + 1]
     int* scratch = cptr + n + 1;                                    // [64]
 
-    const int c = blockIdx.x;       // head class
-    const int s = blockIdx.y;       // sample
     const int64_t g = static_cast<int64_t>(s) * 3 + c;
     const int w = a.w;
     for (int i = threadIdx.x; i < n; i += blockDim.x) fl[i] = a.flags[static_cast<int64_t>(s) * n + i] ? 1 : 0;
@@ -199,6 +199,11 @@ __global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
             ridx[cptr[i] + e] = q;
         }
     }
+}
+
+__global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    build_csr_sample(a, blockIdx.x, blockIdx.y, dsm);   // grid (class, sample)
 }
 
 inline size_t csr_smem_bytes(int n) {

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "deflate_len.cuh"
 #include "flags_csr.cuh"
+#include "mask_pipeline.cuh"
 #include "attn_fwd_f32.cuh"
 #include "attn_fwd_bf16.cuh"
 #include "attn_bwd_bf16.cuh"
@@ -142,6 +143,43 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* c
     });
     dim3 grid(3, csr->B);
     gsa::mask::build_csr_kernel<<<grid, gsa::mask::kThreads, smem, as_stream(stream)>>>(a);
+    return launch_status();
+}
+
+gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w, int32_t* lengths,
+                             uint8_t* flags, gsa_block_csr* csr, int32_t* counters, void* stream) {
+    if (!bytes || !lengths || !flags || !csr || !counters || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES ||
+        L < b || L % b != 0 || w < 0)
+        return GSA_ERR_INVALID_ARGUMENT;
+    const int64_t nblk = L / b;
+    if (csr->B != B || csr->nblk != nblk || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
+        !csr->q_order || !csr->k_order)
+        return GSA_ERR_INVALID_ARGUMENT;
+    if (nblk > GSA_MAX_PIPELINE_BLOCKS) return GSA_ERR_UNSUPPORTED;
+    if (csr->capacity < gsa_csr_capacity(static_cast<int32_t>(nblk))) return GSA_ERR_CAPACITY;
+    using namespace gsa::deflate;
+    const int64_t total = static_cast<int64_t>(B) * nblk;
+    const int64_t grid = (total + kWarps - 1) / kWarps;
+    if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
+    csr->w = w;
+    gsa::mask::CsrArgs a;
+    a.flags = flags;
+    a.nblk = static_cast<int>(nblk);
+    a.w = w;
+    a.cap = csr->capacity;
+    a.row_ptr = csr->row_ptr;
+    a.col_idx = csr->col_idx;
+    a.col_ptr = csr->col_ptr;
+    a.row_idx = csr->row_idx;
+    a.q_order = csr->q_order;
+    a.k_order = csr->k_order;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(gsa::pipeline::mask_pipeline_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    });
+    gsa::pipeline::mask_pipeline_kernel<<<static_cast<unsigned>(grid), 32 * kWarps, kSmemBytes, as_stream(stream)>>>(
+        bytes, L, b, total, lengths, flags, a, counters);
     return launch_status();
 }
 

@@ -146,6 +146,31 @@ int64_t gsa_csr_capacity(int32_t nblk);
 gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* csr, void* stream);
 
 /*
+ * gsa_mask_pipeline — gsa_block_lengths, gsa_literal_flags and
+ * gsa_build_block_csr in one launch, with the same outputs bit for bit.
+ *
+ * The flowchart of the pages (gzip level-1 per block -> r_i > r̄ -> mask per
+ * head class) as one pass: the CTA that finishes the last block of a sample
+ * computes that sample's flags and lists.  No CTA waits for another.
+ *
+ *   bytes, B, L, b   as for gsa_block_lengths; L / b = nblk <= GSA_MAX_PIPELINE_BLOCKS
+ *   w                local window in blocks, >= 0
+ *   lengths          [B][nblk] int32 out
+ *   flags            [B][nblk] uint8 out
+ *   csr              as for gsa_build_block_csr (csr->B == B, csr->nblk == nblk)
+ *   counters         [B] int32 device scratch owned by the caller: zero before
+ *                    the first call; every completed call leaves it zero.
+ *                    Two calls in flight at once must not share it.
+ * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, bad sizes, csr shape),
+ *         GSA_ERR_UNSUPPORTED (nblk > GSA_MAX_PIPELINE_BLOCKS: use the three
+ *         calls), GSA_ERR_CAPACITY (capacity < gsa_csr_capacity(nblk)).
+ */
+#define GSA_MAX_PIPELINE_BLOCKS 1024
+gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w,
+                             int32_t* lengths, uint8_t* flags, gsa_block_csr* csr, int32_t* counters,
+                             void* stream);
+
+/*
  * Attention problem description (host struct).
  *   q, k, v, o, dq, dk, dv: [B][H][L][d] contiguous, element type dtype.
  *   lse: [B][H][L] float32, natural log of the softmax denominator,

@@ -92,6 +92,25 @@ def test_build_csr_rejects_bad_arguments(lib):
     assert f(FAKE, 1, ctypes.byref(nul), NULL) == 1
 
 
+def test_mask_pipeline_rejects_bad_arguments(lib):
+    f = lib.gsa_mask_pipeline
+    c = _csr(B=2, n=8)
+    # bytes, B, L, b, w, lengths, flags, csr, counters, stream; 2 samples x 512 bytes, b=64 -> 8 blocks
+    args = [FAKE, 2, 512, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL]
+    for i in (0, 5, 6, 8):                                   # null device pointers
+        bad = list(args)
+        bad[i] = NULL
+        assert f(*bad) == 1, i
+    assert f(FAKE, 2, 512, 64, -1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1   # negative window
+    assert f(FAKE, 2, 500, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1    # L % b
+    assert f(FAKE, 3, 512, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1    # csr->B != B
+    assert f(FAKE, 2, 1024, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1   # csr->nblk != L / b
+    big = _csr(B=1, n=2048)
+    assert f(FAKE, 1, 2048 * 16, 16, 1, FAKE, FAKE, ctypes.byref(big), FAKE, NULL) == 2   # beyond one launch
+    small = _csr(B=2, n=8, cap=10)
+    assert f(FAKE, 2, 512, 64, 1, FAKE, FAKE, ctypes.byref(small), FAKE, NULL) == 3      # capacity
+
+
 def _desc(B=1, H=4, L=256, d=64, b=64, dtype=1, classes=(0, 0, 1, 2), scale=0.0):
     hc = (ctypes.c_uint8 * len(classes))(*classes)
     return gsa._AttnDesc(B, H, L, d, b, dtype, scale, ctypes.cast(hc, ctypes.c_void_p)), hc
