@@ -39,7 +39,14 @@ namespace deflate {
 
 constexpr int kMaxB = 128;              // largest block handled (bytes)
 constexpr int kWords = kMaxB / 32;      // position bitmask words
-constexpr int kWarps = 4;               // warps (blocks) per CTA
+constexpr int kWarps = 4;               // warps (blocks) per CTA of the one-launch mask stage
+// Warps (blocks) per CTA of the lengths kernel: a CTA's shared memory stays
+// held until its slowest block is done, and block costs vary widely (stored,
+// fixed or dynamic blocks), so small CTAs keep more blocks in flight.
+#ifndef GSA_LEN_WARPS
+#define GSA_LEN_WARPS 1
+#endif
+constexpr int kLenWarps = GSA_LEN_WARPS;
 constexpr int kLitLeaves = kMaxB + 4;   // distinct literal/length symbols + end of block + dummies
 constexpr int kDistLeaves = 32;
 
@@ -471,13 +478,13 @@ __device__ int block_length_warp(WarpSmem& ws, const uint8_t* __restrict__ src, 
     return raw + 18;
 }
 
-__global__ void __launch_bounds__(32 * kWarps)
+__global__ void __launch_bounds__(32 * kLenWarps)
 block_lengths_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_t nblocks_total,
                      int32_t* __restrict__ lengths) {
     extern __shared__ __align__(16) uint8_t dsmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpSmem& ws = reinterpret_cast<WarpSmem*>(dsmem)[warp];
-    const int64_t task = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    const int64_t task = static_cast<int64_t>(blockIdx.x) * kLenWarps + warp;
     if (task >= nblocks_total) return;   // warp-uniform
     const int64_t nblk = L / b;
     const int64_t s = task / nblk, i = task % nblk;
@@ -485,7 +492,8 @@ block_lengths_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_
     if (lane == 0) lengths[task] = len;
 }
 
-constexpr size_t kSmemBytes = sizeof(WarpSmem) * kWarps;
+constexpr size_t kSmemBytes = sizeof(WarpSmem) * kWarps;         // one-launch mask stage
+constexpr size_t kLenSmemBytes = sizeof(WarpSmem) * kLenWarps;   // lengths kernel
 
 }  // namespace deflate
 }  // namespace gsa

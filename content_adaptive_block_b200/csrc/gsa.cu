@@ -98,14 +98,14 @@ gsa_status gsa_block_lengths(const uint8_t* bytes, int32_t B, int64_t L, int32_t
         return GSA_ERR_INVALID_ARGUMENT;
     using namespace gsa::deflate;
     const int64_t total = static_cast<int64_t>(B) * (L / b);
-    const int64_t grid = (total + kWarps - 1) / kWarps;
+    const int64_t grid = (total + kLenWarps - 1) / kLenWarps;
     if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
     static std::once_flag once;
     std::call_once(once, [] {
         cudaFuncSetAttribute(block_lengths_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+                             static_cast<int>(kLenSmemBytes));
     });
-    block_lengths_kernel<<<static_cast<unsigned>(grid), 32 * kWarps, kSmemBytes, as_stream(stream)>>>(
+    block_lengths_kernel<<<static_cast<unsigned>(grid), 32 * kLenWarps, kLenSmemBytes, as_stream(stream)>>>(
         bytes, L, b, total, lengths);
     return launch_status();
 }
