@@ -69,6 +69,7 @@ struct Params {
     __nv_bfloat16* out1;    // dk (dkdv_kernel)
     float scale;
     float scale_log2;
+    int* ticket;            // work counter of the persistent dK/dV kernel (zeroed by dot_kernel)
     uint8_t cls[kMaxHeads];
 };
 
@@ -77,7 +78,8 @@ struct Params {
 template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                   const __nv_bfloat16* __restrict__ dO, float* __restrict__ dvec,
-                                                  int64_t rows) {
+                                                  int64_t rows, int* __restrict__ ticket) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;   // for the persistent dK/dV kernel that follows
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
     constexpr int kRowsPerCta = 256 / kTpr;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
@@ -742,7 +744,32 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
 }
 
+}  // namespace bwd
+}  // namespace gsa
+
+#include "attn_bwd_persist.cuh"
+
+namespace gsa {
+namespace bwd {
+
 // ------------------------------------------------------------ launch
+
+#ifndef GSA_DKV_PERSIST
+#define GSA_DKV_PERSIST 1
+#endif
+
+// Streaming multiprocessors of the current device (cached per device).
+inline int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 template <int D>
 gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
@@ -755,10 +782,22 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     });
     constexpr int kRowsPerCta = 256 / (D / 8);
     dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
-        o, dO, const_cast<float*>(pq.dvec), rows);
+        o, dO, const_cast<float*>(pq.dvec), rows, pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
     dq_kernel<D><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
-    dkdv_kernel<D><<<grid, Shape<D>::kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+    if (D == 64 && GSA_DKV_PERSIST) {
+        static std::once_flag once_p;
+        std::call_once(once_p, [] {
+            cudaFuncSetAttribute(dkdv_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DkvPCfg::kSmemBytes);
+        });
+        const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
+        const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
+        dkdv_persist_kernel<<<static_cast<unsigned>(ctas), DkvPCfg::kThreads, DkvPCfg::kSmemBytes, st>>>(
+            tq, tk, tv, tdo, pkv);
+    } else {
+        dkdv_kernel<D><<<grid, Shape<D>::kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+    }
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
 
@@ -782,6 +821,7 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     base.dvec = work;
     base.scale = scale;
     base.scale_log2 = scale * kLog2e;
+    base.ticket = reinterpret_cast<int*>(work + ((rows + 63) & ~int64_t(63)));   // after D, 256-byte aligned
     for (int h = 0; h < desc->H; ++h) base.cls[h] = cls[h];
     Params pq = base, pkv = base;
     pq.ptr = csr->row_ptr;

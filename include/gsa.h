@@ -216,8 +216,11 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
  *   dV = P^T dO,  dS = P ∘ (dO V^T − D),  dQ = scale · dS K,  dK = scale · dS^T Q,
  * every sum over live pairs only.  o and lse are the forward's outputs.
  *   workspace: device scratch of at least gsa_attn_bwd_workspace(desc) bytes
- *              (holds D, float32 [B][H][L]); its contents need no init.
- * dq, dk, dv are written (not accumulated).  Deterministic: no atomics.
+ *              (holds D, float32 [B][H][L], then a work counter); its
+ *              contents need no init.
+ * dq, dk, dv are written (not accumulated).  Deterministic: each output row
+ * is summed by one CTA in a fixed order (the only atomic hands out work
+ * items).
  * Errors: as gsa_attn_fwd, plus GSA_ERR_CAPACITY when ws_bytes is too small.
  * Only GSA_BF16 is implemented.
  */

@@ -143,7 +143,8 @@ def test_attn_bwd_rejects_bad_arguments(lib):
     c = _csr(n=4)
     d, keep = _desc()
     ws = lib.gsa_attn_bwd_workspace(ctypes.byref(d))
-    assert ws == 4 * 1 * 4 * 256
+    rows = 1 * 4 * 256
+    assert ws == 4 * ((rows + 63) // 64 * 64) + 256   # D (float32 per row), then a work counter
     args = [FAKE] * 6
     assert f(*args[:5], NULL, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws, NULL) == 1
     assert f(*args, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws - 4, NULL) == 3
