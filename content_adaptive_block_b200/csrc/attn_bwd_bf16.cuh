@@ -69,7 +69,7 @@ struct Params {
     __nv_bfloat16* out1;    // dk (dkdv_kernel)
     float scale;
     float scale_log2;
-    int* ticket;            // work counter of the persistent dK/dV kernel (zeroed by dot_kernel)
+    int* ticket;            // work counter of the persistent kernel (dot_kernel zeroes both)
     uint8_t cls[kMaxHeads];
 };
 
@@ -79,7 +79,7 @@ template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                   const __nv_bfloat16* __restrict__ dO, float* __restrict__ dvec,
                                                   int64_t rows, int* __restrict__ ticket) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0;   // for the persistent dK/dV kernel that follows
+    if (blockIdx.x == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels that follow
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
     constexpr int kRowsPerCta = 256 / kTpr;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
@@ -748,6 +748,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 }  // namespace gsa
 
 #include "attn_bwd_persist.cuh"
+#include "attn_bwd_dq_persist.cuh"
 
 namespace gsa {
 namespace bwd {
@@ -756,6 +757,9 @@ namespace bwd {
 
 #ifndef GSA_DKV_PERSIST
 #define GSA_DKV_PERSIST 1
+#endif
+#ifndef GSA_DQ_PERSIST
+#define GSA_DQ_PERSIST 1
 #endif
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -784,7 +788,18 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
         o, dO, const_cast<float*>(pq.dvec), rows, pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
-    dq_kernel<D><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+    if (D == 64 && GSA_DQ_PERSIST) {
+        static std::once_flag once_q;
+        std::call_once(once_q, [] {
+            cudaFuncSetAttribute(dq_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqPCfg::kSmemBytes);
+        });
+        const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
+        const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
+        dq_persist_kernel<<<static_cast<unsigned>(ctas), DqPCfg::kThreads, DqPCfg::kSmemBytes, st>>>(tq, tk, tv,
+                                                                                                     tdo, pq);
+    } else {
+        dq_kernel<D><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+    }
     if (D == 64 && GSA_DKV_PERSIST) {
         static std::once_flag once_p;
         std::call_once(once_p, [] {
@@ -824,6 +839,7 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     base.ticket = reinterpret_cast<int*>(work + ((rows + 63) & ~int64_t(63)));   // after D, 256-byte aligned
     for (int h = 0; h < desc->H; ++h) base.cls[h] = cls[h];
     Params pq = base, pkv = base;
+    pq.ticket = base.ticket + 1;
     pq.ptr = csr->row_ptr;
     pq.idx = csr->col_idx;
     pq.order = csr->q_order;

@@ -113,6 +113,10 @@ gsa_status gsa_literal_flags(const int32_t* lengths, int32_t B, int32_t nblk, ui
  *   k_order [B][3][nblk]    key blocks in the order the backward pass pairs
  *                           them into 128-row key tiles.
  * capacity must be >= gsa_csr_capacity(nblk) (the dense causal count).
+ * Every list holds its own block (i in row i, j in column j), as the mask
+ * equation's I term guarantees; the attention backward at d = 64 relies on
+ * it, and a list given to it without its own block ends in a bounded wait
+ * that sets the device error (gsa_device_error: GSA_ERR_TIMEOUT).
  */
 typedef struct {
     int32_t B;
