@@ -71,3 +71,41 @@ def live_token_pairs(mask: np.ndarray, b: int) -> int:
     live off-diagonal block pair, b*(b+1)/2 per diagonal block."""
     diag = int(np.trace(mask))
     return (int(mask.sum()) - diag) * b * b + diag * b * (b + 1) // 2
+
+
+# ------------------------------------------------ fixed comparison masks
+#
+# Fixed block masks the pages compare against: section "核心公式" (the
+# background paragraph) names BigBird and Longformer as the content-blind
+# baselines, and the arXiv abstract reports both at 8K context.  The pages
+# give no definition, so the published patterns are read at block
+# granularity, intersected with the causal mask like the adaptive one:
+#   Longformer: sliding window of w blocks on each side plus g global blocks
+#     (the first g); a global key block is seen by every later query block and
+#     a global query block sees every earlier key block:
+#     M_ij = 1[j <= i] * (1[i - j <= w] or 1[j < g] or 1[i < g]);
+#   BigBird: the Longformer pattern plus r random key blocks per query block,
+#     drawn causally: R_i = {u_ik mod (i + 1) : k < r} from r given uniform
+#     32-bit words u_ik per query block (the random draws are inputs).
+
+LONGFORMER, BIGBIRD = 0, 1
+
+
+def fixed_block_mask(kind: int, n: int, w: int, g: int, rnd=None) -> np.ndarray:
+    """Boolean [n, n] causal block mask of a fixed pattern.
+
+    kind LONGFORMER or BIGBIRD; w window half-width in blocks, g global
+    blocks; rnd uint32 [n, r] random words of one sample (BigBird only)."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    m = ((i - j) <= w) | (j < g) | (i < g)
+    if kind == BIGBIRD:
+        if rnd is None:
+            raise ValueError("BigBird needs the random words")
+        rnd = np.asarray(rnd, dtype=np.uint64).reshape(n, -1)
+        for row in range(n):
+            for u in rnd[row]:
+                m[row, int(u % np.uint64(row + 1))] = True
+    elif kind != LONGFORMER:
+        raise ValueError(f"unknown fixed mask kind {kind}")
+    return m & (j <= i)

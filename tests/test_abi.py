@@ -27,7 +27,8 @@ def _declared():
 
 def test_header_declares_the_path(lib):
     names = _declared()
-    for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd",
+    for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_mask_pipeline",
+               "gsa_build_fixed_csr", "gsa_attn_fwd",
                "gsa_attn_bwd", "gsa_csr_capacity", "gsa_attn_bwd_workspace", "gsa_device_error",
                "gsa_status_string"):
         assert fn in names
@@ -90,6 +91,27 @@ def test_build_csr_rejects_bad_arguments(lib):
     nul = _csr()
     nul.q_order = None
     assert f(FAKE, 1, ctypes.byref(nul), NULL) == 1
+
+
+def test_build_fixed_csr_rejects_bad_arguments(lib):
+    f = lib.gsa_build_fixed_csr
+    c = _csr(B=2, n=8)
+    # kind, w, g, r, rnd, csr, stream
+    assert f(2, 1, 1, 0, NULL, ctypes.byref(c), NULL) == 1            # unknown kind
+    assert f(-1, 1, 1, 0, NULL, ctypes.byref(c), NULL) == 1
+    assert f(0, -1, 1, 0, NULL, ctypes.byref(c), NULL) == 1           # negative window
+    assert f(0, 1, -1, 0, NULL, ctypes.byref(c), NULL) == 1           # negative globals
+    assert f(1, 1, 1, -1, FAKE, ctypes.byref(c), NULL) == 1           # negative random count
+    assert f(1, 1, 1, 3, NULL, ctypes.byref(c), NULL) == 1            # BigBird picks without words
+    assert f(0, 1, 1, 0, NULL, None, NULL) == 1                       # no csr
+    assert f(1, 1, 1, 9, FAKE, ctypes.byref(c), NULL) == 2            # above GSA_MAX_RANDOM_BLOCKS
+    big = _csr(B=1, n=8193)
+    assert f(0, 1, 1, 0, NULL, ctypes.byref(big), NULL) == 2          # above GSA_MAX_FIXED_BLOCKS
+    small = _csr(B=2, n=8, cap=10)
+    assert f(0, 1, 1, 0, NULL, ctypes.byref(small), NULL) == 3        # capacity
+    nul = _csr(B=2, n=8)
+    nul.row_idx = None
+    assert f(0, 1, 1, 0, NULL, ctypes.byref(nul), NULL) == 1
 
 
 def test_mask_pipeline_rejects_bad_arguments(lib):

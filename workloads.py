@@ -83,6 +83,23 @@ def seq_sweep(L: int) -> Workload:
 SEQ_SWEEP = [4096, 8192, 16384, 32768, 65536]
 
 
+# Fixed comparison masks at block 64 (the 8x8K shape: 128 blocks per sample),
+# with the published defaults of each pattern read at block granularity:
+# BigBird — a 3-block sliding window (w = 1), 2 global blocks, 3 random
+# blocks per query block; Longformer — a 512-token window (256 tokens, w = 4
+# blocks, each side) and one global block.
+FIXED_MASKS = {
+    "bigbird": dict(kind=1, w=1, g=2, r=3),
+    "longformer": dict(kind=0, w=4, g=1, r=0),
+}
+
+
+def random_words(S: int, n: int, r: int, seed: int = 0) -> np.ndarray:
+    """uint32 [S, n, r] uniform words: the random draws of BigBird's picks."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 0xB16B, S, n, r])))
+    return rng.integers(0, 2**32, size=(S, n, r), dtype=np.uint64).astype(np.uint32)
+
+
 def _rng(seed: int, salt: int, s: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, salt, s])))
 
