@@ -383,11 +383,12 @@ def run_ours(args, rank, world, local_rank):
     # ---- mask-stage sweep (secondary metric), rank 0
     mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
     sweep = seq_sweep(gsa, dev) if (rank == 0 and not args.no_seq_sweep) else None
+    variants = mask_variants(gsa, dev) if (rank == 0 and not args.no_mask_variants) else None
 
     if rank != 0:
         return 0
     return report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops,
-                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep)
+                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep, variants)
 
 
 def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_flops):
@@ -478,7 +479,7 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
 
 
 def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops, pairs,
-           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None):
+           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None, variants=None):
     call_ms = {n: float(per_call[:, j].mean()) for j, n in enumerate(names)}
     bwd_ms, fwd_ms = call_ms["gsa_attn_bwd"], call_ms["gsa_attn_fwd"]
     peak_t = peaks["bf16_tflops_sustained"]
@@ -509,6 +510,8 @@ def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flop
         line["mask_stage"] = mask
     if sweep:
         line["seq_sweep"] = sweep
+    if variants:
+        line["mask_variants"] = variants
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line))
@@ -640,6 +643,72 @@ def seq_sweep(gsa, dev, steps=10, warmup=3):
     return out
 
 
+def mask_variants(gsa, dev, steps=10, warmup=3):
+    """The attention (forward + backward) on the 8x8K configuration's inputs
+    under the adaptive gzip mask and under the fixed BigBird and Longformer
+    block masks built by gsa_build_fixed_csr: per mask its list-building
+    time, live fraction and fwd+bwd time and algorithmic TFLOP/s, L2 flushed
+    between steps, CUDA events per step."""
+    import torch
+    wl = W.WORKLOADS["b8_8k"]
+    hc = [int(c) for c in wl.head_classes()]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    x = torch.from_numpy(W.batch_bytes(wl, seed=0)).to(dev)
+    q, k, v, do = W.qkv(wl, seed=0, device=dev, grad=True)
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.S, wl.H, wl.L), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(gsa.gsa_attn_bwd_workspace(q, wl.b, hc), dtype=torch.uint8, device=dev)
+    out = {"metric": "live-block attn TFLOP/s fwd+bwd", "unit": "TFLOP/s",
+           "shape": "8 x 8192 bytes, b=64, 12 heads, d=64, bf16", "masks": {}}
+    lengths = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
+    flags = torch.empty((wl.S, wl.N), dtype=torch.uint8, device=dev)
+    variants = [("gzip", None)] + [(name, cfg) for name, cfg in W.FIXED_MASKS.items()]
+    for name, cfg in variants:
+        csr = gsa.BlockCsr(wl.S, wl.N, dev)
+        if cfg is None:
+            build = (lambda csr=csr: (gsa.gsa_block_lengths(x, wl.b, out=lengths),
+                                      gsa.gsa_literal_flags(lengths, out=flags),
+                                      gsa.gsa_build_block_csr(flags, wl.w, csr)))
+        else:
+            rnd = None
+            if cfg["r"] > 0:
+                rnd = torch.from_numpy(W.random_words(wl.S, wl.N, cfg["r"], seed=0).view(np.int32)).to(dev)
+            build = (lambda cfg=cfg, rnd=rnd, csr=csr:
+                     gsa.gsa_build_fixed_csr(cfg["kind"], wl.S, wl.N, cfg["w"], cfg["g"], rnd, device=dev, csr=csr))
+
+        def one(ev=None):
+            if ev:
+                ev[0].record()
+            build()
+            if ev:
+                ev[1].record()
+            gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse)
+            gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b, dq=dq, dk=dk, dv=dv, workspace=ws)
+            if ev:
+                ev[2].record()
+
+        for _ in range(warmup):
+            flush.zero_()
+            one()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            one(evs[i])
+        torch.cuda.synchronize()
+        assert gsa.gsa_device_error() == 0, "a kernel gave up a bounded wait"
+        t = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(2)] for i in range(steps)]).mean(axis=0)
+        nnz = csr.row_ptr[:, :, -1].cpu().numpy()
+        pairs = sum(live_token_pairs_from_counts(nnz[s], wl.N, wl.b, hc) for s in range(wl.S))
+        flops = 12 * wl.d * pairs
+        out["masks"][name] = {
+            "params": None if cfg is None else {kk: cfg[kk] for kk in ("w", "g", "r")},
+            "build_ms": float(t[0]), "attn_ms": float(t[1]), "attn_tflops": flops / (t[1] * 1e-3) / 1e12,
+            "live_fraction": pairs / (wl.S * wl.H * wl.L * (wl.L + 1) // 2)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,6 +718,8 @@ def main():
     ap.add_argument("--no-mask-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-seq-sweep", action="store_true", help="skip the 4K..64K sequence-length sweep")
+    ap.add_argument("--no-mask-variants", action="store_true",
+                    help="skip the gzip / BigBird / Longformer mask comparison")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw-page CSV export and exit")

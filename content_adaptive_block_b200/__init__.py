@@ -77,6 +77,7 @@ def library():
         lib.gsa_literal_flags.argtypes = [vp, i32, i32, vp, vp]
         lib.gsa_build_block_csr.argtypes = [vp, i32, ctypes.POINTER(_Csr), vp]
         lib.gsa_mask_pipeline.argtypes = [vp, i32, i64, i32, i32, vp, vp, ctypes.POINTER(_Csr), vp, vp]
+        lib.gsa_build_fixed_csr.argtypes = [i32, i32, i32, i32, vp, ctypes.POINTER(_Csr), vp]
         lib.gsa_csr_capacity.argtypes = [i32]
         lib.gsa_csr_capacity.restype = i64
         lib.gsa_attn_fwd.argtypes = [vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc), vp, vp, vp]
@@ -87,8 +88,8 @@ def library():
         lib.gsa_device_error.argtypes = [ctypes.POINTER(i32), i32]
         lib.gsa_status_string.argtypes = [ctypes.c_int]
         lib.gsa_status_string.restype = ctypes.c_char_p
-        for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd",
-                   "gsa_attn_bwd", "gsa_device_error"):
+        for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_mask_pipeline",
+                   "gsa_build_fixed_csr", "gsa_attn_fwd", "gsa_attn_bwd", "gsa_device_error"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -195,6 +196,31 @@ def gsa_build_block_csr(flags: torch.Tensor, w: int, csr: BlockCsr | None = None
     st = csr.struct()
     _check("gsa_build_block_csr", library().gsa_build_block_csr(_ptr(flags), int(w), ctypes.byref(st),
                                                                  _stream(stream)))
+    csr.w = st.w
+    return csr
+
+
+GSA_FIXED_LONGFORMER, GSA_FIXED_BIGBIRD = 0, 1
+
+
+def gsa_build_fixed_csr(kind: int, B: int, nblk: int, w: int, g: int, rnd: torch.Tensor | None = None,
+                        device=None, csr: BlockCsr | None = None, stream=None) -> BlockCsr:
+    """Block lists of a fixed comparison mask (GSA_FIXED_LONGFORMER: window w
+    and g global blocks; GSA_FIXED_BIGBIRD: plus random key blocks from the
+    uint32 words rnd [B, nblk, r]), the same in all three class slots."""
+    r = 0
+    if rnd is not None:
+        _need(rnd, "rnd", torch.int32 if rnd.dtype == torch.int32 else torch.uint32, 3)
+        if tuple(rnd.shape[:2]) != (B, nblk):
+            raise ValueError("rnd must be [B, nblk, r]")
+        r = int(rnd.shape[2])
+        device = rnd.device if device is None else device
+    if csr is None:
+        csr = BlockCsr(B, nblk, device)
+    st = csr.struct()
+    _check("gsa_build_fixed_csr", library().gsa_build_fixed_csr(int(kind), int(w), int(g), r,
+                                                                 _ptr(rnd) if rnd is not None else None,
+                                                                 ctypes.byref(st), _stream(stream)))
     csr.w = st.w
     return csr
 

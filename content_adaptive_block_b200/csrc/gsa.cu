@@ -15,6 +15,10 @@
 #include "deflate_len.cuh"
 #include "flags_csr.cuh"
 #include "mask_pipeline.cuh"
+#include "fixed_csr.cuh"
+
+static_assert(GSA_MAX_FIXED_BLOCKS == gsa::fixed::kMaxBlocks, "header and kernel agree");
+static_assert(GSA_MAX_RANDOM_BLOCKS == gsa::fixed::kMaxRandom, "header and kernel agree");
 #include "attn_fwd_f32.cuh"
 #include "attn_fwd_bf16.cuh"
 #include "attn_bwd_bf16.cuh"
@@ -143,6 +147,43 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* c
     });
     dim3 grid(3, csr->B);
     gsa::mask::build_csr_kernel<<<grid, gsa::mask::kThreads, smem, as_stream(stream)>>>(a);
+    return launch_status();
+}
+
+gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, const uint32_t* rnd,
+                               gsa_block_csr* csr, void* stream) {
+    if (!csr || (kind != GSA_FIXED_LONGFORMER && kind != GSA_FIXED_BIGBIRD) || w < 0 || g < 0 || r < 0)
+        return GSA_ERR_INVALID_ARGUMENT;
+    if (kind == GSA_FIXED_LONGFORMER) r = 0;
+    if (r > 0 && !rnd) return GSA_ERR_INVALID_ARGUMENT;
+    if (csr->B < 1 || csr->nblk < 1 || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
+        !csr->q_order || !csr->k_order)
+        return GSA_ERR_INVALID_ARGUMENT;
+    if (csr->nblk > gsa::fixed::kMaxBlocks || r > gsa::fixed::kMaxRandom) return GSA_ERR_UNSUPPORTED;
+    if (csr->capacity < gsa_csr_capacity(csr->nblk)) return GSA_ERR_CAPACITY;
+    csr->w = w;
+    gsa::fixed::FixedArgs a;
+    a.kind = kind;
+    a.nblk = csr->nblk;
+    a.w = w;
+    a.g = g;
+    a.r = r;
+    a.rnd = rnd;
+    a.cap = csr->capacity;
+    a.row_ptr = csr->row_ptr;
+    a.col_idx = csr->col_idx;
+    a.col_ptr = csr->col_ptr;
+    a.row_idx = csr->row_idx;
+    a.q_order = csr->q_order;
+    a.k_order = csr->k_order;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(gsa::fixed::build_fixed_csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gsa::fixed::smem_bytes(gsa::fixed::kMaxBlocks, gsa::fixed::kMaxRandom)));
+    });
+    dim3 grid(3, csr->B);
+    gsa::fixed::build_fixed_csr_kernel<<<grid, gsa::fixed::kThreads, gsa::fixed::smem_bytes(csr->nblk, r),
+                                         as_stream(stream)>>>(a);
     return launch_status();
 }
 

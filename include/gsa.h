@@ -132,6 +132,33 @@ typedef struct {
     int32_t* k_order;
 } gsa_block_csr;
 
+/*
+ * gsa_build_fixed_csr — the same lists for a fixed, content-blind block mask,
+ * so that the attention calls run the masks the method is compared with.
+ * Background paragraph of section "核心公式" and the arXiv abstract name
+ * BigBird and Longformer as those baselines; the pages do not define them,
+ * so their published patterns are taken at block granularity, causal:
+ *   GSA_FIXED_LONGFORMER: live(i, j) = j <= i and (i - j <= w or j < g or i < g)
+ *     (a sliding window of w blocks each side, the first g blocks global);
+ *   GSA_FIXED_BIGBIRD: the same, or j = u_ik mod (i + 1) for some k < r
+ *     (r random key blocks per query block, drawn causally).
+ *   rnd  device uint32 [csr->B][csr->nblk][r]: the random words u_ik (the
+ *        caller draws them); BigBird with r > 0 only, else ignored (may be NULL).
+ * All three class slots of each sample receive the same lists, so every
+ * head, whatever its class, attends with the fixed mask.  Lists ascend;
+ * q_order is nblk-1 .. 0 (heaviest query blocks first), k_order 0 .. nblk-1.
+ * Errors: GSA_ERR_INVALID_ARGUMENT (unknown kind, w, g or r < 0, null
+ * pointers), GSA_ERR_UNSUPPORTED (nblk > GSA_MAX_FIXED_BLOCKS or
+ * r > GSA_MAX_RANDOM_BLOCKS), GSA_ERR_CAPACITY (capacity <
+ * gsa_csr_capacity(nblk)).
+ */
+#define GSA_FIXED_LONGFORMER 0
+#define GSA_FIXED_BIGBIRD 1
+#define GSA_MAX_FIXED_BLOCKS 8192
+#define GSA_MAX_RANDOM_BLOCKS 8
+gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, const uint32_t* rnd,
+                               gsa_block_csr* csr, void* stream);
+
 /* Worst-case live pairs of one (sample, class): nblk*(nblk+1)/2. */
 int64_t gsa_csr_capacity(int32_t nblk);
 
