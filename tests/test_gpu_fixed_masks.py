@@ -89,7 +89,7 @@ def test_attention_on_fixed_masks(gsa, name):
     n = wl.N
     csr, rnd = _build(gsa, cfg["kind"], wl.S, n, cfg["w"], cfg["g"], cfg["r"], seed=11)
     hc = [int(c) for c in wl.head_classes()]
-    q, k, v, do = W.qkv(wl, seed=3, device="cuda")
+    q, k, v, do = W.qkv(wl, seed=3, device="cuda", grad=True)
     o, lse = gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b)
     dq, dk, dv = gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b)
     torch.cuda.synchronize()
