@@ -225,8 +225,10 @@ def run_reference(args, rank, world):
 _TRAFFIC_CALLS = {
     "gsa_attn_fwd": (["attn_fwd_bf16_kernel<64>"],
                      ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh"]),
-    "gsa_attn_bwd": (["dot_kernel<64>", "dq_kernel<64>", "dkdv_kernel<64>"],
-                     ["content_adaptive_block_b200/csrc/attn_bwd_bf16.cuh"]),
+    "gsa_attn_bwd": (["dot_kernel<64>", "dq_persist_kernel", "dkdv_persist_kernel"],
+                     ["content_adaptive_block_b200/csrc/attn_bwd_bf16.cuh",
+                      "content_adaptive_block_b200/csrc/attn_bwd_persist.cuh",
+                      "content_adaptive_block_b200/csrc/attn_bwd_dq_persist.cuh"]),
 }
 _TRAFFIC_COMMON = ["content_adaptive_block_b200/csrc/common.cuh", "content_adaptive_block_b200/csrc/tiles.cuh",
                    "content_adaptive_block_b200/csrc/gsa.cu"]
