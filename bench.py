@@ -386,11 +386,12 @@ def run_ours(args, rank, world, local_rank):
     mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
     sweep = seq_sweep(gsa, dev) if (rank == 0 and not args.no_seq_sweep) else None
     variants = mask_variants(gsa, dev) if (rank == 0 and not args.no_mask_variants) else None
+    block = lm_block(gsa, dev) if (rank == 0 and not args.no_lm_block) else None
 
     if rank != 0:
         return 0
     return report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops,
-                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep, variants)
+                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep, variants, block)
 
 
 def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_flops):
@@ -481,7 +482,7 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
 
 
 def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops, pairs,
-           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None, variants=None):
+           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None, variants=None, block=None):
     call_ms = {n: float(per_call[:, j].mean()) for j, n in enumerate(names)}
     bwd_ms, fwd_ms = call_ms["gsa_attn_bwd"], call_ms["gsa_attn_fwd"]
     peak_t = peaks["bf16_tflops_sustained"]
@@ -514,6 +515,8 @@ def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flop
         line["seq_sweep"] = sweep
     if variants:
         line["mask_variants"] = variants
+    if block:
+        line["lm_block"] = block
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line))
@@ -711,6 +714,68 @@ def mask_variants(gsa, dev, steps=10, warmup=3):
     return out
 
 
+def lm_block(gsa, dev, steps=10, warmup=3):
+    """One ByteLM block (D = 768, 12 heads, MLP 3072) forward + backward on
+    the 8x8K bench batch under its gzip mask: per step the mask pipeline, the
+    block forward and the block backward, L2 flushed between steps, CUDA
+    events.  FLOPs: the projections' 2 T D (3D + D + 2F) forward and twice
+    that backward, plus the attention's algorithmic 12 d P."""
+    import torch
+    wl = W.WORKLOADS["b8_8k"]
+    c = W.LM_BLOCK
+    D, H, F = c["D"], c["H"], c["F"]
+    hc = [int(v) for v in wl.head_classes()]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    x = torch.from_numpy(W.batch_bytes(wl, seed=0)).to(dev)
+    wt = W.lm_weights(D, F, seed=0, device=dev)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(77)
+    dy = torch.randn((wl.S, wl.L, D), generator=g).bfloat16().to(dev)
+    lengths = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
+    flags = torch.empty((wl.S, wl.N), dtype=torch.uint8, device=dev)
+    counters = torch.zeros(wl.S, dtype=torch.int32, device=dev)
+    csr = gsa.BlockCsr(wl.S, wl.N, dev)
+    y = torch.empty((wl.S, wl.L, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(gsa.gsa_lm_block_workspace(wl.S, wl.L, D, H, F, hc), dtype=torch.uint8, device=dev)
+    grads = {n: torch.empty(wt[n].shape, dtype=torch.float32, device=dev) for n in gsa.LM_WEIGHTS}
+
+    def one(ev=None):
+        if ev:
+            ev[0].record()
+        gsa.gsa_mask_pipeline(x, wl.b, wl.w, csr=csr, lengths=lengths, flags=flags, counters=counters)
+        if ev:
+            ev[1].record()
+        gsa.gsa_lm_block_fwd(x, wt, csr, hc, y=y, workspace=ws)
+        if ev:
+            ev[2].record()
+        gsa.gsa_lm_block_bwd(x, wt, csr, hc, dy, ws, grads=grads)
+        if ev:
+            ev[3].record()
+
+    for _ in range(warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        one(evs[i])
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0, "a kernel gave up a bounded wait"
+    t = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(steps)]).mean(axis=0)
+    T = wl.S * wl.L
+    gemm_fwd = 2.0 * T * D * (3 * D + D + 2 * F)
+    nnz = csr.row_ptr[:, :, -1].cpu().numpy()
+    pairs = sum(live_token_pairs_from_counts(nnz[s], wl.N, wl.b, hc) for s in range(wl.S))
+    attn = 12.0 * 64 * pairs
+    ms = float(t.sum())
+    return {"metric": "ByteLM block TFLOP/s fwd+bwd (projections + live-block attention)", "unit": "TFLOP/s",
+            "shape": f"8 x 8192 bytes, D={D}, H={H} x 64, F={F}, gzip mask b=64 w=2, bf16",
+            "ms": ms, "mask_ms": float(t[0]), "fwd_ms": float(t[1]), "bwd_ms": float(t[2]),
+            "tflops": (3 * gemm_fwd + attn) / (ms * 1e-3) / 1e12, "gemm_gflop": 3 * gemm_fwd / 1e9,
+            "attn_gflop": attn / 1e9, "projections": "cuBLASLt (bf16, fp32 accumulate)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -720,6 +785,7 @@ def main():
     ap.add_argument("--no-mask-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-seq-sweep", action="store_true", help="skip the 4K..64K sequence-length sweep")
+    ap.add_argument("--no-lm-block", action="store_true", help="skip the ByteLM block timing")
     ap.add_argument("--no-mask-variants", action="store_true",
                     help="skip the gzip / BigBird / Longformer mask comparison")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")

@@ -342,6 +342,118 @@ def gsa_attn_bwd_noalloc(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: in
     return dq, dk, dv
 
 
+# ------------------------------------------------------------ ByteLM block
+
+LM_WEIGHTS = ("emb", "ln1_g", "ln1_b", "w_qkv", "w_o", "ln2_g", "ln2_b", "w_1", "w_2")
+_LM_F32 = ("ln1_g", "ln1_b", "ln2_g", "ln2_b")
+
+
+class _LmDesc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("L", ctypes.c_int32), ("D", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("F", ctypes.c_int32), ("b", ctypes.c_int32), ("head_classes", ctypes.c_void_p),
+        ("ln_eps", ctypes.c_float),
+    ]
+
+
+class _LmPtrs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LM_WEIGHTS]
+
+
+def _lm_fns():
+    lib = library()
+    vp = ctypes.c_void_p
+    lib.gsa_lm_block_workspace.argtypes = [ctypes.POINTER(_LmDesc)]
+    lib.gsa_lm_block_workspace.restype = ctypes.c_size_t
+    lib.gsa_lm_block_fwd.argtypes = [vp, ctypes.POINTER(_LmPtrs), ctypes.POINTER(_Csr), ctypes.POINTER(_LmDesc),
+                                     vp, vp, ctypes.c_size_t, vp]
+    lib.gsa_lm_block_fwd.restype = ctypes.c_int
+    lib.gsa_lm_block_bwd.argtypes = [vp, ctypes.POINTER(_LmPtrs), ctypes.POINTER(_Csr), ctypes.POINTER(_LmDesc),
+                                     vp, ctypes.POINTER(_LmPtrs), vp, ctypes.c_size_t, vp]
+    lib.gsa_lm_block_bwd.restype = ctypes.c_int
+    return lib
+
+
+def _lm_desc(B, L, D, H, F, head_classes, b, eps):
+    hc = (ctypes.c_uint8 * H)(*[int(c) for c in head_classes])
+    return _LmDesc(B, L, D, H, F, int(b), ctypes.cast(hc, ctypes.c_void_p), float(eps)), hc
+
+
+def _lm_weights(w: dict):
+    """(D, H, F) of a weight dict, checking dtypes and shapes."""
+    D = w["emb"].shape[1]
+    F = w["w_1"].shape[0]
+    shapes = {"emb": (256, D), "w_qkv": (3 * D, D), "w_o": (D, D), "w_1": (F, D), "w_2": (D, F)}
+    for n in LM_WEIGHTS:
+        _need(w[n], n, torch.float32 if n in _LM_F32 else torch.bfloat16)
+        if tuple(w[n].shape) != shapes.get(n, (D,)):
+            raise ValueError(f"{n} must have shape {shapes.get(n, (D,))}")
+    return D, D // 64, F
+
+
+def gsa_lm_block_workspace(B: int, L: int, D: int, H: int, F: int, head_classes, b: int = 64,
+                           eps: float = 1e-5) -> int:
+    desc, keep = _lm_desc(B, L, D, H, F, head_classes, b, eps)
+    return int(_lm_fns().gsa_lm_block_workspace(ctypes.byref(desc)))
+
+
+def gsa_lm_block_fwd(data: torch.Tensor, weights: dict, csr: BlockCsr, head_classes, b: int = 64,
+                     eps: float = 1e-5, y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     stream=None):
+    """One ByteLM block forward over bytes data [B, L] (uint8): returns
+    (y [B, L, D] bf16, workspace).  Pass the returned workspace to
+    gsa_lm_block_bwd."""
+    _need(data, "data", torch.uint8, 2)
+    B, L = data.shape
+    D, H, F = _lm_weights(weights)
+    lib = _lm_fns()
+    desc, keep = _lm_desc(B, L, D, H, F, head_classes, b, eps)
+    need = int(lib.gsa_lm_block_workspace(ctypes.byref(desc)))
+    if need == 0:
+        raise ValueError("invalid ByteLM block shape")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=data.device)
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=data.device)
+    _need(y, "y", torch.bfloat16)
+    _need(workspace, "workspace")
+    wp = _LmPtrs(*[weights[n].data_ptr() for n in LM_WEIGHTS])
+    st = csr.struct()
+    _check("gsa_lm_block_fwd", lib.gsa_lm_block_fwd(_ptr(data), ctypes.byref(wp), ctypes.byref(st),
+                                                    ctypes.byref(desc), _ptr(y), _ptr(workspace),
+                                                    workspace.numel(), _stream(stream)))
+    del keep
+    return y, workspace
+
+
+def gsa_lm_block_bwd(data: torch.Tensor, weights: dict, csr: BlockCsr, head_classes, dy: torch.Tensor,
+                     workspace: torch.Tensor, b: int = 64, eps: float = 1e-5, grads: dict | None = None,
+                     stream=None) -> dict:
+    """Gradients (float32, one per weight) of <y, dy> for the forward that
+    last used this workspace."""
+    _need(data, "data", torch.uint8, 2)
+    B, L = data.shape
+    D, H, F = _lm_weights(weights)
+    _need(dy, "dy", torch.bfloat16, 3)
+    if tuple(dy.shape) != (B, L, D):
+        raise ValueError("dy must be [B, L, D]")
+    _need(workspace, "workspace")
+    if grads is None:
+        grads = {n: torch.empty(weights[n].shape, dtype=torch.float32, device=data.device) for n in LM_WEIGHTS}
+    for n in LM_WEIGHTS:
+        _need(grads[n], "grad " + n, torch.float32)
+    lib = _lm_fns()
+    desc, keep = _lm_desc(B, L, D, H, F, head_classes, b, eps)
+    wp = _LmPtrs(*[weights[n].data_ptr() for n in LM_WEIGHTS])
+    gp = _LmPtrs(*[grads[n].data_ptr() for n in LM_WEIGHTS])
+    st = csr.struct()
+    _check("gsa_lm_block_bwd", lib.gsa_lm_block_bwd(_ptr(data), ctypes.byref(wp), ctypes.byref(st),
+                                                    ctypes.byref(desc), _ptr(dy), ctypes.byref(gp),
+                                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+    del keep
+    return grads
+
+
 def gsa_device_error(clear: bool = True) -> int:
     """The library's device error word (0 = no kernel gave up a wait)."""
     code = ctypes.c_int32(0)

@@ -2,9 +2,11 @@
 
     python -m content_adaptive_block_b200.build [--force] [--verbose]
 
-One translation unit (csrc/gsa.cu) compiled by nvcc with
+Two translation units (csrc/gsa.cu: the mask stage and the attention;
+csrc/lm_block.cu: the ByteLM block around it) compiled by nvcc with
 -gencode arch=compute_100a,code=sm_100a; the CUDA runtime is linked
-statically, the driver's tensor-map encoder is looked up at run time.
+statically, cuBLASLt (the block's projections) dynamically from the CUDA
+toolkit, and the driver's tensor-map encoder is looked up at run time.
 The ptxas resource report is written next to the library.
 """
 from __future__ import annotations
@@ -18,7 +20,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "gsa.cu")
+SRCS = [os.path.join(HERE, "csrc", "gsa.cu"), os.path.join(HERE, "csrc", "lm_block.cu")]
 OUT_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(OUT_DIR, "libgsa.so")
 REPORT = os.path.join(OUT_DIR, "ptxas_report.txt")
@@ -41,7 +43,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return [SRC] + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [os.path.join(INCLUDE, "gsa.h")]
+    return SRCS + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
 def up_to_date() -> bool:
@@ -56,7 +58,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(OUT_DIR, exist_ok=True)
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, SRC]
+    cuda_lib = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(_nvcc()))), "lib64")
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SRCS, "-L", cuda_lib, "-lcublasLt",
+           "-Xlinker", "-rpath=" + cuda_lib]
     res = subprocess.run(cmd, capture_output=True, text=True)
     with open(REPORT, "w") as f:
         f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)

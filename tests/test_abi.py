@@ -20,7 +20,8 @@ def lib():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "gsa.h")).read()
+    import glob
+    src = "".join(open(p).read() for p in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(gsa_[a-z_0-9]+)\s*\(", src)))
 
@@ -30,7 +31,7 @@ def test_header_declares_the_path(lib):
     for fn in ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_mask_pipeline",
                "gsa_build_fixed_csr", "gsa_attn_fwd",
                "gsa_attn_bwd", "gsa_csr_capacity", "gsa_attn_bwd_workspace", "gsa_device_error",
-               "gsa_status_string"):
+               "gsa_status_string", "gsa_lm_block_workspace", "gsa_lm_block_fwd", "gsa_lm_block_bwd"):
         assert fn in names
 
 
@@ -112,6 +113,41 @@ def test_build_fixed_csr_rejects_bad_arguments(lib):
     nul = _csr(B=2, n=8)
     nul.row_idx = None
     assert f(0, 1, 1, 0, NULL, ctypes.byref(nul), NULL) == 1
+
+
+def _lm(B=2, L=1024, D=256, H=4, F=512, b=64, classes=(0, 0, 1, 2), eps=1e-5):
+    hc = (ctypes.c_uint8 * len(classes))(*classes)
+    return gsa._LmDesc(B, L, D, H, F, b, ctypes.cast(hc, ctypes.c_void_p), eps), hc
+
+
+def test_lm_block_rejects_bad_arguments(lib):
+    gsa._lm_fns()
+    ws = lib.gsa_lm_block_workspace
+    d, k0 = _lm()
+    need = ws(ctypes.byref(d))
+    assert need > 2 * 1024 * (18 * 256 + 4 * 512)
+    for bad in (dict(D=192), dict(H=3, classes=(0, 0, 1)), dict(b=32), dict(L=1000), dict(F=500),
+                dict(classes=(0, 0, 1, 3)), dict(eps=0.0), dict(B=0)):
+        bd, kb = _lm(**bad)
+        assert ws(ctypes.byref(bd)) == 0, bad
+    c = _csr(B=2, n=16)
+    w = gsa._LmPtrs(*([0x1000] * 9))
+    g = gsa._LmPtrs(*([0x1000] * 9))
+    f, fb = lib.gsa_lm_block_fwd, lib.gsa_lm_block_bwd
+    assert f(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, need - 1, NULL) == 3   # capacity
+    assert f(NULL, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, need, NULL) == 1
+    assert f(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), NULL, FAKE, need, NULL) == 1
+    wn = gsa._LmPtrs(*([0x1000] * 8 + [0]))
+    assert f(FAKE, ctypes.byref(wn), ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, need, NULL) == 1
+    big, kg = _lm(D=2304, H=36, classes=(0,) * 36)
+    assert f(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(big), FAKE, FAKE, need, NULL) == 2   # D > 2048
+    assert fb(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), FAKE, ctypes.byref(g), FAKE, need - 1,
+              NULL) == 3
+    assert fb(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), NULL, ctypes.byref(g), FAKE, need,
+              NULL) == 1
+    gn = gsa._LmPtrs(*([0] + [0x1000] * 8))
+    assert fb(FAKE, ctypes.byref(w), ctypes.byref(c), ctypes.byref(d), FAKE, ctypes.byref(gn), FAKE, need,
+              NULL) == 1
 
 
 def test_mask_pipeline_rejects_bad_arguments(lib):

@@ -100,6 +100,32 @@ def random_words(S: int, n: int, r: int, seed: int = 0) -> np.ndarray:
     return rng.integers(0, 2**32, size=(S, n, r), dtype=np.uint64).astype(np.uint32)
 
 
+# One ByteLM block at the width of a 12-block, ~85M-weight byte LM (the
+# paper's 92M / 8K model class): D = 768, 12 heads of 64, MLP 3072, on the
+# 8x8K bench batch; the small shape spans several 128-row tiles with a ragged
+# tail (17 blocks per sample) for exact parity.
+LM_BLOCK = dict(D=768, H=12, F=3072)
+LM_BLOCK_SMALL = dict(S=2, L=17 * 64, D=256, H=4, F=512, w=2)
+
+
+def lm_weights(D: int, F: int, seed: int = 0, device="cpu", std: float = 0.02):
+    """Random-init weights of one block: matrices ~ N(0, std^2) in bf16, the
+    embedding ~ N(0, 1) in bf16, LayerNorm gains ~ 1 + N(0, 0.1^2) and biases
+    ~ N(0, 0.1^2) in float32 (perturbed so their gradients are exercised)."""
+    import torch
+    g = torch.Generator(device="cpu")
+    g.manual_seed(9_000_011 + seed)
+
+    def n(*shape, s=1.0):
+        return torch.randn(*shape, generator=g, dtype=torch.float32) * s
+
+    w = {"emb": n(256, D).bfloat16(), "ln1_g": 1 + n(D, s=0.1), "ln1_b": n(D, s=0.1),
+         "w_qkv": n(3 * D, D, s=std).bfloat16(), "w_o": n(D, D, s=std).bfloat16(),
+         "ln2_g": 1 + n(D, s=0.1), "ln2_b": n(D, s=0.1),
+         "w_1": n(F, D, s=std).bfloat16(), "w_2": n(D, F, s=std).bfloat16()}
+    return {k: v.to(device) for k, v in w.items()}
+
+
 def _rng(seed: int, salt: int, s: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, salt, s])))
 
