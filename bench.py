@@ -454,7 +454,7 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
                 dst.copy_(st[name], non_blocking=True)
             ev["down"][j].record(down)
 
-    e2e_steps = max(4, min(args.steps, 12))
+    e2e_steps = max(4, min(args.steps, 48))   # steady state: one upload and one download of fill/drain
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize()

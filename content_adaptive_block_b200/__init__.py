@@ -52,11 +52,16 @@ class _Csr(ctypes.Structure):
     ]
 
 
+class _AttnLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("qkv_s", "qkv_h", "qkv_l", "o_s", "o_h", "o_l")]
+
+
 class _AttnDesc(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int64),
         ("d", ctypes.c_int32), ("b", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("scale", ctypes.c_float), ("head_classes", ctypes.c_void_p),
+        ("layout", ctypes.c_void_p),
     ]
 
 
@@ -255,30 +260,62 @@ def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None =
 
 # ------------------------------------------------------------------ attention
 
-def _desc(q: torch.Tensor, b: int, head_classes, scale: float):
+def _desc(q: torch.Tensor, b: int, head_classes, scale: float, o: torch.Tensor | None = None):
+    """The call's descriptor; q (and o) may be strided [B, H, L, d] views with
+    contiguous rows, which become the call's layout (None when dense)."""
     B, H, L, d = q.shape
     hc = (ctypes.c_uint8 * H)(*[int(c) for c in head_classes])
     dtype = GSA_F32 if q.dtype == torch.float32 else GSA_BF16
-    return _AttnDesc(B, H, L, d, int(b), dtype, float(scale), ctypes.cast(hc, ctypes.c_void_p)), hc
+    keep = [hc]
+    lay = None
+    if not q.is_contiguous() or (o is not None and not o.is_contiguous()):
+        so = o.stride() if o is not None else q.stride()
+        lay = _AttnLayout(q.stride(0), q.stride(1), q.stride(2), so[0], so[1], so[2])
+        keep.append(lay)
+    desc = _AttnDesc(B, H, L, d, int(b), dtype, float(scale), ctypes.cast(hc, ctypes.c_void_p),
+                     ctypes.cast(ctypes.pointer(lay), ctypes.c_void_p) if lay is not None else None)
+    return desc, keep
+
+
+def _need_rows(t: torch.Tensor, name: str, like: torch.Tensor):
+    """A [B, H, L, d] CUDA tensor of like's dtype, shape and strides, d contiguous."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != like.dtype or t.dim() != 4 or tuple(t.shape) != tuple(like.shape):
+        raise ValueError(f"{name} must be {like.dtype} of shape {tuple(like.shape)}")
+    if t.stride(3) != 1 or t.stride() != like.stride():
+        raise ValueError(f"{name} must have the strides of {like.stride()} with contiguous rows")
 
 
 def gsa_attn_fwd(q, k, v, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,
                  o: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
     """Block-sparse causal attention forward; q, k, v [B, H, L, d] (bf16 or
-    float32).  Returns (o, lse) with lse float32 [B, H, L]."""
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, name, q.dtype, 4)
+    float32), bf16 ones possibly strided views with contiguous rows (k and v
+    with q's strides; o may have its own).  Returns (o, lse) with lse float32
+    [B, H, L]."""
+    if q.dtype == torch.float32:
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _need(t, name, q.dtype, 4)
+    else:
+        _need_rows(q, "q", q)
+        _need_rows(k, "k", q)
+        _need_rows(v, "v", q)
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k and v must have the same shape")
     if len(head_classes) != q.shape[1]:
         raise ValueError("one head class per head")
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    _need(o, "o", q.dtype)
+    if q.dtype == torch.float32:
+        _need(o, "o", q.dtype)
+    else:
+        _need_rows(o, "o", o)
+        if tuple(o.shape) != tuple(q.shape) or o.dtype != q.dtype:
+            raise ValueError("o must match q's shape and dtype")
     _need(lse, "lse", torch.float32)
-    desc, keep = _desc(q, b, head_classes, scale)
+    desc, keep = _desc(q, b, head_classes, scale, o)
     st = csr.struct()
     _check("gsa_attn_fwd", library().gsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(st), ctypes.byref(desc),
                                                   _ptr(o), _ptr(lse), _stream(stream)))
@@ -293,16 +330,26 @@ def gsa_attn_bwd_workspace(q: torch.Tensor, b: int, head_classes) -> int:
 
 def gsa_attn_bwd(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,
                  dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None):
-    """Gradients (dq, dk, dv) of gsa_attn_fwd for upstream gradient do."""
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, name, q.dtype, 4)
-    _need(lse, "lse", torch.float32, 3)
-    if len(head_classes) != q.shape[1]:
-        raise ValueError("one head class per head")
+    """Gradients (dq, dk, dv) of gsa_attn_fwd for upstream gradient do.
+    Strided views as in gsa_attn_fwd: k, v, dq, dk, dv with q's strides, do
+    with o's; dq, dk, dv default to q's strides when q is dense, else they
+    must be given."""
+    if dq is None or dk is None or dv is None:
+        if not q.is_contiguous():
+            raise ValueError("pass dq, dk and dv (with q's strides) for a strided q")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    desc, keep = _desc(q, b, head_classes, scale)
+    for name, t in (("q", q), ("k", k), ("v", v), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _need_rows(t, name, q)
+    _need_rows(o, "o", o)
+    _need_rows(do, "do", o)
+    if tuple(o.shape) != tuple(q.shape):
+        raise ValueError("o must match q's shape")
+    _need(lse, "lse", torch.float32, 3)
+    if len(head_classes) != q.shape[1]:
+        raise ValueError("one head class per head")
+    desc, keep = _desc(q, b, head_classes, scale, o)
     need = int(library().gsa_attn_bwd_workspace(ctypes.byref(desc)))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -328,13 +375,18 @@ def gsa_attn_bwd_noalloc(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: in
     vp = ctypes.c_void_p
     fn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_Csr), ctypes.POINTER(_AttnDesc), vp, vp, vp, vp]
     fn.restype = ctypes.c_int
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, name, q.dtype, 4)
-    _need(lse, "lse", torch.float32, 3)
+    if dq is None or dk is None or dv is None:
+        if not q.is_contiguous():
+            raise ValueError("pass dq, dk and dv (with q's strides) for a strided q")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    desc, keep = _desc(q, b, head_classes, scale)
+    for name, t in (("q", q), ("k", k), ("v", v), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _need_rows(t, name, q)
+    _need_rows(o, "o", o)
+    _need_rows(do, "do", o)
+    _need(lse, "lse", torch.float32, 3)
+    desc, keep = _desc(q, b, head_classes, scale, o)
     st = csr.struct()
     _check("gsa_attn_bwd_noalloc", fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), ctypes.byref(st),
                                       ctypes.byref(desc), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))

@@ -67,6 +67,7 @@ struct Params {
     const float* dvec;      // D_t
     __nv_bfloat16* out0;    // dq (dq_kernel) or dv (dkdv_kernel)
     __nv_bfloat16* out1;    // dk (dkdv_kernel)
+    TokLayout lq;           // layout of q, k, v and of dq, dk, dv
     float scale;
     float scale_log2;
     int* ticket;            // work counter of the persistent kernel (dot_kernel zeroes both)
@@ -75,19 +76,24 @@ struct Params {
 
 // ------------------------------------------------------------ D_t = dO·O
 
+// Grid (S H, L / kRowsPerCta): CTA (s H + h, y) takes the tokens
+// [y kRowsPerCta, (y + 1) kRowsPerCta) of sample s, head h (L is a multiple of 64).
 template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
-                                                  const __nv_bfloat16* __restrict__ dO, float* __restrict__ dvec,
-                                                  int64_t rows, int* __restrict__ ticket) {
-    if (blockIdx.x == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels that follow
+                                                  const __nv_bfloat16* __restrict__ dO, TokLayout lo, int64_t L,
+                                                  int H, float* __restrict__ dvec, int* __restrict__ ticket) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
     constexpr int kRowsPerCta = 256 / kTpr;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
+    const int sh = blockIdx.x, s = sh / H, h = sh - s * H;
+    const int64_t l = static_cast<int64_t>(blockIdx.y) * kRowsPerCta + threadIdx.x / kTpr;
+    const int64_t row = static_cast<int64_t>(sh) * L + l;
     const int part = threadIdx.x % kTpr;
     float acc = 0.f;
-    if (row < rows) {
-        const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
-        const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+    {
+        const int64_t off = s * lo.s + h * lo.h + l * lo.l + part * 8;
+        const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+        const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
         const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
         const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
     }
 #pragma unroll
     for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (row < rows && part == 0) dvec[row] = acc;
+    if (part == 0) dvec[row] = acc;
 }
 
 // ------------------------------------------------------------ dQ
@@ -204,10 +210,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         for (int half = 0; half < 2; ++half) {
             const int blk = half ? qb : qa;
             if (blk < 0) continue;
-            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+            const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at) {
-                tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
-                tma_load_2d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, row);
+                tma_load_4d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s);
+                tma_load_4d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, l0, h, s);
             }
         }
     }
@@ -234,10 +240,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     !mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer))
                     break;
                 mbar_arrive_expect_tx(&full[st], 2 * C::kKVBytes);
-                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(tl.list[n]) * kBlk);
+                const int l0 = tl.list[n] * kBlk;   // token coordinate in the (sample, head)
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_2d(sK + st * C::kKVBytes + at * (kBlk * 128), &tmK, &full[st], at * 64, row);
-                    tma_load_2d(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, row);
+                    tma_load_4d(sK + st * C::kKVBytes + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s);
+                    tma_load_4d(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s);
                 }
             }
         }
@@ -370,7 +376,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             const bool has1 = C::G == 2 && T >= 2;   // dQ_1 holds products only if group 1 had a tile
-            __nv_bfloat16* orow = p.out0 + tok * D;
+            __nv_bfloat16* orow = p.out0 + tok_off(tok, p.L, p.H, p.lq);
             constexpr int kOc = D / (C::G * H);   // output columns per thread (split among a row's threads)
             const int slot = grp * H + hc;
 #pragma unroll
@@ -507,10 +513,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int half = 0; half < 2; ++half) {
             const int blk = half ? kb : ka;
             if (blk < 0) continue;
-            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+            const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at) {
-                tma_load_2d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, row);
-                tma_load_2d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, row);
+                tma_load_4d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, l0, h, s);
+                tma_load_4d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, l0, h, s);
             }
         }
     }
@@ -538,10 +544,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     break;
                 mbar_arrive_expect_tx(&full[st], C::kStageBytes + 2 * C::kVecBytes);
                 const int64_t row64 = head_row0 + static_cast<int64_t>(tl.list[n]) * kBlk;
-                const int row = static_cast<int>(row64);
+                const int l0 = static_cast<int>(row64 - head_row0);   // token coordinate in the (sample, head)
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_2d(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, row);
-                    tma_load_2d(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, row);
+                    tma_load_4d(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, l0, h, s);
+                    tma_load_4d(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, l0, h, s);
                 }
                 bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
                 bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
@@ -712,7 +718,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int slot = grp * H + hc;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok * D;
+                __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok_off(tok, p.L, p.H, p.lq);
                 const float mul = which == 0 ? 1.f : p.scale;
                 const uint32_t col0 = which == 0 ? C::dv_col(0) : C::dk_col(0);
                 const uint32_t col1 = which == 0 ? C::dv_col(1) : C::dk_col(1);
@@ -777,16 +783,16 @@ inline int sm_count() {
 
 template <int D>
 gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                    const __nv_bfloat16* o, const __nv_bfloat16* dO, Params pq, Params pkv, int64_t rows, int S,
-                    int H, int nblk, cudaStream_t st) {
+                    const __nv_bfloat16* o, const __nv_bfloat16* dO, const TokLayout& lo, Params pq, Params pkv,
+                    int S, int H, int nblk, cudaStream_t st) {
     static std::once_flag once;
     std::call_once(once, [] {
         cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemBytes);
         cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvCfg<D>::kSmemBytes);
     });
-    constexpr int kRowsPerCta = 256 / (D / 8);
-    dot_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
-        o, dO, const_cast<float*>(pq.dvec), rows, pkv.ticket);
+    constexpr int kRowsPerCta = 256 / (D / 8);   // 32 or 16: divides L
+    dot_kernel<D><<<dim3(static_cast<unsigned>(S * H), static_cast<unsigned>(pq.L / kRowsPerCta)), 256, 0, st>>>(
+        o, dO, lo, pq.L, pq.H, const_cast<float*>(pq.dvec), pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
     if (D == 64 && GSA_DQ_PERSIST) {
         static std::once_flag once_q;
@@ -818,15 +824,19 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
 
 inline gsa_status launch(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                          const gsa_block_csr* csr, const gsa_attn_desc* desc, const uint8_t* cls, float scale,
-                         void* dq, void* dk, void* dv, float* work, cudaStream_t st) {
+                         void* dq, void* dk, void* dv, float* work, const TokLayout& lq, const TokLayout& lo,
+                         cudaStream_t st) {
     if ((reinterpret_cast<uintptr_t>(lse) & 15u) || (reinterpret_cast<uintptr_t>(work) & 15u))
         return GSA_ERR_INVALID_ARGUMENT;
     const int64_t rows = static_cast<int64_t>(desc->B) * desc->H * desc->L;
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap_bf16(&tq, q, rows, desc->d) || !make_tmap_bf16(&tk, k, rows, desc->d) ||
-        !make_tmap_bf16(&tv, v, rows, desc->d) || !make_tmap_bf16(&tdo, dO, rows, desc->d))
+    if (!make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq) ||
+        !make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq) ||
+        !make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq) ||
+        !make_tmap_tok(&tdo, dO, desc->d, desc->L, desc->H, desc->B, lo))
         return GSA_ERR_CUDA;
     Params base{};
+    base.lq = lq;
     base.cap = csr->capacity;
     base.S = desc->B;
     base.H = desc->H;
@@ -852,8 +862,9 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     pkv.out1 = static_cast<__nv_bfloat16*>(dk);
     const auto* ob = static_cast<const __nv_bfloat16*>(o);
     const auto* dob = static_cast<const __nv_bfloat16*>(dO);
-    if (desc->d == 64) return launch_d<64>(tq, tk, tv, tdo, ob, dob, pq, pkv, rows, desc->B, desc->H, csr->nblk, st);
-    return launch_d<128>(tq, tk, tv, tdo, ob, dob, pq, pkv, rows, desc->B, desc->H, csr->nblk, st);
+    if (desc->d == 64)
+        return launch_d<64>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
+    return launch_d<128>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
 }
 
 }  // namespace bwd

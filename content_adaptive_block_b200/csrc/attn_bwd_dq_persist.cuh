@@ -158,6 +158,7 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 __syncwarp();
             }
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
+            const int s_ = sh / p.H, h_ = sh - s_ * p.H;   // the 4-D maps' head and sample
             if (lane == 0) {
                 // the record slot k & 1 and the Q, dO tile are free once the
                 // previous item's last S, dP completed
@@ -169,9 +170,9 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     for (int half = 0; half < 2; ++half) {
                         const int blk = half ? qb : qa;
                         if (blk < 0) continue;
-                        const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
-                        tma_load_2d(sQ + half * (kBlk * 128), &tmQ, qd_full, 0, row);
-                        tma_load_2d(sDO + half * (kBlk * 128), &tmDO, qd_full, 0, row);
+                        const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
+                        tma_load_4d(sQ + half * (kBlk * 128), &tmQ, qd_full, 0, l0, h_, s_);
+                        tma_load_4d(sDO + half * (kBlk * 128), &tmDO, qd_full, 0, l0, h_, s_);
                     }
                 }
                 int lastw = have ? nwords - 1 : -1;
@@ -193,9 +194,9 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         const uint32_t live = ((ua >> bit) & 1u) | (((ub >> bit) & 1u) << 1);
                         meta[st] = static_cast<uint32_t>(j) | (live << 16) | ((j == last_j ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes);
-                        const int row = static_cast<int>(head_row0 + static_cast<int64_t>(j) * kBlk);
-                        tma_load_2d(stage_k(st), &tmK, &full[st], 0, row);
-                        tma_load_2d(stage_v(st), &tmV, &full[st], 0, row);
+                        const int l0 = j * kBlk;   // token coordinate in the (sample, head)
+                        tma_load_4d(stage_k(st), &tmK, &full[st], 0, l0, h_, s_);
+                        tma_load_4d(stage_v(st), &tmV, &full[st], 0, l0, h_, s_);
                         ++gt;
                     }
                 }
@@ -366,7 +367,7 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(acc_free);   // dQ may take the next item's products
-                    if (my_blk >= 0) store_scaled_bf16(p.out0 + tok * D + c0, ov, p.scale);
+                    if (my_blk >= 0) store_scaled_bf16(p.out0 + tok_off(tok, p.L, p.H, p.lq) + c0, ov, p.scale);
                     break;
                 }
             }

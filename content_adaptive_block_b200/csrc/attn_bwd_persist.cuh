@@ -176,6 +176,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 __syncwarp();
             }
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
+            const int s_ = sh / p.H, h_ = sh - s_ * p.H;   // the 4-D maps' head and sample
             if (lane == 0) {
                 // the record slot k & 1 and the K, V tile are free once the previous
                 // item's last S^T, dP^T completed (every reader of the slot's old
@@ -188,9 +189,9 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     for (int half = 0; half < 2; ++half) {
                         const int blk = half ? kb : ka;
                         if (blk < 0) continue;
-                        const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
-                        tma_load_2d(sK + half * (kBlk * 128), &tmK, kv_full, 0, row);
-                        tma_load_2d(sV + half * (kBlk * 128), &tmV, kv_full, 0, row);
+                        const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
+                        tma_load_4d(sK + half * (kBlk * 128), &tmK, kv_full, 0, l0, h_, s_);
+                        tma_load_4d(sV + half * (kBlk * 128), &tmV, kv_full, 0, l0, h_, s_);
                     }
                 }
                 int lastw = have ? nwords - 1 : -1;
@@ -213,8 +214,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         meta[st] = static_cast<uint32_t>(i) | (live << 16) | ((i == last_i ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes + 2 * C::kVecBytes);
                         const int64_t row64 = head_row0 + static_cast<int64_t>(i) * kBlk;
-                        tma_load_2d(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64));
-                        tma_load_2d(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64));
+                        tma_load_4d(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_);
+                        tma_load_4d(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_);
                         bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
                         bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
                         ++gt;
@@ -415,8 +416,9 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     mbar_arrive(acc_free);   // the accumulators may take the next item's products
                     if (my_blk >= 0) {
                         const int64_t tok = head_row0 + static_cast<int64_t>(my_blk) * kBlk + uu;
-                        store_scaled_bf16(p.out0 + tok * D + c0, ov, 1.f);
-                        store_scaled_bf16(p.out1 + tok * D + c0, ok_, p.scale);
+                        const int64_t off = tok_off(tok, p.L, p.H, p.lq) + c0;
+                        store_scaled_bf16(p.out0 + off, ov, 1.f);
+                        store_scaled_bf16(p.out1 + off, ok_, p.scale);
                     }
                     break;
                 }

@@ -100,6 +100,7 @@ struct FwdParams {
     int S, H, nblk;
     int64_t L;
     __nv_bfloat16* o;
+    TokLayout lo;       // layout of o
     float* lse;
     float scale_log2;   // softmax scale * log2(e)
     uint8_t cls[kMaxHeads];
@@ -173,7 +174,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int qa = p.q_order[g * nblk + 2 * tile];
     const int qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
     const int nwords = (nblk + 31) >> 5;
-    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;   // first row of this (s, h) in the 2-D views
+    const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;   // row of this (s, h)'s first token (LSE index)
 
     // ---- set-up: barriers, TMEM, merged key list
     if (threadIdx.x == 0) {
@@ -200,9 +201,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         for (int half = 0; half < 2; ++half) {
             const int blk = half ? qb : qa;
             if (blk < 0) continue;
-            const int row = static_cast<int>(head_row0 + static_cast<int64_t>(blk) * kBlk);
+            const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at)
-                tma_load_2d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, row);
+                tma_load_4d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s);
         }
     }
     if (warp == 1) {
@@ -270,12 +271,12 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (!mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer)) break;
                 }
                 mbar_arrive_expect_tx(&full[st], 2 * C::kKVBytes);
-                const int row = static_cast<int>(head_row0 + static_cast<int64_t>(list[n]) * kBlk);
+                const int l0 = list[n] * kBlk;   // token coordinate in the (sample, head)
                 uint8_t* dk = sK + st * C::kKVBytes;
                 uint8_t* dv = sV + st * C::kKVBytes;
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_2d(dk + at * (kBlk * 128), &tmK, &full[st], at * 64, row);
-                    tma_load_2d(dv + at * (kBlk * 128), &tmV, &full[st], at * 64, row);
+                    tma_load_4d(dk + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s);
+                    tma_load_4d(dv + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s);
                 }
             }
         }
@@ -467,7 +468,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const float inv = 1.f / lt;
             const bool store = my_blk >= 0;
             const int64_t tok = head_row0 + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
-            __nv_bfloat16* orow = p.o + tok * D;
+            __nv_bfloat16* orow = p.o + tok_off(tok, p.L, p.H, p.lo);
 #pragma unroll
             for (int cb = grp * (D / C::G); cb < (grp + 1) * (D / C::G); cb += 32) {
                 float a[32];

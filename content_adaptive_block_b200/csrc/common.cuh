@@ -144,6 +144,32 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// Element strides of a [sample][head][token][d] tensor whose d values of
+// one token are contiguous: the attention reads and writes Q, K, V, O, dO
+// and the gradients through such a layout (the dense [S][H][L][d] order, or
+// a view of a token-major [S][L][..heads..][d] projection output).
+struct TokLayout {
+    int64_t s, h, l;
+};
+
+// Offset of the token row r = (s H + h) L + l of a tensor with layout t
+// (row numbers stay below 2^31, which the calls check, so 32-bit division).
+__device__ __forceinline__ int64_t tok_off(int64_t r, int64_t L, int H, const TokLayout& t) {
+    const int r32 = static_cast<int>(r), L32 = static_cast<int>(L);
+    const int sh = r32 / L32, l = r32 - sh * L32;
+    const int s = sh / H, h = sh - s * H;
+    return s * t.s + h * t.h + l * t.l;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -354,16 +380,21 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     return fn;
 }
 
-// A bf16 [rows][cols] row-major matrix read in 64 x 64 boxes with the
-// 128-byte swizzle the UMMA descriptors below expect.
-inline bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+// A bf16 [S][H][L][d] tensor with layout t (element strides, multiples of 8)
+// as a 4-D map over (d, L, H, S), read in boxes of 64 tokens x 64 columns of
+// one (sample, head) with the 128-byte swizzle the UMMA descriptors below
+// expect; the box lands in shared memory as [64 tokens][128 B].
+inline bool make_tmap_tok(CUtensorMap* map, const void* base, int64_t d, int64_t L, int64_t H, int64_t S,
+                          const TokLayout& t) {
     auto fn = tmap_encoder();
     if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(S)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(t.l) * 2, static_cast<cuuint64_t>(t.h) * 2,
+                             static_cast<cuuint64_t>(t.s) * 2};
+    cuuint32_t box[4] = {64, 64, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;

@@ -72,6 +72,27 @@ bool csr_ok(const gsa_block_csr* c) {
 }
 
 // Common checks of an attention call; fills the class table.
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The tensors' layouts: dense [B][H][L][d] without desc->layout; with it,
+// strides that are positive multiples of 8 elements (16 bytes, as TMA
+// requires) with each token's d values inside one stride step.
+gsa_status resolve_layout(const gsa_attn_desc* d, gsa::TokLayout* lq, gsa::TokLayout* lo) {
+    const int64_t dense_h = d->L * d->d, dense_s = d->H * dense_h;
+    if (!d->layout) {
+        *lq = *lo = gsa::TokLayout{dense_s, dense_h, d->d};
+        return GSA_OK;
+    }
+    const gsa_attn_layout& y = *d->layout;
+    const int64_t st[6] = {y.qkv_s, y.qkv_h, y.qkv_l, y.o_s, y.o_h, y.o_l};
+    for (int64_t s : st)
+        if (s <= 0 || s % 8 != 0) return GSA_ERR_INVALID_ARGUMENT;
+    if (y.qkv_l < d->d || y.o_l < d->d) return GSA_ERR_INVALID_ARGUMENT;
+    *lq = gsa::TokLayout{y.qkv_s, y.qkv_h, y.qkv_l};
+    *lo = gsa::TokLayout{y.o_s, y.o_h, y.o_l};
+    return GSA_OK;
+}
+
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
     if (!d || !csr || !d->head_classes) return GSA_ERR_INVALID_ARGUMENT;
     if (!csr_ok(csr)) return csr && csr->capacity < gsa_csr_capacity(csr->nblk) ? GSA_ERR_CAPACITY
@@ -234,7 +255,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     const cudaStream_t cs = as_stream(stream);
 
     if (desc->dtype == GSA_F32) {
-        if (desc->b > 128 || !(desc->d == 16 || desc->d == 32 || desc->d == 64 || desc->d == 128))
+        if (desc->b > 128 || !(desc->d == 16 || desc->d == 32 || desc->d == 64 || desc->d == 128) || desc->layout)
             return GSA_ERR_UNSUPPORTED;
         gsa::f32::Params p;
         p.q = static_cast<const float*>(q);
@@ -277,12 +298,16 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     // bf16 tensor-core path
     if (desc->b != gsa::bf16::kBlk || !(desc->d == 64 || desc->d == 128) || csr->nblk > GSA_MAX_BLOCKS_BF16)
         return GSA_ERR_UNSUPPORTED;
-    if (!lse) return GSA_ERR_INVALID_ARGUMENT;
+    if (!lse || !al16(q) || !al16(k) || !al16(v) || !al16(o)) return GSA_ERR_INVALID_ARGUMENT;
     const uint64_t rows = static_cast<uint64_t>(desc->B) * desc->H * desc->L;
     if (rows >= (1ull << 31)) return GSA_ERR_UNSUPPORTED;
+    gsa::TokLayout lq, lo;
+    st = resolve_layout(desc, &lq, &lo);
+    if (st != GSA_OK) return st;
     CUtensorMap tq, tk, tv;
-    if (!gsa::make_tmap_bf16(&tq, q, rows, desc->d) || !gsa::make_tmap_bf16(&tk, k, rows, desc->d) ||
-        !gsa::make_tmap_bf16(&tv, v, rows, desc->d))
+    if (!gsa::make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq) ||
+        !gsa::make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq) ||
+        !gsa::make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq))
         return GSA_ERR_CUDA;
     gsa::bf16::FwdParams p;
     p.row_ptr = csr->row_ptr;
@@ -294,6 +319,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     p.nblk = csr->nblk;
     p.L = desc->L;
     p.o = static_cast<__nv_bfloat16*>(o);
+    p.lo = lo;
     p.lse = lse;
     p.scale_log2 = scale * 1.4426950408889634f;
     std::memcpy(p.cls, cls, desc->H);
@@ -337,9 +363,14 @@ gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void*
         return GSA_ERR_UNSUPPORTED;
     const uint64_t rows = static_cast<uint64_t>(desc->B) * desc->H * desc->L;
     if (rows >= (1ull << 31)) return GSA_ERR_UNSUPPORTED;
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al16(dO) || !al16(dq) || !al16(dk) || !al16(dv))
+        return GSA_ERR_INVALID_ARGUMENT;
+    gsa::TokLayout lq, lo;
+    st = resolve_layout(desc, &lq, &lo);
+    if (st != GSA_OK) return st;
     const float scale = desc->scale > 0.f ? desc->scale : 1.f / std::sqrt(static_cast<float>(desc->d));
     return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, static_cast<float*>(workspace),
-                            as_stream(stream));
+                            lq, lo, as_stream(stream));
 }
 
 gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -357,7 +388,13 @@ gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, con
     float* scratch = noalloc_scratch(&st);
     if (st != GSA_OK) return st;
     const float scale = desc->scale > 0.f ? desc->scale : 1.f / std::sqrt(static_cast<float>(desc->d));
-    return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, scratch, as_stream(stream));
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al16(dO) || !al16(dq) || !al16(dk) || !al16(dv))
+        return GSA_ERR_INVALID_ARGUMENT;
+    gsa::TokLayout lq, lo;
+    st = resolve_layout(desc, &lq, &lo);
+    if (st != GSA_OK) return st;
+    return gsa::bwd::launch(q, k, v, o, lse, dO, csr, desc, cls, scale, dq, dk, dv, scratch, lq, lo,
+                            as_stream(stream));
 }
 
 int64_t gsa_attn_bwd_noalloc_max_rows(void) { return kNoAllocRows; }

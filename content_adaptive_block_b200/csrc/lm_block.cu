@@ -10,10 +10,11 @@
 //
 // Hand-written kernels here: the embedding gather fused with LN1, LayerNorm
 // forward and backward (with deterministic column sums for the gain and bias
-// gradients), the head split / merge between the
-// projections' [token][feature] layout and the attention's [sample][head]
-// [token][64] layout, and the embedding gradient (a deterministic per-byte
-// reduction).  The attention is gsa_attn_fwd / gsa_attn_bwd.  The
+// gradients) and the embedding gradient (a deterministic per-byte
+// reduction).  The attention is gsa_attn_fwd / gsa_attn_bwd, reading Q, K, V
+// straight out of the QKV projection's [token][3][head][64] rows and writing
+// O, dQ, dK, dV in the projections' layouts (gsa_attn_layout), so no head
+// transposes run.  The
 // projections are plain bf16 GEMMs with float32 accumulation and go to
 // cuBLASLt, the residual additions folded into them (D = A B + C) and the
 // GELU and its derivative into their epilogues.
@@ -202,28 +203,6 @@ colsum_kernel(const float* __restrict__ part, int nparts, int D, float* __restri
     }
 }
 
-// ----------------------------------------------------------- head layouts
-// rows [T][nsplit D] (features: part, head, 64) <-> heads[part] [S][H][L][64].
-struct Heads {
-    bf16* p[3];
-};
-
-template <bool TO_HEADS>
-__global__ void heads_kernel(bf16* __restrict__ rows, Heads heads, int nsplit, int64_t T, int L, int H) {
-    const int D = 64 * H;
-    const int64_t width8 = static_cast<int64_t>(nsplit) * D / 8;
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= T * width8) return;
-    const int64_t t = i / width8;
-    const int c = static_cast<int>(i - t * width8) * 8;
-    const int part = c / D, hh = (c % D) >> 6, e = c & 63;
-    const int64_t s = t / L, l = t - s * L;
-    bf16* hp = heads.p[part] + ((s * H + hh) * L + l) * 64 + e;
-    bf16* rp = rows + t * (static_cast<int64_t>(nsplit) * D) + c;
-    if (TO_HEADS) *reinterpret_cast<uint4*>(hp) = *reinterpret_cast<const uint4*>(rp);
-    else *reinterpret_cast<uint4*>(rp) = *reinterpret_cast<const uint4*>(hp);
-}
-
 // ------------------------------------------------------ embedding gradient
 // dE[v][c] = sum over tokens t with bytes[t] == v of dx0[t][c], in a fixed
 // order: CTA (chunk of kEmbChunk tokens, slice of 32 columns) has two warps,
@@ -390,8 +369,8 @@ gsa_status gemm_rm(bool ta, bool tb, int M, int N, int K, const bf16* A, int lda
 
 // ------------------------------------------------------------ workspace
 struct Layout {
-    size_t x0, h, st1, q, k, v, o, lse, om, x1, h2, st2, pre, act, qkv;   // saved by the forward
-    size_t dpre, dh2, dx1, dom, doh, dq, dk, dv, dh, dx0, part, epart, attn_ws;   // backward scratch
+    size_t x0, h, st1, qkv, lse, om, x1, h2, st2, pre, act;       // saved by the forward
+    size_t dpre, dh2, dx1, dom, dqkv, dh, dx0, part, epart, attn_ws;   // backward scratch
     size_t lt, total;
     size_t attn_ws_bytes;
 };
@@ -411,10 +390,7 @@ Layout layout(const gsa_lm_desc* d, const gsa_attn_desc& ad) {
     l.x0 = take(TD);
     l.h = take(TD);
     l.st1 = take(T * 8);
-    l.q = take(TD);
-    l.k = take(TD);
-    l.v = take(TD);
-    l.o = take(TD);
+    l.qkv = take(3 * TD);
     l.lse = take(T * d->H * 4);
     l.om = take(TD);
     l.x1 = take(TD);
@@ -422,15 +398,11 @@ Layout layout(const gsa_lm_desc* d, const gsa_attn_desc& ad) {
     l.st2 = take(T * 8);
     l.pre = take(TF);
     l.act = take(TF);
-    l.qkv = take(3 * TD);
     l.dpre = take(TF);
     l.dh2 = take(TD);
     l.dx1 = take(TD);
     l.dom = take(TD);
-    l.doh = take(TD);
-    l.dq = take(TD);
-    l.dk = take(TD);
-    l.dv = take(TD);
+    l.dqkv = take(3 * TD);
     l.dh = take(TD);
     l.dx0 = take(TD);
     l.part = take(static_cast<size_t>(kLnParts) * 2 * d->D * 4);
@@ -440,6 +412,12 @@ Layout layout(const gsa_lm_desc* d, const gsa_attn_desc& ad) {
     l.lt = take(kLtWorkspace);
     l.total = off;
     return l;
+}
+
+// Q, K, V (and dQ, dK, dV) inside [T][3][H][64] rows; O and dO inside [T][H][64] rows.
+gsa_attn_layout attn_layout(const gsa_lm_desc* d) {
+    const int64_t D = d->D, L = d->L;
+    return gsa_attn_layout{3 * D * L, 64, 3 * D, D * L, 64, D};
 }
 
 gsa_status check(const gsa_lm_desc* d, gsa_attn_desc* ad) {
@@ -457,6 +435,7 @@ gsa_status check(const gsa_lm_desc* d, gsa_attn_desc* ad) {
     ad->dtype = GSA_BF16;
     ad->scale = 0.f;
     ad->head_classes = d->head_classes;
+    ad->layout = nullptr;   // the calls point it at their own layout
     return GSA_OK;
 }
 
@@ -513,15 +492,6 @@ void ln_bwd(int D, const bf16* dy, const bf16* x, const float2* stats, const flo
     colsum_kernel<<<(2 * D + 31) / 32, 256, 0, st>>>(part, kLnParts, D, dg, db);
 }
 
-void heads(bool to_heads, bf16* rows, bf16* p0, bf16* p1, bf16* p2, int nsplit, int64_t T, int L, int H,
-           cudaStream_t st) {
-    Heads hp{{p0, p1, p2}};
-    const int64_t n = T * nsplit * 64 * H / 8;
-    const unsigned grid = static_cast<unsigned>((n + 255) / 256);
-    if (to_heads) heads_kernel<true><<<grid, 256, 0, st>>>(rows, hp, nsplit, T, L, H);
-    else heads_kernel<false><<<grid, 256, 0, st>>>(rows, hp, nsplit, T, L, H);
-}
-
 }  // namespace lm
 }  // namespace gsa
 
@@ -567,14 +537,13 @@ gsa_status gsa_lm_block_fwd(const uint8_t* bytes, const gsa_lm_weights* w, const
     ln_fwd(D, true, bytes, emb, w->ln1_g, w->ln1_b, P(l.x0), P(l.h), reinterpret_cast<float2*>(ws + l.st1), T,
            desc->ln_eps, st);
     GSA_TRY(last_launch());
-    // qkv = h W_qkv^T, then Q, K, V in the attention's head layout
+    // qkv = h W_qkv^T; the attention reads Q, K, V from its rows and writes O as W_o's input rows
     GSA_TRY(gemm_rm(false, true, Mi, 3 * D, D, P(l.h), D, static_cast<const bf16*>(w->w_qkv), D, 0.f, nullptr,
                     3 * D, P(l.qkv), 3 * D, false, lt, st));
-    heads(true, P(l.qkv), P(l.q), P(l.k), P(l.v), 3, T, desc->L, desc->H, st);
-    GSA_TRY(last_launch());
-    GSA_TRY(gsa_attn_fwd(P(l.q), P(l.k), P(l.v), csr, &ad, P(l.o), reinterpret_cast<float*>(ws + l.lse), stream));
-    heads(false, P(l.om), P(l.o), nullptr, nullptr, 1, T, desc->L, desc->H, st);
-    GSA_TRY(last_launch());
+    const gsa_attn_layout al = attn_layout(desc);
+    ad.layout = &al;
+    GSA_TRY(gsa_attn_fwd(P(l.qkv), P(l.qkv) + D, P(l.qkv) + 2 * D, csr, &ad, P(l.om),
+                         reinterpret_cast<float*>(ws + l.lse), stream));
     // x1 = x0 + O W_o^T, h2 = LN2(x1)
     GSA_TRY(gemm_rm(false, true, Mi, D, D, P(l.om), D, static_cast<const bf16*>(w->w_o), D, 1.f, P(l.x0), D,
                     P(l.x1), D, false, lt, st));
@@ -625,20 +594,19 @@ gsa_status gsa_lm_block_bwd(const uint8_t* bytes, const gsa_lm_weights* w, const
     ln_bwd(D, P(l.dh2), P(l.x1), reinterpret_cast<const float2*>(ws + l.st2), w->ln2_g, dyb, P(l.dx1), part,
            g->ln2_g, g->ln2_b, T, st);
     GSA_TRY(last_launch());
-    // attention: dO = dx1 W_o, dW_o = dx1^T O, then the attention's own backward
+    // attention: dO = dx1 W_o, dW_o = dx1^T O, then the attention's own backward (dQ, dK, dV as dqkv rows)
     GSA_TRY(gemm_rm(false, false, Mi, D, D, P(l.dx1), D, static_cast<const bf16*>(w->w_o), D, 0.f, nullptr, D,
                     P(l.dom), D, false, lt, st));
     GSA_TRY(gemm_rm(true, false, D, D, Mi, P(l.dx1), D, P(l.om), D, 0.f, nullptr, D, g->w_o, D, true, lt, st));
-    heads(true, P(l.dom), P(l.doh), nullptr, nullptr, 1, T, desc->L, desc->H, st);
-    GSA_TRY(last_launch());
-    GSA_TRY(gsa_attn_bwd(P(l.q), P(l.k), P(l.v), P(l.o), reinterpret_cast<const float*>(ws + l.lse), P(l.doh), csr,
-                         &ad, P(l.dq), P(l.dk), P(l.dv), ws + l.attn_ws, l.attn_ws_bytes, stream));
-    heads(false, P(l.qkv), P(l.dq), P(l.dk), P(l.dv), 3, T, desc->L, desc->H, st);   // dqkv over qkv
-    GSA_TRY(last_launch());
+    const gsa_attn_layout al = attn_layout(desc);
+    ad.layout = &al;
+    GSA_TRY(gsa_attn_bwd(P(l.qkv), P(l.qkv) + D, P(l.qkv) + 2 * D, P(l.om), reinterpret_cast<const float*>(ws + l.lse),
+                         P(l.dom), csr, &ad, P(l.dqkv), P(l.dqkv) + D, P(l.dqkv) + 2 * D, ws + l.attn_ws,
+                         l.attn_ws_bytes, stream));
     // dW_qkv = dqkv^T h, dh = dqkv W_qkv, dx0 = dx1 + LN1'(dh)
-    GSA_TRY(gemm_rm(true, false, 3 * D, D, Mi, P(l.qkv), 3 * D, P(l.h), D, 0.f, nullptr, D, g->w_qkv, D, true, lt,
+    GSA_TRY(gemm_rm(true, false, 3 * D, D, Mi, P(l.dqkv), 3 * D, P(l.h), D, 0.f, nullptr, D, g->w_qkv, D, true, lt,
                     st));
-    GSA_TRY(gemm_rm(false, false, Mi, D, 3 * D, P(l.qkv), 3 * D, static_cast<const bf16*>(w->w_qkv), D, 0.f,
+    GSA_TRY(gemm_rm(false, false, Mi, D, 3 * D, P(l.dqkv), 3 * D, static_cast<const bf16*>(w->w_qkv), D, 0.f,
                     nullptr, D, P(l.dh), D, false, lt, st));
     ln_bwd(D, P(l.dh), P(l.x0), reinterpret_cast<const float2*>(ws + l.st1), w->ln1_g, P(l.dx1), P(l.dx0), part,
            g->ln1_g, g->ln1_b, T, st);

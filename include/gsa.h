@@ -213,6 +213,21 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
  * (b = 64, d in {64, 128}, nblk <= GSA_MAX_BLOCKS_BF16) with float32
  * accumulation and softmax.
  */
+/*
+ * Layout of the attention tensors, in elements (bf16 calls only).  Element
+ * (sample s, head h, token l, e) of q, k, v, dq, dk and dv is at
+ * s*qkv_s + h*qkv_h + l*qkv_l + e from its base pointer; of o and dO at
+ * s*o_s + h*o_h + l*o_l + e.  Every stride is a positive multiple of 8
+ * (16 bytes, the TMA rule) and the token strides are >= d; the caller keeps
+ * the written tensors (o, dq, dk, dv) free of overlaps.  Example: with one
+ * token-major projection output qkv [B][L][3][H][d], q = qkv, k = qkv + H*d,
+ * v = qkv + 2*H*d and qkv_s = 3*L*H*d, qkv_h = d, qkv_l = 3*H*d.
+ */
+typedef struct {
+    int64_t qkv_s, qkv_h, qkv_l;
+    int64_t o_s, o_h, o_l;
+} gsa_attn_layout;
+
 typedef struct {
     int32_t B, H;
     int64_t L;          /* tokens (bytes) per sample = nblk * b */
@@ -221,6 +236,7 @@ typedef struct {
     int32_t dtype;      /* gsa_dtype */
     float scale;
     const uint8_t* head_classes;
+    const gsa_attn_layout* layout;   /* host; NULL: dense [B][H][L][d] for every tensor */
 } gsa_attn_desc;
 
 /*
@@ -232,10 +248,12 @@ typedef struct {
  * token t in block i,
  *   o_t = Σ_{u in A(t)} softmax_u(scale * q_t·k_u) v_u,
  *   A(t) = { u <= t : block(u) in the CSR row i of (s, c) }.
- *   o [B][H][L][d] out, lse [B][H][L] float32 out (may be NULL for GSA_F32).
+ *   o [B][H][L][d] out (or desc->layout's strides), lse [B][H][L] float32 out
+ *   (dense always; may be NULL for GSA_F32).
  * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, L != nblk*b, shapes that
- * disagree with csr, a class outside 0..2), GSA_ERR_UNSUPPORTED (dtype / b / d
- * outside the kernels above), GSA_ERR_CUDA.
+ * disagree with csr, a class outside 0..2, bf16 tensors not 16-byte aligned,
+ * a layout breaking its rules), GSA_ERR_UNSUPPORTED (dtype / b / d outside the
+ * kernels above, a layout with GSA_F32), GSA_ERR_CUDA.
  */
 gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_block_csr* csr,
                         const gsa_attn_desc* desc, void* o, float* lse, void* stream);

@@ -79,8 +79,8 @@ typedef struct {
 /*
  * Bytes of device workspace the two calls below need (0 for an invalid
  * desc): the activations the forward saves for the backward (about
- * B*L*(18 D + 4 F) bytes), the backward's scratch, the attention backward's
- * workspace and 32 MiB for cuBLASLt.
+ * B*L*(10 D + 4 F) bytes), the backward's scratch (about B*L*(12 D + 2 F)),
+ * the attention backward's workspace and 32 MiB for cuBLASLt.
  */
 size_t gsa_lm_block_workspace(const gsa_lm_desc* desc);
 

@@ -125,7 +125,7 @@ def test_lm_block_rejects_bad_arguments(lib):
     ws = lib.gsa_lm_block_workspace
     d, k0 = _lm()
     need = ws(ctypes.byref(d))
-    assert need > 2 * 1024 * (18 * 256 + 4 * 512)
+    assert need > 2 * 1024 * (22 * 256 + 6 * 512)
     for bad in (dict(D=192), dict(H=3, classes=(0, 0, 1)), dict(b=32), dict(L=1000), dict(F=500),
                 dict(classes=(0, 0, 1, 3)), dict(eps=0.0), dict(B=0)):
         bd, kb = _lm(**bad)
@@ -194,6 +194,26 @@ def test_attn_fwd_rejects_bad_arguments(lib):
     assert f(FAKE, FAKE, FAKE, ctypes.byref(small), ctypes.byref(d), FAKE, FAKE, NULL) == 3
     neg, k6 = _desc(scale=-1.0)
     assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(neg), FAKE, FAKE, NULL) == 1
+
+
+def test_attn_layout_rejects_bad_strides(lib):
+    f = lib.gsa_attn_fwd
+    c = _csr(n=4)
+    good = (3 * 256 * 4 * 64, 64, 3 * 4 * 64, 256 * 4 * 64, 64, 4 * 64)
+    for i, bad in ((0, 12), (1, 0), (2, -64), (2, 32), (5, 8)):   # not a multiple of 8, <= 0, token stride < d
+        s = list(good)
+        s[i] = bad
+        lay = gsa._AttnLayout(*s)
+        d, keep = _desc()
+        d.layout = ctypes.cast(ctypes.pointer(lay), ctypes.c_void_p)
+        assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, NULL) == 1, (i, bad)
+    lay = gsa._AttnLayout(*good)
+    d32, keep = _desc(dtype=0)
+    d32.layout = ctypes.cast(ctypes.pointer(lay), ctypes.c_void_p)
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), ctypes.byref(d32), FAKE, FAKE, NULL) == 2   # float32: dense only
+    d, keep = _desc()
+    odd = ctypes.c_void_p(0x1008)                                 # bf16 tensors must be 16-byte aligned
+    assert f(odd, FAKE, FAKE, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, NULL) == 1
 
 
 def test_attn_bwd_rejects_bad_arguments(lib):
