@@ -76,26 +76,26 @@ struct Params {
 
 // ------------------------------------------------------------ D_t = dO·O
 
-// Grid (S H, L / kRowsPerCta): CTA (s H + h, y) takes the tokens
-// [y kRowsPerCta, (y + 1) kRowsPerCta) of sample s, head h (L is a multiple of 64).
+// Grid (L / kRowsPerCta, y): CTA (x, y) takes the tokens [x kRowsPerCta,
+// (x + 1) kRowsPerCta) of the (sample, head) pairs sh = y, y + gridDim.y, ...
+// (L is a multiple of 64; consecutive CTAs read consecutive rows).
 template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                   const __nv_bfloat16* __restrict__ dO, TokLayout lo, int64_t L,
-                                                  int H, float* __restrict__ dvec, int* __restrict__ ticket) {
+                                                  int H, int SH, float* __restrict__ dvec, int* __restrict__ ticket) {
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
     constexpr int kRowsPerCta = 256 / kTpr;
-    const int sh = blockIdx.x, s = sh / H, h = sh - s * H;
-    const int64_t l = static_cast<int64_t>(blockIdx.y) * kRowsPerCta + threadIdx.x / kTpr;
-    const int64_t row = static_cast<int64_t>(sh) * L + l;
+    const int64_t l = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
     const int part = threadIdx.x % kTpr;
-    float acc = 0.f;
-    {
+    for (int sh = blockIdx.y; sh < SH; sh += gridDim.y) {
+        const int s = sh / H, h = sh - s * H;
         const int64_t off = s * lo.s + h * lo.h + l * lo.l + part * 8;
         const uint4 a = *reinterpret_cast<const uint4*>(o + off);
         const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
         const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
         const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
+        float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 fa = __bfloat1622float2(ah[e]);
@@ -103,10 +103,10 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
             acc = fmaf(fa.x, fb.x, acc);
             acc = fmaf(fa.y, fb.y, acc);
         }
-    }
 #pragma unroll
-    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (part == 0) dvec[row] = acc;
+        for (int o2 = kTpr / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+        if (part == 0) dvec[static_cast<int64_t>(sh) * L + l] = acc;
+    }
 }
 
 // ------------------------------------------------------------ dQ
@@ -153,7 +153,7 @@ struct DqCfg {
     static_assert(kTmemCols * Shape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
-template <int D>
+template <int D, bool K4>   // K4: strided tensors through 4-D maps (see load_rows)
 __global__ void __launch_bounds__(Shape<D>::kThreads, Shape<D>::kCtasPerSm)
 dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
@@ -212,8 +212,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (blk < 0) continue;
             const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at) {
-                tma_load_4d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s);
-                tma_load_4d(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, l0, h, s);
+                load_rows<K4>(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s, head_row0);
+                load_rows<K4>(sDO + at * (128 * 128) + half * (kBlk * 128), &tmDO, q_full, at * 64, l0, h, s, head_row0);
             }
         }
     }
@@ -242,8 +242,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 mbar_arrive_expect_tx(&full[st], 2 * C::kKVBytes);
                 const int l0 = tl.list[n] * kBlk;   // token coordinate in the (sample, head)
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_4d(sK + st * C::kKVBytes + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s);
-                    tma_load_4d(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s);
+                    load_rows<K4>(sK + st * C::kKVBytes + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s, head_row0);
+                    load_rows<K4>(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s, head_row0);
                 }
             }
         }
@@ -376,7 +376,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, kErrTimeoutSoftmax))) {
             tc_fence_after();
             const bool has1 = C::G == 2 && T >= 2;   // dQ_1 holds products only if group 1 had a tile
-            __nv_bfloat16* orow = p.out0 + tok_off(tok, p.L, p.H, p.lq);
+            __nv_bfloat16* orow = p.out0 + (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D);
             constexpr int kOc = D / (C::G * H);   // output columns per thread (split among a row's threads)
             const int slot = grp * H + hc;
 #pragma unroll
@@ -448,7 +448,7 @@ struct DkvCfg {
     static_assert(kTmemCols * Shape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
-template <int D>
+template <int D, bool K4>   // K4: strided tensors through 4-D maps (see load_rows)
 __global__ void __launch_bounds__(Shape<D>::kThreads, Shape<D>::kCtasPerSm)
 dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Params p) {
@@ -515,8 +515,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if (blk < 0) continue;
             const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at) {
-                tma_load_4d(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, l0, h, s);
-                tma_load_4d(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, l0, h, s);
+                load_rows<K4>(sK + at * (128 * 128) + half * (kBlk * 128), &tmK, kv_full, at * 64, l0, h, s, head_row0);
+                load_rows<K4>(sV + at * (128 * 128) + half * (kBlk * 128), &tmV, kv_full, at * 64, l0, h, s, head_row0);
             }
         }
     }
@@ -546,8 +546,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const int64_t row64 = head_row0 + static_cast<int64_t>(tl.list[n]) * kBlk;
                 const int l0 = static_cast<int>(row64 - head_row0);   // token coordinate in the (sample, head)
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_4d(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, l0, h, s);
-                    tma_load_4d(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, l0, h, s);
+                    load_rows<K4>(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, l0, h, s, head_row0);
+                    load_rows<K4>(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, l0, h, s, head_row0);
                 }
                 bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
                 bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
@@ -718,7 +718,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int slot = grp * H + hc;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + tok_off(tok, p.L, p.H, p.lq);
+                __nv_bfloat16* orow = (which == 0 ? p.out0 : p.out1) + (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D);
                 const float mul = which == 0 ? 1.f : p.scale;
                 const uint32_t col0 = which == 0 ? C::dv_col(0) : C::dk_col(0);
                 const uint32_t col1 = which == 0 ? C::dv_col(1) : C::dk_col(1);
@@ -781,43 +781,45 @@ inline int sm_count() {
     return cached[dev];
 }
 
-template <int D>
+template <int D, bool K4>
 gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                     const __nv_bfloat16* o, const __nv_bfloat16* dO, const TokLayout& lo, Params pq, Params pkv,
                     int S, int H, int nblk, cudaStream_t st) {
     static std::once_flag once;
     std::call_once(once, [] {
-        cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemBytes);
-        cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvCfg<D>::kSmemBytes);
+        cudaFuncSetAttribute(dq_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemBytes);
+        cudaFuncSetAttribute(dkdv_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvCfg<D>::kSmemBytes);
     });
     constexpr int kRowsPerCta = 256 / (D / 8);   // 32 or 16: divides L
-    dot_kernel<D><<<dim3(static_cast<unsigned>(S * H), static_cast<unsigned>(pq.L / kRowsPerCta)), 256, 0, st>>>(
-        o, dO, lo, pq.L, pq.H, const_cast<float*>(pq.dvec), pkv.ticket);
+    const int sh_grid = S * H < 65535 ? S * H : 65535;
+    dot_kernel<D><<<dim3(static_cast<unsigned>(pq.L / kRowsPerCta), static_cast<unsigned>(sh_grid)), 256, 0, st>>>(
+        o, dO, lo, pq.L, pq.H, S * H, const_cast<float*>(pq.dvec), pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
     if (D == 64 && GSA_DQ_PERSIST) {
         static std::once_flag once_q;
         std::call_once(once_q, [] {
-            cudaFuncSetAttribute(dq_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqPCfg::kSmemBytes);
+            cudaFuncSetAttribute(dq_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DqPCfg::kSmemBytes);
         });
         const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
         const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
-        dq_persist_kernel<<<static_cast<unsigned>(ctas), DqPCfg::kThreads, DqPCfg::kSmemBytes, st>>>(tq, tk, tv,
-                                                                                                     tdo, pq);
+        dq_persist_kernel<K4><<<static_cast<unsigned>(ctas), DqPCfg::kThreads, DqPCfg::kSmemBytes, st>>>(tq, tk, tv,
+                                                                                                         tdo, pq);
     } else {
-        dq_kernel<D><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
+        dq_kernel<D, K4><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
     }
     if (D == 64 && GSA_DKV_PERSIST) {
         static std::once_flag once_p;
         std::call_once(once_p, [] {
-            cudaFuncSetAttribute(dkdv_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(dkdv_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  DkvPCfg::kSmemBytes);
         });
         const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
         const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
-        dkdv_persist_kernel<<<static_cast<unsigned>(ctas), DkvPCfg::kThreads, DkvPCfg::kSmemBytes, st>>>(
+        dkdv_persist_kernel<K4><<<static_cast<unsigned>(ctas), DkvPCfg::kThreads, DkvPCfg::kSmemBytes, st>>>(
             tq, tk, tv, tdo, pkv);
     } else {
-        dkdv_kernel<D><<<grid, Shape<D>::kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
+        dkdv_kernel<D, K4><<<grid, Shape<D>::kThreads, DkvCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pkv);
     }
     return cudaGetLastError() == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
 }
@@ -829,11 +831,13 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     if ((reinterpret_cast<uintptr_t>(lse) & 15u) || (reinterpret_cast<uintptr_t>(work) & 15u))
         return GSA_ERR_INVALID_ARGUMENT;
     const int64_t rows = static_cast<int64_t>(desc->B) * desc->H * desc->L;
+    // one load kind for all four inputs: 2-D maps only when every one is dense
+    const bool k4 = !is_dense(lq, desc->d, desc->L, desc->H) || !is_dense(lo, desc->d, desc->L, desc->H);
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq) ||
-        !make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq) ||
-        !make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq) ||
-        !make_tmap_tok(&tdo, dO, desc->d, desc->L, desc->H, desc->B, lo))
+    if (!make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
+        !make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
+        !make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
+        !make_tmap_tok(&tdo, dO, desc->d, desc->L, desc->H, desc->B, lo, k4))
         return GSA_ERR_CUDA;
     Params base{};
     base.lq = lq;
@@ -863,8 +867,10 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     const auto* ob = static_cast<const __nv_bfloat16*>(o);
     const auto* dob = static_cast<const __nv_bfloat16*>(dO);
     if (desc->d == 64)
-        return launch_d<64>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
-    return launch_d<128>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
+        return k4 ? launch_d<64, true>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st)
+                  : launch_d<64, false>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
+    return k4 ? launch_d<128, true>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st)
+              : launch_d<128, false>(tq, tk, tv, tdo, ob, dob, lo, pq, pkv, desc->B, desc->H, csr->nblk, st);
 }
 
 }  // namespace bwd

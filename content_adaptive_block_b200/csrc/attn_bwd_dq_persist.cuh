@@ -46,6 +46,7 @@ struct DqPCfg {
     static constexpr int kThreads = 64 + 256;
 };
 
+template <bool K4>   // strided tensors through 4-D maps (see load_rows)
 __global__ void __launch_bounds__(DqPCfg::kThreads, 2)
 dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -171,8 +172,8 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         const int blk = half ? qb : qa;
                         if (blk < 0) continue;
                         const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
-                        tma_load_4d(sQ + half * (kBlk * 128), &tmQ, qd_full, 0, l0, h_, s_);
-                        tma_load_4d(sDO + half * (kBlk * 128), &tmDO, qd_full, 0, l0, h_, s_);
+                        load_rows<K4>(sQ + half * (kBlk * 128), &tmQ, qd_full, 0, l0, h_, s_, head_row0);
+                        load_rows<K4>(sDO + half * (kBlk * 128), &tmDO, qd_full, 0, l0, h_, s_, head_row0);
                     }
                 }
                 int lastw = have ? nwords - 1 : -1;
@@ -195,8 +196,8 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         meta[st] = static_cast<uint32_t>(j) | (live << 16) | ((j == last_j ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes);
                         const int l0 = j * kBlk;   // token coordinate in the (sample, head)
-                        tma_load_4d(stage_k(st), &tmK, &full[st], 0, l0, h_, s_);
-                        tma_load_4d(stage_v(st), &tmV, &full[st], 0, l0, h_, s_);
+                        load_rows<K4>(stage_k(st), &tmK, &full[st], 0, l0, h_, s_, head_row0);
+                        load_rows<K4>(stage_v(st), &tmV, &full[st], 0, l0, h_, s_, head_row0);
                         ++gt;
                     }
                 }
@@ -367,7 +368,7 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(acc_free);   // dQ may take the next item's products
-                    if (my_blk >= 0) store_scaled_bf16(p.out0 + tok_off(tok, p.L, p.H, p.lq) + c0, ov, p.scale);
+                    if (my_blk >= 0) store_scaled_bf16(p.out0 + (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D) + c0, ov, p.scale);
                     break;
                 }
             }

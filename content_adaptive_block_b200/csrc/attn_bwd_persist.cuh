@@ -59,6 +59,7 @@ struct DkvPCfg {
     static constexpr int kThreads = 64 + 256;
 };
 
+template <bool K4>   // strided tensors through 4-D maps (see load_rows)
 __global__ void __launch_bounds__(DkvPCfg::kThreads, 2)
 dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -190,8 +191,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         const int blk = half ? kb : ka;
                         if (blk < 0) continue;
                         const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
-                        tma_load_4d(sK + half * (kBlk * 128), &tmK, kv_full, 0, l0, h_, s_);
-                        tma_load_4d(sV + half * (kBlk * 128), &tmV, kv_full, 0, l0, h_, s_);
+                        load_rows<K4>(sK + half * (kBlk * 128), &tmK, kv_full, 0, l0, h_, s_, head_row0);
+                        load_rows<K4>(sV + half * (kBlk * 128), &tmV, kv_full, 0, l0, h_, s_, head_row0);
                     }
                 }
                 int lastw = have ? nwords - 1 : -1;
@@ -214,8 +215,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         meta[st] = static_cast<uint32_t>(i) | (live << 16) | ((i == last_i ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes + 2 * C::kVecBytes);
                         const int64_t row64 = head_row0 + static_cast<int64_t>(i) * kBlk;
-                        tma_load_4d(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_);
-                        tma_load_4d(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_);
+                        load_rows<K4>(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
+                        load_rows<K4>(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
                         bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
                         bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
                         ++gt;
@@ -416,7 +417,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     mbar_arrive(acc_free);   // the accumulators may take the next item's products
                     if (my_blk >= 0) {
                         const int64_t tok = head_row0 + static_cast<int64_t>(my_blk) * kBlk + uu;
-                        const int64_t off = tok_off(tok, p.L, p.H, p.lq) + c0;
+                        const int64_t off = (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D) + c0;
                         store_scaled_bf16(p.out0 + off, ov, 1.f);
                         store_scaled_bf16(p.out1 + off, ok_, p.scale);
                     }

@@ -136,7 +136,7 @@ struct FwdCfg {
     static_assert(kTmemCols * FwdShape<D>::kCtasPerSm <= 512, "TMEM per SM");
 };
 
-template <int D>
+template <int D, bool K4>   // K4: strided tensors through 4-D maps (see load_rows)
 __global__ void __launch_bounds__(FwdShape<D>::kThreads, FwdShape<D>::kCtasPerSm)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -203,7 +203,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (blk < 0) continue;
             const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
             for (int at = 0; at < C::kAtoms; ++at)
-                tma_load_4d(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s);
+                load_rows<K4>(sQ + at * (128 * 128) + half * (kBlk * 128), &tmQ, q_full, at * 64, l0, h, s, head_row0);
         }
     }
     if (warp == 1) {
@@ -275,8 +275,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 uint8_t* dk = sK + st * C::kKVBytes;
                 uint8_t* dv = sV + st * C::kKVBytes;
                 for (int at = 0; at < C::kAtoms; ++at) {
-                    tma_load_4d(dk + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s);
-                    tma_load_4d(dv + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s);
+                    load_rows<K4>(dk + at * (kBlk * 128), &tmK, &full[st], at * 64, l0, h, s, head_row0);
+                    load_rows<K4>(dv + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s, head_row0);
                 }
             }
         }
@@ -468,7 +468,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const float inv = 1.f / lt;
             const bool store = my_blk >= 0;
             const int64_t tok = head_row0 + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
-            __nv_bfloat16* orow = p.o + tok_off(tok, p.L, p.H, p.lo);
+            __nv_bfloat16* orow = p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D);
 #pragma unroll
             for (int cb = grp * (D / C::G); cb < (grp + 1) * (D / C::G); cb += 32) {
                 float a[32];

@@ -153,6 +153,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Token-tile loads of Q, K, V and dO: K4 selects the 4-D map of a strided
+// layout (coordinates: column, token, head, sample); dense tensors use a 2-D
+// [S H L][d] map (row (s H + h) L + l), which measured ~1 % faster.
+template <bool K4>
+__device__ __forceinline__ void load_rows(void* dst, const CUtensorMap* map, uint64_t* bar, int col, int l0, int h,
+                                          int s, int64_t head_row0) {
+    if constexpr (K4) tma_load_4d(dst, map, bar, col, l0, h, s);
+    else tma_load_2d(dst, map, bar, col, static_cast<int>(head_row0 + l0));
+}
+
 // Element strides of a [sample][head][token][d] tensor whose d values of
 // one token are contiguous: the attention reads and writes Q, K, V, O, dO
 // and the gradients through such a layout (the dense [S][H][L][d] order, or
@@ -380,14 +390,30 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     return fn;
 }
 
+inline bool is_dense(const TokLayout& t, int64_t d, int64_t L, int64_t H) {
+    return t.l == d && t.h == L * d && t.s == H * L * d;
+}
+
 // A bf16 [S][H][L][d] tensor with layout t (element strides, multiples of 8)
 // as a 4-D map over (d, L, H, S), read in boxes of 64 tokens x 64 columns of
 // one (sample, head) with the 128-byte swizzle the UMMA descriptors below
 // expect; the box lands in shared memory as [64 tokens][128 B].
+// k4 false: the tensor is dense and gets the 2-D [S H L][d] map that
+// load_rows<false> reads.
 inline bool make_tmap_tok(CUtensorMap* map, const void* base, int64_t d, int64_t L, int64_t H, int64_t S,
-                          const TokLayout& t) {
+                          const TokLayout& t, bool k4) {
     auto fn = tmap_encoder();
     if (!fn) return false;
+    if (!k4) {
+        if (!is_dense(t, d, L, H)) return false;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(S * H * L)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+        cuuint32_t box[2] = {64, 64};
+        cuuint32_t estr[2] = {1, 1};
+        return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(H),
                           static_cast<cuuint64_t>(S)};
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(t.l) * 2, static_cast<cuuint64_t>(t.h) * 2,

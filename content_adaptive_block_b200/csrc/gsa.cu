@@ -93,6 +93,19 @@ gsa_status resolve_layout(const gsa_attn_desc* d, gsa::TokLayout* lq, gsa::TokLa
     return GSA_OK;
 }
 
+template <int D, bool K4>
+void launch_fwd(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const gsa::bf16::FwdParams& p, cudaStream_t cs) {
+    using C = gsa::bf16::FwdCfg<D>;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
+    });
+    gsa::bf16::attn_fwd_bf16_kernel<D, K4><<<grid, gsa::bf16::FwdShape<D>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv,
+                                                                                                        p);
+}
+
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
     if (!d || !csr || !d->head_classes) return GSA_ERR_INVALID_ARGUMENT;
     if (!csr_ok(csr)) return csr && csr->capacity < gsa_csr_capacity(csr->nblk) ? GSA_ERR_CAPACITY
@@ -304,10 +317,11 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     gsa::TokLayout lq, lo;
     st = resolve_layout(desc, &lq, &lo);
     if (st != GSA_OK) return st;
+    const bool k4 = !gsa::is_dense(lq, desc->d, desc->L, desc->H);
     CUtensorMap tq, tk, tv;
-    if (!gsa::make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq) ||
-        !gsa::make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq) ||
-        !gsa::make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq))
+    if (!gsa::make_tmap_tok(&tq, q, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
+        !gsa::make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
+        !gsa::make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq, k4))
         return GSA_ERR_CUDA;
     gsa::bf16::FwdParams p;
     p.row_ptr = csr->row_ptr;
@@ -324,23 +338,8 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     p.scale_log2 = scale * 1.4426950408889634f;
     std::memcpy(p.cls, cls, desc->H);
     dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
-    if (desc->d == 64) {
-        using C = gsa::bf16::FwdCfg<64>;
-        static std::once_flag once;
-        std::call_once(once, [] {
-            cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes);
-        });
-        gsa::bf16::attn_fwd_bf16_kernel<64><<<grid, gsa::bf16::FwdShape<64>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
-    } else {
-        using C = gsa::bf16::FwdCfg<128>;
-        static std::once_flag once;
-        std::call_once(once, [] {
-            cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-        });
-        gsa::bf16::attn_fwd_bf16_kernel<128><<<grid, gsa::bf16::FwdShape<128>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
-    }
+    if (desc->d == 64) k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
+    else k4 ? launch_fwd<128, true>(grid, tq, tk, tv, p, cs) : launch_fwd<128, false>(grid, tq, tk, tv, p, cs);
     return launch_status();
 }
 
