@@ -223,9 +223,9 @@ def run_reference(args, rank, world):
 # The kernels behind each timed call, and the sources whose hash ties a
 # recorded traffic figure to the code that produced it.
 _TRAFFIC_CALLS = {
-    "gsa_attn_fwd": (["attn_fwd_bf16_kernel<64>"],
+    "gsa_attn_fwd": (["attn_fwd_bf16_kernel<64, 0>"],
                      ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh"]),
-    "gsa_attn_bwd": (["dot_kernel<64>", "dq_persist_kernel", "dkdv_persist_kernel"],
+    "gsa_attn_bwd": (["dot_kernel<64>", "dq_persist_kernel<0>", "dkdv_persist_kernel<0>"],
                      ["content_adaptive_block_b200/csrc/attn_bwd_bf16.cuh",
                       "content_adaptive_block_b200/csrc/attn_bwd_persist.cuh",
                       "content_adaptive_block_b200/csrc/attn_bwd_dq_persist.cuh"]),
@@ -271,6 +271,51 @@ def record_traffic(csv_path, capture):
     with open(os.path.join(ROOT, "profiles", "traffic.json"), "w") as fh:
         json.dump(out, fh, indent=1)
     print(json.dumps(out))
+
+
+_MASK_INST_SOURCES = ["content_adaptive_block_b200/csrc/deflate_len.cuh", "content_adaptive_block_b200/csrc/common.cuh",
+                      "content_adaptive_block_b200/csrc/gsa.cu"]
+
+
+def _sources_hash(sources):
+    import hashlib
+    h = hashlib.sha256()
+    for s in sources:
+        with open(os.path.join(ROOT, s), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def record_mask_inst(csv_path, capture):
+    """Write profiles/mask_inst.json from an ncu raw-page CSV export of one
+    block_lengths_kernel launch on the headline mask point: warp instructions
+    executed per input byte, with the hash of the sources it was built from."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hdr, data = rows[0], rows[2:]
+    col = {h: i for i, h in enumerate(hdr)}
+    row = next(r for r in data if "block_lengths_kernel" in r[col["Kernel Name"]])
+    inst = float(row[col["smsp__inst_executed.sum"]].replace(",", ""))
+    wl = W.mask_sweep(*MASK_POINT)
+    nbytes = wl.S * wl.L
+    rec = {"kernel": "block_lengths_kernel", "workload": f"b{MASK_POINT[0]}_f{MASK_POINT[1]}: {wl.S} x {wl.L} bytes",
+           "warp_inst": inst, "bytes": nbytes, "inst_per_byte": inst / nbytes,
+           "issue_active_pct": float(row[col["smsp__issue_active.avg.pct_of_peak_sustained_active"]]),
+           "warps_active_pct": float(row[col["sm__warps_active.avg.pct_of_peak_sustained_active"]]),
+           "sources": _MASK_INST_SOURCES, "sha256": _sources_hash(_MASK_INST_SOURCES), "capture": capture}
+    with open(os.path.join(ROOT, "profiles", "mask_inst.json"), "w") as fh:
+        json.dump(rec, fh, indent=1)
+    return rec
+
+
+def _mask_inst_record():
+    """Warp instructions per input byte of the lengths kernel, if its sources are unchanged since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "mask_inst.json")) as fh:
+            rec = json.load(fh)
+        return rec if _sources_hash(rec["sources"]) == rec["sha256"] else None
+    except Exception:
+        return None
 
 
 def _traffic_record(kernel):
@@ -583,6 +628,18 @@ def mask_stage(gsa, dev):
             "hbm_frac": (nbytes + out_bytes) / (best_ms * 1e-3) / 1e9 / _peaks()["hbm_gbs"]}
     key = f"b{MASK_POINT[0]}_f{MASK_POINT[1]}"
     out["value"] = out["points"][key]["gbs"]
+    # the lengths kernel is bound by issue (serial parse and Huffman builds per
+    # block), not by its bytes: its roofline is the SM issue rate, 4 warp
+    # instructions per cycle per SM at the maximum clock
+    rec = _mask_inst_record()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = 4.0 * sms * _peaks()["sm_max_mhz"] * 1e6
+    achieved = rec["inst_per_byte"] * out["points"][key]["lengths_gbs"] * 1e9 if rec else None
+    out["roofline"] = {"kernel": "block_lengths_kernel", "bound": "alu", "unit": "warp-inst/s",
+                       "achieved": achieved, "peak": peak, "frac": achieved / peak if rec else None,
+                       "inst_per_byte": rec["inst_per_byte"] if rec else None,
+                       "hbm_frac": out["points"][key]["hbm_frac"],
+                       "note": "instructions per byte from profiles/mask_inst.json (null when the sources changed)"}
     out["workload"] = f"{key}: 256 x 8192 bytes, w=2"
     return out
 
@@ -786,6 +843,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-seq-sweep", action="store_true", help="skip the 4K..64K sequence-length sweep")
     ap.add_argument("--no-lm-block", action="store_true", help="skip the ByteLM block timing")
+    ap.add_argument("--record-mask-inst", metavar="CSV",
+                    help="write profiles/mask_inst.json from an ncu raw-page CSV export and exit")
     ap.add_argument("--no-mask-variants", action="store_true",
                     help="skip the gzip / BigBird / Longformer mask comparison")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
@@ -795,6 +854,9 @@ def main():
     args = ap.parse_args()
     if args.record_traffic:
         record_traffic(args.record_traffic, args.capture)
+        return 0
+    if args.record_mask_inst:
+        print(json.dumps(record_mask_inst(args.record_mask_inst, args.capture)))
         return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
