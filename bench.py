@@ -190,6 +190,32 @@ def cpu_baseline(wl, budget_s=12.0, seed=0):
                       f"turn), float64 numpy; {dt:.1f} s"}
 
 
+# ------------------------------------------------------------ ranks
+# Data-parallel with no exchange on the data path: every rank runs the whole
+# path on its own batch; the only collectives are a barrier around the timed
+# region and the max-over-ranks of the timed milliseconds.
+
+def rank_inputs(wl, rank):
+    """This rank's byte batch: the workload's generator seeded by the rank."""
+    return W.batch_bytes(wl, seed=rank)
+
+
+def max_over_ranks(ms, world, device):
+    """The largest of the ranks' timed milliseconds (a MAX all-reduce)."""
+    if world == 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, work_per_rank, ms_per_step):
+    """Work of all ranks per second at the slowest rank's step time (weak scaling)."""
+    return world * work_per_rank / (ms_per_step * 1e-3)
+
+
 def run_reference(args, rank, world):
     wl = W.WORKLOADS[WORKLOAD]
     if rank != 0:
@@ -350,7 +376,7 @@ def run_ours(args, rank, world, local_rank):
     hc = [int(c) for c in wl.head_classes()]
 
     # ---- inputs (per-rank seed), resident in HBM
-    x_host = W.batch_bytes(wl, seed=rank)
+    x_host = rank_inputs(wl, rank)
     x = torch.from_numpy(x_host).to(dev)
     q, k, v, do = W.qkv(wl, seed=rank, device=dev, grad=True)
     lengths = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
@@ -415,13 +441,9 @@ def run_ours(args, rank, world, local_rank):
     per_call = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(names))]
                          for i in range(args.steps)])
     step_ms = per_call.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_rate(world, step_flops, ms_per_step) / 1e12
 
     # ---- end to end through the API with host buffers
     e2e = None if args.no_e2e else e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev,
@@ -514,12 +536,8 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
     e1.record(stream)
     torch.cuda.synchronize()
     assert gsa.gsa_device_error() == 0, "a kernel gave up a bounded wait"
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    e2e_value = whole_job_rate(world, step_flops, e2e_ms) / 1e12
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": e2e_ms,
             "overlap": "uploads, compute and downloads of consecutive steps on three streams, "
