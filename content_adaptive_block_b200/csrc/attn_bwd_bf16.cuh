@@ -138,7 +138,7 @@ struct DqCfg {
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
     static constexpr int kOffBar = kOffV + kStages * kKVBytes;
     // full[st], empty[st], q_full, s_full[2], ds_full[2], done
-    static constexpr int kNumBars = 2 * kStages + 6;
+    static constexpr int kNumBars = 2 * kStages + 8;   // + drain[2]
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -171,6 +171,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     uint64_t* s_full = q_full + 1;
     uint64_t* ds_full = s_full + 2;
     uint64_t* done = ds_full + 2;   // one phase: every product of the CTA completed
+    uint64_t* drain = done + 1;     // [G] each group's MMA thread at exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -201,6 +202,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(&s_full[1], 1);
         mbar_init(&ds_full[0], 128 * Shape<D>::kHalves);
         mbar_init(&ds_full[1], 128 * Shape<D>::kHalves);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
@@ -231,10 +234,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     tc_fence_after();
     const int T = *tl.count;
     const uint32_t tmem = *tmem_slot;
+    int fills = 0;   // producer: stages issued
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int n = 0; n < T; ++n) {
+            int n = 0;
+            for (; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages &&
                     !mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer))
@@ -246,6 +251,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     load_rows<K4>(sV + st * C::kKVBytes + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s, head_row0);
                 }
             }
+            fills = n;
         }
     } else if (warp >= 2) {
         // warp e = warp - 2: group (e / 4) % G, column half (e / 4) / G
@@ -400,6 +406,20 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a role gave up a wait: the loads and products issued must land before
+        // shared memory and TMEM go (without one, every one of them was waited for)
+        if (warp == 0 && lane == 0) {
+            mbar_wait_drain(q_full, 0);
+            drain_fills(full, C::kStages, fills);
+        }
+        const int e4 = (warp - 2) >> 2;
+        if (warp >= 2 && ((warp - 2) & 3) == 0 && e4 / C::G == 0 && lane == 0) {   // each group's MMA thread
+            umma_commit(&drain[e4 % C::G]);
+            mbar_wait_drain(&drain[e4 % C::G], 0);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
@@ -423,7 +443,7 @@ struct DkvCfg {
     static constexpr int kOffVec = kOffStage + kStages * kStageBytes;   // per stage: LSE[64], D[64]
     static constexpr int kOffBar = kOffVec + kStages * 2 * kVecBytes;
     // full[st], empty[st], kv_full, s_full[2], p_full[2], acc[2], done
-    static constexpr int kNumBars = 2 * kStages + 8;
+    static constexpr int kNumBars = 2 * kStages + 10;   // + drain[2]
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffList = kOffMisc + 16;
     static constexpr int kOffLive = kOffList + kListMaxBlocks * 2;
@@ -466,6 +486,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* p_full = s_full + 2;
     uint64_t* acc = p_full + 2;     // d = 128: group g's dV/dK products of its latest tile completed
     uint64_t* done = acc + 2;       // one phase: every product of the CTA completed
+    uint64_t* drain = done + 1;     // [G] each group's MMA thread at exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     TileList tl;
@@ -504,6 +525,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(&p_full[1], 128 * Shape<D>::kHalves);
         mbar_init(&acc[0], 1);
         mbar_init(&acc[1], 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -534,10 +557,12 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     tc_fence_after();
     const int T = *tl.count;
     const uint32_t tmem = *tmem_slot;
+    int fills = 0;   // producer: stages issued
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int n = 0; n < T; ++n) {
+            int n = 0;
+            for (; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages &&
                     !mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer))
@@ -552,6 +577,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
                 bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
             }
+            fills = n;
         }
     } else if (warp >= 2) {
         // warp e = warp - 2: group (e / 4) % G, column half (e / 4) / G
@@ -744,6 +770,20 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a role gave up a wait: the loads and products issued must land before
+        // shared memory and TMEM go (without one, every one of them was waited for)
+        if (warp == 0 && lane == 0) {
+            mbar_wait_drain(kv_full, 0);
+            drain_fills(full, C::kStages, fills);
+        }
+        const int e4 = (warp - 2) >> 2;
+        if (warp >= 2 && ((warp - 2) & 3) == 0 && e4 / C::G == 0 && lane == 0) {   // each group's MMA thread
+            umma_commit(&drain[e4 % C::G]);
+            mbar_wait_drain(&drain[e4 % C::G], 0);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

@@ -45,7 +45,7 @@ struct DkvPCfg {
     static constexpr int kOffMeta = kOffVec + kStages * 2 * kVecBytes;  // per stage: block | live << 16 | last << 18
     static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
     // full[st], empty[st], kv_full, kv_free, s_full, p_full, acc_done, acc_free, item_full[2]
-    static constexpr int kNumBars = 2 * kStages + 8;
+    static constexpr int kNumBars = 2 * kStages + 9;   // + drain
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
     static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
@@ -86,6 +86,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // elementwise thread to have finished the slot's previous item, so no
     // waiter is ever two phases behind
     uint64_t* item_full = acc_free + 1;
+    uint64_t* drain = item_full + 2;             // the MMA thread's products at exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // [2] item of phase k at rec[k & 1], -1: end
@@ -126,6 +127,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(acc_free, 256);
         mbar_init(&item_full[0], 1);
         mbar_init(&item_full[1], 1);
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -142,10 +144,12 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    int fills = 0, loads = 0;   // producer (lane 0): stages and item tiles issued
     if (warp == 0) {
         // ================= producer: per item its query list, K and V, then one stage per query block
         const int nwords = (nblk + 31) >> 5;
         int gt = 0;   // stages issued so far, across items
+        int nload = 0;   // items whose tile load was issued (lane 0)
         bool ok = true;
         for (int k = 0; ok; ++k) {
             int it = 0;
@@ -186,6 +190,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 rec[k & 1] = (ok && have) ? it : -1;
                 mbar_arrive(&item_full[k & 1]);
                 if (ok && have) {
+                    ++nload;
                     mbar_arrive_expect_tx(kv_full, (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
                     for (int half = 0; half < 2; ++half) {
                         const int blk = half ? kb : ka;
@@ -228,6 +233,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             __syncwarp();   // the bitmaps are rewritten for the next item
             if (!have) break;
         }
+        fills = gt;
+        loads = nload;
     } else if (warp >= 2) {
         // ================= elementwise: two warpgroups splitting the 64 query columns
         constexpr int kCols = 32, kW = 8;
@@ -428,6 +435,19 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a role gave up a wait: the loads and products issued must land before
+        // shared memory and TMEM go (without one, every one of them was waited for)
+        if (warp == 0 && lane == 0) {
+            if (loads > 0) mbar_wait_drain(kv_full, (loads - 1) & 1);
+            drain_fills(full, C::kStages, fills);
+        }
+        if (warp == 2 && lane == 0) {
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

@@ -261,11 +261,14 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     tc_fence_after();
     const int T = *ntiles_slot;
     const uint32_t tmem = *tmem_slot;
+    int fills = 0;          // producer: K / V stages issued
+    int issued_qk = 0, issued_pv = 0;   // MMA thread: QK^T and P V products issued
 
     if (warp == 0) {
         // ================= TMA producer
         if (lane == 0) {
-            for (int n = 0; n < T; ++n) {
+            int n = 0;
+            for (; n < T; ++n) {
                 const int st = n % C::kStages;
                 if (n >= C::kStages) {
                     if (!mbar_wait(&empty[st], ((n / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer)) break;
@@ -279,6 +282,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     load_rows<K4>(dv + at * (kBlk * 128), &tmV, &full[st], at * 64, l0, h, s, head_row0);
                 }
             }
+            fills = n;
         }
     } else if (warp == 1) {
         // ================= MMA issuer
@@ -292,7 +296,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             // its k-th, S buffer k % NS) once its K/V stage is loaded and the
             // group has read that buffer's previous scores; P V of tile na once
             // the group's P is in TMEM.
-            int ns = 0, na = 0;
+            int ns = 0, na = 0;   // QK^T and P V products issued
             PollGuard guard;
             while (ok && na < T) {
                 bool moved = false;
@@ -337,6 +341,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
             }
             if (ok && T > 0) umma_commit(done);
+            issued_qk = ns;
+            issued_pv = na;
         }
         __syncwarp();
     } else {
@@ -494,6 +500,25 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a role gave up a wait: the loads and products issued must land before
+        // shared memory and TMEM go (without one, every one of them was waited for)
+        if (warp == 0 && lane == 0) drain_fills(full, C::kStages, fills);
+        if (warp == 1 && lane == 0) {
+            // tcgen05 products complete in issue order: the phases the last QK^T
+            // and the last P V committed cover every earlier one
+            mbar_wait_drain(q_full, 0);
+            if (issued_qk > 0) {
+                const int n = issued_qk - 1, kq = n / G;
+                mbar_wait_drain(&s_full[(n % G) * NS + kq % NS], (kq / NS) & 1);
+            }
+            if (issued_pv > 0) {
+                const int n = issued_pv - 1;
+                mbar_wait_drain(&p_free[n % G], (n / G) & 1);
+            }
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

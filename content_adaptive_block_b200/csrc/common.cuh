@@ -127,6 +127,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Wait for a phase at a role's exit whatever *abort says, at most
+// kWaitLimitNs: the copies and products a CTA issued must land before it
+// frees its shared memory and TMEM, also when it is giving up.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(kErrTimeoutOther);
+            return false;
+        }
+    }
+}
+
+// The fills 0 .. n-1 of a ring of `stages` slots (fill i into slot i % stages,
+// phase i / stages): the last fill of each slot lands after the earlier ones.
+__device__ __forceinline__ void drain_fills(uint64_t* full, int stages, int n) {
+    for (int st = 0; st < stages && st < n; ++st) {
+        const int last = st + ((n - 1 - st) / stages) * stages;
+        mbar_wait_drain(&full[st], (last / stages) & 1);
+    }
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
