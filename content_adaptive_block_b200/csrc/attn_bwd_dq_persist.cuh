@@ -271,7 +271,7 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const int my_blk = half ? qb : qa;
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + rr;
-            const float lse2 = my_blk >= 0 ? p.lse[tok] * kLog2e : 0.f;
+            const float lse2 = my_blk >= 0 ? p.lse2[tok] : 0.f;
             const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
             for (int ti = 0; ok; ++ti, ++gt) {
                 const int st = gt % C::kStages;

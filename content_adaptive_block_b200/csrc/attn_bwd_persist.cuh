@@ -222,7 +222,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         const int64_t row64 = head_row0 + static_cast<int64_t>(i) * kBlk;
                         load_rows<K4>(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
                         load_rows<K4>(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
-                        bulk_load(stage_lse(st), p.lse + row64, C::kVecBytes, &full[st]);
+                        bulk_load(stage_lse(st), p.lse2 + row64, C::kVecBytes, &full[st]);
                         bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
                         ++gt;
                     }
@@ -339,7 +339,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int cc = 4 * c4 + e;
-                                float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e] * kLog2e));
+                                float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e]));
                                 if (first > cb) pr = cb + cc >= first ? pr : 0.f;
                                 s_[cc] = pr;
                                 d_[cc] = pr * (d_[cc] - dd[e]);

@@ -39,8 +39,8 @@ gsa_status launch_status() {
 // cannot afford cudaMalloc's implicit synchronisation).  For them the
 // backward's per-row scratch (D_t = dO_t · O_t, float32) lives in this
 // fixed array, which every GPU that loads the library holds until exit.
-constexpr int64_t kNoAllocRows = int64_t(1) << 21;   // query rows (B*H*L); 8 MiB
-static __device__ __align__(256) float g_bwd_noalloc_scratch[kNoAllocRows + 64];   // D, then a work counter
+constexpr int64_t kNoAllocRows = int64_t(1) << 21;   // query rows (B*H*L); 16 MiB
+static __device__ __align__(256) float g_bwd_noalloc_scratch[2 * kNoAllocRows + 64];   // D, LSE log2(e), counters
 constexpr int kMaxDevices = 64;
 
 // Device address of the scratch array on the current device, looked up once
@@ -346,7 +346,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
 size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc) {
     if (!desc || desc->B < 1 || desc->H < 1 || desc->L < 1) return 0;
     const size_t rows = static_cast<size_t>(desc->B) * desc->H * desc->L;
-    return sizeof(float) * ((rows + 63) & ~size_t(63)) + 256;   // D, then a work counter
+    return 2 * sizeof(float) * ((rows + 63) & ~size_t(63)) + 256;   // D, LSE log2(e), then work counters
 }
 
 gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,

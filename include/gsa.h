@@ -265,8 +265,8 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
  *   dV = P^T dO,  dS = P ∘ (dO V^T − D),  dQ = scale · dS K,  dK = scale · dS^T Q,
  * every sum over live pairs only.  o and lse are the forward's outputs.
  *   workspace: device scratch of at least gsa_attn_bwd_workspace(desc) bytes
- *              (holds D, float32 [B][H][L], then a work counter); its
- *              contents need no init.
+ *              (holds D and LSE log2(e), float32 [B][H][L] each, then two
+ *              work counters); its contents need no init.
  * dq, dk, dv are written (not accumulated).  Deterministic: each output row
  * is summed by one CTA in a fixed order (the only atomic hands out work
  * items).
@@ -287,9 +287,9 @@ size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc);
  * that hands out every device byte from its pool and forbids other
  * allocations) or cannot afford cudaMalloc's implicit device
  * synchronisation in their loop.  This call needs no workspace argument: its
- * float32 scratch (D_t, one value per query row) is a fixed array compiled
+ * float32 scratch (D_t and LSE_t log2(e), two values per query row) is a fixed array compiled
  * into the library, at most gsa_attn_bwd_noalloc_max_rows() rows
- * (2^21 = B*H*L; 8 MiB, held on every GPU that loads the library until the
+ * (2^21 = B*H*L; 16 MiB, held on every GPU that loads the library until the
  * process exits).  The caller still passes all inputs and outputs, exactly as
  * for gsa_attn_bwd; results are identical.
  *   - Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
