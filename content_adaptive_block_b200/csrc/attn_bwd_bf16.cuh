@@ -24,6 +24,9 @@
 // The bf16 operands written by the elementwise warps stay in TMEM as packed
 // pairs (lane = row, column c = elements 2c, 2c+1), the layout of an M=128
 // A operand, so they never pass through shared memory.
+// At d = 64, steps 2 and 3 run as persistent kernels over the same items
+// (dq_persist_kernel, two CTAs per SM; dkdv_persist_kernel, one CTA per SM
+// with double-buffered scores): attn_bwd_dq_persist.cuh, attn_bwd_persist.cuh.
 #pragma once
 
 #include "common.cuh"
@@ -855,14 +858,14 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     } else {
         dq_kernel<D, K4><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
     }
-    if (D == 64 && GSA_DKV_PERSIST) {
+    if (D == 64 && GSA_DKV_PERSIST) {   // one CTA per SM, double-buffered scores
         static std::once_flag once_p;
         std::call_once(once_p, [] {
             cudaFuncSetAttribute(dkdv_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  DkvPCfg::kSmemBytes);
         });
         const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
-        const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
+        const int64_t ctas = items < sm_count() ? items : sm_count();
         dkdv_persist_kernel<K4><<<static_cast<unsigned>(ctas), DkvPCfg::kThreads, DkvPCfg::kSmemBytes, st>>>(
             tq, tk, tv, tdo, pkv);
     } else {

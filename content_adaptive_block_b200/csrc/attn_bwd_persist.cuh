@@ -1,34 +1,44 @@
-// dK, dV at d = 64 with persistent CTAs.
+// dK, dV at d = 64: one persistent CTA per SM with double-buffered scores.
 //
 // Same products and elementwise arithmetic as dkdv_kernel (see
 // attn_bwd_bf16.cuh): per key tile (two key blocks from the class's key
 // pairing order) over the union of their CSC columns, S^T = K Q^T and
 // dP^T = V dO^T into TMEM, P^T = exp2(S^T c - LSE log2 e) and dS^T = P^T ∘
-// (dP^T - D) by the elementwise warps (two warpgroups splitting the 64 query
-// columns), packed back into TMEM over the scores they replace, then
-// dV += P^T dO and dK += dS^T Q with A from TMEM.
+// (dP^T - D) by the elementwise warps, packed back into TMEM over the scores
+// they replace, then dV += P^T dO and dK += dS^T Q with A from TMEM.
 //
-// What differs: a fixed grid of CTAs (two per SM) takes the work items —
-// (sample·head, key tile) in the heaviest-first order of the plain launch —
-// one at a time from a device counter (dot_kernel zeroes it), and the items
-// follow each other without a gap.  The producer publishes each item (or the
-// end) in a two-slot record ring behind an mbarrier.  The producer
-// warp merges an item's query list itself (a private bitmap, no CTA
-// barrier) and streams the item's Q, dO, LSE and D stages straight after the
-// previous item's, each stage carrying its query block, live bits and an
-// "item's last tile" mark in a word of shared memory; it reloads the K and V
-// tile once the previous item's last S^T, dP^T products completed.  The MMA
-// issuer waits for the previous item's epilogue to have read dV and dK
-// before the new item's first accumulating product.  Phases follow a tile
-// counter running across items.  Every wait is bounded; on a timeout the
-// CTA records an error code and every role leaves.
+// Work: a fixed grid of CTAs (one per SM) takes the work items — (sample·head,
+// key tile) in the heaviest-first order of the plain launch — one at a time
+// from a device counter (dot_kernel zeroes it), with no gap between items.
+// The producer warp publishes each item (or the end) in a two-slot record
+// ring behind mbarriers, merges the item's query list itself (a private
+// bitmap, no CTA barrier) and streams its Q, dO, LSE and D stages straight
+// after the previous item's; each stage carries its query block, live bits
+// and an "item's last tile" mark in a word of shared memory.  K and V are
+// double-buffered per item, so the next item's tile loads while the current
+// one finishes.
+//
+// Overlap: the CTA holds all 512 TMEM columns, two S^T / dP^T buffers, so the
+// scores of tile n + 2 are issued right after the dV, dK products of tile n
+// and are computed while the elementwise warps work on tile n + 1.  Four
+// warpgroups split each tile's 64 query columns into quarters.  Two threads
+// on different warps issue the MMAs, one for S^T and dV, one for dP^T and dK,
+// so each accumulator still sees its products in one fixed order (the result
+// is deterministic) while issue, which dominates with one thread sharing its
+// scheduler with elementwise warps, runs on two schedulers.  The issuers wait
+// for the previous item's epilogue to have read dV and dK before the new
+// item's first accumulating product.  Phases follow a tile counter running
+// across items.  Every wait is bounded; on a timeout the CTA records an error
+// code, drains its loads and products in flight and every role leaves.
+// TMEM: buffer b at 128 b (S^T at +0 with P^T packed over each quarter's
+// first 8 columns, dP^T at +64 with dS^T likewise), dV at 256, dK at 320.
 #pragma once
 
 namespace gsa {
 namespace bwd {
 
 #ifndef GSA_DKVP_STAGES
-#define GSA_DKVP_STAGES 4
+#define GSA_DKVP_STAGES 5
 #endif
 
 struct DkvPCfg {
@@ -38,60 +48,60 @@ struct DkvPCfg {
     static constexpr int kQBytes = kBlk * D * 2;        // one query block of Q or dO
     static constexpr int kVecBytes = kBlk * 4;          // LSE or D of one query block
     static constexpr int kStageBytes = 2 * kQBytes;     // stage: Q, dO (TMA, 1024-aligned)
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = kOffK + kTileBytes;
-    static constexpr int kOffStage = kOffV + kTileBytes;
+    static constexpr int kOffKV = 0;                    // [2 items][K, V]
+    static constexpr int kOffStage = kOffKV + 4 * kTileBytes;
     static constexpr int kOffVec = kOffStage + kStages * kStageBytes;   // per stage: LSE[64], D[64]
     static constexpr int kOffMeta = kOffVec + kStages * 2 * kVecBytes;  // per stage: block | live << 16 | last << 18
     static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
-    // full[st], empty[st], kv_full, kv_free, s_full, p_full, acc_done, acc_free, item_full[2]
-    static constexpr int kNumBars = 2 * kStages + 9;   // + drain
+    // full[st], empty[st], kv_full[2], kv_free[2], s_full[2], p_full[2], acc_done, acc_free,
+    // item_full[2], rec_free[2], drain
+    static constexpr int kNumBars = 2 * kStages + 17;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
     static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
-    static_assert(kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
-    static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
-    static constexpr int kTmemCols = 256;
-    // S^T at 0 (P^T packed over its columns 0..15 and 32..47), dP^T at 64
-    // (dS^T likewise), dV at 128, dK at 192
-    static constexpr uint32_t kTmemDV = 128, kTmemDK = 192;
-    static constexpr int kThreads = 64 + 256;
+    static_assert(kSmemBytes <= 232448 - 1024, "shared memory per CTA");
+    static_assert(kStageBytes % 1024 == 0 && kTileBytes % 1024 == 0, "1024-byte alignment");
+    static constexpr int kTmemCols = 512;
+    static constexpr uint32_t kTmemDV = 256, kTmemDK = 320;
+    static constexpr int kEw = 512;                     // elementwise threads (warps 2 .. 17)
+    static constexpr int kThreads = 64 + kEw + 32;      // + warp 18: the second MMA issuer
 };
 
 template <bool K4>   // strided tensors through 4-D maps (see load_rows)
-__global__ void __launch_bounds__(DkvPCfg::kThreads, 2)
+__global__ void __launch_bounds__(DkvPCfg::kThreads, 1)
 dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const Params p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                     const Params p) {
     using C = DkvPCfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* sK = smem + C::kOffK;
-    uint8_t* sV = smem + C::kOffV;
     uint8_t* sStage = smem + C::kOffStage;
     uint32_t* meta = reinterpret_cast<uint32_t*>(smem + C::kOffMeta);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
     uint64_t* empty = bars + C::kStages;
-    uint64_t* kv_full = bars + 2 * C::kStages;   // phase per item: K, V of the item loaded
-    uint64_t* kv_free = kv_full + 1;             // phase per item: its last S^T, dP^T completed
-    uint64_t* s_full = kv_free + 1;              // phase per tile: S^T, dP^T landed
-    uint64_t* p_full = s_full + 1;               // phase per tile: P^T, dS^T in TMEM (256 arrivals)
-    uint64_t* acc_done = p_full + 1;             // phase per item: its last dV, dK products completed
-    uint64_t* acc_free = acc_done + 1;           // phase per item: its epilogue read dV, dK (256 arrivals)
-    // [2] item k's record (or the end) published: barrier k & 1, phase k >> 1.  One
-    // barrier per record slot: publishing into a slot again needs every
-    // elementwise thread to have finished the slot's previous item, so no
-    // waiter is ever two phases behind
-    uint64_t* item_full = acc_free + 1;
-    uint64_t* drain = item_full + 2;             // the MMA thread's products at exit
+    uint64_t* kv_full = bars + 2 * C::kStages;   // [item & 1], phase item >> 1: K, V of the item loaded
+    uint64_t* kv_free = kv_full + 2;             // [item & 1], phase item >> 1: its last S^T, dP^T completed
+    uint64_t* s_full = kv_free + 2;              // [tile & 1], phase tile >> 1: S^T, dP^T landed
+    // [tile & 1], phase tile >> 1: P^T, dS^T in TMEM (512 arrivals).  Two, because the
+    // issuer is not one of the arriving threads: the elementwise warps may finish tile
+    // n + 1 before the issuer waits for tile n, but not tile n + 2 (its scores are
+    // issued after that wait)
+    uint64_t* p_full = s_full + 2;
+    uint64_t* acc_done = p_full + 2;             // phase per item: its last dV, dK products completed
+    uint64_t* acc_free = acc_done + 1;           // phase per item: its epilogue read dV, dK (512 arrivals)
+    uint64_t* item_full = acc_free + 1;          // [item & 1], phase item >> 1: the item's record published
+    uint64_t* rec_free = item_full + 2;          // [item & 1], phase item >> 1: every elementwise thread read it
+    uint64_t* drain = rec_free + 2;              // the MMA thread's products at exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-    int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // [2] item of phase k at rec[k & 1], -1: end
+    int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // [2] item k at rec[k & 1], -1: end
     uint32_t* bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
     uint32_t* bitsB = bitsA + kListMaxBlocks / 32;
+    auto tile_k = [&](int b) { return smem + C::kOffKV + b * 2 * C::kTileBytes; };
+    auto tile_v = [&](int b) { return smem + C::kOffKV + b * 2 * C::kTileBytes + C::kTileBytes; };
     auto stage_q = [&](int st) { return sStage + st * C::kStageBytes; };
     auto stage_do = [&](int st) { return sStage + st * C::kStageBytes + C::kQBytes; };
     auto stage_lse = [&](int st) { return reinterpret_cast<float*>(smem + C::kOffVec + st * 2 * C::kVecBytes); };
@@ -115,19 +125,23 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     };
 
     if (threadIdx.x == 0) {
+        // two MMA issuers commit to the barriers of products: empty, kv_free, s_full, acc_done, drain
         for (int st = 0; st < C::kStages; ++st) {
             mbar_init(&full[st], 1);
-            mbar_init(&empty[st], 1);
+            mbar_init(&empty[st], 2);
         }
-        mbar_init(kv_full, 1);
-        mbar_init(kv_free, 1);
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 256);
-        mbar_init(acc_done, 1);
-        mbar_init(acc_free, 256);
-        mbar_init(&item_full[0], 1);
-        mbar_init(&item_full[1], 1);
-        mbar_init(drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&kv_full[b], 1);
+            mbar_init(&kv_free[b], 2);
+            mbar_init(&s_full[b], 2);
+            mbar_init(&item_full[b], 1);
+            mbar_init(&rec_free[b], C::kEw);
+        }
+        mbar_init(&p_full[0], C::kEw);
+        mbar_init(&p_full[1], C::kEw);
+        mbar_init(acc_done, 2);
+        mbar_init(acc_free, C::kEw);
+        mbar_init(drain, 2);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -149,7 +163,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= producer: per item its query list, K and V, then one stage per query block
         const int nwords = (nblk + 31) >> 5;
         int gt = 0;   // stages issued so far, across items
-        int nload = 0;   // items whose tile load was issued (lane 0)
+        int nload = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             int it = 0;
@@ -183,24 +197,27 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
             const int s_ = sh / p.H, h_ = sh - s_ * p.H;   // the 4-D maps' head and sample
             if (lane == 0) {
-                // the record slot k & 1 and the K, V tile are free once the previous
-                // item's last S^T, dP^T completed (every reader of the slot's old
-                // record had read it before that product was issued)
-                if (k >= 1 && !mbar_wait(kv_free, (k - 1) & 1, abort_flag, kErrTimeoutProducer)) ok = false;
+                // record slot and K / V buffer k & 1 held item k - 2: every elementwise
+                // thread has read its record, and its last S^T, dP^T completed
+                if (k >= 2 && !(mbar_wait(&rec_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer) &&
+                                mbar_wait(&kv_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer)))
+                    ok = false;
                 rec[k & 1] = (ok && have) ? it : -1;
                 mbar_arrive(&item_full[k & 1]);
                 if (ok && have) {
                     ++nload;
-                    mbar_arrive_expect_tx(kv_full, (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
+                    mbar_arrive_expect_tx(&kv_full[k & 1], (kb >= 0 ? 2 : 1) * 2 * kBlk * D * 2);
                     for (int half = 0; half < 2; ++half) {
                         const int blk = half ? kb : ka;
                         if (blk < 0) continue;
                         const int l0 = blk * kBlk;   // token coordinate in the (sample, head)
-                        load_rows<K4>(sK + half * (kBlk * 128), &tmK, kv_full, 0, l0, h_, s_, head_row0);
-                        load_rows<K4>(sV + half * (kBlk * 128), &tmV, kv_full, 0, l0, h_, s_, head_row0);
+                        load_rows<K4>(tile_k(k & 1) + half * (kBlk * 128), &tmK, &kv_full[k & 1], 0, l0, h_, s_,
+                                      head_row0);
+                        load_rows<K4>(tile_v(k & 1) + half * (kBlk * 128), &tmV, &kv_full[k & 1], 0, l0, h_, s_,
+                                      head_row0);
                     }
                 }
-                int lastw = have ? nwords - 1 : -1;
+                int lastw = (ok && have) ? nwords - 1 : -1;
                 while (lastw >= 0 && (bitsA[lastw] | bitsB[lastw]) == 0u) --lastw;
                 const int last_i = lastw >= 0 ? 32 * lastw + 31 - __clz(bitsA[lastw] | bitsB[lastw]) : -1;
                 for (int w = 0; ok && w <= lastw; ++w) {
@@ -219,9 +236,10 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         const uint32_t live = ((ua >> bit) & 1u) | (((ub >> bit) & 1u) << 1);
                         meta[st] = static_cast<uint32_t>(i) | (live << 16) | ((i == last_i ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes + 2 * C::kVecBytes);
-                        const int64_t row64 = head_row0 + static_cast<int64_t>(i) * kBlk;
-                        load_rows<K4>(stage_q(st), &tmQ, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
-                        load_rows<K4>(stage_do(st), &tmDO, &full[st], 0, static_cast<int>(row64 - head_row0), h_, s_, head_row0);
+                        const int l0 = i * kBlk;
+                        const int64_t row64 = head_row0 + l0;
+                        load_rows<K4>(stage_q(st), &tmQ, &full[st], 0, l0, h_, s_, head_row0);
+                        load_rows<K4>(stage_do(st), &tmDO, &full[st], 0, l0, h_, s_, head_row0);
                         bulk_load(stage_lse(st), p.lse2 + row64, C::kVecBytes, &full[st]);
                         bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
                         ++gt;
@@ -235,53 +253,17 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         fills = gt;
         loads = nload;
-    } else if (warp >= 2) {
-        // ================= elementwise: two warpgroups splitting the 64 query columns
-        constexpr int kCols = 32, kW = 8;
-        const int hc = (warp - 2) >> 2;           // query columns [32 hc, 32 hc + 32)
-        const int c0 = kCols * hc;
+    } else if (warp >= 2 && warp < 18) {
+        // ================= elementwise: four warpgroups, one per quarter of the 64 query columns
+        constexpr int kCols = 16, kW = 8;
+        const int qc = (warp - 2) >> 2;           // query columns [16 qc, 16 qc + 16)
+        const int c0 = kCols * qc;
         const int quad = warp & 3;
         const int u = quad * 32 + lane;           // key row of the tile = TMEM lane
         const int half = u >> 6;
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const bool issuer_warp = warp == 2;       // lane 0 issues every MMA of the CTA
-        constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
-        constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
-        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-        auto issue_s = [&](int st) {   // S^T = K Q^T, dP^T = V dO^T of the stage's query block
-            const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t ak = sdesc_sw128(aK + kk * 32, 16, 1024);
-                const uint64_t bq = sdesc_sw128(aQs + kk * 32, 16, 1024);
-                umma_bf16(tmem, ak, bq, idesc_s, kk > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t av = sdesc_sw128(aV + kk * 32, 16, 1024);
-                const uint64_t bdo = sdesc_sw128(aDOs + kk * 32, 16, 1024);
-                umma_bf16(tmem + 64, av, bdo, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(s_full);
-            if ((meta[st] >> 18) & 1u) umma_commit(kv_free);   // the item's K, V are no longer read
-        };
         bool ok = true;
-        if (issuer_warp) {
-            if (lane == 0) {
-                // the first item's first S^T, dP^T
-                ok = mbar_wait(&item_full[0], 0, abort_flag, kErrTimeoutMma);
-                if (ok && rec[0] >= 0) {
-                    ok = mbar_wait(kv_full, 0, abort_flag, kErrTimeoutMma) &&
-                         mbar_wait(&full[0], 0, abort_flag, kErrTimeoutMma);
-                    if (ok) {
-                        tc_fence_after();
-                        issue_s(0);
-                    }
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-        }
         int gt = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
             if (!__all_sync(0xffffffffu, mbar_wait(&item_full[k & 1], (k >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
@@ -289,6 +271,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 break;
             }
             const int it = rec[k & 1];
+            mbar_arrive(&rec_free[k & 1]);   // the slot may take item k + 2
             if (it < 0) break;
             int sh, ka, kb;
             int64_t g;
@@ -297,7 +280,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
             for (int ti = 0; ok; ++ti, ++gt) {
                 const int st = gt % C::kStages;
-                bool w_ok = mbar_wait(s_full, gt & 1, abort_flag, kErrTimeoutSoftmax);
+                const uint32_t tb = tlane + 128 * (gt & 1);   // this tile's S^T / dP^T buffer
+                bool w_ok = mbar_wait(&s_full[gt & 1], (gt >> 1) & 1, abort_flag, kErrTimeoutSoftmax);
                 w_ok = w_ok && mbar_wait(&full[st], (gt / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
                 if (!__all_sync(0xffffffffu, w_ok)) {
                     ok = false;
@@ -311,24 +295,27 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 // query columns allowed: live block, and in the diagonal block t >= u
                 const int first = !is_live ? kBlk : (i == my_blk ? uu : 0);
                 uint32_t pp[kCols / 2], pd[kCols / 2];
-                if (first >= c0 + kCols) {
+                // the TMEM loads are warp-collective: skip them only when the whole
+                // warp's rows start past this quarter (the diagonal's first column
+                // varies across the warp's lanes; the element mask below covers it)
+                if (__all_sync(0xffffffffu, first >= c0 + kCols)) {
 #pragma unroll
                     for (int e = 0; e < kCols / 2; ++e) pp[e] = pd[e] = 0u;
                 } else {
                     const float4* lse4 = reinterpret_cast<const float4*>(stage_lse(st));
                     const float4* dv4 = reinterpret_cast<const float4*>(stage_d(st));
                     float sv[2][kW], dp[2][kW];
-                    tmem_ldw<kW>(tlane + c0, sv[0]);
-                    tmem_ldw<kW>(tlane + 64 + c0, dp[0]);
+                    tmem_ldw<kW>(tb + c0, sv[0]);
+                    tmem_ldw<kW>(tb + 64 + c0, dp[0]);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
+                    for (int ch = 0; ch < 2; ++ch) {
                         tmem_wait_ld();
-                        if (ch < 3) {
-                            tmem_ldw<kW>(tlane + c0 + kW * (ch + 1), sv[(ch + 1) & 1]);
-                            tmem_ldw<kW>(tlane + 64 + c0 + kW * (ch + 1), dp[(ch + 1) & 1]);
+                        if (ch < 1) {
+                            tmem_ldw<kW>(tb + c0 + kW, sv[1]);
+                            tmem_ldw<kW>(tb + 64 + c0 + kW, dp[1]);
                         }
-                        float* s_ = sv[ch & 1];
-                        float* d_ = dp[ch & 1];
+                        float* s_ = sv[ch];
+                        float* d_ = dp[ch];
                         const int cb = c0 + kW * ch;
 #pragma unroll
                         for (int c4 = 0; c4 < kW / 4; ++c4) {
@@ -353,83 +340,114 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     }
                 }
                 // this thread's P^T and dS^T, packed, over its own (already read) columns
-                tmem_st16u(tlane + c0, pp);
-                tmem_st16u(tlane + 64 + c0, pd);
+                tmem_stn<kCols / 2>(tb + c0, pp);
+                tmem_stn<kCols / 2>(tb + 64 + c0, pd);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(p_full);
-                if (issuer_warp) {
-                    bool go = true;
-                    if (lane == 0) {
-                        go = mbar_wait(p_full, gt & 1, abort_flag, kErrTimeoutMma);
-                        // the item's first accumulating products: the previous item's
-                        // epilogue has read dV and dK
-                        if (go && ti == 0 && k >= 1) go = mbar_wait(acc_free, (k - 1) & 1, abort_flag, kErrTimeoutMma);
-                        if (go) {
-                            tc_fence_after();
-                            const uint32_t aQs = smem_u32(stage_q(st)), aDOs = smem_u32(stage_do(st));
-#pragma unroll
-                            for (int kk = 0; kk < kBlk / 16; ++kk) {
-                                const int h_ = (16 * kk) / kCols;   // the half holding queries 16 kk ..
-                                const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
-                                const uint64_t bdo = sdesc_sw128(aDOs + kk * (16 * 128), kBlk * 128, 1024);
-                                umma_bf16_ts(tmem + C::kTmemDV, tmem + acol, bdo, idesc_acc,
-                                             (ti > 0 || kk > 0) ? 1u : 0u);
-                            }
-#pragma unroll
-                            for (int kk = 0; kk < kBlk / 16; ++kk) {
-                                const int h_ = (16 * kk) / kCols;
-                                const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
-                                const uint64_t bq = sdesc_sw128(aQs + kk * (16 * 128), kBlk * 128, 1024);
-                                umma_bf16_ts(tmem + C::kTmemDK, tmem + 64 + acol, bq, idesc_acc,
-                                             (ti > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            umma_commit(&empty[st]);
-                            if (last) umma_commit(acc_done);
-                            // S^T, dP^T of the next tile, the next item's first after a last tile
-                            bool next = !last;
-                            if (last) {
-                                go = mbar_wait(&item_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag, kErrTimeoutMma);
-                                next = go && rec[(k + 1) & 1] >= 0;
-                            }
-                            if (next) {
-                                const int nst = (gt + 1) % C::kStages;
-                                go = mbar_wait(&full[nst], ((gt + 1) / C::kStages) & 1, abort_flag, kErrTimeoutMma);
-                                if (go && last) go = mbar_wait(kv_full, (k + 1) & 1, abort_flag, kErrTimeoutMma);
-                                if (go) {
-                                    tc_fence_after();
-                                    issue_s(nst);
-                                }
-                            }
-                        }
-                    }
-                    if (!__shfl_sync(0xffffffffu, go, 0)) {
-                        ok = false;
-                        break;
-                    }
-                }
+                mbar_arrive(&p_full[gt & 1]);
                 if (last) {
                     ++gt;
-                    // epilogue of the item: dV, dK of this thread's row, its 32 columns
+                    // epilogue of the item: dV, dK of this thread's row, its 16 columns
                     if (!__all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, abort_flag, kErrTimeoutSoftmax))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    float ov[32], ok_[32];
-                    tmem_ld32(tlane + C::kTmemDV + c0, ov);
-                    tmem_ld32(tlane + C::kTmemDK + c0, ok_);
+                    float ov[16], ok_[16];
+                    tmem_ld16(tlane + C::kTmemDV + c0, ov);
+                    tmem_ld16(tlane + C::kTmemDK + c0, ok_);
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(acc_free);   // the accumulators may take the next item's products
                     if (my_blk >= 0) {
                         const int64_t tok = head_row0 + static_cast<int64_t>(my_blk) * kBlk + uu;
                         const int64_t off = (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D) + c0;
-                        store_scaled_bf16(p.out0 + off, ov, 1.f);
-                        store_scaled_bf16(p.out1 + off, ok_, p.scale);
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            uint4 a, b;
+                            a.x = pack_bf16x2(ov[8 * h2 + 0], ov[8 * h2 + 1]);
+                            a.y = pack_bf16x2(ov[8 * h2 + 2], ov[8 * h2 + 3]);
+                            a.z = pack_bf16x2(ov[8 * h2 + 4], ov[8 * h2 + 5]);
+                            a.w = pack_bf16x2(ov[8 * h2 + 6], ov[8 * h2 + 7]);
+                            b.x = pack_bf16x2(ok_[8 * h2 + 0] * p.scale, ok_[8 * h2 + 1] * p.scale);
+                            b.y = pack_bf16x2(ok_[8 * h2 + 2] * p.scale, ok_[8 * h2 + 3] * p.scale);
+                            b.z = pack_bf16x2(ok_[8 * h2 + 4] * p.scale, ok_[8 * h2 + 5] * p.scale);
+                            b.w = pack_bf16x2(ok_[8 * h2 + 6] * p.scale, ok_[8 * h2 + 7] * p.scale);
+                            *reinterpret_cast<uint4*>(p.out0 + off + 8 * h2) = a;
+                            *reinterpret_cast<uint4*>(p.out1 + off + 8 * h2) = b;
+                        }
                     }
                     break;
                 }
+            }
+        }
+    } else if ((warp == 1 || warp == 18) && lane == 0) {
+        // ================= MMA issuers (lane 0 of warps 1 and 18, on different SM sub-partitions: a
+        // tcgen05.mma takes issue slots its sub-partition's elementwise warps also want).  Warp 1
+        // issues S^T = K Q^T and dV += P^T dO, warp 18 dP^T = V dO^T and dK += dS^T Q: each TMEM
+        // region (S^T and P^T, dP^T and dS^T, dV, dK) is written and read by one thread's products,
+        // in its issue order, so the accumulation order is fixed.  Per tile: dV (dK) of tile n when
+        // its P^T, dS^T are in TMEM, then S^T (dP^T) of tile n + 2.
+        const bool side_s = warp == 1;
+        constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
+        constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
+        int nx = 0, nx_item = 0;   // next tile (and its item) whose scores to issue
+        bool nx_first = true, nx_end = false;
+        // S^T = K Q^T, dP^T = V dO^T of tile nx into buffer nx & 1 (false: a wait gave up)
+        auto issue_next = [&]() -> bool {
+            if (nx_end) return true;
+            if (nx_first) {
+                if (!mbar_wait(&item_full[nx_item & 1], (nx_item >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+                if (rec[nx_item & 1] < 0) {
+                    nx_end = true;
+                    return true;
+                }
+                if (!mbar_wait(&kv_full[nx_item & 1], (nx_item >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+            }
+            const int st = nx % C::kStages;
+            if (!mbar_wait(&full[st], (nx / C::kStages) & 1, abort_flag, kErrTimeoutMma)) return false;
+            tc_fence_after();
+            const bool last = (meta[st] >> 18) & 1u;
+            // this side's operands: K and Q (S^T) or V and dO (dP^T); descriptors built once per
+            // tile and stepped by the K offset (fewer instructions per MMA issue)
+            const uint64_t da = sdesc_sw128(smem_u32(side_s ? tile_k(nx_item & 1) : tile_v(nx_item & 1)), 16, 1024);
+            const uint64_t db = sdesc_sw128(smem_u32(side_s ? stage_q(st) : stage_do(st)), 16, 1024);
+            const uint32_t dst = tmem + 128 * (nx & 1) + (side_s ? 0 : 64);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                umma_bf16(dst, sdesc_advance(da, kk * 32), sdesc_advance(db, kk * 32), idesc_s, kk > 0 ? 1u : 0u);
+            umma_commit(&s_full[nx & 1]);
+            if (last) umma_commit(&kv_free[nx_item & 1]);   // the item's K, V are no longer read
+            ++nx;
+            nx_first = last;
+            if (last) ++nx_item;
+            return true;
+        };
+        bool ok = issue_next() && issue_next();
+        for (int n = 0, k = 0, ti = 0; ok && n < nx; ++n) {
+            ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, abort_flag, kErrTimeoutMma);
+            // the item's first accumulating products: the previous item's epilogue has read dV and dK
+            if (ok && ti == 0 && k >= 1) ok = mbar_wait(acc_free, (k - 1) & 1, abort_flag, kErrTimeoutMma);
+            if (!ok) break;
+            tc_fence_after();
+            const int st = n % C::kStages;
+            const bool last = (meta[st] >> 18) & 1u;
+            // dV += P^T dO or dK += dS^T Q (A from TMEM: quarter kk's 8 packed columns at 16 kk)
+            const uint32_t ab = tmem + 128 * (n & 1) + (side_s ? 0 : 64);
+            const uint32_t acc = tmem + (side_s ? C::kTmemDV : C::kTmemDK);
+            const uint64_t bb = sdesc_sw128(smem_u32(side_s ? stage_do(st) : stage_q(st)), kBlk * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kBlk / 16; ++kk)
+                umma_bf16_ts(acc, ab + 16 * kk, sdesc_advance(bb, kk * (16 * 128)), idesc_acc,
+                             (ti > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&empty[st]);
+            if (last) umma_commit(acc_done);
+            ok = issue_next();   // the scores of tile n + 2 into the buffer this tile's products read
+            if (last) {
+                ++k;
+                ti = 0;
+            } else {
+                ++ti;
             }
         }
     }
@@ -439,10 +457,11 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // a role gave up a wait: the loads and products issued must land before
         // shared memory and TMEM go (without one, every one of them was waited for)
         if (warp == 0 && lane == 0) {
-            if (loads > 0) mbar_wait_drain(kv_full, (loads - 1) & 1);
+            if (loads > 0) mbar_wait_drain(&kv_full[(loads - 1) & 1], ((loads - 1) >> 1) & 1);
+            if (loads > 1) mbar_wait_drain(&kv_full[(loads - 2) & 1], ((loads - 2) >> 1) & 1);
             drain_fills(full, C::kStages, fills);
         }
-        if (warp == 2 && lane == 0) {
+        if ((warp == 1 || warp == 18) && lane == 0) {
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
         }

@@ -283,6 +283,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
     return d;
 }
 
+// The descriptor of the same layout `bytes` further on (a multiple of 16):
+// the start address sits in the low 14 bits in 16-byte units, and shared
+// addresses stay below 2^18, so the addition never carries out of the field.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective;
 // taddr carries the warp's lane quadrant in bits 16..).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
@@ -330,6 +335,13 @@ __device__ __forceinline__ void tmem_ldw(uint32_t taddr, float* v) {
     else tmem_ld8(taddr, v);
 }
 
+// 8 consecutive columns of this thread's lane from 8 raw words.
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 // 16 consecutive columns of this thread's lane from 16 raw words.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -372,9 +384,10 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
 // N (16 or 32) consecutive columns of this thread's lane from N raw words.
 template <int N>
 __device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t* r) {
-    static_assert(N == 16 || N == 32, "store width");
+    static_assert(N == 8 || N == 16 || N == 32, "store width");
     if constexpr (N == 32) tmem_st32u(taddr, r);
-    else tmem_st16u(taddr, r);
+    else if constexpr (N == 16) tmem_st16u(taddr, r);
+    else tmem_st8u(taddr, r);
 }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
