@@ -70,6 +70,10 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 #ifndef GSA_FWD64_STAGES
 #define GSA_FWD64_STAGES 5
 #endif
+// d = 64 through the persistent kernel (attn_fwd_persist.cuh).
+#ifndef GSA_FWD_PERSIST
+#define GSA_FWD_PERSIST 1
+#endif
 #ifndef GSA_FWD128_STAGES
 #define GSA_FWD128_STAGES 5
 #endif
@@ -103,6 +107,7 @@ struct FwdParams {
     TokLayout lo;       // layout of o
     float* lse;
     float scale_log2;   // softmax scale * log2(e)
+    int* ticket;        // persistent kernel: work counter, CTAs finished (both zero at launch)
     uint8_t cls[kMaxHeads];
 };
 
@@ -527,3 +532,5 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
 }  // namespace bf16
 }  // namespace gsa
+
+#include "attn_fwd_persist.cuh"

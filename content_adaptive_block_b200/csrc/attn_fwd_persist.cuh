@@ -1,0 +1,500 @@
+// Forward at d = 64 with persistent CTAs.
+//
+// Same products and softmax arithmetic as attn_fwd_bf16_kernel<64> (one
+// softmax warpgroup, two S buffers, P packed to bf16 in TMEM, O rescaled only
+// when the running max grows by more than 8 in log2 units), but a fixed grid
+// of CTAs (two per SM) takes the work items — (sample·head, query tile of two
+// blocks from the class's pairing order), heaviest tile first — one at a time
+// from a device counter.  With ~12 key tiles per item on the gzip masks, a
+// CTA per item spends about as long on barrier and TMEM set-up, the key-list
+// merge, the pipeline fill and the epilogue as on its tiles; here those
+// overlap the previous item's tiles:
+//   warp 0   producer: takes an item, merges its two CSR rows (private
+//            bitmaps), publishes it in a two-slot record ring, loads its Q
+//            into one of two Q buffers, then streams its key blocks' K and V
+//            into the stage ring straight after the previous item's, each
+//            stage carrying its block, live bit per half and an "item's last
+//            tile" mark in a metadata word;
+//   warp 1   TMEM owner; one thread issues QK^T and P V in tile order
+//            across items, event-driven (QK^T of the next item starts as soon
+//            as its Q and K are in and an S buffer is free);
+//   warps 2-5 softmax, one thread per query row; after an item's last tile
+//            the same threads normalise O and store it with the LSE, so O is
+//            read before they release the next item's first P, whose P V
+//            overwrites it.
+// The counter is one of a ring of device-global slots picked per launch; the
+// launch's last CTA to leave returns its slot to zero.  An item without a
+// live key block (no mask built here has one: every row holds its diagonal
+// block) gets O = 0 and LSE = -inf from the producer.  Every wait is bounded;
+// on a timeout the CTA records an error code, drains its loads and products
+// in flight and every role leaves.
+// TMEM: S[b] at 64 b, O at 128, P (32 packed columns) at 192.
+#pragma once
+
+namespace gsa {
+namespace bf16 {
+
+#ifndef GSA_FWDP_STAGES
+#define GSA_FWDP_STAGES 4
+#endif
+
+struct FwdPCfg {
+    static constexpr int D = 64;
+    static constexpr int kStages = GSA_FWDP_STAGES;
+    static constexpr int kQBytes = 128 * D * 2;         // Q tile (two query blocks)
+    static constexpr int kKVBytes = kBlk * D * 2;       // one key block of K or V
+    static constexpr int kStageBytes = 2 * kKVBytes;    // stage: K, V (1024-aligned)
+    static constexpr int kOffQ = 0;                     // [2 items]
+    static constexpr int kOffStage = kOffQ + 2 * kQBytes;
+    static constexpr int kOffMeta = kOffStage + kStages * kStageBytes;   // per stage: block | live << 16 | last << 18
+    static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
+    // full[st], empty[st], q_full[2], q_free[2], s_full[2], s_free[2], p_full, p_free, acc_done,
+    // item_full[2], rec_free[2], drain
+    static constexpr int kNumBars = 2 * kStages + 16;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
+    static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
+    static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
+    static constexpr int kSmemBytes = kEnd + 1024;
+    static_assert(kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
+    static_assert(kQBytes % 1024 == 0 && kStageBytes % 1024 == 0, "1024-byte alignment");
+    static constexpr int kTmemCols = 256;
+    static constexpr uint32_t kTmemS = 0, kTmemO = 128, kTmemP = 192;
+    static constexpr int kThreads = 64 + 128;
+};
+
+template <bool K4>   // strided tensors through 4-D maps (see load_rows)
+__global__ void __launch_bounds__(FwdPCfg::kThreads, 2)
+attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using C = FwdPCfg;
+    constexpr int D = C::D;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sStage = smem + C::kOffStage;
+    uint32_t* meta = reinterpret_cast<uint32_t*>(smem + C::kOffMeta);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + C::kStages;
+    uint64_t* q_full = bars + 2 * C::kStages;   // [2] Q of item k in buffer k & 1 loaded (phase k >> 1)
+    uint64_t* q_free = q_full + 2;              // [2] item k's last QK^T completed (phase k >> 1)
+    uint64_t* s_full = q_free + 2;              // [2] QK^T of tile n landed in S[n & 1] (phase n >> 1)
+    uint64_t* s_free = s_full + 2;              // [2] the softmax read S[n & 1] (128 arrivals)
+    uint64_t* p_full = s_free + 2;              // P of tile n in TMEM (128 arrivals, phase n & 1)
+    uint64_t* p_free = p_full + 1;              // P V of tile n completed (phase n & 1)
+    uint64_t* acc_done = p_free + 1;            // item k's last P V completed (phase k & 1)
+    // [2] item k's record (or the end) published in slot k & 1 (phase k >> 1);
+    // the slot is written again once the softmax threads read it (rec_free)
+    // and the MMA thread issued the item's last QK^T (q_free)
+    uint64_t* item_full = acc_done + 1;
+    uint64_t* rec_free = item_full + 2;
+    uint64_t* drain = rec_free + 2;             // the MMA thread's products at exit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
+    uint32_t* bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
+    uint32_t* bitsB = bitsA + kListMaxBlocks / 32;
+    auto q_buf = [&](int b) { return smem + C::kOffQ + b * C::kQBytes; };
+    auto stage_k = [&](int st) { return sStage + st * C::kStageBytes; };
+    auto stage_v = [&](int st) { return sStage + st * C::kStageBytes + C::kKVBytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = p.nblk;
+    const int SH = p.S * p.H;
+    const int items = SH * ((nblk + 1) / 2);
+    // item it: query tile it / SH (heaviest first), sample-head it % SH
+    auto item_keys = [&](int it, int& sh, int& qa, int& qb, int64_t& g) {
+        sh = it % SH;
+        const int tile = it / SH;
+        const int s = sh / p.H, h = sh % p.H;
+        g = static_cast<int64_t>(s) * 3 + p.cls[h];
+        qa = p.q_order[g * nblk + 2 * tile];
+        qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < C::kStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_free[b], 1);
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_free[b], 128);
+            mbar_init(&item_full[b], 1);
+            mbar_init(&rec_free[b], 128);
+        }
+        mbar_init(p_full, 128);
+        mbar_init(p_free, 1);
+        mbar_init(acc_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    int fills = 0, loads = 0;   // producer (lane 0): stages and Q tiles issued
+    if (warp == 0) {
+        // ================= producer
+        const int nwords = (nblk + 31) >> 5;
+        int gt = 0;      // stages issued so far, across items
+        int k = 0;       // items published
+        bool ok = true;
+        while (ok) {
+            int it = 0;
+            if (lane == 0) it = atomicAdd(p.ticket, 1);
+            it = __shfl_sync(0xffffffffu, it, 0);
+            const bool have = it < items;
+            int sh = 0, qa = 0, qb = -1;
+            int64_t g = 0;
+            bool any = false;
+            if (have) {
+                item_keys(it, sh, qa, qb, g);
+                // union of the two CSR rows, ascending, with a live bit per query half
+                for (int w = lane; w < nwords; w += 32) {
+                    bitsA[w] = 0u;
+                    bitsB[w] = 0u;
+                }
+                __syncwarp();
+                const int32_t* rp = p.row_ptr + g * (nblk + 1);
+                const int32_t* ci = p.col_idx + g * p.cap;
+                for (int e = rp[qa] + lane; e < rp[qa + 1]; e += 32) {
+                    const int j = ci[e];
+                    atomicOr(&bitsA[j >> 5], 1u << (j & 31));
+                }
+                if (qb >= 0) {
+                    for (int e = rp[qb] + lane; e < rp[qb + 1]; e += 32) {
+                        const int j = ci[e];
+                        atomicOr(&bitsB[j >> 5], 1u << (j & 31));
+                    }
+                }
+                __syncwarp();
+                uint32_t u = 0u;
+                for (int w = lane; w < nwords; w += 32) u |= bitsA[w] | bitsB[w];
+                any = __any_sync(0xffffffffu, u != 0u);
+            }
+            const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
+            if (have && !any) {
+                // no live key block: the softmax over an empty set
+                for (int half = 0; half < 2; ++half) {
+                    const int blk = half ? qb : qa;
+                    if (blk < 0) continue;
+                    for (int rr = lane; rr < kBlk; rr += 32) {
+                        const int64_t tok = head_row0 + static_cast<int64_t>(blk) * kBlk + rr;
+                        uint4* orow = reinterpret_cast<uint4*>(p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D));
+#pragma unroll
+                        for (int e = 0; e < D * 2 / 16; ++e) orow[e] = make_uint4(0u, 0u, 0u, 0u);
+                        p.lse[tok] = -INFINITY;
+                    }
+                }
+                __syncwarp();   // the bitmaps are rewritten for the next item
+                continue;
+            }
+            const int s_ = sh / p.H, h_ = sh - s_ * p.H;   // the 4-D maps' head and sample
+            if (lane == 0) {
+                // slot k & 1 and Q buffer k & 1 held item k - 2
+                if (k >= 2) {
+                    ok = mbar_wait(&rec_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer) &&
+                         mbar_wait(&q_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer);
+                }
+                rec[k & 1] = (ok && have) ? it : -1;
+                mbar_arrive(&item_full[k & 1]);
+                if (ok && have) {
+                    mbar_arrive_expect_tx(&q_full[k & 1], (qb >= 0 ? 2 : 1) * kBlk * D * 2);
+                    for (int half = 0; half < 2; ++half) {
+                        const int blk = half ? qb : qa;
+                        if (blk < 0) continue;
+                        load_rows<K4>(q_buf(k & 1) + half * (kBlk * 128), &tmQ, &q_full[k & 1], 0, blk * kBlk, h_,
+                                      s_, head_row0);
+                    }
+                    ++loads;
+                }
+                int lastw = (ok && have) ? nwords - 1 : -1;
+                while (lastw >= 0 && (bitsA[lastw] | bitsB[lastw]) == 0u) --lastw;
+                const int last_j = lastw >= 0 ? 32 * lastw + 31 - __clz(bitsA[lastw] | bitsB[lastw]) : -1;
+                for (int w = 0; ok && w <= lastw; ++w) {
+                    const uint32_t ua = bitsA[w], ub = bitsB[w];
+                    uint32_t u = ua | ub;
+                    while (u) {
+                        const int bit = __ffs(u) - 1;
+                        u &= u - 1;
+                        const int j = 32 * w + bit;
+                        const int st = gt % C::kStages;
+                        if (gt >= C::kStages &&
+                            !mbar_wait(&empty[st], ((gt / C::kStages) - 1) & 1, abort_flag, kErrTimeoutProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t live = ((ua >> bit) & 1u) | (((ub >> bit) & 1u) << 1);
+                        meta[st] = static_cast<uint32_t>(j) | (live << 16) | ((j == last_j ? 1u : 0u) << 18);
+                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                        load_rows<K4>(stage_k(st), &tmK, &full[st], 0, j * kBlk, h_, s_, head_row0);
+                        load_rows<K4>(stage_v(st), &tmV, &full[st], 0, j * kBlk, h_, s_, head_row0);
+                        ++gt;
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            gt = __shfl_sync(0xffffffffu, gt, 0);
+            ++k;
+            __syncwarp();   // the bitmaps are rewritten for the next item
+            if (!have) break;
+        }
+        fills = gt;
+    } else if (warp == 1) {
+        // ================= MMA issuer: QK^T of tile ns and P V of tile na, in tile order across items
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+            int ns = 0, kq = 0;     // QK^T: tiles issued, item of tile ns
+            int na = 0, ta = 0;     // P V: tiles issued, tile index of na within its item
+            bool item_open = false, qk_end = false, ok = true;
+            PollGuard guard;
+            while (ok && !(qk_end && na == ns)) {
+                bool moved = false;
+                if (!qk_end) {
+                    if (!item_open) {
+                        if (mbar_test(&item_full[kq & 1], (kq >> 1) & 1)) {
+                            if (rec[kq & 1] < 0) qk_end = true;
+                            else item_open = true;
+                            moved = true;
+                        }
+                    } else {
+                        const int st = ns % C::kStages, sb = ns & 1;
+                        if (mbar_test(&q_full[kq & 1], (kq >> 1) & 1) &&
+                            mbar_test(&full[st], (ns / C::kStages) & 1) &&
+                            (ns < 2 || mbar_test(&s_free[sb], ((ns - 2) >> 1) & 1))) {
+                            tc_fence_after();
+                            const uint64_t da = sdesc_sw128(smem_u32(q_buf(kq & 1)), 16, 1024);
+                            const uint64_t db = sdesc_sw128(smem_u32(stage_k(st)), 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                umma_bf16(tmem + C::kTmemS + 64 * sb, sdesc_advance(da, kk * 32),
+                                          sdesc_advance(db, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
+                            umma_commit(&s_full[sb]);
+                            if ((meta[st] >> 18) & 1u) {   // the item's Q is no longer read
+                                umma_commit(&q_free[kq & 1]);
+                                ++kq;
+                                item_open = false;
+                            }
+                            ++ns;
+                            moved = true;
+                        }
+                    }
+                }
+                if (na < ns && mbar_test(p_full, na & 1)) {
+                    tc_fence_after();
+                    const int st = na % C::kStages;
+                    const bool last = (meta[st] >> 18) & 1u;
+                    const uint64_t bv = sdesc_sw128(smem_u32(stage_v(st)), kBlk * 128, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk)
+                        umma_bf16_ts(tmem + C::kTmemO, tmem + C::kTmemP + kk * 8, sdesc_advance(bv, kk * (16 * 128)),
+                                     idesc_pv, (ta > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(p_free);
+                    umma_commit(&empty[st]);
+                    if (last) {
+                        umma_commit(acc_done);
+                        ta = 0;
+                    } else {
+                        ++ta;
+                    }
+                    ++na;
+                    moved = true;
+                }
+                if (moved) guard.progress();
+                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax warpgroup (warps 2..5), one thread per query row
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;         // query row in the tile = TMEM lane
+        const int half = r >> 6;
+        const int rr = r & 63;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const uint32_t tO = tl + C::kTmemO;
+        const uint32_t tP = tl + C::kTmemP;
+        bool ok = true;
+        int n = 0;   // tiles done so far, across items
+        for (int k = 0; ok; ++k) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&item_full[k & 1], (k >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                ok = false;
+                break;
+            }
+            const int it = rec[k & 1];
+            mbar_arrive(&rec_free[k & 1]);
+            if (it < 0) break;
+            int sh, qa, qb;
+            int64_t g;
+            item_keys(it, sh, qa, qb, g);
+            const int my_blk = half ? qb : qa;
+            float m = -INFINITY, l = 0.f;   // running max (log2 units) and sum of this row
+            for (;; ++n) {
+                const int sb = n & 1, st = n % C::kStages;
+                const uint32_t tS = tl + C::kTmemS + 64 * sb;
+                bool w_ok = mbar_wait(&s_full[sb], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax);
+                // the stage's metadata came with its loads
+                w_ok = w_ok && mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
+                if (!__all_sync(0xffffffffu, w_ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t mt = meta[st];
+                const int j = static_cast<int>(mt & 0xffffu);
+                const bool is_live = (mt >> (16 + half)) & 1u;
+                const bool last_tile = (mt >> 18) & 1u;
+                const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);   // visible columns 0..last
+                // pass 1: raw-score maximum (the scale is positive)
+                float mx = -INFINITY;
+                if (last >= 0) {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        float v[32];
+                        tmem_ld32(tS + 32 * ch, v);
+                        tmem_wait_ld();
+                        if (last < 32 * ch + 31) {
+#pragma unroll
+                            for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : -INFINITY;
+                        }
+                        mx = fmaxf(mx, max_reduce<32>(v));
+                    }
+                }
+                mx *= p.scale_log2;
+                const float m_new = fmaxf(m, mx);
+                float alpha = 1.f;
+                bool rescale = false;
+                float m_use = m;
+                if (m == -INFINITY) {
+                    m_use = m_new;
+                } else if (m_new > m + kRescaleThreshold) {
+                    m_use = m_new;
+                    alpha = ex2(m - m_new);
+                    rescale = true;
+                }
+                const float msafe = m_use == -INFINITY ? 0.f : m_use;
+                // pass 2: p = 2^(s * scale * log2 e - m), packed to bf16
+                uint32_t pk[32];
+                float sum = 0.f;
+                if (last < 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) pk[e] = 0u;
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        float v[32];
+                        tmem_ld32(tS + 32 * ch, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int cc = 0; cc < 32; ++cc) v[cc] = ex2(fmaf(v[cc], p.scale_log2, -msafe));
+                        if (last < 32 * ch + 31) {
+#pragma unroll
+                            for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : 0.f;
+                        }
+                        sum += sum_reduce<32>(v);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                    }
+                }
+                l = l * alpha + sum;
+                m = m_use;
+                // the scores are in registers: S[sb] may take a later QK^T
+                tc_fence_before();
+                mbar_arrive(&s_free[sb]);
+                // P and O were last used by the P V product of the previous tile
+                if (n >= 1 &&
+                    !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st32u(tP, pk);
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int cb = 0; cb < D; cb += 32) {
+                        float ov[32];
+                        tmem_ld32(tO + cb, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                        tmem_st32(tO + cb, ov);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(p_full);
+                if (last_tile) {
+                    ++n;
+                    // epilogue: O / l of this row and its LSE
+                    if (!__all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, abort_flag, kErrTimeoutSoftmax))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const bool store = my_blk >= 0;
+                    const int64_t tok =
+                        static_cast<int64_t>(sh) * p.L + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
+                    __nv_bfloat16* orow = p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D);
+                    const float inv = 1.f / l;
+#pragma unroll
+                    for (int cb = 0; cb < D; cb += 32) {
+                        float a[32];
+                        tmem_ld32(tO + cb, a);
+                        tmem_wait_ld();
+                        if (store) store_scaled_bf16(orow + cb, a, inv);
+                    }
+                    if (store) p.lse[tok] = (m + log2f(l)) * 0.69314718055994531f;
+                    break;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        // a role gave up a wait: the loads and products issued must land before
+        // shared memory and TMEM go (without one, every one of them was waited for)
+        if (warp == 0 && lane == 0) {
+            for (int b = 0; b < 2; ++b) {
+                const int kl = loads - 1 - ((loads - 1 - b) & 1);   // last item loaded into buffer b
+                if (loads > b) mbar_wait_drain(&q_full[b], (kl >> 1) & 1);
+            }
+            drain_fills(full, C::kStages, fills);
+        }
+        if (warp == 1 && lane == 0) {
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if (threadIdx.x == 0) {
+        // the launch's last CTA returns the counter slot to zero (its producer
+        // took its last ticket before this point, like every other CTA's)
+        __threadfence();
+        if (atomicAdd(p.ticket + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+            atomicExch(p.ticket, 0);
+            atomicExch(p.ticket + 1, 0);
+            __threadfence();
+        }
+    }
+}
+
+}  // namespace bf16
+}  // namespace gsa

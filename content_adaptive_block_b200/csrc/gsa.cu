@@ -66,6 +66,31 @@ float* noalloc_scratch(gsa_status* st) {
     return addr[dev];
 }
 
+// ---- work counters of the persistent forward
+//
+// The forward takes no workspace, so its persistent kernel draws items from
+// one of these slots (work counter, CTAs finished), a different slot per
+// launch in turn; the launch's last CTA returns its slot to zero.  Up to
+// kFwdSlots forward launches may therefore be in flight at once.
+constexpr int kFwdSlots = 256;
+static __device__ int g_fwd_tickets[2 * kFwdSlots];
+
+int* fwd_ticket_slot() {
+    static std::mutex mu;
+    static int* addr[kMaxDevices] = {};
+    static unsigned next[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fwd_tickets) != cudaSuccess || !p) return nullptr;
+        addr[dev] = static_cast<int*>(p);
+    }
+    const unsigned slot = next[dev]++ % kFwdSlots;
+    return addr[dev] + 2 * slot;
+}
+
 bool csr_ok(const gsa_block_csr* c) {
     return c && c->B >= 1 && c->nblk >= 1 && c->row_ptr && c->col_idx && c->col_ptr && c->row_idx && c->q_order &&
            c->k_order && c->capacity >= gsa_csr_capacity(c->nblk);
@@ -104,6 +129,18 @@ void launch_fwd(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const C
     });
     gsa::bf16::attn_fwd_bf16_kernel<D, K4><<<grid, gsa::bf16::FwdShape<D>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv,
                                                                                                         p);
+}
+
+template <bool K4>
+void launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const gsa::bf16::FwdParams& p, cudaStream_t cs) {
+    using C = gsa::bf16::FwdPCfg;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(gsa::bf16::attn_fwd_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
+    });
+    gsa::bf16::attn_fwd_persist_kernel<K4><<<ctas, C::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
 }
 
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
@@ -323,7 +360,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
         !gsa::make_tmap_tok(&tk, k, desc->d, desc->L, desc->H, desc->B, lq, k4) ||
         !gsa::make_tmap_tok(&tv, v, desc->d, desc->L, desc->H, desc->B, lq, k4))
         return GSA_ERR_CUDA;
-    gsa::bf16::FwdParams p;
+    gsa::bf16::FwdParams p{};
     p.row_ptr = csr->row_ptr;
     p.col_idx = csr->col_idx;
     p.q_order = csr->q_order;
@@ -338,8 +375,16 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     p.scale_log2 = scale * 1.4426950408889634f;
     std::memcpy(p.cls, cls, desc->H);
     dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
-    if (desc->d == 64) k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
-    else k4 ? launch_fwd<128, true>(grid, tq, tk, tv, p, cs) : launch_fwd<128, false>(grid, tq, tk, tv, p, cs);
+    if (desc->d == 64 && GSA_FWD_PERSIST) {
+        p.ticket = fwd_ticket_slot();
+        if (!p.ticket) return GSA_ERR_CUDA;
+        const int64_t items = static_cast<int64_t>(desc->B) * desc->H * ((csr->nblk + 1) / 2);
+        const int64_t ctas = items < 2 * gsa::bwd::sm_count() ? items : 2 * gsa::bwd::sm_count();
+        k4 ? launch_fwd_persist<true>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs)
+           : launch_fwd_persist<false>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs);
+    } else if (desc->d == 64) {
+        k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
+    } else k4 ? launch_fwd<128, true>(grid, tq, tk, tv, p, cs) : launch_fwd<128, false>(grid, tq, tk, tv, p, cs);
     return launch_status();
 }
 
