@@ -1,34 +1,44 @@
 // Forward at d = 64 with persistent CTAs.
 //
-// Same products and softmax arithmetic as attn_fwd_bf16_kernel<64> (one
-// softmax warpgroup, two S buffers, P packed to bf16 in TMEM, O rescaled only
-// when the running max grows by more than 8 in log2 units), but a fixed grid
-// of CTAs (two per SM) takes the work items — (sample·head, query tile of two
-// blocks from the class's pairing order), heaviest tile first — one at a time
-// from a device counter.  With ~12 key tiles per item on the gzip masks, a
-// CTA per item spends about as long on barrier and TMEM set-up, the key-list
-// merge, the pipeline fill and the epilogue as on its tiles; here those
-// overlap the previous item's tiles:
+// Same products as attn_fwd_bf16_kernel<64> — S = Q K^T per key block, an
+// online softmax in exp2 with O rescaled only when a running max grows by
+// more than 8 (log2 units), P packed to bf16 in TMEM as the A operand of
+// O += P V — organised for the short items of the gzip masks (~12 key tiles
+// per 128-row query tile):
+//   persistent CTAs: a fixed grid (two per SM) takes the work items —
+//     (sample·head, query tile of two blocks from the class's pairing
+//     order), heaviest tile first — one at a time from a device counter, so
+//     set-up, key-list merge, pipeline fill and epilogue overlap the
+//     previous item's tiles;
+//   column split: two softmax warpgroups, A with key columns 0..31 of every
+//     tile and B with columns 32..63, each with its own running max m_h,
+//     sum l_h and accumulator O_h = Σ P_h V_h (split-key online softmax), so
+//     no value crosses warps per tile; they combine once per item:
+//     m = max(m_A, m_B), O = Σ_h O_h 2^(m_h - m) / Σ_h l_h 2^(m_h - m).
+//     Each thread reads its 32 scores from TMEM once and writes its packed
+//     P over its own, already-read score columns.
+// Roles:
 //   warp 0   producer: takes an item, merges its two CSR rows (private
 //            bitmaps), publishes it in a two-slot record ring, loads its Q
 //            into one of two Q buffers, then streams its key blocks' K and V
 //            into the stage ring straight after the previous item's, each
 //            stage carrying its block, live bit per half and an "item's last
 //            tile" mark in a metadata word;
-//   warp 1   TMEM owner; one thread issues QK^T and P V in tile order
-//            across items, event-driven (QK^T of the next item starts as soon
-//            as its Q and K are in and an S buffer is free);
-//   warps 2-5 softmax, one thread per query row; after an item's last tile
-//            the same threads normalise O and store it with the LSE, so O is
-//            read before they release the next item's first P, whose P V
-//            overwrites it.
+//   warp 1   TMEM owner; one thread issues QK^T and P V in tile order across
+//            items, event-driven.  tcgen05 products of one thread run in
+//            issue order, so the QK^T of tile n + 2 goes into the S buffer of
+//            tile n right after the P V products that read its P;
+//   warps 2-9 softmax warpgroups; after an item's last tile the same threads
+//            normalise O and store it with the LSE, so O is read before they
+//            release the next item's first P, whose P V overwrites it.
 // The counter is one of a ring of device-global slots picked per launch; the
 // launch's last CTA to leave returns its slot to zero.  An item without a
 // live key block (no mask built here has one: every row holds its diagonal
 // block) gets O = 0 and LSE = -inf from the producer.  Every wait is bounded;
 // on a timeout the CTA records an error code, drains its loads and products
 // in flight and every role leaves.
-// TMEM: S[b] at 64 b, O at 128, P (32 packed columns) at 192.
+// TMEM: S[b] at 64 b (P_A packed over its columns 0..15, P_B over 32..47),
+// O_A at 128, O_B at 192.
 #pragma once
 
 namespace gsa {
@@ -48,18 +58,22 @@ struct FwdPCfg {
     static constexpr int kOffStage = kOffQ + 2 * kQBytes;
     static constexpr int kOffMeta = kOffStage + kStages * kStageBytes;   // per stage: block | live << 16 | last << 18
     static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
-    // full[st], empty[st], q_full[2], q_free[2], s_full[2], s_free[2], p_full, p_free, acc_done,
+    // full[st], empty[st], q_full[2], q_free[2], s_full[2], p_full[2], p_free, acc_done,
     // item_full[2], rec_free[2], drain
-    static constexpr int kNumBars = 2 * kStages + 16;
+    static constexpr int kNumBars = 2 * kStages + 15;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
     static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
-    static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
+    // [item parity][2 halves][m, l][128 rows]: a warp writes a buffer again only after
+    // the next item's pair barrier, which the other warp reaches after its reads
+    static constexpr int kOffMl = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
+    static constexpr int kEnd = kOffMl + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
     static_assert(kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
     static_assert(kQBytes % 1024 == 0 && kStageBytes % 1024 == 0, "1024-byte alignment");
     static constexpr int kTmemCols = 256;
-    static constexpr uint32_t kTmemS = 0, kTmemO = 128, kTmemP = 192;
-    static constexpr int kThreads = 64 + 128;
+    static constexpr uint32_t kTmemS = 0, kTmemO = 128;   // O_h at 128 + 64 h
+    static constexpr int kSoftmax = 256;                  // two warpgroups
+    static constexpr int kThreads = 64 + kSoftmax;
 };
 
 template <bool K4>   // strided tensors through 4-D maps (see load_rows)
@@ -78,9 +92,8 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     uint64_t* q_full = bars + 2 * C::kStages;   // [2] Q of item k in buffer k & 1 loaded (phase k >> 1)
     uint64_t* q_free = q_full + 2;              // [2] item k's last QK^T completed (phase k >> 1)
     uint64_t* s_full = q_free + 2;              // [2] QK^T of tile n landed in S[n & 1] (phase n >> 1)
-    uint64_t* s_free = s_full + 2;              // [2] the softmax read S[n & 1] (128 arrivals)
-    uint64_t* p_full = s_free + 2;              // P of tile n in TMEM (128 arrivals, phase n & 1)
-    uint64_t* p_free = p_full + 1;              // P V of tile n completed (phase n & 1)
+    uint64_t* p_full = s_full + 2;              // [2] P of tile n over S[n & 1] (256 arrivals, phase n >> 1)
+    uint64_t* p_free = p_full + 2;              // P V of tile n completed (phase n & 1)
     uint64_t* acc_done = p_free + 1;            // item k's last P V completed (phase k & 1)
     // [2] item k's record (or the end) published in slot k & 1 (phase k >> 1);
     // the slot is written again once the softmax threads read it (rec_free)
@@ -120,11 +133,10 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             mbar_init(&q_full[b], 1);
             mbar_init(&q_free[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 128);
+            mbar_init(&p_full[b], C::kSoftmax);
             mbar_init(&item_full[b], 1);
-            mbar_init(&rec_free[b], 128);
+            mbar_init(&rec_free[b], C::kSoftmax);
         }
-        mbar_init(p_full, 128);
         mbar_init(p_free, 1);
         mbar_init(acc_done, 1);
         mbar_init(drain, 1);
@@ -271,9 +283,9 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         }
                     } else {
                         const int st = ns % C::kStages, sb = ns & 1;
-                        if (mbar_test(&q_full[kq & 1], (kq >> 1) & 1) &&
-                            mbar_test(&full[st], (ns / C::kStages) & 1) &&
-                            (ns < 2 || mbar_test(&s_free[sb], ((ns - 2) >> 1) & 1))) {
+                        // S[sb] held tile ns - 2: its P V products are issued (in order before this QK^T)
+                        if (ns < na + 2 && mbar_test(&q_full[kq & 1], (kq >> 1) & 1) &&
+                            mbar_test(&full[st], (ns / C::kStages) & 1)) {
                             tc_fence_after();
                             const uint64_t da = sdesc_sw128(smem_u32(q_buf(kq & 1)), 16, 1024);
                             const uint64_t db = sdesc_sw128(smem_u32(stage_k(st)), 16, 1024);
@@ -292,15 +304,18 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         }
                     }
                 }
-                if (na < ns && mbar_test(p_full, na & 1)) {
+                if (na < ns && mbar_test(&p_full[na & 1], (na >> 1) & 1)) {
                     tc_fence_after();
                     const int st = na % C::kStages;
                     const bool last = (meta[st] >> 18) & 1u;
                     const uint64_t bv = sdesc_sw128(smem_u32(stage_v(st)), kBlk * 128, 1024);
+                    // O_h += P_h V[32 h .. 32 h + 31]: key chunk kk (16 keys) of half kk / 2 sits at
+                    // packed column 32 (kk / 2) + 8 (kk % 2) of the S buffer
+                    const uint32_t ap = tmem + C::kTmemS + 64 * (na & 1);
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk)
-                        umma_bf16_ts(tmem + C::kTmemO, tmem + C::kTmemP + kk * 8, sdesc_advance(bv, kk * (16 * 128)),
-                                     idesc_pv, (ta > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
+                                     sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
                     umma_commit(p_free);
                     umma_commit(&empty[st]);
                     if (last) {
@@ -318,14 +333,16 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         __syncwarp();
     } else {
-        // ================= softmax warpgroup (warps 2..5), one thread per query row
-        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;         // query row in the tile = TMEM lane
+        // ================= softmax warpgroups (warps 2..9): one thread per query row and column half
+        const int hc = (warp - 2) >> 2;          // key columns [32 hc, 32 hc + 32), accumulator O_hc
+        const int c0 = 32 * hc;
+        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;          // query row in the tile = TMEM lane
         const int half = r >> 6;
         const int rr = r & 63;
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const uint32_t tO = tl + C::kTmemO;
-        const uint32_t tP = tl + C::kTmemP;
+        const uint32_t tO = tl + C::kTmemO + 64 * hc;
+        float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
         bool ok = true;
         int n = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
@@ -340,10 +357,10 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             int64_t g;
             item_keys(it, sh, qa, qb, g);
             const int my_blk = half ? qb : qa;
-            float m = -INFINITY, l = 0.f;   // running max (log2 units) and sum of this row
+            float m = -INFINITY, l = 0.f;   // running max (log2 units) and sum of this row's half
             for (;; ++n) {
                 const int sb = n & 1, st = n % C::kStages;
-                const uint32_t tS = tl + C::kTmemS + 64 * sb;
+                const uint32_t tS = tl + C::kTmemS + 64 * sb + c0;
                 bool w_ok = mbar_wait(&s_full[sb], (n >> 1) & 1, abort_flag, kErrTimeoutSoftmax);
                 // the stage's metadata came with its loads
                 w_ok = w_ok && mbar_wait(&full[st], (n / C::kStages) & 1, abort_flag, kErrTimeoutSoftmax);
@@ -356,23 +373,17 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 const int j = static_cast<int>(mt & 0xffffu);
                 const bool is_live = (mt >> (16 + half)) & 1u;
                 const bool last_tile = (mt >> 18) & 1u;
-                const int last = !is_live ? -1 : (j == my_blk ? rr : kBlk - 1);   // visible columns 0..last
-                // pass 1: raw-score maximum (the scale is positive)
-                float mx = -INFINITY;
-                if (last >= 0) {
+                // visible columns of this half: 0 .. lim (none below 0)
+                const int lim = (!is_live ? -1 : (j == my_blk ? rr : kBlk - 1)) - c0;
+                float v[32];
+                tmem_ld32(tS, v);
+                tmem_wait_ld();
+                if (lim < 31) {
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        float v[32];
-                        tmem_ld32(tS + 32 * ch, v);
-                        tmem_wait_ld();
-                        if (last < 32 * ch + 31) {
-#pragma unroll
-                            for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : -INFINITY;
-                        }
-                        mx = fmaxf(mx, max_reduce<32>(v));
-                    }
+                    for (int cc = 0; cc < 32; ++cc) v[cc] = cc <= lim ? v[cc] : -INFINITY;
                 }
-                mx *= p.scale_log2;
+                // raw-score maximum (the scale is positive), then p = 2^(s * scale * log2 e - m)
+                const float mx = max_reduce<32>(v) * p.scale_log2;
                 const float m_new = fmaxf(m, mx);
                 float alpha = 1.f;
                 bool rescale = false;
@@ -385,42 +396,22 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     rescale = true;
                 }
                 const float msafe = m_use == -INFINITY ? 0.f : m_use;
-                // pass 2: p = 2^(s * scale * log2 e - m), packed to bf16
-                uint32_t pk[32];
-                float sum = 0.f;
-                if (last < 0) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) pk[e] = 0u;
-                } else {
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        float v[32];
-                        tmem_ld32(tS + 32 * ch, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int cc = 0; cc < 32; ++cc) v[cc] = ex2(fmaf(v[cc], p.scale_log2, -msafe));
-                        if (last < 32 * ch + 31) {
-#pragma unroll
-                            for (int cc = 0; cc < 32; ++cc) v[cc] = 32 * ch + cc <= last ? v[cc] : 0.f;
-                        }
-                        sum += sum_reduce<32>(v);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[16 * ch + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                    }
-                }
-                l = l * alpha + sum;
+                for (int cc = 0; cc < 32; ++cc) v[cc] = ex2(fmaf(v[cc], p.scale_log2, -msafe));   // masked: 2^-inf = 0
+                l = l * alpha + sum_reduce<32>(v);
                 m = m_use;
-                // the scores are in registers: S[sb] may take a later QK^T
-                tc_fence_before();
-                mbar_arrive(&s_free[sb]);
-                // P and O were last used by the P V product of the previous tile
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                // P over this thread's own, already-read score columns
+                tmem_st16u(tS, pk);
+                // O_hc was last written by the P V products of the previous tile
                 if (n >= 1 &&
                     !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                tmem_st32u(tP, pk);
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                     for (int cb = 0; cb < D; cb += 32) {
@@ -434,28 +425,37 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                mbar_arrive(&p_full[sb]);
                 if (last_tile) {
                     ++n;
-                    // epilogue: O / l of this row and its LSE
+                    // epilogue: combine the halves, O / l for this thread's 32 output columns, LSE
+                    float* mlk = ml + (k & 1) * (4 * 128);
+                    mlk[(hc * 2 + 0) * 128 + r] = m;
+                    mlk[(hc * 2 + 1) * 128 + r] = l;
+                    pair_barrier(quad);
+                    const float mA = mlk[0 * 128 + r], lA = mlk[1 * 128 + r];
+                    const float mB = mlk[2 * 128 + r], lB = mlk[3 * 128 + r];
                     if (!__all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, abort_flag, kErrTimeoutSoftmax))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const bool store = my_blk >= 0;
-                    const int64_t tok =
-                        static_cast<int64_t>(sh) * p.L + static_cast<int64_t>(store ? my_blk : 0) * kBlk + rr;
-                    __nv_bfloat16* orow = p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D);
-                    const float inv = 1.f / l;
+                    const float mm = fmaxf(mA, mB);
+                    const float wA = mA == -INFINITY ? 0.f : ex2(mA - mm);
+                    const float wB = mB == -INFINITY ? 0.f : ex2(mB - mm);
+                    const float lt = lA * wA + lB * wB;
+                    float a[32], b2[32];
+                    tmem_ld32(tl + C::kTmemO + c0, a);
+                    tmem_ld32(tl + C::kTmemO + 64 + c0, b2);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int cb = 0; cb < D; cb += 32) {
-                        float a[32];
-                        tmem_ld32(tO + cb, a);
-                        tmem_wait_ld();
-                        if (store) store_scaled_bf16(orow + cb, a, inv);
+                    for (int e = 0; e < 32; ++e) a[e] = fmaf(b2[e], wB, a[e] * wA);
+                    if (my_blk >= 0) {
+                        const int64_t tok = static_cast<int64_t>(sh) * p.L + static_cast<int64_t>(my_blk) * kBlk + rr;
+                        __nv_bfloat16* orow = p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D);
+                        store_scaled_bf16(orow + c0, a, 1.f / lt);
+                        if (hc == 0) p.lse[tok] = (mm + log2f(lt)) * 0.69314718055994531f;
                     }
-                    if (store) p.lse[tok] = (m + log2f(l)) * 0.69314718055994531f;
                     break;
                 }
             }
