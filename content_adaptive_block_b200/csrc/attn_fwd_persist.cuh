@@ -24,8 +24,9 @@
 //            into the stage ring straight after the previous item's, each
 //            stage carrying its block, live bit per half and an "item's last
 //            tile" mark in a metadata word;
-//   warp 1   TMEM owner; one thread issues QK^T and P V in tile order across
-//            items, event-driven.  tcgen05 products of one thread run in
+//   warp 1   TMEM owner; issues QK^T and P V in tile order across items,
+//            event-driven: the warp runs the loop converged, one elected
+//            lane issues.  tcgen05 products of one thread run in
 //            issue order, so the QK^T of tile n + 2 goes into the S buffer of
 //            tile n right after the P V products that read its P;
 //   warps 2-9 softmax warpgroups; after an item's last tile the same threads
@@ -264,74 +265,80 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         fills = gt;
     } else if (warp == 1) {
-        // ================= MMA issuer: QK^T of tile ns and P V of tile na, in tile order across items
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
-            int ns = 0, kq = 0;     // QK^T: tiles issued, item of tile ns
-            int na = 0, ta = 0;     // P V: tiles issued, tile index of na within its item
-            bool item_open = false, qk_end = false, ok = true;
-            PollGuard guard;
-            while (ok && !(qk_end && na == ns)) {
-                bool moved = false;
-                if (!qk_end) {
-                    if (!item_open) {
-                        if (mbar_test(&item_full[kq & 1], (kq >> 1) & 1)) {
-                            if (rec[kq & 1] < 0) qk_end = true;
-                            else item_open = true;
-                            moved = true;
-                        }
-                    } else {
-                        const int st = ns % C::kStages, sb = ns & 1;
-                        // S[sb] held tile ns - 2: its P V products are issued (in order before this QK^T)
-                        if (ns < na + 2 && mbar_test(&q_full[kq & 1], (kq >> 1) & 1) &&
-                            mbar_test(&full[st], (ns / C::kStages) & 1)) {
-                            tc_fence_after();
-                            const uint64_t da = sdesc_sw128(smem_u32(q_buf(kq & 1)), 16, 1024);
-                            const uint64_t db = sdesc_sw128(smem_u32(stage_k(st)), 16, 1024);
+        // ================= MMA issuer: QK^T of tile ns and P V of tile na, in tile order across
+        // items.  The whole warp runs the loop converged (decisions by vote), one elected lane
+        // issues: the loop state and every operand stay warp-uniform.
+        constexpr uint32_t idesc_qk = idesc_bf16(128, kBlk, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, D, 1);
+        const auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
+        int ns = 0, kq = 0;     // QK^T: tiles issued, item of tile ns
+        int na = 0, ta = 0;     // P V: tiles issued, tile index of na within its item
+        bool item_open = false, qk_end = false, q_ready = false, ok = true;
+        PollGuard guard;
+        while (ok && !(qk_end && na == ns)) {
+            bool moved = false;
+            if (!qk_end) {
+                if (!item_open) {
+                    if (all(mbar_test(&item_full[kq & 1], (kq >> 1) & 1))) {
+                        if (rec[kq & 1] < 0) qk_end = true;
+                        else item_open = true;
+                        q_ready = false;
+                        moved = true;
+                    }
+                } else {
+                    const int st = ns % C::kStages, sb = ns & 1;
+                    // S[sb] held tile ns - 2: its P V products are issued (in order before this QK^T)
+                    if (!q_ready) q_ready = all(mbar_test(&q_full[kq & 1], (kq >> 1) & 1));
+                    if (ns < na + 2 && q_ready && all(mbar_test(&full[st], (ns / C::kStages) & 1))) {
+                        tc_fence_after();
+                        const uint64_t da = sdesc_sw128(smem_u32(q_buf(kq & 1)), 16, 1024);
+                        const uint64_t db = sdesc_sw128(smem_u32(stage_k(st)), 16, 1024);
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                umma_bf16(tmem + C::kTmemS + 64 * sb, sdesc_advance(da, kk * 32),
-                                          sdesc_advance(db, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
-                            umma_commit(&s_full[sb]);
-                            if ((meta[st] >> 18) & 1u) {   // the item's Q is no longer read
-                                umma_commit(&q_free[kq & 1]);
-                                ++kq;
-                                item_open = false;
-                            }
-                            ++ns;
-                            moved = true;
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_bf16_w(tmem + C::kTmemS + 64 * sb, sdesc_advance(da, kk * 32),
+                                        sdesc_advance(db, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
+                        umma_commit_w(&s_full[sb]);
+                        if ((meta[st] >> 18) & 1u) {   // the item's Q is no longer read
+                            umma_commit_w(&q_free[kq & 1]);
+                            ++kq;
+                            item_open = false;
                         }
+                        ++ns;
+                        moved = true;
                     }
                 }
-                if (na < ns && mbar_test(&p_full[na & 1], (na >> 1) & 1)) {
-                    tc_fence_after();
-                    const int st = na % C::kStages;
-                    const bool last = (meta[st] >> 18) & 1u;
-                    const uint64_t bv = sdesc_sw128(smem_u32(stage_v(st)), kBlk * 128, 1024);
-                    // O_h += P_h V[32 h .. 32 h + 31]: key chunk kk (16 keys) of half kk / 2 sits at
-                    // packed column 32 (kk / 2) + 8 (kk % 2) of the S buffer
-                    const uint32_t ap = tmem + C::kTmemS + 64 * (na & 1);
+            }
+            if (na < ns && all(mbar_test(&p_full[na & 1], (na >> 1) & 1))) {
+                tc_fence_after();
+                const int st = na % C::kStages;
+                const bool last = (meta[st] >> 18) & 1u;
+                const uint64_t bv = sdesc_sw128(smem_u32(stage_v(st)), kBlk * 128, 1024);
+                // O_h += P_h V[32 h .. 32 h + 31]: key chunk kk (16 keys) of half kk / 2 sits at
+                // packed column 32 (kk / 2) + 8 (kk % 2) of the S buffer
+                const uint32_t ap = tmem + C::kTmemS + 64 * (na & 1);
 #pragma unroll
-                    for (int kk = 0; kk < kBlk / 16; ++kk)
-                        umma_bf16_ts(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
-                                     sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
-                    umma_commit(p_free);
-                    umma_commit(&empty[st]);
-                    if (last) {
-                        umma_commit(acc_done);
-                        ta = 0;
-                    } else {
-                        ++ta;
-                    }
-                    ++na;
-                    moved = true;
+                for (int kk = 0; kk < kBlk / 16; ++kk)
+                    umma_bf16_ts_w(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
+                                   sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
+                umma_commit_w(p_free);
+                umma_commit_w(&empty[st]);
+                if (last) {
+                    umma_commit_w(acc_done);
+                    ta = 0;
+                } else {
+                    ++ta;
                 }
-                if (moved) guard.progress();
-                else if (guard.stalled(abort_flag, kErrTimeoutMma)) ok = false;
+                ++na;
+                moved = true;
+            }
+            if (moved) {
+                guard.progress();
+            } else {
+                bool stop = false;
+                if (lane == 0) stop = guard.stalled(abort_flag, kErrTimeoutMma);
+                if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) ok = false;
             }
         }
-        __syncwarp();
     } else {
         // ================= softmax warpgroups (warps 2..9): one thread per query row and column half
         const int hc = (warp - 2) >> 2;          // key columns [32 hc, 32 hc + 32), accumulator O_hc
@@ -474,9 +481,9 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             }
             drain_fills(full, C::kStages, fills);
         }
-        if (warp == 1 && lane == 0) {
-            umma_commit(drain);
-            mbar_wait_drain(drain, 0);
+        if (warp == 1) {
+            umma_commit_w(drain);   // the lane that issued the products
+            if (lane == 0) mbar_wait_drain(drain, 0);
         }
         __syncthreads();
     }
