@@ -59,9 +59,9 @@ struct FwdPCfg {
     static constexpr int kOffStage = kOffQ + 2 * kQBytes;
     static constexpr int kOffMeta = kOffStage + kStages * kStageBytes;   // per stage: block | live << 16 | last << 18
     static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
-    // full[st], empty[st], q_full[2], q_free[2], s_full[2], p_full[2], p_free, acc_done,
+    // full[st], empty[st], q_full[2], q_free[2], s_full[2], p_full[2], acc_done,
     // item_full[2], rec_free[2], drain
-    static constexpr int kNumBars = 2 * kStages + 15;
+    static constexpr int kNumBars = 2 * kStages + 14;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
     static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
     // [item parity][2 halves][m, l][128 rows]: a warp writes a buffer again only after
@@ -89,13 +89,12 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     uint32_t* meta = reinterpret_cast<uint32_t*>(smem + C::kOffMeta);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
-    uint64_t* empty = bars + C::kStages;
+    uint64_t* empty = bars + C::kStages;        // P V of the stage's tile completed (also: O quiescent)
     uint64_t* q_full = bars + 2 * C::kStages;   // [2] Q of item k in buffer k & 1 loaded (phase k >> 1)
     uint64_t* q_free = q_full + 2;              // [2] item k's last QK^T completed (phase k >> 1)
     uint64_t* s_full = q_free + 2;              // [2] QK^T of tile n landed in S[n & 1] (phase n >> 1)
     uint64_t* p_full = s_full + 2;              // [2] P of tile n over S[n & 1] (256 arrivals, phase n >> 1)
-    uint64_t* p_free = p_full + 2;              // P V of tile n completed (phase n & 1)
-    uint64_t* acc_done = p_free + 1;            // item k's last P V completed (phase k & 1)
+    uint64_t* acc_done = p_full + 2;            // item k's last P V completed (phase k & 1)
     // [2] item k's record (or the end) published in slot k & 1 (phase k >> 1);
     // the slot is written again once the softmax threads read it (rec_free)
     // and the MMA thread issued the item's last QK^T (q_free)
@@ -138,7 +137,6 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             mbar_init(&item_full[b], 1);
             mbar_init(&rec_free[b], C::kSoftmax);
         }
-        mbar_init(p_free, 1);
         mbar_init(acc_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -308,7 +306,11 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     }
                 }
             }
-            if (na < ns && all(mbar_test(&p_full[na & 1], (na >> 1) & 1))) {
+            // with no QK^T issuable before it, block on the next P (the hardware suspends the
+            // warp until the phase completes or a time limit passes)
+            const bool only_pv = qk_end || ns >= na + 2;
+            if (na < ns && all(only_pv ? mbar_try_wait(&p_full[na & 1], (na >> 1) & 1)
+                                       : mbar_test(&p_full[na & 1], (na >> 1) & 1))) {
                 tc_fence_after();
                 const int st = na % C::kStages;
                 const bool last = (meta[st] >> 18) & 1u;
@@ -320,7 +322,6 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 for (int kk = 0; kk < kBlk / 16; ++kk)
                     umma_bf16_ts_w(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
                                    sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
-                umma_commit_w(p_free);
                 umma_commit_w(&empty[st]);
                 if (last) {
                     umma_commit_w(acc_done);
@@ -390,7 +391,7 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     for (int cc = 0; cc < 32; ++cc) v[cc] = cc <= lim ? v[cc] : -INFINITY;
                 }
                 // raw-score maximum (the scale is positive), then p = 2^(s * scale * log2 e - m)
-                const float mx = max_reduce<32>(v) * p.scale_log2;
+                const float mx = max_reduce3_32(v) * p.scale_log2;
                 const float m_new = fmaxf(m, mx);
                 float alpha = 1.f;
                 bool rescale = false;
@@ -403,18 +404,27 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     rescale = true;
                 }
                 const float msafe = m_use == -INFINITY ? 0.f : m_use;
+                const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-msafe, -msafe);
 #pragma unroll
-                for (int cc = 0; cc < 32; ++cc) v[cc] = ex2(fmaf(v[cc], p.scale_log2, -msafe));   // masked: 2^-inf = 0
-                l = l * alpha + sum_reduce<32>(v);
+                for (int e = 0; e < 16; ++e) {   // masked: 2^-inf = 0
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(v[2 * e], v[2 * e + 1]), sc2, nm2), x0, x1);
+                    v[2 * e] = ex2(x0);
+                    v[2 * e + 1] = ex2(x1);
+                }
+                l = l * alpha + sum_reduce2_32(v);
                 m = m_use;
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 // P over this thread's own, already-read score columns
                 tmem_st16u(tS, pk);
-                // O_hc was last written by the P V products of the previous tile
-                if (n >= 1 &&
-                    !__all_sync(0xffffffffu, mbar_wait(p_free, (n - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+                // O_hc was last written by the P V products of the previous tile, which complete
+                // the phase of its stage's empty barrier (one phase per use of the stage; this
+                // wait, taken every tile, keeps the softmax at most one phase behind)
+                if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(&empty[(n - 1) % C::kStages],
+                                                                 ((n - 1) / C::kStages) & 1, abort_flag,
+                                                                 kErrTimeoutSoftmax))) {
                     ok = false;
                     break;
                 }

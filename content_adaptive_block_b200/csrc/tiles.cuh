@@ -141,6 +141,32 @@ __device__ __forceinline__ float sum_reduce(const float* v) {
     return t[0];
 }
 
+// Maximum of 32 values with three-input max: 17 instructions, depth 4.
+__device__ __forceinline__ float max_reduce3_32(const float* v) {
+    float t[11], u[4];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) t[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    t[10] = fmaxf(v[30], v[31]);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) u[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+    u[3] = fmaxf(t[9], t[10]);
+    return fmaxf(fmax3(u[0], u[1], u[2]), u[3]);
+}
+
+// Sum of 32 values as 16 packed pairs (v[2i], v[2i+1]): 16 instructions, depth 5.
+__device__ __forceinline__ float sum_reduce2_32(const float* v) {
+    uint64_t t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = f2_add(f2_pack(v[4 * i], v[4 * i + 1]), f2_pack(v[4 * i + 2], v[4 * i + 3]));
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
+    float lo, hi;
+    f2_unpack(t[0], lo, hi);
+    return lo + hi;
+}
+
 // 32 fp32 values times `mul` as bf16 to global memory (16-byte stores).
 __device__ __forceinline__ void store_scaled_bf16(__nv_bfloat16* dst, const float* v, float mul) {
 #pragma unroll
