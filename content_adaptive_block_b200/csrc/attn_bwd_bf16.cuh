@@ -67,8 +67,8 @@ struct Params {
     int S, H, nblk;
     int64_t L;
     const float* lse;
-    const float* lse2;      // LSE_t log2(e), written next to D_t by dot_kernel
-    const float* dvec;      // D_t
+    const float* nlse2;     // -LSE_t log2(e), written next to -D_t by dot_kernel
+    const float* ndvec;     // -D_t (negated: the exponent and dS take them as addends)
     __nv_bfloat16* out0;    // dq (dq_kernel) or dv (dkdv_kernel)
     __nv_bfloat16* out1;    // dk (dkdv_kernel)
     TokLayout lq;           // layout of q, k, v and of dq, dk, dv
@@ -86,8 +86,8 @@ struct Params {
 template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                   const __nv_bfloat16* __restrict__ dO, TokLayout lo, int64_t L,
-                                                  int H, int SH, float* __restrict__ dvec,
-                                                  const float* __restrict__ lse, float* __restrict__ lse2,
+                                                  int H, int SH, float* __restrict__ ndvec,
+                                                  const float* __restrict__ lse, float* __restrict__ nlse2,
                                                   int* __restrict__ ticket) {
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
@@ -113,8 +113,8 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
         for (int o2 = kTpr / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
         if (part == 0) {
             const int64_t row = static_cast<int64_t>(sh) * L + l;
-            dvec[row] = acc;
-            lse2[row] = lse[row] * kLog2e;   // the backward's exponents are in log2 units
+            ndvec[row] = -acc;
+            nlse2[row] = -(lse[row] * kLog2e);   // the backward's exponents are in log2 units
         }
     }
 }
@@ -279,8 +279,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int rr = r & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + rr;
-        const float lse2 = my_blk >= 0 ? p.lse2[tok] : 0.f;
-        const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
+        const float nlse2 = my_blk >= 0 ? p.nlse2[tok] : 0.f;
+        const float ndt = my_blk >= 0 ? p.ndvec[tok] : 0.f;
         // the group's MMA issuer: lane 0 of its first warp
         const bool issuer_warp = ((warp - 2) & 3) == 0 && hc == 0;
         constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
@@ -345,7 +345,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const float* d_ = dp[ch & 1];
                     const int cb = c0 + kW * ch;   // first key column of the chunk
 #pragma unroll
-                    for (int cc = 0; cc < kW; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, -lse2)) * (d_[cc] - dt);
+                    for (int cc = 0; cc < kW; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, nlse2)) * (d_[cc] + ndt);
                     if (last < cb + kW - 1) {
 #pragma unroll
                         for (int cc = 0; cc < kW; ++cc) s_[cc] = cb + cc <= last ? s_[cc] : 0.f;
@@ -584,8 +584,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     load_rows<K4>(stage_q(st) + at * (kBlk * 128), &tmQ, &full[st], at * 64, l0, h, s, head_row0);
                     load_rows<K4>(stage_do(st) + at * (kBlk * 128), &tmDO, &full[st], at * 64, l0, h, s, head_row0);
                 }
-                bulk_load(stage_lse(st), p.lse2 + row64, C::kVecBytes, &full[st]);
-                bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
+                bulk_load(stage_lse(st), p.nlse2 + row64, C::kVecBytes, &full[st]);
+                bulk_load(stage_d(st), p.ndvec + row64, C::kVecBytes, &full[st]);
             }
             fills = n;
         }
@@ -684,10 +684,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int cc = 4 * c4 + e;
-                            float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e]));
+                            float pr = ex2(fmaf(s_[cc], p.scale_log2, lv[e]));
                             if (first > cb) pr = cb + cc >= first ? pr : 0.f;
                             s_[cc] = pr;
-                            d_[cc] = pr * (d_[cc] - dd[e]);
+                            d_[cc] = pr * (d_[cc] + dd[e]);
                         }
                     }
 #pragma unroll
@@ -843,7 +843,7 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     constexpr int kRowsPerCta = 256 / (D / 8);   // 32 or 16: divides L
     const int sh_grid = S * H < 65535 ? S * H : 65535;
     dot_kernel<D><<<dim3(static_cast<unsigned>(pq.L / kRowsPerCta), static_cast<unsigned>(sh_grid)), 256, 0, st>>>(
-        o, dO, lo, pq.L, pq.H, S * H, const_cast<float*>(pq.dvec), pq.lse, const_cast<float*>(pq.lse2), pkv.ticket);
+        o, dO, lo, pq.L, pq.H, S * H, const_cast<float*>(pq.ndvec), pq.lse, const_cast<float*>(pq.nlse2), pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
     if (D == 64 && GSA_DQ_PERSIST) {
         static std::once_flag once_q;
@@ -897,8 +897,8 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     base.nblk = csr->nblk;
     base.L = desc->L;
     base.lse = lse;
-    base.lse2 = work + ((rows + 63) & ~int64_t(63));   // after D, 256-byte aligned
-    base.dvec = work;
+    base.nlse2 = work + ((rows + 63) & ~int64_t(63));   // after -D, 256-byte aligned
+    base.ndvec = work;
     base.scale = scale;
     base.scale_log2 = scale * kLog2e;
     base.ticket = reinterpret_cast<int*>(work + 2 * ((rows + 63) & ~int64_t(63)));   // after D and LSE2

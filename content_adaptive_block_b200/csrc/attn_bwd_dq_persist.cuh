@@ -224,38 +224,40 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int half = r >> 6;
         const int rr = r & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const bool issuer_warp = warp == 2;       // lane 0 issues every MMA of the CTA
+        // warp 2 issues every MMA of the CTA: converged, by vote, one elected lane issuing (the
+        // loop state and operands stay warp-uniform)
+        const bool issuer_warp = warp == 2;
+        const auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kErrTimeoutMma));
+        };
         constexpr uint32_t idesc_s = idesc_bf16(128, kBlk, 0);
         constexpr uint32_t idesc_dq = idesc_bf16(128, D, 1);
         const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO);
         auto issue_s = [&](int st) {   // S = Q K^T, dP = dO V^T of the stage's key block
             const uint32_t aKs = smem_u32(stage_k(st)), aVs = smem_u32(stage_v(st));
+            const uint64_t dq_ = sdesc_sw128(aQ, 16, 1024), dk_ = sdesc_sw128(aKs, 16, 1024);
+            const uint64_t ddo = sdesc_sw128(aDO, 16, 1024), dv_ = sdesc_sw128(aVs, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-                umma_bf16(tmem, sdesc_sw128(aQ + kk * 32, 16, 1024), sdesc_sw128(aKs + kk * 32, 16, 1024), idesc_s,
-                          kk > 0 ? 1u : 0u);
+                umma_bf16_w(tmem, sdesc_advance(dq_, kk * 32), sdesc_advance(dk_, kk * 32), idesc_s, kk > 0 ? 1u : 0u);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-                umma_bf16(tmem + 64, sdesc_sw128(aDO + kk * 32, 16, 1024), sdesc_sw128(aVs + kk * 32, 16, 1024),
-                          idesc_s, kk > 0 ? 1u : 0u);
-            umma_commit(s_full);
-            if ((meta[st] >> 18) & 1u) umma_commit(qd_free);   // the item's Q, dO are no longer read
+                umma_bf16_w(tmem + 64, sdesc_advance(ddo, kk * 32), sdesc_advance(dv_, kk * 32), idesc_s,
+                            kk > 0 ? 1u : 0u);
+            umma_commit_w(s_full);
+            if ((meta[st] >> 18) & 1u) umma_commit_w(qd_free);   // the item's Q, dO are no longer read
         };
         bool ok = true;
         if (issuer_warp) {
-            if (lane == 0) {
-                // the first item's first S, dP
-                ok = mbar_wait(&item_full[0], 0, abort_flag, kErrTimeoutMma);
-                if (ok && rec[0] >= 0) {
-                    ok = mbar_wait(qd_full, 0, abort_flag, kErrTimeoutMma) &&
-                         mbar_wait(&full[0], 0, abort_flag, kErrTimeoutMma);
-                    if (ok) {
-                        tc_fence_after();
-                        issue_s(0);
-                    }
+            // the first item's first S, dP
+            ok = wait_all(&item_full[0], 0);
+            if (ok && rec[0] >= 0) {
+                ok = wait_all(qd_full, 0) && wait_all(&full[0], 0);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
                 }
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
         }
         int gt = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
@@ -271,8 +273,9 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const int my_blk = half ? qb : qa;
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
             const int64_t tok = head_row0 + static_cast<int64_t>(my_blk < 0 ? 0 : my_blk) * kBlk + rr;
-            const float lse2 = my_blk >= 0 ? p.lse2[tok] : 0.f;
-            const float dt = my_blk >= 0 ? p.dvec[tok] : 0.f;
+            const float nlse2 = my_blk >= 0 ? p.nlse2[tok] : 0.f;
+            const float ndt = my_blk >= 0 ? p.ndvec[tok] : 0.f;
+            const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(nlse2, nlse2), nd2 = f2_pack(ndt, ndt);
             for (int ti = 0; ok; ++ti, ++gt) {
                 const int st = gt % C::kStages;
                 bool w_ok = mbar_wait(s_full, gt & 1, abort_flag, kErrTimeoutSoftmax);
@@ -307,7 +310,12 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         const float* d_ = dp[ch & 1];
                         const int cb = c0 + kW * ch;
 #pragma unroll
-                        for (int cc = 0; cc < kW; ++cc) s_[cc] = ex2(fmaf(s_[cc], p.scale_log2, -lse2)) * (d_[cc] - dt);
+                        for (int e = 0; e < kW / 2; ++e) {   // dS = 2^(S c - LSE log2 e) (dP - D), in pairs
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(s_[2 * e], s_[2 * e + 1]), sc2, nl2), x0, x1);
+                            const uint64_t pr = f2_pack(ex2(x0), ex2(x1));
+                            f2_unpack(f2_mul(pr, f2_add(f2_pack(d_[2 * e], d_[2 * e + 1]), nd2)), s_[2 * e], s_[2 * e + 1]);
+                        }
                         if (lastc < cb + kW - 1) {
 #pragma unroll
                             for (int cc = 0; cc < kW; ++cc) s_[cc] = cb + cc <= lastc ? s_[cc] : 0.f;
@@ -322,42 +330,38 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 tc_fence_before();
                 mbar_arrive(p_full);
                 if (issuer_warp) {
-                    bool go = true;
-                    if (lane == 0) {
-                        go = mbar_wait(p_full, gt & 1, abort_flag, kErrTimeoutMma);
-                        // the item's first accumulating product: the previous item's
-                        // epilogue has read dQ
-                        if (go && ti == 0 && k >= 1) go = mbar_wait(acc_free, (k - 1) & 1, abort_flag, kErrTimeoutMma);
-                        if (go) {
-                            tc_fence_after();
-                            const uint32_t aKs = smem_u32(stage_k(st));
+                    bool go = wait_all(p_full, gt & 1);
+                    // the item's first accumulating product: the previous item's epilogue has read dQ
+                    if (go && ti == 0 && k >= 1) go = wait_all(acc_free, (k - 1) & 1);
+                    if (go) {
+                        tc_fence_after();
+                        const uint64_t bk = sdesc_sw128(smem_u32(stage_k(st)), kBlk * 128, 1024);
 #pragma unroll
-                            for (int kk = 0; kk < kBlk / 16; ++kk) {
-                                const int h_ = (16 * kk) / kCols;   // the half holding keys 16 kk ..
-                                const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
-                                const uint64_t bd = sdesc_sw128(aKs + kk * (16 * 128), kBlk * 128, 1024);
-                                umma_bf16_ts(tmem + C::kTmemDQ, tmem + acol, bd, idesc_dq, (ti > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            umma_commit(&empty[st]);
-                            if (last) umma_commit(acc_done);
-                            // S, dP of the next tile, the next item's first after a last tile
-                            bool next = !last;
-                            if (last) {
-                                go = mbar_wait(&item_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag, kErrTimeoutMma);
-                                next = go && rec[(k + 1) & 1] >= 0;
-                            }
-                            if (next) {
-                                const int nst = (gt + 1) % C::kStages;
-                                go = mbar_wait(&full[nst], ((gt + 1) / C::kStages) & 1, abort_flag, kErrTimeoutMma);
-                                if (go && last) go = mbar_wait(qd_full, (k + 1) & 1, abort_flag, kErrTimeoutMma);
-                                if (go) {
-                                    tc_fence_after();
-                                    issue_s(nst);
-                                }
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            const int h_ = (16 * kk) / kCols;   // the half holding keys 16 kk ..
+                            const uint32_t acol = kCols * h_ + (16 * kk - kCols * h_) / 2;
+                            umma_bf16_ts_w(tmem + C::kTmemDQ, tmem + acol, sdesc_advance(bk, kk * (16 * 128)), idesc_dq,
+                                           (ti > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit_w(&empty[st]);
+                        if (last) umma_commit_w(acc_done);
+                        // S, dP of the next tile, the next item's first after a last tile
+                        bool next = !last;
+                        if (last) {
+                            go = wait_all(&item_full[(k + 1) & 1], ((k + 1) >> 1) & 1);
+                            next = go && rec[(k + 1) & 1] >= 0;
+                        }
+                        if (next) {
+                            const int nst = (gt + 1) % C::kStages;
+                            go = wait_all(&full[nst], ((gt + 1) / C::kStages) & 1);
+                            if (go && last) go = wait_all(qd_full, (k + 1) & 1);
+                            if (go) {
+                                tc_fence_after();
+                                issue_s(nst);
                             }
                         }
                     }
-                    if (!__shfl_sync(0xffffffffu, go, 0)) {
+                    if (!go) {
                         ok = false;
                         break;
                     }
@@ -390,9 +394,9 @@ dq_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             if (loads > 0) mbar_wait_drain(qd_full, (loads - 1) & 1);
             drain_fills(full, C::kStages, fills);
         }
-        if (warp == 2 && lane == 0) {
-            umma_commit(drain);
-            mbar_wait_drain(drain, 0);
+        if (warp == 2) {
+            umma_commit_w(drain);   // from the lane that issued the products
+            if (lane == 0) mbar_wait_drain(drain, 0);
         }
         __syncthreads();
     }

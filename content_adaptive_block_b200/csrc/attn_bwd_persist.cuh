@@ -240,8 +240,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         const int64_t row64 = head_row0 + l0;
                         load_rows<K4>(stage_q(st), &tmQ, &full[st], 0, l0, h_, s_, head_row0);
                         load_rows<K4>(stage_do(st), &tmDO, &full[st], 0, l0, h_, s_, head_row0);
-                        bulk_load(stage_lse(st), p.lse2 + row64, C::kVecBytes, &full[st]);
-                        bulk_load(stage_d(st), p.dvec + row64, C::kVecBytes, &full[st]);
+                        bulk_load(stage_lse(st), p.nlse2 + row64, C::kVecBytes, &full[st]);
+                        bulk_load(stage_d(st), p.ndvec + row64, C::kVecBytes, &full[st]);
                         ++gt;
                     }
                 }
@@ -263,6 +263,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int half = u >> 6;
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
         bool ok = true;
         int gt = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
@@ -324,12 +325,19 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                             const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
+                            for (int e = 0; e < 4; e += 2) {   // P^T = 2^(S^T c - LSE log2 e), dS^T = P^T (dP^T - D), in pairs
                                 const int cc = 4 * c4 + e;
-                                float pr = ex2(fmaf(s_[cc], p.scale_log2, -lv[e]));
-                                if (first > cb) pr = cb + cc >= first ? pr : 0.f;
-                                s_[cc] = pr;
-                                d_[cc] = pr * (d_[cc] - dd[e]);
+                                float x0, x1;
+                                f2_unpack(f2_fma(f2_pack(s_[cc], s_[cc + 1]), sc2, f2_pack(lv[e], lv[e + 1])), x0, x1);
+                                float p0 = ex2(x0), p1 = ex2(x1);
+                                if (first > cb) {
+                                    p0 = cb + cc >= first ? p0 : 0.f;
+                                    p1 = cb + cc + 1 >= first ? p1 : 0.f;
+                                }
+                                s_[cc] = p0;
+                                s_[cc + 1] = p1;
+                                f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(d_[cc], d_[cc + 1]), f2_pack(dd[e], dd[e + 1]))),
+                                          d_[cc], d_[cc + 1]);
                             }
                         }
 #pragma unroll
@@ -381,9 +389,11 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
         }
-    } else if ((warp == 1 || warp == 18) && lane == 0) {
-        // ================= MMA issuers (lane 0 of warps 1 and 18, on different SM sub-partitions: a
-        // tcgen05.mma takes issue slots its sub-partition's elementwise warps also want).  Warp 1
+    } else if (warp == 1 || warp == 18) {
+        // ================= MMA issuers (warps 1 and 18, on different SM sub-partitions: a
+        // tcgen05.mma takes issue slots its sub-partition's elementwise warps also want).  Each
+        // warp runs its loop converged (waits by vote) and one elected lane issues, so the loop
+        // state and operands stay warp-uniform.  Warp 1
         // issues S^T = K Q^T and dV += P^T dO, warp 18 dP^T = V dO^T and dK += dS^T Q: each TMEM
         // region (S^T and P^T, dP^T and dS^T, dV, dK) is written and read by one thread's products,
         // in its issue order, so the accumulation order is fixed.  Per tile: dV (dK) of tile n when
@@ -393,19 +403,22 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         constexpr uint32_t idesc_acc = idesc_bf16(128, D, 1);
         int nx = 0, nx_item = 0;   // next tile (and its item) whose scores to issue
         bool nx_first = true, nx_end = false;
+        const auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kErrTimeoutMma));
+        };
         // S^T = K Q^T, dP^T = V dO^T of tile nx into buffer nx & 1 (false: a wait gave up)
         auto issue_next = [&]() -> bool {
             if (nx_end) return true;
             if (nx_first) {
-                if (!mbar_wait(&item_full[nx_item & 1], (nx_item >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+                if (!wait_all(&item_full[nx_item & 1], (nx_item >> 1) & 1)) return false;
                 if (rec[nx_item & 1] < 0) {
                     nx_end = true;
                     return true;
                 }
-                if (!mbar_wait(&kv_full[nx_item & 1], (nx_item >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+                if (!wait_all(&kv_full[nx_item & 1], (nx_item >> 1) & 1)) return false;
             }
             const int st = nx % C::kStages;
-            if (!mbar_wait(&full[st], (nx / C::kStages) & 1, abort_flag, kErrTimeoutMma)) return false;
+            if (!wait_all(&full[st], (nx / C::kStages) & 1)) return false;
             tc_fence_after();
             const bool last = (meta[st] >> 18) & 1u;
             // this side's operands: K and Q (S^T) or V and dO (dP^T); descriptors built once per
@@ -415,9 +428,9 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const uint32_t dst = tmem + 128 * (nx & 1) + (side_s ? 0 : 64);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-                umma_bf16(dst, sdesc_advance(da, kk * 32), sdesc_advance(db, kk * 32), idesc_s, kk > 0 ? 1u : 0u);
-            umma_commit(&s_full[nx & 1]);
-            if (last) umma_commit(&kv_free[nx_item & 1]);   // the item's K, V are no longer read
+                umma_bf16_w(dst, sdesc_advance(da, kk * 32), sdesc_advance(db, kk * 32), idesc_s, kk > 0 ? 1u : 0u);
+            umma_commit_w(&s_full[nx & 1]);
+            if (last) umma_commit_w(&kv_free[nx_item & 1]);   // the item's K, V are no longer read
             ++nx;
             nx_first = last;
             if (last) ++nx_item;
@@ -425,9 +438,9 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         };
         bool ok = issue_next() && issue_next();
         for (int n = 0, k = 0, ti = 0; ok && n < nx; ++n) {
-            ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, abort_flag, kErrTimeoutMma);
+            ok = wait_all(&p_full[n & 1], (n >> 1) & 1);
             // the item's first accumulating products: the previous item's epilogue has read dV and dK
-            if (ok && ti == 0 && k >= 1) ok = mbar_wait(acc_free, (k - 1) & 1, abort_flag, kErrTimeoutMma);
+            if (ok && ti == 0 && k >= 1) ok = wait_all(acc_free, (k - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             const int st = n % C::kStages;
@@ -438,10 +451,10 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const uint64_t bb = sdesc_sw128(smem_u32(side_s ? stage_do(st) : stage_q(st)), kBlk * 128, 1024);
 #pragma unroll
             for (int kk = 0; kk < kBlk / 16; ++kk)
-                umma_bf16_ts(acc, ab + 16 * kk, sdesc_advance(bb, kk * (16 * 128)), idesc_acc,
-                             (ti > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(&empty[st]);
-            if (last) umma_commit(acc_done);
+                umma_bf16_ts_w(acc, ab + 16 * kk, sdesc_advance(bb, kk * (16 * 128)), idesc_acc,
+                               (ti > 0 || kk > 0) ? 1u : 0u);
+            umma_commit_w(&empty[st]);
+            if (last) umma_commit_w(acc_done);
             ok = issue_next();   // the scores of tile n + 2 into the buffer this tile's products read
             if (last) {
                 ++k;
@@ -461,9 +474,9 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (loads > 1) mbar_wait_drain(&kv_full[(loads - 2) & 1], ((loads - 2) >> 1) & 1);
             drain_fills(full, C::kStages, fills);
         }
-        if ((warp == 1 || warp == 18) && lane == 0) {
-            umma_commit(drain);
-            mbar_wait_drain(drain, 0);
+        if (warp == 1 || warp == 18) {
+            umma_commit_w(drain);   // from the lane that issued the products
+            if (lane == 0) mbar_wait_drain(drain, 0);
         }
         __syncthreads();
     }
