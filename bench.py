@@ -249,8 +249,9 @@ def run_reference(args, rank, world):
 # The kernels behind each timed call, and the sources whose hash ties a
 # recorded traffic figure to the code that produced it.
 _TRAFFIC_CALLS = {
-    "gsa_attn_fwd": (["attn_fwd_bf16_kernel<64, 0>"],
-                     ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh"]),
+    "gsa_attn_fwd": (["attn_fwd_persist_kernel<0>"],
+                     ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh",
+                      "content_adaptive_block_b200/csrc/attn_fwd_persist.cuh"]),
     "gsa_attn_bwd": (["dot_kernel<64>", "dq_persist_kernel<0>", "dkdv_persist_kernel<0>"],
                      ["content_adaptive_block_b200/csrc/attn_bwd_bf16.cuh",
                       "content_adaptive_block_b200/csrc/attn_bwd_persist.cuh",

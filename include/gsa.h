@@ -250,6 +250,11 @@ typedef struct {
  *   A(t) = { u <= t : block(u) in the CSR row i of (s, c) }.
  *   o [B][H][L][d] out (or desc->layout's strides), lse [B][H][L] float32 out
  *   (dense always; may be NULL for GSA_F32).
+ * bf16 at d = 64 runs persistent CTAs that draw work items from a counter in
+ * the library's device memory: one of 256 slots, taken in turn per call and
+ * returned to zero by the call's last CTA, so up to 256 such calls may be in
+ * flight at once (on any streams) on one device.  A query row with no live
+ * key (no mask built by this library has one) gets o = 0 and lse = -inf.
  * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, L != nblk*b, shapes that
  * disagree with csr, a class outside 0..2, bf16 tensors not 16-byte aligned,
  * a layout breaking its rules), GSA_ERR_UNSUPPORTED (dtype / b / d outside the
@@ -265,7 +270,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
  *   dV = P^T dO,  dS = P ∘ (dO V^T − D),  dQ = scale · dS K,  dK = scale · dS^T Q,
  * every sum over live pairs only.  o and lse are the forward's outputs.
  *   workspace: device scratch of at least gsa_attn_bwd_workspace(desc) bytes
- *              (holds D and LSE log2(e), float32 [B][H][L] each, then two
+ *              (holds -D and -LSE log2(e), float32 [B][H][L] each, then two
  *              work counters); its contents need no init.
  * dq, dk, dv are written (not accumulated).  Deterministic: each output row
  * is summed by one CTA in a fixed order (the only atomic hands out work

@@ -222,7 +222,7 @@ def test_attn_bwd_rejects_bad_arguments(lib):
     d, keep = _desc()
     ws = lib.gsa_attn_bwd_workspace(ctypes.byref(d))
     rows = 1 * 4 * 256
-    assert ws == 2 * 4 * ((rows + 63) // 64 * 64) + 256   # D and LSE log2(e) (float32 per row), then counters
+    assert ws == 2 * 4 * ((rows + 63) // 64 * 64) + 256   # -D and -LSE log2(e) (float32 per row), then counters
     args = [FAKE] * 6
     assert f(*args[:5], NULL, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws, NULL) == 1
     assert f(*args, ctypes.byref(c), ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws - 4, NULL) == 3
