@@ -29,9 +29,12 @@
 //            lane issues.  tcgen05 products of one thread run in
 //            issue order, so the QK^T of tile n + 2 goes into the S buffer of
 //            tile n right after the P V products that read its P;
-//   warps 2-9 softmax warpgroups; after an item's last tile the same threads
-//            normalise O and store it with the LSE, so O is read before they
-//            release the next item's first P, whose P V overwrites it.
+//   warps 2-9 softmax warpgroups.  An item's epilogue (O / l and the LSE)
+//            runs inside the next item's first tile, between storing its P
+//            and releasing it: the wait for the previous tile's P V, taken
+//            every tile, has by then shown the item's last product complete,
+//            and O is read before the P V that overwrites it is issued.  The
+//            item's query blocks come with its record, from shared memory.
 // The counter is one of a ring of device-global slots picked per launch; the
 // launch's last CTA to leave returns its slot to zero.  An item without a
 // live key block (no mask built here has one: every row holds its diagonal
@@ -59,13 +62,13 @@ struct FwdPCfg {
     static constexpr int kOffStage = kOffQ + 2 * kQBytes;
     static constexpr int kOffMeta = kOffStage + kStages * kStageBytes;   // per stage: block | live << 16 | last << 18
     static constexpr int kOffBar = kOffMeta + ((kStages * 4 + 7) & ~7);
-    // full[st], empty[st], q_full[2], q_free[2], s_full[2], p_full[2], acc_done,
-    // item_full[2], rec_free[2], drain
-    static constexpr int kNumBars = 2 * kStages + 14;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
-    static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
+    // full[st], empty[st], q_full[2], q_free[2], s_full[2], p_full[2], item_full[2], rec_free[2],
+    // drain, ml_full[4]
+    static constexpr int kNumBars = 2 * kStages + 17;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort, item record[2][2]
+    static constexpr int kOffBits = kOffMisc + 32;            // producer's two bitmaps
     // [item parity][2 halves][m, l][128 rows]: a warp writes a buffer again only after
-    // the next item's pair barrier, which the other warp reaches after its reads
+    // the next item's exchange phase, which the other warp joins after its reads
     static constexpr int kOffMl = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kEnd = kOffMl + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
@@ -94,15 +97,18 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     uint64_t* q_free = q_full + 2;              // [2] item k's last QK^T completed (phase k >> 1)
     uint64_t* s_full = q_free + 2;              // [2] QK^T of tile n landed in S[n & 1] (phase n >> 1)
     uint64_t* p_full = s_full + 2;              // [2] P of tile n over S[n & 1] (256 arrivals, phase n >> 1)
-    uint64_t* acc_done = p_full + 2;            // item k's last P V completed (phase k & 1)
     // [2] item k's record (or the end) published in slot k & 1 (phase k >> 1);
     // the slot is written again once the softmax threads read it (rec_free)
     // and the MMA thread issued the item's last QK^T (q_free)
-    uint64_t* item_full = acc_done + 1;
+    uint64_t* item_full = p_full + 2;
     uint64_t* rec_free = item_full + 2;
     uint64_t* drain = rec_free + 2;             // the MMA thread's products at exit
+    // [quadrant] both halves' (m, l) of an item's rows are in shared memory (64 arrivals: the
+    // quadrant's two softmax warps; phase per item)
+    uint64_t* ml_full = drain + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    // record slot b: rec[2 b] = item (-1: the end), rec[2 b + 1] = qa | (qb + 1) << 16
     int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
     uint32_t* bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
     uint32_t* bitsB = bitsA + kListMaxBlocks / 32;
@@ -137,8 +143,8 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             mbar_init(&item_full[b], 1);
             mbar_init(&rec_free[b], C::kSoftmax);
         }
-        mbar_init(acc_done, 1);
         mbar_init(drain, 1);
+        for (int q = 0; q < 4; ++q) mbar_init(&ml_full[q], 64);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -218,7 +224,8 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     ok = mbar_wait(&rec_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer) &&
                          mbar_wait(&q_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer);
                 }
-                rec[k & 1] = (ok && have) ? it : -1;
+                rec[2 * (k & 1)] = (ok && have) ? it : -1;
+                rec[2 * (k & 1) + 1] = qa | ((qb + 1) << 16);
                 mbar_arrive(&item_full[k & 1]);
                 if (ok && have) {
                     mbar_arrive_expect_tx(&q_full[k & 1], (qb >= 0 ? 2 : 1) * kBlk * D * 2);
@@ -278,7 +285,7 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             if (!qk_end) {
                 if (!item_open) {
                     if (all(mbar_test(&item_full[kq & 1], (kq >> 1) & 1))) {
-                        if (rec[kq & 1] < 0) qk_end = true;
+                        if (rec[2 * (kq & 1)] < 0) qk_end = true;
                         else item_open = true;
                         q_ready = false;
                         moved = true;
@@ -323,12 +330,7 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     umma_bf16_ts_w(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
                                    sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
                 umma_commit_w(&empty[st]);
-                if (last) {
-                    umma_commit_w(acc_done);
-                    ta = 0;
-                } else {
-                    ++ta;
-                }
+                ta = last ? 0 : ta + 1;
                 ++na;
                 moved = true;
             }
@@ -351,6 +353,44 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t tO = tl + C::kTmemO + 64 * hc;
         float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
+        // the previous item's epilogue, run once its last P V completed: combine the halves'
+        // (m, l) through shared memory (double-buffered by item parity: a warp writes a buffer
+        // again only after the next item's exchange phase, which the other warp joins after its
+        // reads; a bounded mbarrier wait, so a partner that gave up cannot hang it), then O / l
+        // for this thread's 32 output columns and the LSE.  False: a wait gave up.
+        struct Pending {
+            bool on = false;
+            int parity = 0;
+            int64_t tok = -1;   // this row's token (-1: no row)
+            float m = 0.f, l = 0.f;
+        } pend;
+        auto epilogue = [&]() -> bool {
+            float* mlk = ml + pend.parity * (4 * 128);
+            mlk[(hc * 2 + 0) * 128 + r] = pend.m;
+            mlk[(hc * 2 + 1) * 128 + r] = pend.l;
+            mbar_arrive(&ml_full[quad]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&ml_full[quad], pend.parity, abort_flag, kErrTimeoutSoftmax)))
+                return false;
+            const float mA = mlk[0 * 128 + r], lA = mlk[1 * 128 + r];
+            const float mB = mlk[2 * 128 + r], lB = mlk[3 * 128 + r];
+            const float mm = fmaxf(mA, mB);
+            const float wA = mA == -INFINITY ? 0.f : ex2(mA - mm);
+            const float wB = mB == -INFINITY ? 0.f : ex2(mB - mm);
+            const float lt = lA * wA + lB * wB;
+            float a[32], b2[32];
+            tmem_ld32(tl + C::kTmemO + c0, a);
+            tmem_ld32(tl + C::kTmemO + 64 + c0, b2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) a[e] = fmaf(b2[e], wB, a[e] * wA);
+            if (pend.tok >= 0) {
+                __nv_bfloat16* orow = p.o + (K4 ? tok_off(pend.tok, p.L, p.H, p.lo) : pend.tok * D);
+                store_scaled_bf16(orow + c0, a, rcp_approx(lt));
+                if (hc == 0) p.lse[pend.tok] = (mm + lg2_approx(lt)) * 0.69314718055994531f;
+            }
+            pend.on = false;
+            return true;
+        };
         bool ok = true;
         int n = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
@@ -358,13 +398,24 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 ok = false;
                 break;
             }
-            const int it = rec[k & 1];
+            const int it = rec[2 * (k & 1)];
+            const int qw = rec[2 * (k & 1) + 1];
             mbar_arrive(&rec_free[k & 1]);
-            if (it < 0) break;
-            int sh, qa, qb;
-            int64_t g;
-            item_keys(it, sh, qa, qb, g);
-            const int my_blk = half ? qb : qa;
+            if (it < 0) {
+                // the last item's epilogue: its last P V (tile n - 1) completes the stage's phase
+                if (pend.on) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&empty[(n - 1) % C::kStages], ((n - 1) / C::kStages) & 1,
+                                                           abort_flag, kErrTimeoutSoftmax))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!epilogue()) ok = false;
+                }
+                break;
+            }
+            const int sh = it % SH;
+            const int my_blk = half ? (qw >> 16) - 1 : (qw & 0xffff);
             float m = -INFINITY, l = 0.f;   // running max (log2 units) and sum of this row's half
             for (;; ++n) {
                 const int sb = n & 1, st = n % C::kStages;
@@ -429,6 +480,11 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     break;
                 }
                 tc_fence_after();
+                // the previous item's O: read before this tile's P V overwrites it
+                if (pend.on && !epilogue()) {
+                    ok = false;
+                    break;
+                }
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                     for (int cb = 0; cb < D; cb += 32) {
@@ -445,34 +501,12 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 mbar_arrive(&p_full[sb]);
                 if (last_tile) {
                     ++n;
-                    // epilogue: combine the halves, O / l for this thread's 32 output columns, LSE
-                    float* mlk = ml + (k & 1) * (4 * 128);
-                    mlk[(hc * 2 + 0) * 128 + r] = m;
-                    mlk[(hc * 2 + 1) * 128 + r] = l;
-                    pair_barrier(quad);
-                    const float mA = mlk[0 * 128 + r], lA = mlk[1 * 128 + r];
-                    const float mB = mlk[2 * 128 + r], lB = mlk[3 * 128 + r];
-                    if (!__all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, abort_flag, kErrTimeoutSoftmax))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const float mm = fmaxf(mA, mB);
-                    const float wA = mA == -INFINITY ? 0.f : ex2(mA - mm);
-                    const float wB = mB == -INFINITY ? 0.f : ex2(mB - mm);
-                    const float lt = lA * wA + lB * wB;
-                    float a[32], b2[32];
-                    tmem_ld32(tl + C::kTmemO + c0, a);
-                    tmem_ld32(tl + C::kTmemO + 64 + c0, b2);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = fmaf(b2[e], wB, a[e] * wA);
-                    if (my_blk >= 0) {
-                        const int64_t tok = static_cast<int64_t>(sh) * p.L + static_cast<int64_t>(my_blk) * kBlk + rr;
-                        __nv_bfloat16* orow = p.o + (K4 ? tok_off(tok, p.L, p.H, p.lo) : tok * D);
-                        store_scaled_bf16(orow + c0, a, 1.f / lt);
-                        if (hc == 0) p.lse[tok] = (mm + log2f(lt)) * 0.69314718055994531f;
-                    }
+                    pend.on = true;
+                    pend.parity = k & 1;
+                    pend.tok = my_blk >= 0 ? static_cast<int64_t>(sh) * p.L + static_cast<int64_t>(my_blk) * kBlk + rr
+                                           : -1;
+                    pend.m = m;
+                    pend.l = l;
                     break;
                 }
             }

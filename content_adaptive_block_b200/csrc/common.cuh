@@ -433,6 +433,19 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 1/x and log2(x) on the special-function unit (approximate: about 1 ulp and
+// 2^-22 relative in the normal range; flush-to-zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Packed fp32 pairs (sm_100): two lanes of IEEE single precision in one
 // 64-bit register, one instruction for both (the same rounding as two scalar
 // operations).
