@@ -56,8 +56,8 @@ struct DkvPCfg {
     // full[st], empty[st], kv_full[2], kv_free[2], s_full[2], p_full[2], acc_done, acc_free,
     // item_full[2], rec_free[2], drain
     static constexpr int kNumBars = 2 * kStages + 17;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2]
-    static constexpr int kOffBits = kOffMisc + 16;                       // producer's two bitmaps
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;              // tmem base, abort, item record[2][2]
+    static constexpr int kOffBits = kOffMisc + 32;                       // producer's two bitmaps
     static constexpr int kEnd = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
     static_assert(kSmemBytes <= 232448 - 1024, "shared memory per CTA");
@@ -97,7 +97,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint64_t* drain = rec_free + 2;              // the MMA thread's products at exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-    int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // [2] item k at rec[k & 1], -1: end
+    // record slot b: rec[2 b] = item (-1: the end), rec[2 b + 1] = ka | (kb + 1) << 16
+    int* rec = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
     uint32_t* bitsA = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
     uint32_t* bitsB = bitsA + kListMaxBlocks / 32;
     auto tile_k = [&](int b) { return smem + C::kOffKV + b * 2 * C::kTileBytes; };
@@ -202,7 +203,8 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (k >= 2 && !(mbar_wait(&rec_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer) &&
                                 mbar_wait(&kv_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, kErrTimeoutProducer)))
                     ok = false;
-                rec[k & 1] = (ok && have) ? it : -1;
+                rec[2 * (k & 1)] = (ok && have) ? it : -1;
+                rec[2 * (k & 1) + 1] = ka | ((kb + 1) << 16);
                 mbar_arrive(&item_full[k & 1]);
                 if (ok && have) {
                     ++nload;
@@ -264,6 +266,44 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int uu = u & 63;
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        // The previous item's epilogue (dV, dK of this thread's row, its 16 columns) runs inside
+        // the next item's first tile, after its P^T, dS^T are stored and before they are released:
+        // by then the item's last products have long been issued, and the accumulators are read
+        // (acc_free) before the next item's first accumulating products, which wait for it.
+        struct Pending {
+            bool on = false;
+            int parity = 0;
+            int64_t tok = -1;   // this row's token (-1: no row)
+        } pend;
+        auto epilogue = [&]() -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_done, pend.parity, abort_flag, kErrTimeoutSoftmax))) return false;
+            tc_fence_after();
+            float ov[16], ok_[16];
+            tmem_ld16(tlane + C::kTmemDV + c0, ov);
+            tmem_ld16(tlane + C::kTmemDK + c0, ok_);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(acc_free);   // the accumulators may take the next item's products
+            if (pend.tok >= 0) {
+                const int64_t off = (K4 ? tok_off(pend.tok, p.L, p.H, p.lq) : pend.tok * D) + c0;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint4 a, b;
+                    a.x = pack_bf16x2(ov[8 * h2 + 0], ov[8 * h2 + 1]);
+                    a.y = pack_bf16x2(ov[8 * h2 + 2], ov[8 * h2 + 3]);
+                    a.z = pack_bf16x2(ov[8 * h2 + 4], ov[8 * h2 + 5]);
+                    a.w = pack_bf16x2(ov[8 * h2 + 6], ov[8 * h2 + 7]);
+                    b.x = pack_bf16x2(ok_[8 * h2 + 0] * p.scale, ok_[8 * h2 + 1] * p.scale);
+                    b.y = pack_bf16x2(ok_[8 * h2 + 2] * p.scale, ok_[8 * h2 + 3] * p.scale);
+                    b.z = pack_bf16x2(ok_[8 * h2 + 4] * p.scale, ok_[8 * h2 + 5] * p.scale);
+                    b.w = pack_bf16x2(ok_[8 * h2 + 6] * p.scale, ok_[8 * h2 + 7] * p.scale);
+                    *reinterpret_cast<uint4*>(p.out0 + off + 8 * h2) = a;
+                    *reinterpret_cast<uint4*>(p.out1 + off + 8 * h2) = b;
+                }
+            }
+            pend.on = false;
+            return true;
+        };
         bool ok = true;
         int gt = 0;   // tiles done so far, across items
         for (int k = 0; ok; ++k) {
@@ -271,13 +311,15 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 ok = false;
                 break;
             }
-            const int it = rec[k & 1];
+            const int it = rec[2 * (k & 1)];
+            const int kw = rec[2 * (k & 1) + 1];
             mbar_arrive(&rec_free[k & 1]);   // the slot may take item k + 2
-            if (it < 0) break;
-            int sh, ka, kb;
-            int64_t g;
-            item_keys(it, sh, ka, kb, g);
-            const int my_blk = half ? kb : ka;
+            if (it < 0) {
+                if (pend.on && !epilogue()) ok = false;   // the last item's
+                break;
+            }
+            const int sh = it % SH;
+            const int my_blk = half ? (kw >> 16) - 1 : (kw & 0xffff);
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
             for (int ti = 0; ok; ++ti, ++gt) {
                 const int st = gt % C::kStages;
@@ -351,40 +393,17 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tmem_stn<kCols / 2>(tb + c0, pp);
                 tmem_stn<kCols / 2>(tb + 64 + c0, pd);
                 tmem_wait_st();
+                if (pend.on && !epilogue()) {   // the previous item's dV, dK
+                    ok = false;
+                    break;
+                }
                 tc_fence_before();
                 mbar_arrive(&p_full[gt & 1]);
                 if (last) {
                     ++gt;
-                    // epilogue of the item: dV, dK of this thread's row, its 16 columns
-                    if (!__all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, abort_flag, kErrTimeoutSoftmax))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    float ov[16], ok_[16];
-                    tmem_ld16(tlane + C::kTmemDV + c0, ov);
-                    tmem_ld16(tlane + C::kTmemDK + c0, ok_);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(acc_free);   // the accumulators may take the next item's products
-                    if (my_blk >= 0) {
-                        const int64_t tok = head_row0 + static_cast<int64_t>(my_blk) * kBlk + uu;
-                        const int64_t off = (K4 ? tok_off(tok, p.L, p.H, p.lq) : tok * D) + c0;
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            uint4 a, b;
-                            a.x = pack_bf16x2(ov[8 * h2 + 0], ov[8 * h2 + 1]);
-                            a.y = pack_bf16x2(ov[8 * h2 + 2], ov[8 * h2 + 3]);
-                            a.z = pack_bf16x2(ov[8 * h2 + 4], ov[8 * h2 + 5]);
-                            a.w = pack_bf16x2(ov[8 * h2 + 6], ov[8 * h2 + 7]);
-                            b.x = pack_bf16x2(ok_[8 * h2 + 0] * p.scale, ok_[8 * h2 + 1] * p.scale);
-                            b.y = pack_bf16x2(ok_[8 * h2 + 2] * p.scale, ok_[8 * h2 + 3] * p.scale);
-                            b.z = pack_bf16x2(ok_[8 * h2 + 4] * p.scale, ok_[8 * h2 + 5] * p.scale);
-                            b.w = pack_bf16x2(ok_[8 * h2 + 6] * p.scale, ok_[8 * h2 + 7] * p.scale);
-                            *reinterpret_cast<uint4*>(p.out0 + off + 8 * h2) = a;
-                            *reinterpret_cast<uint4*>(p.out1 + off + 8 * h2) = b;
-                        }
-                    }
+                    pend.on = true;
+                    pend.parity = k & 1;
+                    pend.tok = my_blk >= 0 ? head_row0 + static_cast<int64_t>(my_blk) * kBlk + uu : -1;
                     break;
                 }
             }
@@ -411,7 +430,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (nx_end) return true;
             if (nx_first) {
                 if (!wait_all(&item_full[nx_item & 1], (nx_item >> 1) & 1)) return false;
-                if (rec[nx_item & 1] < 0) {
+                if (rec[2 * (nx_item & 1)] < 0) {
                     nx_end = true;
                     return true;
                 }
