@@ -151,3 +151,37 @@ def test_b1_64k_sampled(gsa):
                     np.random.default_rng(1).integers(0, wl.N, 12).tolist()))
     pairs = {(0, 0), (0, 7), (0, 8), (0, 11), (0, 12), (0, 15)}
     _compare(o, lse, q, k, v, fl, wl.w, hc, wl.b, TOL_BF16, TOL_LSE_BF16, pairs=pairs, q_blocks=qb)
+
+
+def test_bf16_concurrent_streams_and_counter_slots(gsa):
+    """The d=64 bf16 forward's persistent CTAs draw items from a device-global
+    counter slot per call: four calls in flight on four streams, and more calls
+    in a row than there are slots, give the outputs of one call at a time,
+    bit for bit (each item's arithmetic does not depend on the CTA taking it)."""
+    wl = W.WORKLOADS["b8_4k"]
+    fl = _flags_for(W.batch_bytes(wl), wl.b)
+    hc = list(wl.head_classes())
+    csr = gsa.gsa_build_block_csr(torch.from_numpy(fl.astype(np.uint8)).cuda(), wl.w)
+    ins = [[t.cuda() for t in W.qkv(wl, seed=seed)] for seed in range(4)]
+    want = []
+    for q, k, v in ins:
+        o, lse = gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b)
+        want.append((o.clone(), lse.clone()))
+    torch.cuda.synchronize()
+    outs = [(torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)) for q, _, _ in ins]
+    streams = [torch.cuda.Stream() for _ in ins]
+    for (q, k, v), (o, lse), st in zip(ins, outs, streams):
+        st.wait_stream(torch.cuda.current_stream())
+        gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse, stream=st)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    for (o, lse), (wo, wlse) in zip(outs, want):
+        assert torch.equal(o, wo) and torch.equal(lse, wlse)
+    # more calls than counter slots (256): every slot comes back to zero
+    q, k, v = ins[0]
+    o, lse = outs[0]
+    for _ in range(300):
+        gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    assert torch.equal(o, want[0][0]) and torch.equal(lse, want[0][1])
