@@ -70,6 +70,67 @@ def live_token_pairs_from_counts(nnz_sc, n, b, head_classes):
 
 # ------------------------------------------------------------------ clocks
 
+class NvmlClockSampler:
+    """SM clock and clock-event (throttle) reasons read through NVML every 10 ms
+    from a background thread while the timed loop runs (read-only queries; the
+    main thread releases the GIL while it waits on the GPU).  Same summary as
+    ClockSampler; start() raises when NVML or the device is not available."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.device = device_index
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.stop_flag = None
+
+    def start(self):
+        import threading
+        import pynvml as nv
+        import torch
+        nv.nvmlInit()
+        u = str(torch.cuda.get_device_properties(self.device).uuid)
+        handle = nv.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        self.nv, self.handle = nv, handle
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        self.masks = [(name, getattr(nv, const)) for name, const in self.REASONS]
+        self.stop_flag = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                    why = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    self.rows.append((sm, why))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        if not self.rows:
+            return None
+        sm = [float(r[0]) for r in self.rows]
+        reasons = sorted({name for _, why in self.rows for name, m in self.masks if why & m})
+        loaded = [x for x in sm if x > 0.5 * self.max_mhz] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
+                "samples": len(self.rows), "source": "nvml, 10 ms"}
+
+
 class ClockSampler:
     """nvidia-smi sampling of the SM clock and throttle reasons while running."""
 
@@ -424,12 +485,18 @@ def run_ours(args, rank, world, local_rank):
     step_flops = fwd_flops + bwd_flops
     dense_pairs = wl.S * wl.H * wl.L * (wl.L + 1) // 2
 
-    sampler = ClockSampler(local_rank) if rank == 0 else None
+    sampler = None
+    if rank == 0:
+        # NVML in a thread (many samples inside a short timed region); nvidia-smi when NVML is absent
+        try:
+            sampler = NvmlClockSampler(local_rank)
+            sampler.start()
+        except Exception:
+            sampler = ClockSampler(local_rank)
+            sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
