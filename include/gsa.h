@@ -253,8 +253,9 @@ typedef struct {
  * bf16 at d = 64 runs persistent CTAs that draw work items from a counter in
  * the library's device memory: one of 256 slots, taken in turn per call and
  * returned to zero by the call's last CTA, so up to 256 such calls may be in
- * flight at once (on any streams) on one device.  A query row with no live
- * key (no mask built by this library has one) gets o = 0 and lse = -inf.
+ * flight at once (on any streams) on one device.  Every query row needs at
+ * least one live key, as in every mask built by this library (each block
+ * sees itself); a row without one has no defined output.
  * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, L != nblk*b, shapes that
  * disagree with csr, a class outside 0..2, bf16 tensors not 16-byte aligned,
  * a layout breaking its rules), GSA_ERR_UNSUPPORTED (dtype / b / d outside the
