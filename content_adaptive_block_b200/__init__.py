@@ -22,9 +22,10 @@ import torch
 
 __all__ = [
     "GsaError", "BlockCsr", "HEAD_LOCAL", "HEAD_LITERAL", "HEAD_HYBRID",
-    "gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_csr_capacity",
-    "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_attn_bwd_noalloc", "gsa_device_error",
-    "gsa_status_string", "library", "library_path",
+    "gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_build_fixed_csr", "gsa_mask_pipeline",
+    "gsa_csr_capacity", "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_attn_bwd_noalloc",
+    "gsa_attn_bwd_noalloc_max_rows", "gsa_lm_block_workspace", "gsa_lm_block_fwd", "gsa_lm_block_bwd",
+    "gsa_device_error", "gsa_status_string", "library", "library_path",
 ]
 
 HEAD_LOCAL, HEAD_LITERAL, HEAD_HYBRID = 0, 1, 2
@@ -361,6 +362,14 @@ def gsa_attn_bwd(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale
         _stream(stream)))
     del keep
     return dq, dk, dv
+
+
+def gsa_attn_bwd_noalloc_max_rows() -> int:
+    """Query rows (B·H·L) the built-in scratch of gsa_attn_bwd_noalloc holds."""
+    fn = library().gsa_attn_bwd_noalloc_max_rows
+    fn.argtypes = []
+    fn.restype = ctypes.c_int64
+    return int(fn())
 
 
 def gsa_attn_bwd_noalloc(q, k, v, o, lse, do, csr: BlockCsr, head_classes, b: int, scale: float = 0.0,

@@ -240,3 +240,23 @@ def test_python_binding_refuses_cpu_tensors(lib):
         gsa.gsa_block_lengths(torch.zeros((1, 64), dtype=torch.uint8), 64)
     with pytest.raises(ValueError):
         gsa.gsa_literal_flags(torch.zeros((1, 4), dtype=torch.int32))
+
+
+def test_binding_mirrors_every_header_function():
+    """The Python binding exposes each C entry point of include/*.h under the
+    same name (and lists it in __all__)."""
+    import re
+    import content_adaptive_block_b200 as gsa
+    names = set()
+    for h in ("gsa.h", "gsa_lm.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        names |= set(re.findall(r"^[A-Za-z_][\w \*]*?\b(gsa_\w+)\s*\(", text, re.M))
+    assert len(names) >= 16, names
+    for n in sorted(names):
+        assert callable(getattr(gsa, n, None)), n
+        assert n in gsa.__all__, n
+
+
+def test_noalloc_max_rows_through_the_binding():
+    import content_adaptive_block_b200 as gsa
+    assert gsa.gsa_attn_bwd_noalloc_max_rows() == 1 << 21
