@@ -43,7 +43,8 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return SRCS + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    return (SRCS + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(HERE, "csrc", "*.h")) +
+            glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def up_to_date() -> bool:

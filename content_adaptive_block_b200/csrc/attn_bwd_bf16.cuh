@@ -835,22 +835,18 @@ template <int D, bool K4>
 gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                     const __nv_bfloat16* o, const __nv_bfloat16* dO, const TokLayout& lo, Params pq, Params pkv,
                     int S, int H, int nblk, cudaStream_t st) {
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(dq_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemBytes);
-        cudaFuncSetAttribute(dkdv_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvCfg<D>::kSmemBytes);
-    });
+    const bool persist_q = D == 64 && GSA_DQ_PERSIST, persist_kv = D == 64 && GSA_DKV_PERSIST;
+    if (!(persist_q ? smem_opt_in(dq_persist_kernel<K4>, DqPCfg::kSmemBytes)
+                    : smem_opt_in(dq_kernel<D, K4>, DqCfg<D>::kSmemBytes)) ||
+        !(persist_kv ? smem_opt_in(dkdv_persist_kernel<K4>, DkvPCfg::kSmemBytes)
+                     : smem_opt_in(dkdv_kernel<D, K4>, DkvCfg<D>::kSmemBytes)))
+        return GSA_ERR_CUDA;
     constexpr int kRowsPerCta = 256 / (D / 8);   // 32 or 16: divides L
     const int sh_grid = S * H < 65535 ? S * H : 65535;
     dot_kernel<D><<<dim3(static_cast<unsigned>(pq.L / kRowsPerCta), static_cast<unsigned>(sh_grid)), 256, 0, st>>>(
         o, dO, lo, pq.L, pq.H, S * H, const_cast<float*>(pq.ndvec), pq.lse, const_cast<float*>(pq.nlse2), pkv.ticket);
     dim3 grid(S * H, (nblk + 1) / 2);
-    if (D == 64 && GSA_DQ_PERSIST) {
-        static std::once_flag once_q;
-        std::call_once(once_q, [] {
-            cudaFuncSetAttribute(dq_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DqPCfg::kSmemBytes);
-        });
+    if (persist_q) {
         const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
         const int64_t ctas = items < 2 * sm_count() ? items : 2 * sm_count();
         dq_persist_kernel<K4><<<static_cast<unsigned>(ctas), DqPCfg::kThreads, DqPCfg::kSmemBytes, st>>>(tq, tk, tv,
@@ -858,12 +854,7 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     } else {
         dq_kernel<D, K4><<<grid, Shape<D>::kThreads, DqCfg<D>::kSmemBytes, st>>>(tq, tk, tv, tdo, pq);
     }
-    if (D == 64 && GSA_DKV_PERSIST) {   // one CTA per SM, double-buffered scores
-        static std::once_flag once_p;
-        std::call_once(once_p, [] {
-            cudaFuncSetAttribute(dkdv_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DkvPCfg::kSmemBytes);
-        });
+    if (persist_kv) {   // one CTA per SM, double-buffered scores
         const int64_t items = static_cast<int64_t>(S) * H * ((nblk + 1) / 2);
         const int64_t ctas = items < sm_count() ? items : sm_count();
         dkdv_persist_kernel<K4><<<static_cast<unsigned>(ctas), DkvPCfg::kThreads, DkvPCfg::kSmemBytes, st>>>(

@@ -12,6 +12,8 @@
 
 #include <mutex>
 
+#include "host_attr.h"
+
 namespace gsa {
 
 // Codes kernels leave in the device error word (read by gsa_device_error).

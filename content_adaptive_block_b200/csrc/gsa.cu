@@ -119,28 +119,22 @@ gsa_status resolve_layout(const gsa_attn_desc* d, gsa::TokLayout* lq, gsa::TokLa
 }
 
 template <int D, bool K4>
-void launch_fwd(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const gsa::bf16::FwdParams& p, cudaStream_t cs) {
+gsa_status launch_fwd(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const gsa::bf16::FwdParams& p, cudaStream_t cs) {
     using C = gsa::bf16::FwdCfg<D>;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(gsa::bf16::attn_fwd_bf16_kernel<D, K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes);
-    });
+    if (!gsa::smem_opt_in(gsa::bf16::attn_fwd_bf16_kernel<D, K4>, C::kSmemBytes)) return GSA_ERR_CUDA;
     gsa::bf16::attn_fwd_bf16_kernel<D, K4><<<grid, gsa::bf16::FwdShape<D>::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv,
                                                                                                         p);
+    return launch_status();
 }
 
 template <bool K4>
-void launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const gsa::bf16::FwdParams& p, cudaStream_t cs) {
+gsa_status launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const gsa::bf16::FwdParams& p, cudaStream_t cs) {
     using C = gsa::bf16::FwdPCfg;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(gsa::bf16::attn_fwd_persist_kernel<K4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes);
-    });
+    if (!gsa::smem_opt_in(gsa::bf16::attn_fwd_persist_kernel<K4>, C::kSmemBytes)) return GSA_ERR_CUDA;
     gsa::bf16::attn_fwd_persist_kernel<K4><<<ctas, C::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+    return launch_status();
 }
 
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
@@ -169,29 +163,28 @@ int64_t gsa_csr_capacity(int32_t nblk) {
 }
 
 gsa_status gsa_block_lengths(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t* lengths, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_block_lengths");
     if (!bytes || !lengths || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES || L < b || L % b != 0)
         return GSA_ERR_INVALID_ARGUMENT;
     using namespace gsa::deflate;
     const int64_t total = static_cast<int64_t>(B) * (L / b);
     const int64_t grid = (total + kLenWarps - 1) / kLenWarps;
     if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(block_lengths_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kLenSmemBytes));
-    });
+    if (!gsa::smem_opt_in(block_lengths_kernel, static_cast<int>(kLenSmemBytes))) return GSA_ERR_CUDA;
     block_lengths_kernel<<<static_cast<unsigned>(grid), 32 * kLenWarps, kLenSmemBytes, as_stream(stream)>>>(
         bytes, L, b, total, lengths);
     return launch_status();
 }
 
 gsa_status gsa_literal_flags(const int32_t* lengths, int32_t B, int32_t nblk, uint8_t* flags, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_literal_flags");
     if (!lengths || !flags || B < 1 || nblk < 1) return GSA_ERR_INVALID_ARGUMENT;
     gsa::mask::literal_flags_kernel<<<B, 256, 0, as_stream(stream)>>>(lengths, nblk, flags);
     return launch_status();
 }
 
 gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* csr, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_build_block_csr");
     if (!flags || !csr || w < 0) return GSA_ERR_INVALID_ARGUMENT;
     if (csr->B < 1 || csr->nblk < 1 || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
         !csr->q_order || !csr->k_order)
@@ -211,11 +204,9 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* c
     a.q_order = csr->q_order;
     a.k_order = csr->k_order;
     const size_t smem = gsa::mask::csr_smem_bytes(csr->nblk);
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(gsa::mask::build_csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gsa::mask::csr_smem_bytes(gsa::mask::kMaxBlocksCsr)));
-    });
+    if (!gsa::smem_opt_in(gsa::mask::build_csr_kernel,
+                          static_cast<int>(gsa::mask::csr_smem_bytes(gsa::mask::kMaxBlocksCsr))))
+        return GSA_ERR_CUDA;
     dim3 grid(3, csr->B);
     gsa::mask::build_csr_kernel<<<grid, gsa::mask::kThreads, smem, as_stream(stream)>>>(a);
     return launch_status();
@@ -223,6 +214,7 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* c
 
 gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, const uint32_t* rnd,
                                gsa_block_csr* csr, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_build_fixed_csr");
     if (!csr || (kind != GSA_FIXED_LONGFORMER && kind != GSA_FIXED_BIGBIRD) || w < 0 || g < 0 || r < 0)
         return GSA_ERR_INVALID_ARGUMENT;
     if (kind == GSA_FIXED_LONGFORMER) r = 0;
@@ -247,11 +239,9 @@ gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, co
     a.row_idx = csr->row_idx;
     a.q_order = csr->q_order;
     a.k_order = csr->k_order;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(gsa::fixed::build_fixed_csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gsa::fixed::smem_bytes(gsa::fixed::kMaxBlocks, gsa::fixed::kMaxRandom)));
-    });
+    if (!gsa::smem_opt_in(gsa::fixed::build_fixed_csr_kernel,
+                          static_cast<int>(gsa::fixed::smem_bytes(gsa::fixed::kMaxBlocks, gsa::fixed::kMaxRandom))))
+        return GSA_ERR_CUDA;
     dim3 grid(3, csr->B);
     gsa::fixed::build_fixed_csr_kernel<<<grid, gsa::fixed::kThreads, gsa::fixed::smem_bytes(csr->nblk, r),
                                          as_stream(stream)>>>(a);
@@ -260,6 +250,7 @@ gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, co
 
 gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w, int32_t* lengths,
                              uint8_t* flags, gsa_block_csr* csr, int32_t* counters, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_mask_pipeline");
     if (!bytes || !lengths || !flags || !csr || !counters || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES ||
         L < b || L % b != 0 || w < 0)
         return GSA_ERR_INVALID_ARGUMENT;
@@ -285,11 +276,7 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     a.row_idx = csr->row_idx;
     a.q_order = csr->q_order;
     a.k_order = csr->k_order;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(gsa::pipeline::mask_pipeline_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
-    });
+    if (!gsa::smem_opt_in(gsa::pipeline::mask_pipeline_kernel, static_cast<int>(kSmemBytes))) return GSA_ERR_CUDA;
     gsa::pipeline::mask_pipeline_kernel<<<static_cast<unsigned>(grid), 32 * kWarps, kSmemBytes, as_stream(stream)>>>(
         bytes, L, b, total, lengths, flags, a, counters);
     return launch_status();
@@ -297,6 +284,7 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
 
 gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_block_csr* csr,
                         const gsa_attn_desc* desc, void* o, float* lse, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_attn_fwd");
     if (!q || !k || !v || !o) return GSA_ERR_INVALID_ARGUMENT;
     uint8_t cls[GSA_MAX_HEADS];
     gsa_status st = check_attn(desc, csr, cls);
@@ -325,17 +313,14 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
         std::memcpy(p.cls, cls, desc->H);
         dim3 grid(csr->nblk, desc->H, desc->B);
         const size_t smem = 3u * desc->b * desc->d * sizeof(float);
-        static std::once_flag once;
-        std::call_once(once, [] {
-            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 3 * 128 * 16 * 4);
-            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 3 * 128 * 32 * 4);
-            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 3 * 128 * 64 * 4);
-            cudaFuncSetAttribute(gsa::f32::attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 3 * 128 * 128 * 4);
-        });
+        bool opted = false;
+        switch (desc->d) {
+            case 16: opted = gsa::smem_opt_in(gsa::f32::attn_fwd_f32_kernel<16>, 3 * 128 * 16 * 4); break;
+            case 32: opted = gsa::smem_opt_in(gsa::f32::attn_fwd_f32_kernel<32>, 3 * 128 * 32 * 4); break;
+            case 64: opted = gsa::smem_opt_in(gsa::f32::attn_fwd_f32_kernel<64>, 3 * 128 * 64 * 4); break;
+            default: opted = gsa::smem_opt_in(gsa::f32::attn_fwd_f32_kernel<128>, 3 * 128 * 128 * 4); break;
+        }
+        if (!opted) return GSA_ERR_CUDA;
         switch (desc->d) {
             case 16: gsa::f32::attn_fwd_f32_kernel<16><<<grid, 128, smem, cs>>>(p); break;
             case 32: gsa::f32::attn_fwd_f32_kernel<32><<<grid, 128, smem, cs>>>(p); break;
@@ -380,12 +365,12 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
         if (!p.ticket) return GSA_ERR_CUDA;
         const int64_t items = static_cast<int64_t>(desc->B) * desc->H * ((csr->nblk + 1) / 2);
         const int64_t ctas = items < 2 * gsa::bwd::sm_count() ? items : 2 * gsa::bwd::sm_count();
-        k4 ? launch_fwd_persist<true>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs)
-           : launch_fwd_persist<false>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs);
-    } else if (desc->d == 64) {
-        k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
-    } else k4 ? launch_fwd<128, true>(grid, tq, tk, tv, p, cs) : launch_fwd<128, false>(grid, tq, tk, tv, p, cs);
-    return launch_status();
+        return k4 ? launch_fwd_persist<true>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs)
+                  : launch_fwd_persist<false>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs);
+    }
+    if (desc->d == 64)
+        return k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
+    return k4 ? launch_fwd<128, true>(grid, tq, tk, tv, p, cs) : launch_fwd<128, false>(grid, tq, tk, tv, p, cs);
 }
 
 size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc) {
@@ -397,6 +382,7 @@ size_t gsa_attn_bwd_workspace(const gsa_attn_desc* desc) {
 gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                         const gsa_block_csr* csr, const gsa_attn_desc* desc, void* dq, void* dk, void* dv,
                         void* workspace, size_t ws_bytes, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_attn_bwd");
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return GSA_ERR_INVALID_ARGUMENT;
     uint8_t cls[GSA_MAX_HEADS];
     gsa_status st = check_attn(desc, csr, cls);
@@ -420,6 +406,7 @@ gsa_status gsa_attn_bwd(const void* q, const void* k, const void* v, const void*
 gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                                 const void* dO, const gsa_block_csr* csr, const gsa_attn_desc* desc, void* dq,
                                 void* dk, void* dv, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_attn_bwd_noalloc");
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GSA_ERR_INVALID_ARGUMENT;
     uint8_t cls[GSA_MAX_HEADS];
     gsa_status st = check_attn(desc, csr, cls);
@@ -444,6 +431,7 @@ gsa_status gsa_attn_bwd_noalloc(const void* q, const void* k, const void* v, con
 int64_t gsa_attn_bwd_noalloc_max_rows(void) { return kNoAllocRows; }
 
 gsa_status gsa_device_error(int32_t* code, int32_t clear) {
+    const gsa::CallRange nvtx_range("gsa_device_error");
     if (!code) return GSA_ERR_INVALID_ARGUMENT;
     if (cudaDeviceSynchronize() != cudaSuccess) return GSA_ERR_CUDA;
     int v = 0;

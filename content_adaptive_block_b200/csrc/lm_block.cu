@@ -29,6 +29,7 @@
 
 #include "gsa.h"
 #include "gsa_lm.h"
+#include "host_attr.h"
 
 namespace gsa {
 namespace lm {
@@ -466,30 +467,32 @@ void ln_fwd(int D, bool gather, const uint8_t* bytes, const bf16* src, const flo
 }
 
 template <int NC>
-void ln_bwd_launch(const bf16* dy, const bf16* x, const float2* stats, const float* g, const bf16* dres, bf16* dx,
+bool ln_bwd_launch(const bf16* dy, const bf16* x, const float2* stats, const float* g, const bf16* dres, bf16* dx,
                    float* part, int64_t T, cudaStream_t st) {
     constexpr int kSmem = kLnWarps * 2 * 256 * NC * 4;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(ln_bwd_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    });
+    if (!gsa::smem_opt_in(ln_bwd_kernel<NC>, kSmem)) return false;
     const int64_t rpc = (T + kLnParts - 1) / kLnParts;
     ln_bwd_kernel<NC><<<kLnParts, 32 * kLnWarps, kSmem, st>>>(dy, x, stats, g, dres, dx, part, T, rpc);
+    return true;
 }
 
-void ln_bwd(int D, const bf16* dy, const bf16* x, const float2* stats, const float* g, const bf16* dres, bf16* dx,
+// False when the kernel could not be opted in to its shared memory (nothing launched).
+bool ln_bwd(int D, const bf16* dy, const bf16* x, const float2* stats, const float* g, const bf16* dres, bf16* dx,
             float* part, float* dg, float* db, int64_t T, cudaStream_t st) {
+    bool ok = false;
     switch (D / 256) {
-        case 1: ln_bwd_launch<1>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 2: ln_bwd_launch<2>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 3: ln_bwd_launch<3>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 4: ln_bwd_launch<4>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 5: ln_bwd_launch<5>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 6: ln_bwd_launch<6>(dy, x, stats, g, dres, dx, part, T, st); break;
-        case 7: ln_bwd_launch<7>(dy, x, stats, g, dres, dx, part, T, st); break;
-        default: ln_bwd_launch<8>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 1: ok = ln_bwd_launch<1>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 2: ok = ln_bwd_launch<2>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 3: ok = ln_bwd_launch<3>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 4: ok = ln_bwd_launch<4>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 5: ok = ln_bwd_launch<5>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 6: ok = ln_bwd_launch<6>(dy, x, stats, g, dres, dx, part, T, st); break;
+        case 7: ok = ln_bwd_launch<7>(dy, x, stats, g, dres, dx, part, T, st); break;
+        default: ok = ln_bwd_launch<8>(dy, x, stats, g, dres, dx, part, T, st); break;
     }
+    if (!ok) return false;
     colsum_kernel<<<(2 * D + 31) / 32, 256, 0, st>>>(part, kLnParts, D, dg, db);
+    return true;
 }
 
 }  // namespace lm
@@ -514,6 +517,7 @@ size_t gsa_lm_block_workspace(const gsa_lm_desc* desc) {
 
 gsa_status gsa_lm_block_fwd(const uint8_t* bytes, const gsa_lm_weights* w, const gsa_block_csr* csr,
                             const gsa_lm_desc* desc, void* y, void* workspace, size_t ws_bytes, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_lm_block_fwd");
     gsa_attn_desc ad;
     GSA_TRY(check(desc, &ad));
     if (!bytes || !w || !csr || !y || !workspace || !w->emb || !w->ln1_g || !w->ln1_b || !w->w_qkv || !w->w_o ||
@@ -560,6 +564,7 @@ gsa_status gsa_lm_block_fwd(const uint8_t* bytes, const gsa_lm_weights* w, const
 gsa_status gsa_lm_block_bwd(const uint8_t* bytes, const gsa_lm_weights* w, const gsa_block_csr* csr,
                             const gsa_lm_desc* desc, const void* dy, const gsa_lm_grads* g, void* workspace,
                             size_t ws_bytes, void* stream) {
+    const gsa::CallRange nvtx_range("gsa_lm_block_bwd");
     gsa_attn_desc ad;
     GSA_TRY(check(desc, &ad));
     if (!bytes || !w || !csr || !dy || !g || !workspace || !w->emb || !w->ln1_g || !w->w_qkv || !w->w_o ||
@@ -591,8 +596,9 @@ gsa_status gsa_lm_block_bwd(const uint8_t* bytes, const gsa_lm_weights* w, const
     GSA_TRY(gemm_rm(false, false, Mi, D, F, P(l.dpre), F, static_cast<const bf16*>(w->w_1), D, 0.f, nullptr, D,
                     P(l.dh2), D, false, lt, st));
     // dx1 = dy + LN2'(dh2)
-    ln_bwd(D, P(l.dh2), P(l.x1), reinterpret_cast<const float2*>(ws + l.st2), w->ln2_g, dyb, P(l.dx1), part,
-           g->ln2_g, g->ln2_b, T, st);
+    if (!ln_bwd(D, P(l.dh2), P(l.x1), reinterpret_cast<const float2*>(ws + l.st2), w->ln2_g, dyb, P(l.dx1), part,
+                g->ln2_g, g->ln2_b, T, st))
+        return GSA_ERR_CUDA;
     GSA_TRY(last_launch());
     // attention: dO = dx1 W_o, dW_o = dx1^T O, then the attention's own backward (dQ, dK, dV as dqkv rows)
     GSA_TRY(gemm_rm(false, false, Mi, D, D, P(l.dx1), D, static_cast<const bf16*>(w->w_o), D, 0.f, nullptr, D,
@@ -608,16 +614,14 @@ gsa_status gsa_lm_block_bwd(const uint8_t* bytes, const gsa_lm_weights* w, const
                     st));
     GSA_TRY(gemm_rm(false, false, Mi, D, 3 * D, P(l.dqkv), 3 * D, static_cast<const bf16*>(w->w_qkv), D, 0.f,
                     nullptr, D, P(l.dh), D, false, lt, st));
-    ln_bwd(D, P(l.dh), P(l.x0), reinterpret_cast<const float2*>(ws + l.st1), w->ln1_g, P(l.dx1), P(l.dx0), part,
-           g->ln1_g, g->ln1_b, T, st);
+    if (!ln_bwd(D, P(l.dh), P(l.x0), reinterpret_cast<const float2*>(ws + l.st1), w->ln1_g, P(l.dx1), P(l.dx0),
+                part, g->ln1_g, g->ln1_b, T, st))
+        return GSA_ERR_CUDA;
     GSA_TRY(last_launch());
     // dE: per byte value, the sum of its tokens' dx0 rows
     const int nchunks = static_cast<int>((T + kEmbChunk - 1) / kEmbChunk);
     float* epart = reinterpret_cast<float*>(ws + l.epart);
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(embed_part_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmbSmem);
-    });
+    if (!gsa::smem_opt_in(embed_part_kernel, kEmbSmem)) return GSA_ERR_CUDA;
     embed_part_kernel<<<dim3(nchunks, D / kEmbCols), 32 * kEmbWarps, kEmbSmem, st>>>(bytes, P(l.dx0), T, D,
                                                                                       epart);
     embed_reduce_kernel<<<(256 * D + 255) / 256, 256, 0, st>>>(epart, nchunks, D, g->emb);

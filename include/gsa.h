@@ -253,7 +253,12 @@ typedef struct {
  * bf16 at d = 64 runs persistent CTAs that draw work items from a counter in
  * the library's device memory: one of 256 slots, taken in turn per call and
  * returned to zero by the call's last CTA, so up to 256 such calls may be in
- * flight at once (on any streams) on one device.  Every query row needs at
+ * flight at once (on any streams) on one device.  The slot is chosen on the
+ * host when the call is made: a call captured into a CUDA graph keeps its
+ * slot for every replay, so replays of that graph must not overlap one
+ * another, nor run beside 256 or more later eager calls (which wrap round
+ * onto the same slot); overlapping users of one slot skip or repeat work
+ * items without any error being reported.  Every query row needs at
  * least one live key, as in every mask built by this library (each block
  * sees itself); a row without one has no defined output.
  * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, L != nblk*b, shapes that

@@ -63,7 +63,7 @@ def fake_torch_uuid(monkeypatch):
 def _run(monkeypatch, samples, n_min):
     nv, state = _fake_nvml(samples)
     monkeypatch.setitem(sys.modules, "pynvml", nv)
-    s = bench.NvmlClockSampler(0, period_s=0.001)
+    s = bench.NvmlClockSampler(0, period_s=0.001, spawn=False)
     s.start()
     t0 = time.time()
     while state["i"] < n_min and time.time() - t0 < 5:

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import workloads as W
+from parity_sampling import class_pairs
 from oracle import attention as oatt, deflate1, flags as oflags, mask as omask
 
 pytestmark = pytest.mark.gpu
@@ -87,11 +88,8 @@ def test_bwd_b8_8k_sampled(gsa):
     got = _run(gsa, q, k, v, do, fl, wl.w, wl.head_classes(), wl.b)
     hc = wl.head_classes()
     rng = np.random.default_rng(5)
-    pairs = set()
-    for cls in (0, 1, 2):
-        heads = [h for h in range(wl.H) if hc[h] == cls]
-        for _ in range(3):
-            pairs.add((int(rng.integers(wl.S)), int(rng.choice(heads))))
+    pairs = class_pairs(wl.S, hc, 4, seed=5)   # 4 distinct (sample, head) per class
+    assert len(pairs) == 12
     blocks = sorted(set([0, 1, wl.N - 1] + rng.integers(0, wl.N, 10).tolist()))
     _compare(got, q, k, v, do, fl, wl.w, hc, wl.b, pairs=pairs, q_blocks=blocks, k_blocks=blocks)
 
@@ -106,5 +104,6 @@ def test_bwd_b1_64k_sampled(gsa):
     lit = np.nonzero(fl[0])[0]
     blocks = sorted(set([0, 1, wl.N - 1, int(lit[0]), int(lit[-1]), int(lit[len(lit) // 2])] +
                         np.random.default_rng(2).integers(0, wl.N, 8).tolist()))
-    pairs = {(0, 0), (0, 8), (0, 11), (0, 12), (0, 15)}
+    pairs = class_pairs(wl.S, hc, 4, seed=2)   # 4 distinct heads per class (the one sample)
+    assert len(pairs) == 12
     _compare(got, q, k, v, do, fl, wl.w, hc, wl.b, pairs=pairs, q_blocks=blocks, k_blocks=blocks)

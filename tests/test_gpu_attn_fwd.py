@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import workloads as W
+from parity_sampling import class_pairs
 from oracle import attention as oatt, deflate1, flags as oflags, mask as omask
 
 pytestmark = pytest.mark.gpu
@@ -130,12 +131,8 @@ def test_b8_8k_sampled(gsa):
     q, k, v = W.qkv(wl, seed=0)
     o, lse = _run_fwd(gsa, q, k, v, fl, wl.w, wl.head_classes(), wl.b)
     hc = wl.head_classes()
-    rng = np.random.default_rng(0)
-    pairs = set()
-    for cls in (0, 1, 2):
-        heads = [h for h in range(wl.H) if hc[h] == cls]
-        for _ in range(4):
-            pairs.add((int(rng.integers(wl.S)), int(rng.choice(heads))))
+    pairs = class_pairs(wl.S, hc, 4, seed=0)   # 4 distinct (sample, head) per class
+    assert len(pairs) == 12
     _compare(o, lse, q, k, v, fl, wl.w, hc, wl.b, TOL_BF16, TOL_LSE_BF16, pairs=pairs)
 
 
@@ -149,7 +146,8 @@ def test_b1_64k_sampled(gsa):
     lit = np.nonzero(fl[0])[0]
     qb = sorted(set([0, 1, wl.N - 1, int(lit[-1]), int(lit[len(lit) // 2])] +
                     np.random.default_rng(1).integers(0, wl.N, 12).tolist()))
-    pairs = {(0, 0), (0, 7), (0, 8), (0, 11), (0, 12), (0, 15)}
+    pairs = class_pairs(wl.S, hc, 4, seed=1)   # 4 distinct heads per class (the one sample)
+    assert len(pairs) == 12
     _compare(o, lse, q, k, v, fl, wl.w, hc, wl.b, TOL_BF16, TOL_LSE_BF16, pairs=pairs, q_blocks=qb)
 
 

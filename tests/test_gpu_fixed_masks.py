@@ -107,7 +107,7 @@ def test_attention_on_fixed_masks(gsa, name):
         rows = np.concatenate([np.arange(i * wl.b, (i + 1) * wl.b) for i in qb])
         keys = np.concatenate([np.arange(j * wl.b, (j + 1) * wl.b) for j in kb])
         assert np.abs(got[0][s, h, rows] - o_ref[rows]).max() <= 2e-2
-        assert np.abs(got[1][s, h, rows] - lse_ref[rows]).max() <= 2e-2
+        assert np.abs(got[1][s, h, rows] - lse_ref[rows]).max() <= 1e-3   # LSE bar of every bf16 test
         for g_, r_, idx in ((got[2], dq_ref, rows), (got[3], dk_ref, keys), (got[4], dv_ref, keys)):
             err = np.linalg.norm(g_[s, h, idx] - r_[idx]) / np.linalg.norm(r_[idx])
             assert err <= 2e-2, (name, s, h, err)

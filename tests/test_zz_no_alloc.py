@@ -5,7 +5,9 @@ the library, so the caller passes no workspace.
 
 Checked through the C ABI against gsa_attn_bwd (which takes a caller-made
 workspace) on two calls in a row, within the backward's tolerance (relative
-L2 <= 2e-2 per gradient), plus the host-side size limit.  This file is
+L2 <= 2e-2 per gradient); bit for bit over calls whose shapes change in
+between (the array is shared and never cleared); plus the host-side size
+limit.  This file is
 collected last so a run that stops at the first failure has run the rest."""
 import ctypes
 
@@ -71,6 +73,43 @@ def test_noalloc_matches_workspace_backward(gsa, d):
         for got, want in zip((dq, dk, dv), ref):
             assert torch.isfinite(got.float()).all(), call
             assert _rel(got, want) <= TOL_REL_L2, call
+
+
+def _call_noalloc(fn, gsa, q, k, v, o, lse, do, csr, hc, b):
+    S, H, L, d = q.shape
+    hcs = (ctypes.c_uint8 * H)(*hc)
+    desc = gsa._AttnDesc(S, H, L, d, b, 1, 0.0, ctypes.cast(hcs, ctypes.c_void_p))
+    st = csr.struct()
+    dq, dk, dv = torch.full_like(q, float("nan")), torch.full_like(k, float("nan")), torch.full_like(v, float("nan"))
+    rc = fn(*(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, o, lse, do)), ctypes.byref(st), ctypes.byref(desc),
+            *(ctypes.c_void_p(t.data_ptr()) for t in (dq, dk, dv)),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, gsa.gsa_status_string(rc)
+    return dq, dk, dv
+
+
+def test_noalloc_shape_changes_between_calls(gsa):
+    """The shared array keeps the last call's contents and its regions sit at
+    offsets that depend on B*H*L: a large call, a smaller one, then the large
+    one again must each give gsa_attn_bwd's gradients (with a fresh workspace)
+    bit for bit, since both run the same deterministic kernels."""
+    lib = gsa.library()
+    fn = _noalloc_fn(lib, gsa)
+    b = 64
+    shapes = [(2, 4, 9, 64, 1), (1, 3, 5, 64, 2), (2, 4, 9, 64, 1), (1, 2, 7, 128, 1)]
+    for i, (S, H, n, d, w) in enumerate(shapes):
+        hc = [(0, 1, 2, 2)[h % 4] for h in range(H)]
+        rng = np.random.default_rng(100 + i)
+        fl = torch.from_numpy((rng.random((S, n)) < 0.5).astype(np.uint8)).cuda()
+        csr = gsa.gsa_build_block_csr(fl, w)
+        q, k, v, do = (t.cuda() for t in W.random_tensors((S, H, n * b, d), 4, torch.bfloat16, seed=200 + i))
+        o, lse = gsa.gsa_attn_fwd(q, k, v, csr, hc, b)
+        ref = gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, b)
+        got = _call_noalloc(fn, gsa, q, k, v, o, lse, do, csr, hc, b)
+        torch.cuda.synchronize()
+        assert gsa.gsa_device_error() == 0
+        for name, g_, r_ in zip(("dq", "dk", "dv"), got, ref):
+            assert torch.equal(g_, r_), (i, name)
 
 
 def test_noalloc_rejects_rows_beyond_its_scratch(gsa):
