@@ -1,0 +1,575 @@
+// Per-block gzip level-1 compressed length, one block per lane.
+//
+// Gzip-guided Sparse Attention (daiwk.github.io reproduction of arXiv
+// 2607.21752), section "核心公式", r_i equation: the information signal of
+// block i is |gzip(x_{ib:(i+1)b})|, each block compressed alone at gzip
+// level 1.  The length is that of Python's gzip.compress(block, 1): 18
+// framing bytes plus the raw DEFLATE stream (RFC 1951) zlib's level 1
+// writes.  No stream is produced; each lane walks the decisions zlib makes
+// for its block and sums the bits.
+//
+// Why one block per lane.  The work per block is a chain of small
+// data-dependent steps (a greedy parse, three heap-ordered Huffman builds),
+// so a warp per block leaves most lanes idle: here the 32 lanes of a warp
+// take 32 consecutive blocks and run the same steps side by side.  Each lane
+// keeps its block's state in shared memory as 32-bit words at
+// [word][lane], so lane l always hits bank l whatever word it reads: no
+// bank conflicts although the lanes' indices differ.
+//
+// The decisions (the same as zlib level 1):
+//  * parse: at each position with >= 3 bytes left, the earlier positions
+//    with the same 15-bit hash ((x0 << 10) ^ (x1 << 5) ^ x2) that were
+//    entered into the hash chains are tried, most recent first, at most 4;
+//    the first longest match wins (strictly longer than the best so far,
+//    starting from 2) and the search stops at 8 bytes (or the bytes left);
+//    a match of 8 extends up to 258 (or the bytes left).  Position 0 is
+//    never a source (zlib's empty-slot sentinel).  The current position is
+//    entered before the next one is looked at; after a match of at most 4
+//    bytes that leaves >= 3 bytes, its inner positions are entered too,
+//    after a longer one they are skipped.  The chains here are short bucket
+//    lists (64 buckets on the hash's low bits) filtered by the full hash,
+//    which visits exactly zlib's chain in the same order.
+//  * trees: the literal/length and distance codes are Huffman codes built
+//    with zlib's heap discipline: leaves in increasing symbol order, a
+//    1-based binary min-heap on (frequency, subtree depth), ties left to the
+//    heap's own order (right child taken on equality, the moving node kept
+//    on equality), a parent one deeper than its deeper child; an alphabet of
+//    fewer than two symbols gets dummy symbols of frequency 1.  With at most
+//    129 symbols of total frequency <= 129 no code can exceed 15 bits (a
+//    Huffman code of depth 16 needs a total frequency of at least the 18th
+//    Fibonacci number), so only the code-length code (limit 7) can overflow;
+//    it gets zlib's repair (leaves moved down to the deepest level that is
+//    not full, then lengths dealt out again in the order the nodes left the
+//    heap).
+//  * header: the code lengths of each alphabet are run-length coded
+//    separately with zlib's run rules, counted in closed form per maximal
+//    run of equal lengths (see add_run).
+//  * block kind (zlib >= 1.2.12): stored (b + 5 bytes) when b + 4 <=
+//    min(fixed, dynamic) bytes, else fixed when it is no larger than
+//    dynamic, else dynamic.
+#pragma once
+
+#include "common.cuh"
+
+namespace gsa {
+namespace deflate_lane {
+
+constexpr int kBuckets = 64;            // hash-chain buckets per block (low 6 hash bits)
+
+// Per-lane word layout (offsets in words; word i of lane l is at
+// smem[i * 32 + l] of the warp's region).  Phase A (parse) and phase B
+// (trees) overlap: the literal counts survive until their leaves are
+// gathered, which writes only nodes 0 .. leaves-1.
+template <int MAXB>
+struct Layout {
+    static constexpr int kMaxLeaves = MAXB + 2;            // symbols of one tree (+ dummies)
+    static constexpr int kXb = 0;                          // block bytes, 4 per word, zero padded
+    static constexpr int kXw = MAXB / 4 + 3;
+    static constexpr int kPos = kXb + kXw;                 // per position: hash | bucket link << 16 | byte << 24
+    static constexpr int kHeads = kPos + MAXB;             // bucket heads, 4 positions per word
+    static constexpr int kPhaseA = kHeads + kBuckets / 4;
+    static constexpr int kCnt = kPhaseA > kMaxLeaves ? kPhaseA : kMaxLeaves;   // literal/length counts, 4 per word
+    static constexpr int kNode = 0;                        // parent | symbol << 9 | freq << 18 | bits << 27
+    static constexpr int kHeap = 2 * kMaxLeaves;           // (freq << 8 | depth) << 9 | node, 1-based
+    static constexpr int kDcnt = (kCnt + 72 > kHeap + kMaxLeaves + 1) ? kCnt + 72 : kHeap + kMaxLeaves + 1;
+    static constexpr int kBlf = kDcnt + 8;                 // code-length symbol counts, one per word
+    static constexpr int kWords = kBlf + 19;
+    // code-length tree (<= 19 leaves, 37 nodes, 20 heap entries): its nodes in
+    // heap-exit order, above its heap entries, over words dead by then
+    static constexpr int kOrder = kHeap + 24;
+    static_assert(kOrder + 40 <= kBlf, "the heap-exit order stays clear of the code-length counts");
+    static_assert(kCnt >= kMaxLeaves, "gathering leaves leaves the counts intact");
+};
+
+// Fixed-code length of a literal/length symbol (RFC 1951 section 3.2.6).
+__device__ __forceinline__ int fixed_len(int s) { return s < 144 ? 8 : (s < 256 ? 9 : (s < 280 ? 7 : 8)); }
+
+// Length 3..258 -> code - 257 (0..28) and its extra bits.
+__device__ __forceinline__ void length_code(int len, int& code, int& extra) {
+    if (len == 258) {
+        code = 28;
+        extra = 0;
+        return;
+    }
+    const int v = len - 3;
+    if (v < 8) {
+        code = v;
+        extra = 0;
+        return;
+    }
+    const int e = (31 - __clz(v)) - 2;
+    code = 4 * e + 4 + ((v >> e) - 4);
+    extra = e;
+}
+
+// Distance 1..32768 -> code 0..29 and its extra bits.
+__device__ __forceinline__ void dist_code(int dist, int& code, int& extra) {
+    const int v = dist - 1;
+    if (v < 4) {
+        code = v;
+        extra = 0;
+        return;
+    }
+    const int e = (31 - __clz(v)) - 1;
+    code = 2 * e + 2 + ((v >> e) & 1);
+    extra = e;
+}
+
+// One lane's view of its words.
+struct LaneMem {
+    uint32_t* p;   // warp region + lane
+    __device__ __forceinline__ uint32_t ld(int i) const { return p[i * 32]; }
+    __device__ __forceinline__ void st(int i, uint32_t v) const { p[i * 32] = v; }
+};
+
+// 4 bytes of the block starting at byte k (little endian; k + 4 within the padded words).
+template <int MAXB>
+__device__ __forceinline__ uint32_t load4(const LaneMem& m, int k) {
+    const int w = Layout<MAXB>::kXb + (k >> 2);
+    return __funnelshift_r(m.ld(w), m.ld(w + 1), (k & 3) * 8);
+}
+
+// Leading equal bytes of a and b (as loaded by load4), 0..4.
+__device__ __forceinline__ int equal_bytes(uint32_t a, uint32_t b) {
+    const uint32_t d = a ^ b;
+    return d ? (__ffs(d) - 1) >> 3 : 4;
+}
+
+// Sift the heap entry at k down (zlib's heap discipline; comparisons on the
+// key bits above the node id).
+template <int MAXB>
+__device__ __forceinline__ void sift_down(const LaneMem& m, int len, int k) {
+    constexpr int H = Layout<MAXB>::kHeap;
+    const uint32_t v = m.ld(H + k);
+    const uint32_t kv = v | 511u;
+    int j = k << 1;
+    while (j <= len) {
+        uint32_t cj = m.ld(H + j);
+        if (j < len) {
+            const uint32_t cr = m.ld(H + j + 1);
+            if ((cr | 511u) <= (cj | 511u)) {
+                ++j;
+                cj = cr;
+            }
+        }
+        if (kv <= (cj | 511u)) break;
+        m.st(H + k, cj);
+        k = j;
+        j <<= 1;
+    }
+    m.st(H + k, v);
+}
+
+// Huffman tree over the nleaf leaves in node words 0 .. nleaf-1 (symbol and
+// frequency set, parent 0).  Writes each node's parent and, for every node,
+// its code length (bits 27..31).  track: record the heap-exit order at
+// kOrder (needed for the repair of a length-limited tree).  Returns the
+// number of nodes.
+template <int MAXB>
+__device__ int build_tree(const LaneMem& m, int nleaf, bool track) {
+    using Y = Layout<MAXB>;
+    for (int i = 0; i < nleaf; ++i) m.st(Y::kHeap + 1 + i, ((m.ld(Y::kNode + i) >> 18 & 511u) << 17) | i);
+    int len = nleaf;
+    for (int k = len >> 1; k >= 1; --k) sift_down<MAXB>(m, len, k);
+    int next = nleaf, no = 0;
+    do {
+        const uint32_t a = m.ld(Y::kHeap + 1);
+        m.st(Y::kHeap + 1, m.ld(Y::kHeap + len));
+        --len;
+        sift_down<MAXB>(m, len, 1);
+        const uint32_t b = m.ld(Y::kHeap + 1);
+        const int na = a & 511u, nb = b & 511u;
+        m.st(Y::kNode + na, m.ld(Y::kNode + na) | next);
+        m.st(Y::kNode + nb, m.ld(Y::kNode + nb) | next);
+        if (track) {
+            m.st(Y::kOrder + no, na);
+            m.st(Y::kOrder + no + 1, nb);
+            no += 2;
+        }
+        const uint32_t ka = a >> 9, kb = b >> 9;
+        const uint32_t da = ka & 255u, db = kb & 255u;
+        const uint32_t key = (((ka >> 8) + (kb >> 8)) << 8) | ((da > db ? da : db) + 1u);
+        m.st(Y::kNode + next, 0u);
+        m.st(Y::kHeap + 1, (key << 9) | next);
+        ++next;
+        sift_down<MAXB>(m, len, 1);
+    } while (len >= 2);
+    if (track) m.st(Y::kOrder + no, m.ld(Y::kHeap + 1) & 511u);
+    // lengths, parents before children (a parent's id is above its children's)
+    for (int id = next - 2; id >= 0; --id) {
+        const uint32_t w = m.ld(Y::kNode + id);
+        const uint32_t pb = m.ld(Y::kNode + (w & 511u)) >> 27;
+        m.st(Y::kNode + id, (w & 0x07ffffffu) | ((pb + 1u) << 27));
+    }
+    return next;
+}
+
+// Code-length symbols of a maximal run of R copies of length v (zlib's run
+// rules with the run starting after a different length or an array start):
+// counts into the code-length counts, returns the extra bits.
+template <int MAXB>
+__device__ __forceinline__ int add_run(const LaneMem& m, int v, int R) {
+    constexpr int F = Layout<MAXB>::kBlf;
+    if (R <= 0) return 0;
+    if (v == 0) {
+        int n18 = R / 138;
+        const int r = R - 138 * n18;
+        int x = 0;
+        if (r >= 11) ++n18;
+        else if (r >= 3) {
+            m.st(F + 17, m.ld(F + 17) + 1);
+            x += 3;
+        } else if (r > 0) m.st(F + 0, m.ld(F + 0) + r);
+        if (n18) m.st(F + 18, m.ld(F + 18) + n18);
+        return x + 7 * n18;
+    }
+    int nv, n16;
+    if (R < 4) {
+        nv = R;
+        n16 = 0;
+    } else {
+        nv = 1;
+        n16 = 1;
+        if (R > 7) {
+            const int rest = R - 7;
+            n16 += rest / 6;
+            const int r = rest % 6;
+            if (r >= 3) ++n16;
+            else nv += r;
+        }
+    }
+    m.st(F + v, m.ld(F + v) + nv);
+    if (n16) m.st(F + 16, m.ld(F + 16) + n16);
+    return 2 * n16;
+}
+
+// gzip length (18 + raw DEFLATE bytes) of the lane's block of n bytes, whose
+// bytes are already in its words (zero padded).
+template <int MAXB>
+__device__ int lane_block_length(const LaneMem& m, int n) {
+    using Y = Layout<MAXB>;
+    // ---- per position: byte, and the 3-byte hash where >= 3 bytes are left
+    {
+        uint32_t h = 0;
+        for (int q = 0; q < n; ++q) {
+            const uint32_t xq = (m.ld(Y::kXb + (q >> 2)) >> ((q & 3) * 8)) & 255u;
+            uint32_t w = xq << 24;
+            if (q + 2 < n) {
+                const uint32_t x2 = (m.ld(Y::kXb + ((q + 2) >> 2)) >> (((q + 2) & 3) * 8)) & 255u;
+                if (q == 0) {
+                    const uint32_t x1 = (m.ld(Y::kXb) >> 8) & 255u;
+                    h = (xq << 10) ^ (x1 << 5) ^ x2;
+                } else {
+                    h = ((h << 5) ^ x2);
+                }
+                h &= 0x7fffu;
+                w |= h;
+            }
+            m.st(Y::kPos + q, w);
+        }
+    }
+    for (int i = 0; i < kBuckets / 4; ++i) m.st(Y::kHeads + i, 0u);
+    for (int i = 0; i < 72; ++i) m.st(Y::kCnt + i, 0u);
+    for (int i = 0; i < 8; ++i) m.st(Y::kDcnt + i, 0u);
+
+    // enter position q (>= 3 bytes left) into its bucket; w = its position word
+    auto insert = [&](int q, uint32_t w) {
+        const uint32_t bk = w & (kBuckets - 1);
+        const int hw = Y::kHeads + (bk >> 2);
+        const uint32_t sh = (bk & 3u) * 8u;
+        const uint32_t heads = m.ld(hw);
+        m.st(Y::kPos + q, w | (((heads >> sh) & 255u) << 16));
+        m.st(hw, (heads & ~(255u << sh)) | (static_cast<uint32_t>(q) << sh));
+    };
+
+    // ---- greedy parse
+    int fix = 7;       // fixed-code bits (end of block included), extra bits included
+    int extra = 0;     // extra bits of the length and distance codes
+    int p = 0;
+    while (p < n) {
+        const int rem = n - p;
+        const uint32_t wp = m.ld(Y::kPos + p);
+        int mlen = 0, mpos = 0;
+        if (rem >= 3) {
+            const uint32_t h = wp & 0x7fffu;
+            const uint32_t bk = h & (kBuckets - 1);
+            uint32_t c = (m.ld(Y::kHeads + (bk >> 2)) >> ((bk & 3u) * 8u)) & 255u;
+            insert(p, wp);
+            if (c != 0u) {
+                const int nice = rem < 8 ? rem : 8;
+                uint32_t p0 = 0, p1 = 0;
+                bool loaded = false;
+                int best = 2, nc = 0;
+                while (c != 0u && nc < 4) {
+                    const uint32_t wc = m.ld(Y::kPos + c);
+                    if ((wc & 0x7fffu) == h) {
+                        ++nc;
+                        if (!loaded) {
+                            p0 = load4<MAXB>(m, p);
+                            p1 = load4<MAXB>(m, p + 4);
+                            loaded = true;
+                        }
+                        int len = equal_bytes(load4<MAXB>(m, c), p0);
+                        if (len == 4) len += equal_bytes(load4<MAXB>(m, c + 4), p1);
+                        if (len > nice) len = nice;
+                        if (len > best) {
+                            best = len;
+                            mpos = static_cast<int>(c);
+                            if (len >= nice) break;
+                        }
+                    }
+                    c = (wc >> 16) & 255u;
+                }
+                if (best >= 8 && rem > 8) {
+                    const int lim = rem < 258 ? rem : 258;
+                    int k = 8;
+                    while (k < lim) {
+                        const int e = equal_bytes(load4<MAXB>(m, mpos + k), load4<MAXB>(m, p + k));
+                        k += e;
+                        if (e < 4) break;
+                    }
+                    best = k < lim ? k : lim;
+                }
+                if (best >= 3) mlen = best < rem ? best : rem;
+            }
+        }
+        if (mlen >= 3) {
+            int lc, le, dc, de;
+            length_code(mlen, lc, le);
+            dist_code(p - mpos, dc, de);
+            const int sym = 257 + lc;
+            m.st(Y::kCnt + (sym >> 2), m.ld(Y::kCnt + (sym >> 2)) + (1u << ((sym & 3) * 8)));
+            m.st(Y::kDcnt + (dc >> 2), m.ld(Y::kDcnt + (dc >> 2)) + (1u << ((dc & 3) * 8)));
+            extra += le + de;
+            fix += fixed_len(sym) + 5 + le + de;
+            if (mlen <= 4 && rem - mlen >= 3)
+                for (int q = p + 1; q < p + mlen; ++q) insert(q, m.ld(Y::kPos + q));
+            p += mlen;
+        } else {
+            const uint32_t xp = wp >> 24;
+            m.st(Y::kCnt + (xp >> 2), m.ld(Y::kCnt + (xp >> 2)) + (1u << ((xp & 3) * 8)));
+            fix += xp < 144 ? 8 : 9;
+            p += 1;
+        }
+    }
+    // end of block
+    m.st(Y::kCnt + 64, m.ld(Y::kCnt + 64) + 1u);
+
+    // ---- literal/length tree: leaves in symbol order (never fewer than two:
+    // end of block and at least one literal)
+    int nleaf = 0;
+    for (int wd = 0; wd < 72; ++wd) {
+        uint32_t v = m.ld(Y::kCnt + wd);
+        while (v) {
+            const int j = (__ffs(v) - 1) >> 3;
+            const uint32_t f = (v >> (8 * j)) & 255u;
+            v &= ~(255u << (8 * j));
+            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
+            ++nleaf;
+        }
+    }
+    for (int i = 0; i < 19; ++i) m.st(Y::kBlf + i, 0u);
+    build_tree<MAXB>(m, nleaf, false);
+    int dyn = extra;
+    int blx = 0;   // extra bits of the code-length symbols
+    {
+        // data bits, and the run-length coding of lengths 0 .. max symbol
+        int prev = -1, rv = -1, rl = 0;
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = m.ld(Y::kNode + i);
+            const int s = (w >> 9) & 511u, v = w >> 27;
+            dyn += static_cast<int>((w >> 18) & 511u) * v;
+            const int gap = s - prev - 1;
+            if (gap > 0 || v != rv) {
+                blx += add_run<MAXB>(m, rv, rl);
+                blx += add_run<MAXB>(m, 0, gap);
+                rv = v;
+                rl = 1;
+            } else {
+                ++rl;
+            }
+            prev = s;
+        }
+        blx += add_run<MAXB>(m, rv, rl);
+    }
+
+    // ---- distance tree (dummies for fewer than two codes)
+    {
+        nleaf = 0;
+        int max_code = -1;
+        for (int wd = 0; wd < 8; ++wd) {
+            uint32_t v = m.ld(Y::kDcnt + wd);
+            while (v) {
+                const int j = (__ffs(v) - 1) >> 3;
+                const uint32_t f = (v >> (8 * j)) & 255u;
+                v &= ~(255u << (8 * j));
+                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
+                max_code = 4 * wd + j;
+                ++nleaf;
+            }
+        }
+        while (nleaf < 2) {
+            const int s = max_code < 2 ? ++max_code : 0;
+            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (1u << 18));
+            ++nleaf;
+        }
+        build_tree<MAXB>(m, nleaf, false);
+        // lengths by code, 4 bits each (codes 0 .. 29), dummies included; data bits of real codes
+        uint64_t dlo = 0, dhi = 0;
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = m.ld(Y::kNode + i);
+            const int s = (w >> 9) & 511u;
+            const uint64_t v = w >> 27;
+            if (s < 16) dlo |= v << (4 * s);
+            else dhi |= v << (4 * (s - 16));
+        }
+        for (int wd = 0; wd < 8; ++wd) {   // real codes only (dummies cost nothing net)
+            uint32_t cv = m.ld(Y::kDcnt + wd);
+            while (cv) {
+                const int j = (__ffs(cv) - 1) >> 3;
+                const int f = (cv >> (8 * j)) & 255u;
+                cv &= ~(255u << (8 * j));
+                const int s = 4 * wd + j;
+                const int len = static_cast<int>(((s < 16 ? dlo >> (4 * s) : dhi >> (4 * (s - 16)))) & 15u);
+                dyn += f * len;
+            }
+        }
+        int rv = -1, rl = 0;
+        for (int s = 0; s <= max_code; ++s) {
+            const int v = static_cast<int>(((s < 16 ? dlo >> (4 * s) : dhi >> (4 * (s - 16)))) & 15u);
+            if (v == rv) {
+                ++rl;
+            } else {
+                blx += add_run<MAXB>(m, rv, rl);
+                rv = v;
+                rl = 1;
+            }
+        }
+        blx += add_run<MAXB>(m, rv, rl);
+    }
+
+    // ---- code-length tree (limit 7 bits, with zlib's repair)
+    uint64_t bllen = 0;   // 3 bits per code-length symbol
+    int blbits = blx;
+    {
+        nleaf = 0;
+        int max_code = -1;
+        for (int s = 0; s < 19; ++s) {
+            const uint32_t f = m.ld(Y::kBlf + s);
+            if (f) {
+                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (f << 18));
+                max_code = s;
+                ++nleaf;
+            }
+        }
+        const int nreal = nleaf;
+        while (nleaf < 2) {
+            const int s = max_code < 2 ? ++max_code : 0;
+            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (1u << 18));
+            ++nleaf;
+        }
+        const int nodes = build_tree<MAXB>(m, nleaf, true);
+        // overflow: nodes whose length passed 7 (each clamped in turn from its clamped parent)
+        int overflow = 0;
+        uint64_t count = 0;   // leaves per length 0..7, 8 bits each
+        for (int id = nodes - 1; id >= 0; --id) {
+            const uint32_t w = m.ld(Y::kNode + id);
+            int d = static_cast<int>(w >> 27);
+            if (id < nodes - 1) {
+                const int pd = static_cast<int>(m.ld(Y::kNode + (w & 511u)) >> 27);
+                d = pd + 1;
+                if (d > 7) {
+                    d = 7;
+                    ++overflow;
+                }
+                m.st(Y::kNode + id, (w & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
+            }
+            if (id < nleaf) count += uint64_t(1) << (8 * d);
+        }
+        if (overflow > 0) {
+            do {
+                int d = 6;
+                while (((count >> (8 * d)) & 255u) == 0) --d;
+                count -= uint64_t(1) << (8 * d);
+                count += uint64_t(2) << (8 * (d + 1));
+                count -= uint64_t(1) << 56;
+                overflow -= 2;
+            } while (overflow > 0);
+            int r = 0;
+            for (int d = 7; d != 0; --d) {
+                int c = static_cast<int>((count >> (8 * d)) & 255u);
+                while (c != 0) {
+                    const int nd = static_cast<int>(m.ld(Y::kOrder + r));
+                    ++r;
+                    if (nd >= nleaf) continue;
+                    m.st(Y::kNode + nd, (m.ld(Y::kNode + nd) & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
+                    --c;
+                }
+            }
+        }
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = m.ld(Y::kNode + i);
+            const int s = (w >> 9) & 511u;
+            bllen |= static_cast<uint64_t>(w >> 27) << (3 * s);
+            if (i < nreal) blbits += static_cast<int>((w >> 18) & 511u) * static_cast<int>(w >> 27);
+        }
+    }
+    // code-length code lengths sent: RFC order, trailing zeros trimmed, at least 4
+    constexpr uint64_t kOrderNibbles = 0xF1E2D3C4B5A69780ull;   // 16, 17, 18 then 0 8 7 9 6 10 5 11 4 12 3 13 2 14 1 15
+    int hclen = 4;
+    for (int i = 18; i >= 4; --i) {
+        const int sym = static_cast<int>((kOrderNibbles >> (4 * (i - 3))) & 15u);
+        if ((bllen >> (3 * sym)) & 7u) {
+            hclen = i + 1;
+            break;
+        }
+    }
+    dyn += blbits + 5 + 5 + 4 + 3 * hclen;
+
+    int opt = (dyn + 3 + 7) >> 3;
+    const int stat = (fix + 3 + 7) >> 3;
+    if (stat <= opt) opt = stat;
+    const int raw = (n + 4 <= opt) ? n + 5 : opt;
+    return raw + 18;
+}
+
+// Per-lane words a warp needs, and warps per CTA, for blocks of at most MAXB bytes.
+template <int MAXB>
+struct KernelShape {
+    static constexpr int kWarpBytes = Layout<MAXB>::kWords * 32 * 4;
+    static constexpr int kWarps = 1;
+    static constexpr int kSmemBytes = kWarpBytes * kWarps;
+};
+
+// Lengths of blocks task0 .. task0 + 31 of the batch, one per lane: the
+// warp stages its 32 blocks (contiguous bytes) into the lanes' words with
+// coalesced loads, then each lane runs its block.
+template <int MAXB>
+__global__ void __launch_bounds__(32 * KernelShape<MAXB>::kWarps)
+block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblocks_total,
+                          int32_t* __restrict__ lengths) {
+    using Y = Layout<MAXB>;
+    extern __shared__ __align__(16) uint32_t lsmem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* region = lsmem + static_cast<size_t>(warp) * Y::kWords * 32;
+    const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * 32;
+    if (task0 >= nblocks_total) return;   // warp-uniform
+    const int nb = nblocks_total - task0 < 32 ? static_cast<int>(nblocks_total - task0) : 32;
+    // zero every lane's byte words, then scatter the warp's nb * b contiguous bytes
+    for (int i = 0; i < Y::kXw; ++i) region[(Y::kXb + i) * 32 + lane] = 0u;
+    __syncwarp();
+    const uint8_t* src = bytes + task0 * b;
+    uint8_t* r8 = reinterpret_cast<uint8_t*>(region);
+    for (int j = lane; j < nb * b; j += 32) {
+        const int blk = j / b, k = j - blk * b;
+        r8[((Y::kXb + (k >> 2)) * 32 + blk) * 4 + (k & 3)] = src[j];
+    }
+    __syncwarp();
+    if (lane < nb) {
+        const LaneMem m{region + lane};
+        lengths[task0 + lane] = lane_block_length<MAXB>(m, b);
+    }
+}
+
+}  // namespace deflate_lane
+}  // namespace gsa

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "deflate_len.cuh"
+#include "deflate_lane.cuh"
 #include "flags_csr.cuh"
 #include "mask_pipeline.cuh"
 #include "fixed_csr.cuh"
@@ -137,6 +138,20 @@ gsa_status launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtens
     return launch_status();
 }
 
+// The lengths kernel for blocks of at most MAXB bytes: 32 blocks per warp,
+// one per lane.
+template <int MAXB>
+gsa_status launch_lengths_lane(const uint8_t* bytes, int b, int64_t total, int32_t* lengths, cudaStream_t cs) {
+    using K = gsa::deflate_lane::KernelShape<MAXB>;
+    const int64_t per_cta = 32 * K::kWarps;
+    const int64_t grid = (total + per_cta - 1) / per_cta;
+    if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
+    if (!gsa::smem_opt_in(gsa::deflate_lane::block_lengths_lane_kernel<MAXB>, K::kSmemBytes)) return GSA_ERR_CUDA;
+    gsa::deflate_lane::block_lengths_lane_kernel<MAXB><<<static_cast<unsigned>(grid), 32 * K::kWarps, K::kSmemBytes,
+                                                         cs>>>(bytes, b, total, lengths);
+    return launch_status();
+}
+
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
     if (!d || !csr || !d->head_classes) return GSA_ERR_INVALID_ARGUMENT;
     if (!csr_ok(csr)) return csr && csr->capacity < gsa_csr_capacity(csr->nblk) ? GSA_ERR_CAPACITY
@@ -166,14 +181,10 @@ gsa_status gsa_block_lengths(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     const gsa::CallRange nvtx_range("gsa_block_lengths");
     if (!bytes || !lengths || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES || L < b || L % b != 0)
         return GSA_ERR_INVALID_ARGUMENT;
-    using namespace gsa::deflate;
     const int64_t total = static_cast<int64_t>(B) * (L / b);
-    const int64_t grid = (total + kLenWarps - 1) / kLenWarps;
-    if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
-    if (!gsa::smem_opt_in(block_lengths_kernel, static_cast<int>(kLenSmemBytes))) return GSA_ERR_CUDA;
-    block_lengths_kernel<<<static_cast<unsigned>(grid), 32 * kLenWarps, kLenSmemBytes, as_stream(stream)>>>(
-        bytes, L, b, total, lengths);
-    return launch_status();
+    if (b <= 32) return launch_lengths_lane<32>(bytes, b, total, lengths, as_stream(stream));
+    if (b <= 64) return launch_lengths_lane<64>(bytes, b, total, lengths, as_stream(stream));
+    return launch_lengths_lane<128>(bytes, b, total, lengths, as_stream(stream));
 }
 
 gsa_status gsa_literal_flags(const int32_t* lengths, int32_t B, int32_t nblk, uint8_t* flags, void* stream) {
