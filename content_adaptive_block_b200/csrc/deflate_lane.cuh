@@ -65,20 +65,36 @@ struct Layout {
     static constexpr int kMaxLeaves = MAXB + 2;            // symbols of one tree (+ dummies)
     static constexpr int kXb = 0;                          // block bytes, 4 per word, zero padded
     static constexpr int kXw = MAXB / 4 + 3;
-    static constexpr int kPos = kXb + kXw;                 // per position: hash | bucket link << 16 | byte << 24
+    static constexpr int kPos = kXb + kXw;                 // per position: hash | previous bucket-mate << 15
     static constexpr int kHeads = kPos + MAXB;             // bucket heads, 4 positions per word
     static constexpr int kPhaseA = kHeads + kBuckets / 4;
     static constexpr int kCnt = kPhaseA > kMaxLeaves ? kPhaseA : kMaxLeaves;   // literal/length counts, 4 per word
     static constexpr int kNode = 0;                        // parent | symbol << 9 | freq << 18 | bits << 27
     static constexpr int kHeap = 2 * kMaxLeaves;           // (freq << 8 | depth) << 9 | node, 1-based
     static constexpr int kDcnt = (kCnt + 72 > kHeap + kMaxLeaves + 1) ? kCnt + 72 : kHeap + kMaxLeaves + 1;
-    static constexpr int kBlf = kDcnt + 8;                 // code-length symbol counts, one per word
-    static constexpr int kWords = kBlf + 19;
     // code-length tree (<= 19 leaves, 37 nodes, 20 heap entries): its nodes in
     // heap-exit order, above its heap entries, over words dead by then
     static constexpr int kOrder = kHeap + 24;
-    static_assert(kOrder + 40 <= kBlf, "the heap-exit order stays clear of the code-length counts");
+    static constexpr int kWords = (kDcnt + 8 > kOrder + 40) ? kDcnt + 8 : kOrder + 40;
     static_assert(kCnt >= kMaxLeaves, "gathering leaves leaves the counts intact");
+};
+
+// The 19 code-length symbol counts (each < 512) in three registers, 9 bits
+// apiece: symbol s in word s / 7 at bit 9 (s % 7).
+struct ClCounts {
+    uint64_t w[3] = {0, 0, 0};
+    __device__ __forceinline__ void add(int s, int n) {
+        const uint64_t d = static_cast<uint64_t>(n) << (9 * (s % 7));
+        const int k = s / 7;
+        if (k == 0) w[0] += d;
+        else if (k == 1) w[1] += d;
+        else w[2] += d;
+    }
+    __device__ __forceinline__ int get(int s) const {
+        const int k = s / 7;
+        const uint64_t x = k == 0 ? w[0] : (k == 1 ? w[1] : w[2]);
+        return static_cast<int>((x >> (9 * (s % 7))) & 511u);
+    }
 };
 
 // Fixed-code length of a literal/length symbol (RFC 1951 section 3.2.6).
@@ -206,10 +222,8 @@ __device__ int build_tree(const LaneMem& m, int nleaf, bool track) {
 
 // Code-length symbols of a maximal run of R copies of length v (zlib's run
 // rules with the run starting after a different length or an array start):
-// counts into the code-length counts, returns the extra bits.
-template <int MAXB>
-__device__ __forceinline__ int add_run(const LaneMem& m, int v, int R) {
-    constexpr int F = Layout<MAXB>::kBlf;
+// counts into cl, returns the extra bits.
+__device__ __forceinline__ int add_run(ClCounts& cl, int v, int R) {
     if (R <= 0) return 0;
     if (v == 0) {
         int n18 = R / 138;
@@ -217,10 +231,10 @@ __device__ __forceinline__ int add_run(const LaneMem& m, int v, int R) {
         int x = 0;
         if (r >= 11) ++n18;
         else if (r >= 3) {
-            m.st(F + 17, m.ld(F + 17) + 1);
+            cl.add(17, 1);
             x += 3;
-        } else if (r > 0) m.st(F + 0, m.ld(F + 0) + r);
-        if (n18) m.st(F + 18, m.ld(F + 18) + n18);
+        } else if (r > 0) cl.add(0, r);
+        if (n18) cl.add(18, n18);
         return x + 7 * n18;
     }
     int nv, n16;
@@ -238,95 +252,187 @@ __device__ __forceinline__ int add_run(const LaneMem& m, int v, int R) {
             else nv += r;
         }
     }
-    m.st(F + v, m.ld(F + v) + nv);
-    if (n16) m.st(F + 16, m.ld(F + 16) + n16);
+    cl.add(v, nv);
+    if (n16) cl.add(16, n16);
     return 2 * n16;
 }
 
-// gzip length (18 + raw DEFLATE bytes) of the lane's block of n bytes, whose
-// bytes are already in its words (zero padded).
-template <int MAXB>
-__device__ int lane_block_length(const LaneMem& m, int n) {
-    using Y = Layout<MAXB>;
-    // ---- per position: byte, and the 3-byte hash where >= 3 bytes are left
-    {
-        uint32_t h = 0;
-        for (int q = 0; q < n; ++q) {
-            const uint32_t xq = (m.ld(Y::kXb + (q >> 2)) >> ((q & 3) * 8)) & 255u;
-            uint32_t w = xq << 24;
-            if (q + 2 < n) {
-                const uint32_t x2 = (m.ld(Y::kXb + ((q + 2) >> 2)) >> (((q + 2) & 3) * 8)) & 255u;
-                if (q == 0) {
-                    const uint32_t x1 = (m.ld(Y::kXb) >> 8) & 255u;
-                    h = (xq << 10) ^ (x1 << 5) ^ x2;
-                } else {
-                    h = ((h << 5) ^ x2);
-                }
-                h &= 0x7fffu;
-                w |= h;
+// Huffman cost (sum of frequency x code length) of at most four symbol
+// counts, zeros ignored; a lone symbol costs one bit per occurrence (zlib
+// gives it a dummy sibling).  Closed forms on the sorted counts
+// v0 <= v1 <= v2 <= v3: four symbols merge v0 + v1 first, then the two
+// smallest of (v0 + v1, v2, v3).
+__device__ __forceinline__ int huffman_cost4(int a, int b, int c, int d) {
+    int v0 = a, v1 = b, v2 = c, v3 = d, t;
+#define GSA_CX(x, y) \
+    t = min(x, y);   \
+    y = max(x, y);   \
+    x = t;
+    GSA_CX(v0, v1) GSA_CX(v2, v3) GSA_CX(v0, v2) GSA_CX(v1, v3) GSA_CX(v1, v2)
+#undef GSA_CX
+    const int total = v0 + v1 + v2 + v3;
+    if (v0 > 0) {
+        const int m1 = v0 + v1;
+        return m1 + min(m1, v3) + v2 + total;
+    }
+    if (v1 > 0) return 2 * (v1 + v2) + v3;
+    if (v2 > 0) return v2 + v3;
+    return v3;
+}
+
+// Lowest position in RFC 1951's code-length order (16 17 18 0 8 7 9 6 10 5
+// 11 4 12 3 13 2 14 1 15) of a code length that a Huffman code over U >= 2
+// symbols must use, taken as the larger of two facts: some length is at
+// most floor(log2 U), some length is at least ceil(log2 U) (Kraft).  The
+// header sends the code-length code lengths up to the last nonzero one in
+// that order, so it sends at least this position + 1 of them.
+__device__ __forceinline__ int min_order_pos(int U) {
+    const int fl = 31 - __clz(U);                  // floor(log2 U)
+    const int cl = fl + ((U & (U - 1)) ? 1 : 0);   // ceil(log2 U)
+    // best (lowest) position among lengths <= fl: 8 -> 4, 7 -> 5, 6 -> 7, 5 -> 9, 4 -> 11, 3 -> 13, 2 -> 15, 1 -> 17
+    const int lo = fl >= 8 ? 4 : (fl == 7 ? 5 : (fl == 6 ? 7 : 9 + 2 * (5 - (fl < 1 ? 1 : fl))));
+    // lowest position among lengths >= cl: 8 -> 4 while cl <= 8; 9 -> 6, 10 -> 8, 11 -> 10, ...
+    const int hi = cl <= 8 ? 4 : 2 * cl - 12;
+    return lo > hi ? lo : hi;
+}
+
+// Code-length symbols of a zero run of R >= 1 (zlib's rules), as counts
+// of symbols 0, 17, 18 and their extra bits.
+__device__ __forceinline__ void zero_run_counts(int R, int& z0, int& z17, int& z18, int& ext) {
+    int n18 = R / 138;
+    const int r = R - 138 * n18;
+    if (r >= 11) ++n18;
+    else if (r >= 3) {
+        ++z17;
+        ext += 3;
+    } else z0 += r;
+    z18 += n18;
+    ext += 7 * n18;
+}
+
+// Code-length symbols of the zero runs between used symbols of an
+// alphabet (its used-symbol bitmask, NWD words), and a lower bound on those
+// of its used symbols: islands of m consecutive used symbols send each
+// length alone when m <= 3 and at least two symbols (a length, a repeat)
+// otherwise.  Zero runs after the last used symbol are not sent.
+template <int NWD>
+__device__ __forceinline__ void run_counts(const uint32_t (&um)[NWD], int& z0, int& z17, int& z18, int& zext,
+                                           int& nz) {
+    bool ones = false;
+    int run = 0;   // length of the current run (of ones or zeros)
+#pragma unroll
+    for (int k = 0; k < NWD; ++k) {
+        const uint32_t w = um[k];
+        int i = 0;
+        while (i < 32) {
+            const uint32_t x = ones ? ~w : w;   // the next bit that ends the current run
+            const uint32_t rest = x >> i;
+            const int len = rest ? __ffs(rest) - 1 : 32 - i;
+            run += len;
+            i += len;
+            if (i < 32) {   // run ends at bit i
+                if (ones) nz += run <= 3 ? run : 2;
+                else if (run > 0) zero_run_counts(run, z0, z17, z18, zext);
+                ones = !ones;
+                run = 0;
             }
-            m.st(Y::kPos + q, w);
         }
     }
+    if (ones) nz += run <= 3 ? run : 2;
+}
+
+// gzip length (18 + raw DEFLATE bytes) of the lane's block of n bytes, whose
+// bytes are already in its words (zero padded).  lanes: the warp's lanes
+// that hold a block (all of them call this together).
+template <int MAXB>
+__device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
+    using Y = Layout<MAXB>;
+    constexpr int NW = MAXB / 32;   // words of the per-position bitmasks
+    // ---- prepass, the same steps on every lane: each position with >= 3
+    // bytes left gets its hash and its previous bucket-mate (64 buckets on the
+    // hash's low bits; 0 ends a list, as position 0 is never a match source)
     for (int i = 0; i < kBuckets / 4; ++i) m.st(Y::kHeads + i, 0u);
     for (int i = 0; i < 72; ++i) m.st(Y::kCnt + i, 0u);
     for (int i = 0; i < 8; ++i) m.st(Y::kDcnt + i, 0u);
+    {
+        uint32_t h = 0;
+        for (int q = 0; q + 2 < n; ++q) {
+            const uint32_t x2 = (m.ld(Y::kXb + ((q + 2) >> 2)) >> (((q + 2) & 3) * 8)) & 255u;
+            if (q == 0) {
+                const uint32_t w0 = m.ld(Y::kXb);
+                h = ((w0 & 255u) << 10) ^ (((w0 >> 8) & 255u) << 5) ^ x2;
+            } else {
+                h = (h << 5) ^ x2;
+            }
+            h &= 0x7fffu;
+            const uint32_t bk = h & (kBuckets - 1);
+            const int hw = Y::kHeads + (bk >> 2);
+            const uint32_t sh = (bk & 3u) * 8u;
+            const uint32_t heads = m.ld(hw);
+            m.st(Y::kPos + q, h | (((heads >> sh) & 255u) << 15));
+            m.st(hw, (heads & ~(255u << sh)) | (static_cast<uint32_t>(q) << sh));
+        }
+    }
 
-    // enter position q (>= 3 bytes left) into its bucket; w = its position word
-    auto insert = [&](int q, uint32_t w) {
-        const uint32_t bk = w & (kBuckets - 1);
-        const int hw = Y::kHeads + (bk >> 2);
-        const uint32_t sh = (bk & 3u) * 8u;
-        const uint32_t heads = m.ld(hw);
-        m.st(Y::kPos + q, w | (((heads >> sh) & 255u) << 16));
-        m.st(hw, (heads & ~(255u << sh)) | (static_cast<uint32_t>(q) << sh));
+    // ---- greedy parse.  Candidates for p: its earlier bucket-mates with the
+    // same hash that were entered into the chains (a bitmask in registers),
+    // newest first.  Literal positions are marked and counted afterwards.
+    uint32_t ins[NW], lit[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) ins[k] = lit[k] = 0u;
+    auto bit = [&](const uint32_t (&a)[NW], uint32_t q) -> bool {
+        uint32_t w = 0;
+#pragma unroll
+        for (int k = 0; k < NW; ++k)
+            if (k == static_cast<int>(q >> 5)) w = a[k];
+        return (w >> (q & 31u)) & 1u;
     };
-
-    // ---- greedy parse
+    auto set = [&](uint32_t (&a)[NW], int q) {
+#pragma unroll
+        for (int k = 0; k < NW; ++k)
+            if (k == (q >> 5)) a[k] |= 1u << (q & 31);
+    };
     int fix = 7;       // fixed-code bits (end of block included), extra bits included
     int extra = 0;     // extra bits of the length and distance codes
     int p = 0;
     while (p < n) {
         const int rem = n - p;
-        const uint32_t wp = m.ld(Y::kPos + p);
         int mlen = 0, mpos = 0;
         if (rem >= 3) {
+            const uint32_t wp = m.ld(Y::kPos + p);
             const uint32_t h = wp & 0x7fffu;
-            const uint32_t bk = h & (kBuckets - 1);
-            uint32_t c = (m.ld(Y::kHeads + (bk >> 2)) >> ((bk & 3u) * 8u)) & 255u;
-            insert(p, wp);
-            if (c != 0u) {
+            uint32_t q = (wp >> 15) & 127u;
+            set(ins, p);
+            if (q != 0u) {
                 const int nice = rem < 8 ? rem : 8;
-                uint32_t p0 = 0, p1 = 0;
-                bool loaded = false;
+                const uint32_t p0 = load4<MAXB>(m, p), p1 = load4<MAXB>(m, p + 4);
                 int best = 2, nc = 0;
-                while (c != 0u && nc < 4) {
-                    const uint32_t wc = m.ld(Y::kPos + c);
-                    if ((wc & 0x7fffu) == h) {
+                while (q != 0u && nc < 4) {
+                    const uint32_t wq = m.ld(Y::kPos + q);
+                    if ((wq & 0x7fffu) == h && bit(ins, q)) {
                         ++nc;
-                        if (!loaded) {
-                            p0 = load4<MAXB>(m, p);
-                            p1 = load4<MAXB>(m, p + 4);
-                            loaded = true;
-                        }
-                        int len = equal_bytes(load4<MAXB>(m, c), p0);
-                        if (len == 4) len += equal_bytes(load4<MAXB>(m, c + 4), p1);
+                        const uint32_t q0 = load4<MAXB>(m, q), q1 = load4<MAXB>(m, q + 4);
+                        int len = equal_bytes(q0, p0);
+                        if (len == 4) len += equal_bytes(q1, p1);
                         if (len > nice) len = nice;
                         if (len > best) {
                             best = len;
-                            mpos = static_cast<int>(c);
+                            mpos = static_cast<int>(q);
                             if (len >= nice) break;
                         }
                     }
-                    c = (wc >> 16) & 255u;
+                    q = (wq >> 15) & 127u;
                 }
                 if (best >= 8 && rem > 8) {
                     const int lim = rem < 258 ? rem : 258;
                     int k = 8;
-                    while (k < lim) {
-                        const int e = equal_bytes(load4<MAXB>(m, mpos + k), load4<MAXB>(m, p + k));
+                    while (k < lim) {   // 8 bytes per step
+                        const uint32_t a0 = load4<MAXB>(m, mpos + k), b0 = load4<MAXB>(m, p + k);
+                        const uint32_t a1 = load4<MAXB>(m, mpos + k + 4), b1 = load4<MAXB>(m, p + k + 4);
+                        int e = equal_bytes(a0, b0);
+                        if (e == 4) e += equal_bytes(a1, b1);
                         k += e;
-                        if (e < 4) break;
+                        if (e < 8) break;
                     }
                     best = k < lim ? k : lim;
                 }
@@ -343,17 +449,103 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
             extra += le + de;
             fix += fixed_len(sym) + 5 + le + de;
             if (mlen <= 4 && rem - mlen >= 3)
-                for (int q = p + 1; q < p + mlen; ++q) insert(q, m.ld(Y::kPos + q));
+                for (int q = p + 1; q < p + mlen; ++q) set(ins, q);
             p += mlen;
         } else {
-            const uint32_t xp = wp >> 24;
-            m.st(Y::kCnt + (xp >> 2), m.ld(Y::kCnt + (xp >> 2)) + (1u << ((xp & 3) * 8)));
-            fix += xp < 144 ? 8 : 9;
+            set(lit, p);
             p += 1;
+        }
+    }
+    // literal counts, the same steps on every lane
+    for (int q = 0; q < n; ++q) {
+        if (bit(lit, q)) {
+            const uint32_t xq = (m.ld(Y::kXb + (q >> 2)) >> ((q & 3) * 8)) & 255u;
+            m.st(Y::kCnt + (xq >> 2), m.ld(Y::kCnt + (xq >> 2)) + (1u << ((xq & 3) * 8)));
+            fix += xq < 144 ? 8 : 9;
         }
     }
     // end of block
     m.st(Y::kCnt + 64, m.ld(Y::kCnt + 64) + 1u);
+    const int stat = (fix + 3 + 7) >> 3;
+
+    // ---- a lower bound on the dynamic block's bits, from the counts alone:
+    //  * data: at least the entropy of each alphabet's symbol counts (a lone
+    //    distance code costs exactly one bit per use);
+    //  * header: 5 + 5 + 4 bits, 3 bits per code-length code length sent
+    //    (at least min_order_pos + 1 of them), and the code-length symbols:
+    //    those of the zero runs between used symbols are known exactly
+    //    (symbols 0, 17, 18 and their extra bits), the islands of used
+    //    symbols need at least the counts run_counts gives, and coding all
+    //    of them costs at least the Huffman cost of those four counts
+    //    (merging symbols and lowering counts never raise a Huffman cost).
+    // When the bound shows fixed (or stored) coding no larger than dynamic,
+    // zlib's choice follows without building any tree.
+    int result = -1;
+    {
+        uint32_t um[9];   // used literal/length symbols 0 .. 287
+        float slog = 0.f;
+        int T = 0;
+#pragma unroll
+        for (int k = 0; k < 9; ++k) um[k] = 0u;
+#pragma unroll
+        for (int wd = 0; wd < 72; ++wd) {
+            const uint32_t v = m.ld(Y::kCnt + wd);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int f = static_cast<int>((v >> (8 * j)) & 255u);
+                T += f;
+                slog += static_cast<float>(f) * lg2_approx(static_cast<float>(f > 1 ? f : 1));
+            }
+            // bytes that are nonzero -> 4 bits (positions 21..24 of the product)
+            uint32_t t = v | (v >> 4);
+            t |= t >> 2;
+            t |= t >> 1;
+            t &= 0x01010101u;
+            um[wd >> 3] |= ((t * 0x204081u) >> 21 & 15u) << (4 * (wd & 7));
+        }
+        int U = 0;
+#pragma unroll
+        for (int k = 0; k < 9; ++k) U += __popc(um[k]);
+        int z0 = 0, z17 = 0, z18 = 0, zext = 0, nz = 0;
+        run_counts<9>(um, z0, z17, z18, zext, nz);
+        float data = static_cast<float>(T) * lg2_approx(static_cast<float>(T)) - slog;   // U >= 2 always
+        // distance codes, with zlib's dummies for fewer than two codes
+        int Td = 0, dmax = -1;
+        float slogd = 0.f;
+        uint32_t ud[1] = {0u};
+#pragma unroll
+        for (int wd = 0; wd < 8; ++wd) {
+            const uint32_t v = m.ld(Y::kDcnt + wd);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int f = static_cast<int>((v >> (8 * j)) & 255u);
+                Td += f;
+                slogd += static_cast<float>(f) * lg2_approx(static_cast<float>(f > 1 ? f : 1));
+                if (f) ud[0] |= 1u << (4 * wd + j);
+            }
+        }
+        const int Ud = __popc(ud[0]);
+        if (ud[0]) dmax = 31 - __clz(ud[0]);
+        int dbits_int = 0;
+        if (Ud >= 2) data += static_cast<float>(Td) * lg2_approx(static_cast<float>(Td)) - slogd;
+        else dbits_int = Td;   // zero or one code: one bit per use
+        for (int u = Ud; u < 2; ++u) {
+            const int sd = dmax < 2 ? ++dmax : 0;
+            ud[0] |= 1u << sd;
+        }
+        run_counts<1>(ud, z0, z17, z18, zext, nz);
+        int pos = min_order_pos(U);
+        const int pd = min_order_pos(Ud > 2 ? Ud : 2);
+        if (pd > pos) pos = pd;
+        const int hclen_lb = pos + 1 > 4 ? pos + 1 : 4;
+        // data bits rounded down with half a bit to spare for the approximate logarithms
+        const int data_lb = static_cast<int>(floorf(data - 0.5f)) + dbits_int;
+        const int lb = data_lb + extra + 5 + 5 + 4 + 3 * hclen_lb + huffman_cost4(z0, z17, z18, nz) + zext;
+        if (lb >= fix) result = (n + 4 <= stat) ? n + 5 : stat;   // fixed no larger than dynamic
+        else if (((lb + 3 + 7) >> 3) >= n + 4 && stat >= n + 4) result = n + 5;   // stored
+    }
+    if (__all_sync(lanes, result >= 0)) return result + 18;
+    if (result >= 0) return result + 18;   // this lane waits while the others build their trees
 
     // ---- literal/length tree: leaves in symbol order (never fewer than two:
     // end of block and at least one literal)
@@ -368,7 +560,7 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
             ++nleaf;
         }
     }
-    for (int i = 0; i < 19; ++i) m.st(Y::kBlf + i, 0u);
+    ClCounts cl;
     build_tree<MAXB>(m, nleaf, false);
     int dyn = extra;
     int blx = 0;   // extra bits of the code-length symbols
@@ -377,20 +569,20 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
         int prev = -1, rv = -1, rl = 0;
         for (int i = 0; i < nleaf; ++i) {
             const uint32_t w = m.ld(Y::kNode + i);
-            const int s = (w >> 9) & 511u, v = w >> 27;
+            const int sy = (w >> 9) & 511u, v = w >> 27;
             dyn += static_cast<int>((w >> 18) & 511u) * v;
-            const int gap = s - prev - 1;
+            const int gap = sy - prev - 1;
             if (gap > 0 || v != rv) {
-                blx += add_run<MAXB>(m, rv, rl);
-                blx += add_run<MAXB>(m, 0, gap);
+                blx += add_run(cl, rv, rl);
+                blx += add_run(cl, 0, gap);
                 rv = v;
                 rl = 1;
             } else {
                 ++rl;
             }
-            prev = s;
+            prev = sy;
         }
-        blx += add_run<MAXB>(m, rv, rl);
+        blx += add_run(cl, rv, rl);
     }
 
     // ---- distance tree (dummies for fewer than two codes)
@@ -408,9 +600,10 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
                 ++nleaf;
             }
         }
+        const int nreal = nleaf;
         while (nleaf < 2) {
-            const int s = max_code < 2 ? ++max_code : 0;
-            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (1u << 18));
+            const int sd = max_code < 2 ? ++max_code : 0;
+            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sd) << 9) | (1u << 18));
             ++nleaf;
         }
         build_tree<MAXB>(m, nleaf, false);
@@ -418,34 +611,24 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
         uint64_t dlo = 0, dhi = 0;
         for (int i = 0; i < nleaf; ++i) {
             const uint32_t w = m.ld(Y::kNode + i);
-            const int s = (w >> 9) & 511u;
+            const int sd = (w >> 9) & 511u;
             const uint64_t v = w >> 27;
-            if (s < 16) dlo |= v << (4 * s);
-            else dhi |= v << (4 * (s - 16));
-        }
-        for (int wd = 0; wd < 8; ++wd) {   // real codes only (dummies cost nothing net)
-            uint32_t cv = m.ld(Y::kDcnt + wd);
-            while (cv) {
-                const int j = (__ffs(cv) - 1) >> 3;
-                const int f = (cv >> (8 * j)) & 255u;
-                cv &= ~(255u << (8 * j));
-                const int s = 4 * wd + j;
-                const int len = static_cast<int>(((s < 16 ? dlo >> (4 * s) : dhi >> (4 * (s - 16)))) & 15u);
-                dyn += f * len;
-            }
+            if (sd < 16) dlo |= v << (4 * sd);
+            else dhi |= v << (4 * (sd - 16));
+            if (i < nreal) dyn += static_cast<int>((w >> 18) & 511u) * static_cast<int>(v);
         }
         int rv = -1, rl = 0;
-        for (int s = 0; s <= max_code; ++s) {
-            const int v = static_cast<int>(((s < 16 ? dlo >> (4 * s) : dhi >> (4 * (s - 16)))) & 15u);
+        for (int sd = 0; sd <= max_code; ++sd) {
+            const int v = static_cast<int>(((sd < 16 ? dlo >> (4 * sd) : dhi >> (4 * (sd - 16)))) & 15u);
             if (v == rv) {
                 ++rl;
             } else {
-                blx += add_run<MAXB>(m, rv, rl);
+                blx += add_run(cl, rv, rl);
                 rv = v;
                 rl = 1;
             }
         }
-        blx += add_run<MAXB>(m, rv, rl);
+        blx += add_run(cl, rv, rl);
     }
 
     // ---- code-length tree (limit 7 bits, with zlib's repair)
@@ -454,18 +637,18 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
     {
         nleaf = 0;
         int max_code = -1;
-        for (int s = 0; s < 19; ++s) {
-            const uint32_t f = m.ld(Y::kBlf + s);
+        for (int sy = 0; sy < 19; ++sy) {
+            const int f = cl.get(sy);
             if (f) {
-                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (f << 18));
-                max_code = s;
+                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (static_cast<uint32_t>(f) << 18));
+                max_code = sy;
                 ++nleaf;
             }
         }
         const int nreal = nleaf;
         while (nleaf < 2) {
-            const int s = max_code < 2 ? ++max_code : 0;
-            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(s) << 9) | (1u << 18));
+            const int sy = max_code < 2 ? ++max_code : 0;
+            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (1u << 18));
             ++nleaf;
         }
         const int nodes = build_tree<MAXB>(m, nleaf, true);
@@ -476,8 +659,8 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
             const uint32_t w = m.ld(Y::kNode + id);
             int d = static_cast<int>(w >> 27);
             if (id < nodes - 1) {
-                const int pd = static_cast<int>(m.ld(Y::kNode + (w & 511u)) >> 27);
-                d = pd + 1;
+                const int pdp = static_cast<int>(m.ld(Y::kNode + (w & 511u)) >> 27);
+                d = pdp + 1;
                 if (d > 7) {
                     d = 7;
                     ++overflow;
@@ -509,17 +692,17 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
         }
         for (int i = 0; i < nleaf; ++i) {
             const uint32_t w = m.ld(Y::kNode + i);
-            const int s = (w >> 9) & 511u;
-            bllen |= static_cast<uint64_t>(w >> 27) << (3 * s);
+            const int sy = (w >> 9) & 511u;
+            bllen |= static_cast<uint64_t>(w >> 27) << (3 * sy);
             if (i < nreal) blbits += static_cast<int>((w >> 18) & 511u) * static_cast<int>(w >> 27);
         }
     }
     // code-length code lengths sent: RFC order, trailing zeros trimmed, at least 4
-    constexpr uint64_t kOrderNibbles = 0xF1E2D3C4B5A69780ull;   // 16, 17, 18 then 0 8 7 9 6 10 5 11 4 12 3 13 2 14 1 15
+    constexpr uint64_t kOrderNibbles = 0xF1E2D3C4B5A69780ull;   // order positions 3..18: 0 8 7 9 6 10 5 11 4 12 3 13 2 14 1 15
     int hclen = 4;
     for (int i = 18; i >= 4; --i) {
-        const int sym = static_cast<int>((kOrderNibbles >> (4 * (i - 3))) & 15u);
-        if ((bllen >> (3 * sym)) & 7u) {
+        const int sy = static_cast<int>((kOrderNibbles >> (4 * (i - 3))) & 15u);
+        if ((bllen >> (3 * sy)) & 7u) {
             hclen = i + 1;
             break;
         }
@@ -527,7 +710,6 @@ __device__ int lane_block_length(const LaneMem& m, int n) {
     dyn += blbits + 5 + 5 + 4 + 3 * hclen;
 
     int opt = (dyn + 3 + 7) >> 3;
-    const int stat = (fix + 3 + 7) >> 3;
     if (stat <= opt) opt = stat;
     const int raw = (n + 4 <= opt) ? n + 5 : opt;
     return raw + 18;
@@ -567,7 +749,8 @@ block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblo
     __syncwarp();
     if (lane < nb) {
         const LaneMem m{region + lane};
-        lengths[task0 + lane] = lane_block_length<MAXB>(m, b);
+        const unsigned lanes = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+        lengths[task0 + lane] = lane_block_length<MAXB>(m, b, lanes);
     }
 }
 
