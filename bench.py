@@ -390,7 +390,7 @@ def record_traffic(csv_path, capture):
     print(json.dumps(out))
 
 
-_MASK_INST_SOURCES = ["content_adaptive_block_b200/csrc/deflate_len.cuh", "content_adaptive_block_b200/csrc/common.cuh",
+_MASK_INST_SOURCES = ["content_adaptive_block_b200/csrc/deflate_lane.cuh", "content_adaptive_block_b200/csrc/common.cuh",
                       "content_adaptive_block_b200/csrc/gsa.cu"]
 
 
@@ -405,17 +405,17 @@ def _sources_hash(sources):
 
 def record_mask_inst(csv_path, capture):
     """Write profiles/mask_inst.json from an ncu raw-page CSV export of one
-    block_lengths_kernel launch on the headline mask point: warp instructions
+    launch of the lengths kernel on the headline mask point: warp instructions
     executed per input byte, with the hash of the sources it was built from."""
     import csv
     rows = list(csv.reader(open(csv_path)))
     hdr, data = rows[0], rows[2:]
     col = {h: i for i, h in enumerate(hdr)}
-    row = next(r for r in data if "block_lengths_kernel" in r[col["Kernel Name"]])
+    row = next(r for r in data if "block_lengths" in r[col["Kernel Name"]])
     inst = float(row[col["smsp__inst_executed.sum"]].replace(",", ""))
     wl = W.mask_sweep(*MASK_POINT)
     nbytes = wl.S * wl.L
-    rec = {"kernel": "block_lengths_kernel", "workload": f"b{MASK_POINT[0]}_f{MASK_POINT[1]}: {wl.S} x {wl.L} bytes",
+    rec = {"kernel": row[col["Kernel Name"]].split("(")[0], "workload": f"b{MASK_POINT[0]}_f{MASK_POINT[1]}: {wl.S} x {wl.L} bytes",
            "warp_inst": inst, "bytes": nbytes, "inst_per_byte": inst / nbytes,
            "issue_active_pct": float(row[col["smsp__issue_active.avg.pct_of_peak_sustained_active"]]),
            "warps_active_pct": float(row[col["sm__warps_active.avg.pct_of_peak_sustained_active"]]),
@@ -549,13 +549,14 @@ def run_ours(args, rank, world, local_rank):
     # ---- mask-stage sweep (secondary metric), rank 0
     mask = mask_stage(gsa, dev) if (rank == 0 and not args.no_mask_sweep) else None
     sweep = seq_sweep(gsa, dev) if (rank == 0 and not args.no_seq_sweep) else None
+    cfgs = config_lines(gsa, dev) if (rank == 0 and not args.no_configs) else None
     variants = mask_variants(gsa, dev) if (rank == 0 and not args.no_mask_variants) else None
     block = lm_block(gsa, dev) if (rank == 0 and not args.no_lm_block) else None
 
     if rank != 0:
         return 0
     return report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops,
-                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep, variants, block)
+                  pairs, dense_pairs, launches_per_step, e2e, clocks, mask, sweep, variants, block, cfgs)
 
 
 def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_flops):
@@ -642,7 +643,7 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
 
 
 def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flops, bwd_flops, step_flops, pairs,
-           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None, variants=None, block=None):
+           dense_pairs, launches_per_step, e2e, clocks, mask, sweep=None, variants=None, block=None, cfgs=None):
     call_ms = {n: float(per_call[:, j].mean()) for j, n in enumerate(names)}
     bwd_ms, fwd_ms = call_ms["gsa_attn_bwd"], call_ms["gsa_attn_fwd"]
     # the calls are event-timed one by one inside a short region: the burst peak is their denominator
@@ -672,6 +673,8 @@ def report(args, wl, world, peaks, per_call, names, ms_per_step, value, fwd_flop
     }
     if mask:
         line["mask_stage"] = mask
+    if cfgs:
+        line["configs"] = cfgs
     if sweep:
         line["seq_sweep"] = sweep
     if variants:
@@ -744,19 +747,88 @@ def mask_stage(gsa, dev):
             "hbm_frac": (nbytes + out_bytes) / (best_ms * 1e-3) / 1e9 / _peaks()["hbm_gbs"]}
     key = f"b{MASK_POINT[0]}_f{MASK_POINT[1]}"
     out["value"] = out["points"][key]["gbs"]
-    # the lengths kernel is bound by issue (serial parse and Huffman builds per
-    # block), not by its bytes: its roofline is the SM issue rate, 4 warp
-    # instructions per cycle per SM at the maximum clock
+    # graded against HBM: bytes in (input) and out (lengths, flags, lists) over
+    # the stage's time.  The lengths kernel is latency-bound integer code far
+    # below that; its issue-rate use (warp instructions per byte from an ncu
+    # capture, 4 per cycle per SM at the maximum clock) is reported beside it.
     rec = _mask_inst_record()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    peak = 4.0 * sms * _peaks()["sm_max_mhz"] * 1e6
-    achieved = rec["inst_per_byte"] * out["points"][key]["lengths_gbs"] * 1e9 if rec else None
-    out["roofline"] = {"kernel": "block_lengths_kernel", "bound": "alu", "unit": "warp-inst/s",
-                       "achieved": achieved, "peak": peak, "frac": achieved / peak if rec else None,
+    peak_issue = 4.0 * sms * _peaks()["sm_max_mhz"] * 1e6
+    pt = out["points"][key]
+    issue = rec["inst_per_byte"] * pt["lengths_gbs"] * 1e9 if rec else None
+    out["roofline"] = {"kernel": "lengths + flags + lists", "bound": "hbm", "unit": "GB/s",
+                       "achieved": (pt["bytes_in"] + pt["bytes_out"]) / (pt["ms"] * 1e-3) / 1e9,
+                       "peak": _peaks()["hbm_gbs"], "frac": pt["hbm_frac"],
                        "inst_per_byte": rec["inst_per_byte"] if rec else None,
-                       "hbm_frac": out["points"][key]["hbm_frac"],
+                       "issue_frac": issue / peak_issue if rec else None,
                        "note": "instructions per byte from profiles/mask_inst.json (null when the sources changed)"}
     out["workload"] = f"{key}: 256 x 8192 bytes, w=2"
+    return out
+
+
+def config_lines(gsa, dev, steps=20, warmup=3):
+    """The attention calls on the other workloads: tiny fp32 (forward), 8 x 4K
+    (forward) and 1 x 64K (d = 128, forward and backward), each call timed
+    alone with CUDA events, L2 flushed before every call.  Per call the
+    algorithmic work (live token pairs P: forward 4 d P FLOPs, backward 8 d P)
+    and bytes (forward Q, K, V, O and LSE; backward Q, K, V, O, dO, LSE in and
+    dQ, dK, dV out, once each), reported as FLOP/s against the bf16 burst peak
+    and GB/s against the measured HBM copy bandwidth: the 4K and 64K calls
+    sit near or below the ridge point, so their HBM fraction is the bar."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks = _peaks()
+    out = {"unit_flops": "TFLOP/s", "unit_bytes": "GB/s", "peak_tflops": peaks["bf16_tflops"],
+           "peak_gbs": peaks["hbm_gbs"], "workloads": {}}
+    for name in ("tiny_fp32", "b8_4k", "b1_64k"):
+        wl = W.WORKLOADS[name]
+        hc = [int(c) for c in wl.head_classes()]
+        x = torch.from_numpy(W.batch_bytes(wl, seed=0)).to(dev)
+        flags = gsa.gsa_literal_flags(gsa.gsa_block_lengths(x, wl.b))
+        csr = gsa.gsa_build_block_csr(flags, wl.w)
+        f32 = wl.dtype == "f32"
+        q, k, v, do = W.qkv(wl, seed=0, device=dev, grad=True)
+        o = torch.empty_like(q)
+        lse = torch.empty((wl.S, wl.H, wl.L), dtype=torch.float32, device=dev)
+        calls = [("fwd", lambda: gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse))]
+        if wl.backward:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            ws = torch.empty(gsa.gsa_attn_bwd_workspace(q, wl.b, hc), dtype=torch.uint8, device=dev)
+            calls.append(("bwd", lambda: gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b, dq=dq, dk=dk, dv=dv,
+                                                          workspace=ws)))
+        nnz = csr.row_ptr[:, :, -1].cpu().numpy()
+        pairs = sum(live_token_pairs_from_counts(nnz[s], wl.N, wl.b, hc) for s in range(wl.S))
+        esz = 4 if f32 else 2
+        tensor = wl.S * wl.H * wl.L * wl.d * esz
+        vec = wl.S * wl.H * wl.L * 4
+        rec = {"config": workload_desc(wl), "live_token_pairs": pairs,
+               "literal_blocks": float(flags.float().sum(dim=1).mean().item()),
+               "live_fraction": pairs / (wl.S * wl.H * wl.L * (wl.L + 1) // 2)}
+        for label, fn in calls:
+            for _ in range(warmup):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for e0, e1 in evs:
+                flush.zero_()
+                e0.record()
+                fn()
+                e1.record()
+            torch.cuda.synchronize()
+            assert gsa.gsa_device_error() == 0, "a kernel gave up a bounded wait"
+            ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+            flops = (4 if label == "fwd" else 8) * wl.d * pairs
+            nbytes = 4 * tensor + vec if label == "fwd" else 8 * tensor + vec
+            tf = flops / (ms * 1e-3) / 1e12
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            rec[label] = {"ms": ms, "gflop": flops / 1e9, "mbytes": nbytes / 1e6, "tflops": tf,
+                          "frac_of_burst": tf / peaks["bf16_tflops"], "gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                          "bound": "hbm" if flops / nbytes < peaks["bf16_tflops"] * 1e3 / peaks["hbm_gbs"] else "tensor"}
+            if f32:
+                rec[label]["note"] = "float32 CUDA-core path (parity configuration); launch-bound at this size"
+        out["workloads"][name] = rec
+        del q, k, v, do, o
     return out
 
 
@@ -949,6 +1021,45 @@ def lm_block(gsa, dev, steps=10, warmup=3):
             "attn_gflop": attn / 1e9, "projections": "cuBLASLt (bf16, fp32 accumulate)"}
 
 
+def profile_lengths():
+    """gsa_block_lengths three times on the headline mask point (256 x 8192
+    bytes, b = 64, high-entropy fraction 0.3): a short program for an ncu
+    capture of the lengths kernel."""
+    import torch
+    import content_adaptive_block_b200 as gsa
+    from content_adaptive_block_b200 import build
+    build.build()
+    wl = W.mask_sweep(*MASK_POINT)
+    x = torch.from_numpy(W.batch_bytes(wl)).cuda()
+    for _ in range(3):
+        gsa.gsa_block_lengths(x, wl.b)
+    torch.cuda.synchronize()
+    print("lengths ok")
+    return 0
+
+
+def profile_attn(name):
+    """The mask and the attention calls of one workload, three times (a short
+    program for an ncu capture of one attention kernel)."""
+    import torch
+    import content_adaptive_block_b200 as gsa
+    from content_adaptive_block_b200 import build
+    build.build()
+    wl = W.WORKLOADS[name]
+    hc = [int(c) for c in wl.head_classes()]
+    x = torch.from_numpy(W.batch_bytes(wl)).cuda()
+    csr = gsa.gsa_build_block_csr(gsa.gsa_literal_flags(gsa.gsa_block_lengths(x, wl.b)), wl.w)
+    q, k, v, do = W.qkv(wl, seed=0, device="cuda", grad=True)
+    for _ in range(3):
+        o, lse = gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b)
+        if wl.backward:
+            gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    print("attn ok")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -958,6 +1069,8 @@ def main():
     ap.add_argument("--no-mask-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-seq-sweep", action="store_true", help="skip the 4K..64K sequence-length sweep")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the tiny / 8x4K / 1x64K attention call timings")
     ap.add_argument("--no-lm-block", action="store_true", help="skip the ByteLM block timing")
     ap.add_argument("--record-mask-inst", metavar="CSV",
                     help="write profiles/mask_inst.json from an ncu raw-page CSV export and exit")
@@ -967,7 +1080,15 @@ def main():
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw-page CSV export and exit")
     ap.add_argument("--capture", default="", help="the ncu command recorded with --record-traffic")
+    ap.add_argument("--profile-lengths", action="store_true",
+                    help="run gsa_block_lengths three times on the headline mask point and exit (for ncu)")
+    ap.add_argument("--profile-attn", metavar="WORKLOAD", choices=sorted(W.WORKLOADS),
+                    help="run the workload's attention calls three times and exit (for ncu)")
     args = ap.parse_args()
+    if args.profile_lengths:
+        return profile_lengths()
+    if args.profile_attn:
+        return profile_attn(args.profile_attn)
     if args.record_traffic:
         record_traffic(args.record_traffic, args.capture)
         return 0

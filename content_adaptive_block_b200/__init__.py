@@ -46,7 +46,7 @@ class GsaError(RuntimeError):
 class _Csr(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int32), ("nblk", ctypes.c_int32), ("w", ctypes.c_int32),
-        ("reserved", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("classes", ctypes.c_int32), ("capacity", ctypes.c_int64),
         ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
         ("col_ptr", ctypes.c_void_p), ("row_idx", ctypes.c_void_p),
         ("q_order", ctypes.c_void_p), ("k_order", ctypes.c_void_p),
@@ -81,7 +81,7 @@ def library():
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
         lib.gsa_block_lengths.argtypes = [vp, i32, i64, i32, vp, vp]
         lib.gsa_literal_flags.argtypes = [vp, i32, i32, vp, vp]
-        lib.gsa_build_block_csr.argtypes = [vp, i32, ctypes.POINTER(_Csr), vp]
+        lib.gsa_build_block_csr.argtypes = [vp, i32, vp, i32, ctypes.POINTER(_Csr), vp]
         lib.gsa_mask_pipeline.argtypes = [vp, i32, i64, i32, i32, vp, vp, ctypes.POINTER(_Csr), vp, vp]
         lib.gsa_build_fixed_csr.argtypes = [i32, i32, i32, i32, vp, ctypes.POINTER(_Csr), vp]
         lib.gsa_csr_capacity.argtypes = [i32]
@@ -169,6 +169,7 @@ class BlockCsr:
         cap = gsa_csr_capacity(nblk) if capacity is None else int(capacity)
         i32 = dict(dtype=torch.int32, device=device)
         self.B, self.nblk, self.capacity, self.w = B, nblk, cap, -1
+        self.classes = 0   # bitmask of the head classes whose lists were built
         self.row_ptr = torch.empty((B, 3, nblk + 1), **i32)
         self.col_idx = torch.empty((B, 3, cap), **i32)
         self.col_ptr = torch.empty((B, 3, nblk + 1), **i32)
@@ -177,7 +178,7 @@ class BlockCsr:
         self.k_order = torch.empty((B, 3, nblk), **i32)
 
     def struct(self) -> _Csr:
-        return _Csr(self.B, self.nblk, self.w, 0, self.capacity,
+        return _Csr(self.B, self.nblk, self.w, self.classes, self.capacity,
                     self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_ptr.data_ptr(),
                     self.row_idx.data_ptr(), self.q_order.data_ptr(), self.k_order.data_ptr())
 
@@ -193,16 +194,23 @@ class BlockCsr:
         return [ri[cp[j]: cp[j + 1]] for j in range(self.nblk)]
 
 
-def gsa_build_block_csr(flags: torch.Tensor, w: int, csr: BlockCsr | None = None, stream=None) -> BlockCsr:
-    """Block lists of the mask for all three head classes from literal flags."""
+def gsa_build_block_csr(flags: torch.Tensor, w: int, csr: BlockCsr | None = None, stream=None,
+                        head_classes=None) -> BlockCsr:
+    """Block lists of the mask from literal flags: for the classes in
+    head_classes (one per head), or for all three classes when it is None."""
     _need(flags, "flags", torch.uint8, 2)
     B, n = flags.shape
     if csr is None:
         csr = BlockCsr(B, n, flags.device)
     st = csr.struct()
-    _check("gsa_build_block_csr", library().gsa_build_block_csr(_ptr(flags), int(w), ctypes.byref(st),
-                                                                 _stream(stream)))
-    csr.w = st.w
+    hc, H = None, 0
+    if head_classes is not None:
+        H = len(head_classes)
+        hc = (ctypes.c_uint8 * H)(*[int(c) for c in head_classes])
+    _check("gsa_build_block_csr", library().gsa_build_block_csr(_ptr(flags), int(w),
+                                                                 ctypes.cast(hc, ctypes.c_void_p) if hc else None,
+                                                                 H, ctypes.byref(st), _stream(stream)))
+    csr.w, csr.classes = st.w, st.classes
     return csr
 
 
@@ -227,7 +235,7 @@ def gsa_build_fixed_csr(kind: int, B: int, nblk: int, w: int, g: int, rnd: torch
     _check("gsa_build_fixed_csr", library().gsa_build_fixed_csr(int(kind), int(w), int(g), r,
                                                                  _ptr(rnd) if rnd is not None else None,
                                                                  ctypes.byref(st), _stream(stream)))
-    csr.w = st.w
+    csr.w, csr.classes = st.w, st.classes
     return csr
 
 
@@ -255,7 +263,7 @@ def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None =
     _check("gsa_mask_pipeline", library().gsa_mask_pipeline(_ptr(data), B, L, int(b), int(w), _ptr(lengths),
                                                              _ptr(flags), ctypes.byref(st), _ptr(counters),
                                                              _stream(stream)))
-    csr.w = st.w
+    csr.w, csr.classes = st.w, st.classes
     return lengths, flags, csr
 
 

@@ -83,6 +83,7 @@ struct CsrArgs {
     int32_t* row_idx;
     int32_t* q_order;
     int32_t* k_order;
+    int cls[3];   // the classes built: CTA column x of the list kernel builds class cls[x]
 };
 
 __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
@@ -203,7 +204,7 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm) {
 
 __global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
     extern __shared__ __align__(16) uint8_t dsm[];
-    build_csr_sample(a, blockIdx.x, blockIdx.y, dsm);   // grid (class, sample)
+    build_csr_sample(a, a.cls[blockIdx.x], blockIdx.y, dsm);   // grid (classes built, sample)
 }
 
 inline size_t csr_smem_bytes(int n) {

@@ -162,6 +162,7 @@ gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t*
     if (!(d->scale >= 0.f) || !std::isfinite(d->scale)) return GSA_ERR_INVALID_ARGUMENT;
     for (int h = 0; h < d->H; ++h) {
         if (d->head_classes[h] > 2) return GSA_ERR_INVALID_ARGUMENT;
+        if (!((csr->classes >> d->head_classes[h]) & 1)) return GSA_ERR_INVALID_ARGUMENT;   // lists not built
         cls[h] = d->head_classes[h];
     }
     if (d->dtype != GSA_F32 && d->dtype != GSA_BF16) return GSA_ERR_INVALID_ARGUMENT;
@@ -194,15 +195,24 @@ gsa_status gsa_literal_flags(const int32_t* lengths, int32_t B, int32_t nblk, ui
     return launch_status();
 }
 
-gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* csr, void* stream) {
+gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, const uint8_t* head_classes, int32_t H,
+                               gsa_block_csr* csr, void* stream) {
     const gsa::CallRange nvtx_range("gsa_build_block_csr");
     if (!flags || !csr || w < 0) return GSA_ERR_INVALID_ARGUMENT;
+    int classes = 7;
+    if (head_classes) {
+        if (H < 1 || H > GSA_MAX_HEADS) return GSA_ERR_INVALID_ARGUMENT;
+        classes = 0;
+        for (int h = 0; h < H; ++h) {
+            if (head_classes[h] > 2) return GSA_ERR_INVALID_ARGUMENT;
+            classes |= 1 << head_classes[h];
+        }
+    }
     if (csr->B < 1 || csr->nblk < 1 || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
         !csr->q_order || !csr->k_order)
         return GSA_ERR_INVALID_ARGUMENT;
     if (csr->nblk > gsa::mask::kMaxBlocksCsr) return GSA_ERR_UNSUPPORTED;
     if (csr->capacity < gsa_csr_capacity(csr->nblk)) return GSA_ERR_CAPACITY;
-    csr->w = w;
     gsa::mask::CsrArgs a;
     a.flags = flags;
     a.nblk = csr->nblk;
@@ -214,11 +224,16 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* c
     a.row_idx = csr->row_idx;
     a.q_order = csr->q_order;
     a.k_order = csr->k_order;
+    int ncls = 0;
+    for (int c = 0; c < 3; ++c)
+        if ((classes >> c) & 1) a.cls[ncls++] = c;
     const size_t smem = gsa::mask::csr_smem_bytes(csr->nblk);
     if (!gsa::smem_opt_in(gsa::mask::build_csr_kernel,
                           static_cast<int>(gsa::mask::csr_smem_bytes(gsa::mask::kMaxBlocksCsr))))
         return GSA_ERR_CUDA;
-    dim3 grid(3, csr->B);
+    csr->w = w;
+    csr->classes = classes;
+    dim3 grid(ncls, csr->B);
     gsa::mask::build_csr_kernel<<<grid, gsa::mask::kThreads, smem, as_stream(stream)>>>(a);
     return launch_status();
 }
@@ -236,6 +251,7 @@ gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, co
     if (csr->nblk > gsa::fixed::kMaxBlocks || r > gsa::fixed::kMaxRandom) return GSA_ERR_UNSUPPORTED;
     if (csr->capacity < gsa_csr_capacity(csr->nblk)) return GSA_ERR_CAPACITY;
     csr->w = w;
+    csr->classes = 7;
     gsa::fixed::FixedArgs a;
     a.kind = kind;
     a.nblk = csr->nblk;
@@ -276,7 +292,11 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     const int64_t grid = (total + kWarps - 1) / kWarps;
     if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
     csr->w = w;
+    csr->classes = 7;
     gsa::mask::CsrArgs a;
+    a.cls[0] = 0;
+    a.cls[1] = 1;
+    a.cls[2] = 2;
     a.flags = flags;
     a.nblk = static_cast<int>(nblk);
     a.w = w;

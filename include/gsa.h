@@ -122,7 +122,7 @@ typedef struct {
     int32_t B;
     int32_t nblk;
     int32_t w;          /* set by gsa_build_block_csr */
-    int32_t reserved;
+    int32_t classes;    /* bit c set: the lists of head class c were built (set by the builders) */
     int64_t capacity;   /* entries per (sample, class) in col_idx and row_idx */
     int32_t* row_ptr;
     int32_t* col_idx;
@@ -163,18 +163,25 @@ gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, co
 int64_t gsa_csr_capacity(int32_t nblk);
 
 /*
- * gsa_build_block_csr — the lists above from the literal flags.
+ * gsa_build_block_csr — the lists above from the literal flags, for the head
+ * classes the heads use.
  *
- *   flags  [csr->B][csr->nblk] uint8 (nonzero = literal)
- *   w      local window in blocks, >= 0
- *   csr    host struct; its B, nblk, capacity and device pointers are read,
- *          w is written.
- * Head classes are not an argument: the lists are built for all three classes
- * and each attention head picks its class.
- * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, sizes < 1, w < 0),
- *         GSA_ERR_CAPACITY (capacity < gsa_csr_capacity(nblk)).
+ *   flags         [csr->B][csr->nblk] uint8 (nonzero = literal)
+ *   w             local window in blocks, >= 0
+ *   head_classes  host [H], each 0, 1 or 2 (gsa_head_class): the lists are
+ *                 built only for the classes that appear (a class's slots of
+ *                 the arrays are left untouched otherwise); NULL builds all
+ *                 three (H is then ignored)
+ *   H             heads, 1 .. GSA_MAX_HEADS (when head_classes is given)
+ *   csr           host struct; its B, nblk, capacity and device pointers are
+ *                 read, w and classes (the bitmask of classes built) are written.
+ * The attention calls reject a head whose class's lists were not built.
+ * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, sizes < 1, w < 0, H out of
+ *         range, a class outside 0..2), GSA_ERR_CAPACITY (capacity <
+ *         gsa_csr_capacity(nblk)).
  */
-gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, gsa_block_csr* csr, void* stream);
+gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, const uint8_t* head_classes, int32_t H,
+                               gsa_block_csr* csr, void* stream);
 
 /*
  * gsa_mask_pipeline — gsa_block_lengths, gsa_literal_flags and

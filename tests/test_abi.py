@@ -75,23 +75,39 @@ def test_literal_flags_rejects_bad_arguments(lib):
     assert f(FAKE, 1, 0, FAKE, NULL) == 1
 
 
-def _csr(B=1, n=4, cap=None):
+def _csr(B=1, n=4, cap=None, classes=7):
     p = 0x1000
-    return gsa._Csr(B, n, 0, 0, gsa.gsa_csr_capacity(n) if cap is None else cap, p, p, p, p, p, p)
+    return gsa._Csr(B, n, 0, classes, gsa.gsa_csr_capacity(n) if cap is None else cap, p, p, p, p, p, p)
 
 
 def test_build_csr_rejects_bad_arguments(lib):
     f = lib.gsa_build_block_csr
     c = _csr()
-    assert f(NULL, 1, ctypes.byref(c), NULL) == 1
-    assert f(FAKE, -1, ctypes.byref(c), NULL) == 1          # negative window
+    assert f(NULL, 1, NULL, 0, ctypes.byref(c), NULL) == 1
+    assert f(FAKE, -1, NULL, 0, ctypes.byref(c), NULL) == 1          # negative window
     c0 = _csr(B=0)
-    assert f(FAKE, 1, ctypes.byref(c0), NULL) == 1
+    assert f(FAKE, 1, NULL, 0, ctypes.byref(c0), NULL) == 1
     small = _csr(n=8, cap=10)
-    assert f(FAKE, 1, ctypes.byref(small), NULL) == 3       # capacity
+    assert f(FAKE, 1, NULL, 0, ctypes.byref(small), NULL) == 3       # capacity
     nul = _csr()
     nul.q_order = None
-    assert f(FAKE, 1, ctypes.byref(nul), NULL) == 1
+    assert f(FAKE, 1, NULL, 0, ctypes.byref(nul), NULL) == 1
+    hc = (ctypes.c_uint8 * 3)(0, 3, 1)
+    assert f(FAKE, 1, ctypes.cast(hc, ctypes.c_void_p), 3, ctypes.byref(c), NULL) == 1   # class 3
+    hc = (ctypes.c_uint8 * 1)(0)
+    assert f(FAKE, 1, ctypes.cast(hc, ctypes.c_void_p), 0, ctypes.byref(c), NULL) == 1   # H = 0
+
+
+def test_attention_rejects_heads_of_classes_not_built(lib):
+    # lists of the local class only (classes = 0b001): a literal head is refused before any launch
+    c = _csr(B=1, n=4, classes=1)
+    hc = (ctypes.c_uint8 * 2)(0, 1)
+    d = gsa._AttnDesc(1, 2, 256, 64, 64, 1, 0.0, ctypes.cast(hc, ctypes.c_void_p))
+    p = FAKE
+    assert lib.gsa_attn_fwd(p, p, p, ctypes.byref(c), ctypes.byref(d), p, p, NULL) == 1
+    hc[1] = 0
+    c.classes = 0
+    assert lib.gsa_attn_fwd(p, p, p, ctypes.byref(c), ctypes.byref(d), p, p, NULL) == 1
 
 
 def test_build_fixed_csr_rejects_bad_arguments(lib):

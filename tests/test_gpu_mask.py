@@ -160,3 +160,40 @@ def test_pipeline_end_to_end_mask(gsa):
     for s in range(wl.S):
         for c in (0, 1, 2):
             assert csr.rows(s, c) == [list(r) for r in omask.row_lists(omask.block_mask(want_fl[s], wl.w, c))]
+
+
+@pytest.mark.parametrize("head_classes", [[0, 0], [1], [2, 2, 1], [1, 0, 2]])
+def test_block_lists_for_the_classes_in_use(gsa, head_classes):
+    """gsa_build_block_csr with head classes builds the lists of exactly the
+    classes that appear (the other classes' slots keep what they held) and
+    records them; attention on those heads matches the all-class build bit
+    for bit, and a head of a class not built is refused."""
+    B, n, w, b, d = 2, 33, 2, 64, 64
+    rng = np.random.default_rng(len(head_classes))
+    fl = torch.from_numpy((rng.random((B, n)) < 0.4).astype(np.uint8)).cuda()
+    full = gsa.gsa_build_block_csr(fl, w)
+    part = gsa.BlockCsr(B, n, fl.device)
+    for t in (part.row_ptr, part.col_ptr, part.q_order, part.k_order, part.col_idx, part.row_idx):
+        t.fill_(-7)
+    gsa.gsa_build_block_csr(fl, w, part, head_classes=head_classes)
+    torch.cuda.synchronize()
+    want = sum(1 << c for c in set(head_classes))
+    assert part.classes == want and full.classes == 7
+    for c in range(3):
+        if (want >> c) & 1:
+            for s in range(B):
+                assert part.rows(s, c) == full.rows(s, c) and part.cols(s, c) == full.cols(s, c)
+            assert torch.equal(part.q_order[:, c], full.q_order[:, c])
+            assert torch.equal(part.k_order[:, c], full.k_order[:, c])
+        else:
+            assert (part.row_ptr[:, c] == -7).all() and (part.q_order[:, c] == -7).all()
+    H = len(head_classes)
+    q, k, v = (t.cuda() for t in W.random_tensors((B, H, n * b, d), 3, torch.bfloat16, seed=40 + H))
+    o1, l1 = gsa.gsa_attn_fwd(q, k, v, full, head_classes, b)
+    o2, l2 = gsa.gsa_attn_fwd(q, k, v, part, head_classes, b)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    missing = [c for c in range(3) if not (want >> c) & 1]
+    if missing:
+        with pytest.raises(RuntimeError):
+            gsa.gsa_attn_fwd(q, k, v, part, [missing[0]] * H, b)

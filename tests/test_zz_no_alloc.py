@@ -125,7 +125,7 @@ def test_noalloc_rejects_rows_beyond_its_scratch(gsa):
     hcs = (ctypes.c_uint8 * H)(*([0] * H))
     desc = gsa._AttnDesc(S, H, n * b, 64, b, 1, 0.0, ctypes.cast(hcs, ctypes.c_void_p))
     fake = 0x1000
-    st = gsa._Csr(S, n, 1, 0, gsa.gsa_csr_capacity(n), fake, fake, fake, fake, fake, fake)
+    st = gsa._Csr(S, n, 1, 7, gsa.gsa_csr_capacity(n), fake, fake, fake, fake, fake, fake)
     p = ctypes.c_void_p(fake)
     rc = fn(p, p, p, p, p, p, ctypes.byref(st), ctypes.byref(desc), p, p, p, ctypes.c_void_p(0))
     assert rc == 3   # GSA_ERR_CAPACITY
