@@ -54,8 +54,11 @@ def _peaks():
 
 
 def workload_desc(wl):
+    hc = [int(c) for c in wl.head_classes()]
+    split = "/".join(str(hc.count(c)) for c in (0, 1, 2))
     return (f"{wl.name}: batch {wl.S} x {wl.L} bytes, b={wl.b} ({wl.N} blocks), w={wl.w}, "
-            f"{wl.H} heads (6 local/3 literal/3 hybrid), d={wl.d}, {wl.dtype}, fwd+bwd")
+            f"{wl.H} heads ({split} local/literal/hybrid), d={wl.d}, {wl.dtype}, "
+            f"{'fwd+bwd' if wl.backward else 'fwd'}")
 
 
 def live_token_pairs_from_counts(nnz_sc, n, b, head_classes):
