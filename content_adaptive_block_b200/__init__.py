@@ -82,7 +82,7 @@ def library():
         lib.gsa_block_lengths.argtypes = [vp, i32, i64, i32, vp, vp]
         lib.gsa_literal_flags.argtypes = [vp, i32, i32, vp, vp]
         lib.gsa_build_block_csr.argtypes = [vp, i32, vp, i32, ctypes.POINTER(_Csr), vp]
-        lib.gsa_mask_pipeline.argtypes = [vp, i32, i64, i32, i32, vp, vp, ctypes.POINTER(_Csr), vp, vp]
+        lib.gsa_mask_pipeline.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, vp, ctypes.POINTER(_Csr), vp, vp]
         lib.gsa_build_fixed_csr.argtypes = [i32, i32, i32, i32, vp, ctypes.POINTER(_Csr), vp]
         lib.gsa_csr_capacity.argtypes = [i32]
         lib.gsa_csr_capacity.restype = i64
@@ -182,13 +182,20 @@ class BlockCsr:
                     self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_ptr.data_ptr(),
                     self.row_idx.data_ptr(), self.q_order.data_ptr(), self.k_order.data_ptr())
 
+    def slot(self, s: int, c: int) -> int:
+        """The sample whose slot holds (s, c)'s lists: sample 0's for the local
+        class when it is stored once (classes bit 3)."""
+        return 0 if (c == 0 and self.classes & 8) else s
+
     def rows(self, s: int, c: int) -> list:
         """Key-block list of every query block of (sample s, class c), on the host."""
+        s = self.slot(s, c)
         rp = self.row_ptr[s, c].cpu().tolist()
         ci = self.col_idx[s, c, : rp[-1]].cpu().tolist()
         return [ci[rp[i]: rp[i + 1]] for i in range(self.nblk)]
 
     def cols(self, s: int, c: int) -> list:
+        s = self.slot(s, c)
         cp = self.col_ptr[s, c].cpu().tolist()
         ri = self.row_idx[s, c, : cp[-1]].cpu().tolist()
         return [ri[cp[j]: cp[j + 1]] for j in range(self.nblk)]
@@ -241,9 +248,10 @@ def gsa_build_fixed_csr(kind: int, B: int, nblk: int, w: int, g: int, rnd: torch
 
 def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None = None,
                       lengths: torch.Tensor | None = None, flags: torch.Tensor | None = None,
-                      counters: torch.Tensor | None = None, stream=None):
+                      counters: torch.Tensor | None = None, stream=None, head_classes=None):
     """lengths -> flags -> block lists in one launch; returns (lengths, flags, csr).
-    counters (int32 [B], zero, left zero by each call) may be passed to avoid
+    The local class's lists are stored once (sample 0's slot).  counters (int32,
+    at least one element, zero, left zero by each call) may be passed to avoid
     allocating one per call."""
     _need(data, "data", torch.uint8, 2)
     B, L = data.shape
@@ -255,14 +263,19 @@ def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None =
     if csr is None:
         csr = BlockCsr(B, n, data.device)
     if counters is None:
-        counters = torch.zeros(B, dtype=torch.int32, device=data.device)
+        counters = torch.zeros(1, dtype=torch.int32, device=data.device)
     _need(lengths, "lengths", torch.int32)
     _need(flags, "flags", torch.uint8)
     _need(counters, "counters", torch.int32)
     st = csr.struct()
-    _check("gsa_mask_pipeline", library().gsa_mask_pipeline(_ptr(data), B, L, int(b), int(w), _ptr(lengths),
-                                                             _ptr(flags), ctypes.byref(st), _ptr(counters),
-                                                             _stream(stream)))
+    hc, H = None, 0
+    if head_classes is not None:
+        H = len(head_classes)
+        hc = (ctypes.c_uint8 * H)(*[int(c) for c in head_classes])
+    _check("gsa_mask_pipeline", library().gsa_mask_pipeline(_ptr(data), B, L, int(b), int(w),
+                                                             ctypes.cast(hc, ctypes.c_void_p) if hc else None, H,
+                                                             _ptr(lengths), _ptr(flags), ctypes.byref(st),
+                                                             _ptr(counters), _stream(stream)))
     csr.w, csr.classes = st.w, st.classes
     return lengths, flags, csr
 

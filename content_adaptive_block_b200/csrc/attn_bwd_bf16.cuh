@@ -76,6 +76,7 @@ struct Params {
     float scale_log2;
     int* ticket;            // work counter of the persistent kernel (dot_kernel zeroes both)
     uint8_t cls[kMaxHeads];
+    int local_once;   // the local class's lists are stored once, in sample 0's slot
 };
 
 // ------------------------------------------------------------ D_t = dO·O
@@ -197,7 +198,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
     const int qa = p.order[g * nblk + 2 * tile];
     const int qb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
     const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
@@ -518,7 +519,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
     const int ka = p.order[g * nblk + 2 * tile];
     const int kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
     const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
@@ -894,6 +895,7 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     base.scale_log2 = scale * kLog2e;
     base.ticket = reinterpret_cast<int*>(work + 2 * ((rows + 63) & ~int64_t(63)));   // after D and LSE2
     for (int h = 0; h < desc->H; ++h) base.cls[h] = cls[h];
+    base.local_once = (csr->classes >> 3) & 1;
     Params pq = base, pkv = base;
     pq.ticket = base.ticket + 1;
     pq.ptr = csr->row_ptr;

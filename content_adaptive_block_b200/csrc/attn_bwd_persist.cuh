@@ -120,7 +120,7 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         sh = it % SH;
         const int tile = it / SH;
         const int s = sh / p.H, h = sh % p.H;
-        g = static_cast<int64_t>(s) * 3 + p.cls[h];
+        g = (p.cls[h] == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + p.cls[h];
         ka = p.order[g * nblk + 2 * tile];
         kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
     };

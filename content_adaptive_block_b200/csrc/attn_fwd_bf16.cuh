@@ -109,6 +109,7 @@ struct FwdParams {
     float scale_log2;   // softmax scale * log2(e)
     int* ticket;        // persistent kernel: work counter, CTAs finished (both zero at launch)
     uint8_t cls[kMaxHeads];
+    int local_once;   // the local class's lists are stored once, in sample 0's slot
 };
 
 template <int D>
@@ -175,7 +176,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
     const int qa = p.q_order[g * nblk + 2 * tile];
     const int qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
     const int nwords = (nblk + 31) >> 5;

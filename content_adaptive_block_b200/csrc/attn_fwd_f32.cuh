@@ -33,6 +33,7 @@ struct Params {
     int64_t L;
     float scale;
     uint8_t cls[kMaxHeads];
+    int local_once;   // the local class's lists are stored once, in sample 0's slot
 };
 
 template <int D>
@@ -44,7 +45,7 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(Params p) {
     float* sv = sk + b * D;       // [b][D]
     const int i = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int c = p.cls[h];
-    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
     const int64_t head_off = (static_cast<int64_t>(s) * p.H + h) * p.L;
     const int r = threadIdx.x;
     const int64_t row0 = head_off + static_cast<int64_t>(i) * b;

@@ -125,7 +125,7 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         sh = it % SH;
         const int tile = it / SH;
         const int s = sh / p.H, h = sh % p.H;
-        g = static_cast<int64_t>(s) * 3 + p.cls[h];
+        g = (p.cls[h] == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + p.cls[h];
         qa = p.q_order[g * nblk + 2 * tile];
         qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
     };

@@ -723,21 +723,14 @@ struct KernelShape {
     static constexpr int kSmemBytes = kWarpBytes * kWarps;
 };
 
-// Lengths of blocks task0 .. task0 + 31 of the batch, one per lane: the
-// warp stages its 32 blocks (contiguous bytes) into the lanes' words with
-// coalesced loads, then each lane runs its block.
+// Lengths of the nb (<= 32) blocks task0 .. task0 + nb - 1 of the batch, one
+// per lane, into lengths[task0 ..]: the warp stages its blocks (contiguous
+// bytes) into the lanes' words of region with coalesced loads, then each lane
+// runs its block.  Whole warp.
 template <int MAXB>
-__global__ void __launch_bounds__(32 * KernelShape<MAXB>::kWarps)
-block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblocks_total,
-                          int32_t* __restrict__ lengths) {
+__device__ __forceinline__ void warp_block_lengths(uint32_t* region, const uint8_t* __restrict__ bytes, int b,
+                                                   int64_t task0, int nb, int32_t* __restrict__ lengths, int lane) {
     using Y = Layout<MAXB>;
-    extern __shared__ __align__(16) uint32_t lsmem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* region = lsmem + static_cast<size_t>(warp) * Y::kWords * 32;
-    const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * 32;
-    if (task0 >= nblocks_total) return;   // warp-uniform
-    const int nb = nblocks_total - task0 < 32 ? static_cast<int>(nblocks_total - task0) : 32;
-    // zero every lane's byte words, then scatter the warp's nb * b contiguous bytes
     for (int i = 0; i < Y::kXw; ++i) region[(Y::kXb + i) * 32 + lane] = 0u;
     __syncwarp();
     const uint8_t* src = bytes + task0 * b;
@@ -752,6 +745,23 @@ block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblo
         const unsigned lanes = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
         lengths[task0 + lane] = lane_block_length<MAXB>(m, b, lanes);
     }
+    __syncwarp();   // the region may be restaged next
+}
+
+// Lengths of blocks task0 .. task0 + 31 of the batch, one per lane (see
+// warp_block_lengths), one warp per CTA.
+template <int MAXB>
+__global__ void __launch_bounds__(32 * KernelShape<MAXB>::kWarps)
+block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblocks_total,
+                          int32_t* __restrict__ lengths) {
+    using Y = Layout<MAXB>;
+    extern __shared__ __align__(16) uint32_t lsmem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* region = lsmem + static_cast<size_t>(warp) * Y::kWords * 32;
+    const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * 32;
+    if (task0 >= nblocks_total) return;   // warp-uniform
+    const int nb = nblocks_total - task0 < 32 ? static_cast<int>(nblocks_total - task0) : 32;
+    warp_block_lengths<MAXB>(region, bytes, b, task0, nb, lengths, lane);
 }
 
 }  // namespace deflate_lane

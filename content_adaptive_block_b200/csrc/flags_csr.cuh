@@ -91,8 +91,9 @@ __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
 
 // Lists of class c for sample s, by the whole CTA (any multiple of 32
 // threads up to 1024); dsm holds csr_smem_bytes(nblk).  Reads the flags from
-// a.flags, so a CTA that wrote them must synchronise first.
-__device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm) {
+// a.flags (a CTA that wrote them must synchronise first), or, with
+// flags_ready, finds them (0 / 1) already in dsm[0 .. nblk).
+__device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, bool flags_ready = false) {
     const int n = a.nblk;
     uint8_t* fl = dsm;                                              // [n]
     int* pre = reinterpret_cast<int*>(dsm + ((n + 15) & ~15));      // [n] inclusive literal count
@@ -103,7 +104,8 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm) {
 
     const int64_t g = static_cast<int64_t>(s) * 3 + c;
     const int w = a.w;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) fl[i] = a.flags[static_cast<int64_t>(s) * n + i] ? 1 : 0;
+    if (!flags_ready)
+        for (int i = threadIdx.x; i < n; i += blockDim.x) fl[i] = a.flags[static_cast<int64_t>(s) * n + i] ? 1 : 0;
     __syncthreads();
 
     // literal prefix counts: each thread scans a contiguous chunk

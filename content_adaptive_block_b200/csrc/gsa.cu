@@ -12,7 +12,6 @@
 #include "gsa.h"
 
 #include "common.cuh"
-#include "deflate_len.cuh"
 #include "deflate_lane.cuh"
 #include "flags_csr.cuh"
 #include "mask_pipeline.cuh"
@@ -152,6 +151,34 @@ gsa_status launch_lengths_lane(const uint8_t* bytes, int b, int64_t total, int32
     return launch_status();
 }
 
+// The one-launch mask stage for blocks of at most MAXB bytes: a cooperative
+// launch (every CTA resident: the phases meet at a grid barrier) of as many
+// CTAs as fit on the device at once, at most one per 32-block chunk group.
+template <int MAXB>
+gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
+    using S = gsa::pipeline::Shape<MAXB>;
+    auto kernel = gsa::pipeline::mask_pipeline_kernel<MAXB>;
+    if (!gsa::smem_opt_in(kernel, static_cast<int>(S::kSmemBytes))) return GSA_ERR_CUDA;
+    int dev = 0, per_sm = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * S::kWarps, S::kSmemBytes) !=
+            cudaSuccess ||
+        per_sm < 1)
+        return GSA_ERR_CUDA;
+    const int64_t chunks = (P.total + 31) / 32;
+    const int64_t need = (chunks + S::kWarps - 1) / S::kWarps;
+    const int64_t jobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    int64_t grid = static_cast<int64_t>(per_sm) * sms;
+    const int64_t want = need > jobs ? need : jobs;
+    if (want < grid) grid = want;
+    void* args[] = {const_cast<gsa::pipeline::PipeArgs*>(&P)};
+    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel),
+                                                      dim3(static_cast<unsigned>(grid)),
+                                                      dim3(32 * S::kWarps), args, S::kSmemBytes, cs);
+    return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {
     if (!d || !csr || !d->head_classes) return GSA_ERR_INVALID_ARGUMENT;
     if (!csr_ok(csr)) return csr && csr->capacity < gsa_csr_capacity(csr->nblk) ? GSA_ERR_CAPACITY
@@ -275,28 +302,42 @@ gsa_status gsa_build_fixed_csr(int32_t kind, int32_t w, int32_t g, int32_t r, co
     return launch_status();
 }
 
-gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w, int32_t* lengths,
-                             uint8_t* flags, gsa_block_csr* csr, int32_t* counters, void* stream) {
+gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w,
+                             const uint8_t* head_classes, int32_t H, int32_t* lengths, uint8_t* flags,
+                             gsa_block_csr* csr, int32_t* counter, void* stream) {
     const gsa::CallRange nvtx_range("gsa_mask_pipeline");
-    if (!bytes || !lengths || !flags || !csr || !counters || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES ||
+    if (!bytes || !lengths || !flags || !csr || !counter || B < 1 || b < 1 || b > GSA_MAX_BLOCK_BYTES ||
         L < b || L % b != 0 || w < 0)
         return GSA_ERR_INVALID_ARGUMENT;
     const int64_t nblk = L / b;
     if (csr->B != B || csr->nblk != nblk || !csr->row_ptr || !csr->col_idx || !csr->col_ptr || !csr->row_idx ||
         !csr->q_order || !csr->k_order)
         return GSA_ERR_INVALID_ARGUMENT;
+    int classes = 7;
+    if (head_classes) {
+        if (H < 1 || H > GSA_MAX_HEADS) return GSA_ERR_INVALID_ARGUMENT;
+        classes = 0;
+        for (int h = 0; h < H; ++h) {
+            if (head_classes[h] > 2) return GSA_ERR_INVALID_ARGUMENT;
+            classes |= 1 << head_classes[h];
+        }
+    }
     if (nblk > GSA_MAX_PIPELINE_BLOCKS) return GSA_ERR_UNSUPPORTED;
     if (csr->capacity < gsa_csr_capacity(static_cast<int32_t>(nblk))) return GSA_ERR_CAPACITY;
-    using namespace gsa::deflate;
     const int64_t total = static_cast<int64_t>(B) * nblk;
-    const int64_t grid = (total + kWarps - 1) / kWarps;
-    if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
-    csr->w = w;
-    csr->classes = 7;
-    gsa::mask::CsrArgs a;
-    a.cls[0] = 0;
-    a.cls[1] = 1;
-    a.cls[2] = 2;
+    gsa::pipeline::PipeArgs P{};
+    P.bytes = bytes;
+    P.b = b;
+    P.B = B;
+    P.nblk = static_cast<int>(nblk);
+    P.total = total;
+    P.lengths = lengths;
+    P.flags = flags;
+    P.counter = counter;
+    P.local_once = classes & 1;
+    for (int c = 1; c < 3; ++c)
+        if ((classes >> c) & 1) P.per[P.nper++] = c;
+    gsa::mask::CsrArgs& a = P.a;
     a.flags = flags;
     a.nblk = static_cast<int>(nblk);
     a.w = w;
@@ -307,10 +348,14 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     a.row_idx = csr->row_idx;
     a.q_order = csr->q_order;
     a.k_order = csr->k_order;
-    if (!gsa::smem_opt_in(gsa::pipeline::mask_pipeline_kernel, static_cast<int>(kSmemBytes))) return GSA_ERR_CUDA;
-    gsa::pipeline::mask_pipeline_kernel<<<static_cast<unsigned>(grid), 32 * kWarps, kSmemBytes, as_stream(stream)>>>(
-        bytes, L, b, total, lengths, flags, a, counters);
-    return launch_status();
+    gsa_status st;
+    if (b <= 32) st = launch_pipeline<32>(P, as_stream(stream));
+    else if (b <= 64) st = launch_pipeline<64>(P, as_stream(stream));
+    else st = launch_pipeline<128>(P, as_stream(stream));
+    if (st != GSA_OK) return st;
+    csr->w = w;
+    csr->classes = classes | (P.local_once ? 8 : 0);
+    return GSA_OK;
 }
 
 gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_block_csr* csr,
@@ -342,6 +387,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
         p.L = desc->L;
         p.scale = scale;
         std::memcpy(p.cls, cls, desc->H);
+        p.local_once = (csr->classes >> 3) & 1;
         dim3 grid(csr->nblk, desc->H, desc->B);
         const size_t smem = 3u * desc->b * desc->d * sizeof(float);
         bool opted = false;
@@ -390,6 +436,7 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     p.lse = lse;
     p.scale_log2 = scale * 1.4426950408889634f;
     std::memcpy(p.cls, cls, desc->H);
+    p.local_once = (csr->classes >> 3) & 1;
     dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
     if (desc->d == 64 && GSA_FWD_PERSIST) {
         p.ticket = fwd_ticket_slot();

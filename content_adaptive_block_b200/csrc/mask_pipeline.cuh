@@ -3,84 +3,139 @@
 //
 // Gzip-guided Sparse Attention (daiwk.github.io), flowchart and section
 // "核心公式": gzip level-1 per block, r_i > r̄ per sample, then the mask of
-// each head class.  The flags of a sample need every one of its lengths, so
-// the stages meet per sample: each CTA (four warps, one block each, as in the
-// lengths kernel) adds the number of blocks it finished for each sample to a
-// per-sample counter after a fence; the CTA whose addition completes a
-// sample computes that sample's flags and its three classes' lists with all
-// 128 threads, reusing the shared memory of the lengths phase, and resets the
-// counter.  No CTA waits for another, so nothing can stall.
+// each head class.  The flags of a sample need all of its lengths, so the
+// launch is cooperative (every CTA resident at once) with two phases and one
+// grid barrier between them:
+//   1. lengths: every warp takes chunks of 32 consecutive blocks, one block
+//      per lane, exactly as the lengths kernel does (deflate_lane.cuh);
+//   2. lists: jobs (sample, class) spread over all CTAs.  A job sums its
+//      sample's lengths, sets the flags (len_i * nblk > Σ len) in shared
+//      memory — the sample's first job also writes them out — and builds the
+//      class's lists.  The local class's lists depend only on (nblk, w)
+//      (mask equation: |i - j| <= w intersected with causality), so they are
+//      built once, into sample 0's slot, and the attention calls read that
+//      slot for every sample.
+// The barrier: each CTA adds one to a counter in caller-owned memory and
+// waits (bounded by a time limit, after which it records an error code and
+// leaves) until all have; each CTA adds one more as it leaves, and the last
+// to leave sets the counter back to zero for the next call.
 #pragma once
 
-#include "deflate_len.cuh"
+#include "deflate_lane.cuh"
 #include "flags_csr.cuh"
 
 namespace gsa {
 namespace pipeline {
 
-constexpr int kMaxBlocks = 1024;   // block lists built in the lengths phase's shared memory
-// the list scratch of build_csr_sample (csr_smem_bytes) fits in the lengths phase's
-static_assert(sizeof(deflate::WarpSmem) * deflate::kWarps >=
-                  ((kMaxBlocks + 15) & ~15) + 4 * (2 * kMaxBlocks + 2 * (kMaxBlocks + 1) + 64),
-              "list scratch fits in the lengths scratch");
+constexpr int kMaxBlocks = 1024;   // blocks per sample (the lists' scratch sits in the CTA's shared memory)
 
-__global__ void __launch_bounds__(32 * deflate::kWarps)
-mask_pipeline_kernel(const uint8_t* __restrict__ bytes, int64_t L, int b, int64_t nblocks_total,
-                     int32_t* __restrict__ lengths, uint8_t* __restrict__ flags, mask::CsrArgs a,
-                     int* __restrict__ counters) {
-    extern __shared__ __align__(16) uint8_t dsmem[];
-    __shared__ int fin[deflate::kWarps];
-    __shared__ int nfin;
-    __shared__ long long part[deflate::kWarps];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nblk = L / b;
-    const int64_t task0 = static_cast<int64_t>(blockIdx.x) * deflate::kWarps;
-    const int64_t task = task0 + warp;
-    if (task < nblocks_total) {
-        deflate::WarpSmem& ws = reinterpret_cast<deflate::WarpSmem*>(dsmem)[warp];
-        const int64_t s = task / nblk, i = task % nblk;
-        const int len = deflate::block_length_warp(ws, bytes + s * L + i * b, b, lane);
-        if (lane == 0) {
-            lengths[task] = len;
-            __threadfence();   // ordered before this CTA's counter update
-        }
-    }
+template <int MAXB>
+struct Shape {
+    // warps per CTA: as many as fit (up to 16) in 220 KB of shared memory; the
+    // list jobs run on all of them
+    static constexpr int kWarpBytes = deflate_lane::Layout<MAXB>::kWords * 128;
+    static constexpr int kWarps = 220 * 1024 / kWarpBytes < 16 ? 220 * 1024 / kWarpBytes : 16;
+    static constexpr size_t kLengthsBytes = static_cast<size_t>(kWarps) * kWarpBytes;
+    static constexpr size_t kListBytes = ((kMaxBlocks + 15) & ~15) + 4 * (2 * kMaxBlocks + 2 * (kMaxBlocks + 1) + 64);
+    static constexpr size_t kSmemBytes = kLengthsBytes > kListBytes ? kLengthsBytes : kListBytes;
+};
+
+struct PipeArgs {
+    const uint8_t* bytes;
+    int b;
+    int B;
+    int nblk;
+    int64_t total;        // B * nblk blocks
+    int32_t* lengths;     // [B][nblk]
+    uint8_t* flags;       // [B][nblk]
+    mask::CsrArgs a;
+    int* counter;         // the grid barrier's counter (zero between calls)
+    int nper;             // classes built per sample (those other than a local class built once)
+    int per[3];           // ... and which
+    int local_once;       // 1: the local class is in use, built once into sample 0's slot
+};
+
+// All CTAs of the grid reach this point (thread 0 of each waits, bounded);
+// false when the wait gave up.
+__device__ __forceinline__ bool grid_barrier(int* counter, int target) {
+    __shared__ int ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        // this CTA's blocks, per sample (consecutive tasks: samples ascend)
-        nfin = 0;
-        int64_t t = task0;
-        const int64_t tend = task0 + deflate::kWarps < nblocks_total ? task0 + deflate::kWarps : nblocks_total;
-        while (t < tend) {
-            const int64_t s = t / nblk;
-            const int64_t send = (s + 1) * nblk < tend ? (s + 1) * nblk : tend;
-            const int cnt = static_cast<int>(send - t);
-            if (atomicAdd(&counters[s], cnt) + cnt == nblk) fin[nfin++] = static_cast<int>(s);
-            t = send;
+        __threadfence();   // this CTA's lengths before its arrival
+        atomicAdd(counter, 1);
+        ok = 1;
+        const unsigned long long t0 = globaltimer_ns();
+        for (uint32_t it = 0;; ++it) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+            if (v >= target) break;
+            __nanosleep(256);   // leave the SM's issue slots to the warps still computing lengths
+            if ((it & 15u) == 15u && globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_error(kErrTimeoutOther);
+                ok = 0;
+                break;
+            }
         }
+        __threadfence();
     }
     __syncthreads();
-    for (int f = 0; f < nfin; ++f) {
-        const int s = fin[f];
-        __threadfence();   // the other CTAs' lengths of this sample are visible
-        const int32_t* row = lengths + static_cast<int64_t>(s) * nblk;
+    return ok != 0;
+}
+
+template <int MAXB>
+__global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel(const PipeArgs P) {
+    constexpr int kWarps = Shape<MAXB>::kWarps;
+    extern __shared__ __align__(16) uint8_t dsmem[];
+    __shared__ long long part[kWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- phase 1: lengths, chunks of 32 blocks per warp
+    {
+        uint32_t* region = reinterpret_cast<uint32_t*>(dsmem) +
+                           static_cast<size_t>(warp) * deflate_lane::Layout<MAXB>::kWords * 32;
+        const int64_t nchunks = (P.total + 31) / 32;
+        for (int64_t ch = static_cast<int64_t>(blockIdx.x) * kWarps + warp; ch < nchunks;
+             ch += static_cast<int64_t>(gridDim.x) * kWarps) {
+            const int64_t task0 = ch * 32;
+            const int nb = P.total - task0 < 32 ? static_cast<int>(P.total - task0) : 32;
+            deflate_lane::warp_block_lengths<MAXB>(region, P.bytes, P.b, task0, nb, P.lengths, lane);
+        }
+    }
+    if (!grid_barrier(P.counter, static_cast<int>(gridDim.x))) return;
+
+    // ---- phase 2: (sample, class) jobs.  Per sample max(nper, 1) jobs (one
+    // writes the flags even when no per-sample class is built), then the
+    // local class once.
+    const int n = P.nblk;
+    const int jobs_per = P.nper > 0 ? P.nper : 1;
+    const int njobs = P.B * jobs_per + P.local_once;
+    uint8_t* fl = dsmem;   // the list builder's flag scratch: dsm[0 .. n)
+    for (int j = blockIdx.x; j < njobs; j += gridDim.x) {
+        const bool local = j == P.B * jobs_per;
+        const int s = local ? 0 : j / jobs_per;
+        const int k = local ? 0 : j % jobs_per;
+        const int c = local ? 0 : (P.nper > 0 ? P.per[k] : -1);
+        __syncthreads();   // the previous job's scratch
+        const int32_t* row = P.lengths + static_cast<int64_t>(s) * n;
         long long acc = 0;
-        for (int i = threadIdx.x; i < nblk; i += blockDim.x) acc += __ldcg(row + i);
+        for (int i = threadIdx.x; i < n; i += blockDim.x) acc += __ldcg(row + i);
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (lane == 0) part[warp] = acc;
         __syncthreads();
         long long total = 0;
-        for (int k = 0; k < deflate::kWarps; ++k) total += part[k];
-        uint8_t* frow = flags + static_cast<int64_t>(s) * nblk;
-        for (int i = threadIdx.x; i < nblk; i += blockDim.x)
-            frow[i] = static_cast<long long>(__ldcg(row + i)) * nblk > total ? 1 : 0;
-        __syncthreads();
-        for (int c = 0; c < 3; ++c) {
-            mask::build_csr_sample(a, c, s, dsmem);
-            __syncthreads();
+        for (int w = 0; w < kWarps; ++w) total += part[w];
+        const bool write = !local && k == 0;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint8_t f = static_cast<long long>(__ldcg(row + i)) * n > total ? 1 : 0;
+            fl[i] = f;
+            if (write) P.flags[static_cast<int64_t>(s) * n + i] = f;
         }
-        if (threadIdx.x == 0) counters[s] = 0;   // ready for the next call
+        if (c >= 0) mask::build_csr_sample(P.a, c, s, dsmem, true);
     }
+
+    // ---- leave: the last CTA out resets the counter for the next call
+    __syncthreads();
+    if (threadIdx.x == 0 && atomicAdd(P.counter, 1) == 2 * static_cast<int>(gridDim.x) - 1) *P.counter = 0;
 }
 
 }  // namespace pipeline

@@ -122,7 +122,8 @@ typedef struct {
     int32_t B;
     int32_t nblk;
     int32_t w;          /* set by gsa_build_block_csr */
-    int32_t classes;    /* bit c set: the lists of head class c were built (set by the builders) */
+    int32_t classes;    /* bit c set: the lists of head class c were built; bit 3: the local
+                           class's lists are stored once, in sample 0's slot (set by the builders) */
     int64_t capacity;   /* entries per (sample, class) in col_idx and row_idx */
     int32_t* row_ptr;
     int32_t* col_idx;
@@ -185,28 +186,39 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, const uint8_t* h
 
 /*
  * gsa_mask_pipeline — gsa_block_lengths, gsa_literal_flags and
- * gsa_build_block_csr in one launch, with the same outputs bit for bit.
+ * gsa_build_block_csr in one launch.
  *
  * The flowchart of the pages (gzip level-1 per block -> r_i > r̄ -> mask per
- * head class) as one pass: the CTA that finishes the last block of a sample
- * computes that sample's flags and lists.  No CTA waits for another.
+ * head class) as one pass: a cooperative launch whose CTAs first compute all
+ * lengths, meet at a grid barrier, then share out the (sample, class) list
+ * jobs, each of which computes its sample's flags.  The local class's lists
+ * depend only on (nblk, w): they are built once, into sample 0's slot, and
+ * csr->classes gets bit 3 (value 8) to say so; the attention calls then read
+ * that slot for every sample.  Lengths, flags and the other classes' lists
+ * are those of the three calls, bit for bit.
  *
  *   bytes, B, L, b   as for gsa_block_lengths; L / b = nblk <= GSA_MAX_PIPELINE_BLOCKS
  *   w                local window in blocks, >= 0
+ *   head_classes, H  as for gsa_build_block_csr (NULL: all three classes)
  *   lengths          [B][nblk] int32 out
  *   flags            [B][nblk] uint8 out
  *   csr              as for gsa_build_block_csr (csr->B == B, csr->nblk == nblk)
- *   counters         [B] int32 device scratch owned by the caller: zero before
- *                    the first call; every completed call leaves it zero.
- *                    Two calls in flight at once must not share it.
- * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, bad sizes, csr shape),
- *         GSA_ERR_UNSUPPORTED (nblk > GSA_MAX_PIPELINE_BLOCKS: use the three
- *         calls), GSA_ERR_CAPACITY (capacity < gsa_csr_capacity(nblk)).
+ *   counter          one int32 of device scratch owned by the caller (the
+ *                    grid barrier's counter): zero before the first call;
+ *                    every completed call leaves it zero.  Two calls in
+ *                    flight at once must not share it.  After a call whose
+ *                    barrier timed out (a device error code is recorded) it
+ *                    must be zeroed again.
+ * Errors: GSA_ERR_INVALID_ARGUMENT (null pointers, bad sizes, csr shape, H or
+ *         a class out of range), GSA_ERR_UNSUPPORTED (nblk >
+ *         GSA_MAX_PIPELINE_BLOCKS: use the three calls), GSA_ERR_CAPACITY
+ *         (capacity < gsa_csr_capacity(nblk)), GSA_ERR_CUDA (the cooperative
+ *         launch was refused).
  */
 #define GSA_MAX_PIPELINE_BLOCKS 1024
 gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t b, int32_t w,
-                             int32_t* lengths, uint8_t* flags, gsa_block_csr* csr, int32_t* counters,
-                             void* stream);
+                             const uint8_t* head_classes, int32_t H, int32_t* lengths, uint8_t* flags,
+                             gsa_block_csr* csr, int32_t* counter, void* stream);
 
 /*
  * Attention problem description (host struct).

@@ -169,20 +169,25 @@ def test_lm_block_rejects_bad_arguments(lib):
 def test_mask_pipeline_rejects_bad_arguments(lib):
     f = lib.gsa_mask_pipeline
     c = _csr(B=2, n=8)
-    # bytes, B, L, b, w, lengths, flags, csr, counters, stream; 2 samples x 512 bytes, b=64 -> 8 blocks
-    args = [FAKE, 2, 512, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL]
-    for i in (0, 5, 6, 8):                                   # null device pointers
-        bad = list(args)
-        bad[i] = NULL
-        assert f(*bad) == 1, i
-    assert f(FAKE, 2, 512, 64, -1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1   # negative window
-    assert f(FAKE, 2, 500, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1    # L % b
-    assert f(FAKE, 3, 512, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1    # csr->B != B
-    assert f(FAKE, 2, 1024, 64, 1, FAKE, FAKE, ctypes.byref(c), FAKE, NULL) == 1   # csr->nblk != L / b
+    # bytes, B, L, b, w, head_classes, H, lengths, flags, csr, counter, stream; 2 samples x 512 bytes, b=64
+    def call(**kw):
+        a = dict(bytes=FAKE, B=2, L=512, b=64, w=1, hc=NULL, H=0, lengths=FAKE, flags=FAKE, csr=ctypes.byref(c),
+                 counter=FAKE)
+        a.update(kw)
+        return f(a["bytes"], a["B"], a["L"], a["b"], a["w"], a["hc"], a["H"], a["lengths"], a["flags"], a["csr"],
+                 a["counter"], NULL)
+    for name in ("bytes", "lengths", "flags", "counter"):       # null device pointers
+        assert call(**{name: NULL}) == 1, name
+    assert call(w=-1) == 1                                       # negative window
+    assert call(L=500) == 1                                      # L % b
+    assert call(B=3) == 1                                        # csr->B != B
+    assert call(L=1024) == 1                                     # csr->nblk != L / b
+    hc = (ctypes.c_uint8 * 2)(0, 5)
+    assert call(hc=ctypes.cast(hc, ctypes.c_void_p), H=2) == 1   # a class outside 0..2
     big = _csr(B=1, n=2048)
-    assert f(FAKE, 1, 2048 * 16, 16, 1, FAKE, FAKE, ctypes.byref(big), FAKE, NULL) == 2   # beyond one launch
+    assert call(B=1, L=2048 * 16, b=16, csr=ctypes.byref(big)) == 2   # beyond one launch
     small = _csr(B=2, n=8, cap=10)
-    assert f(FAKE, 2, 512, 64, 1, FAKE, FAKE, ctypes.byref(small), FAKE, NULL) == 3      # capacity
+    assert call(csr=ctypes.byref(small)) == 3                    # capacity
 
 
 def _desc(B=1, H=4, L=256, d=64, b=64, dtype=1, classes=(0, 0, 1, 2), scale=0.0):

@@ -3,8 +3,9 @@ the three separate calls, which test_gpu_mask.py pins to the oracle, and its
 lengths against the oracle directly: every output must match bit for bit.
 Cases cover CTAs that straddle samples (blocks per sample not a multiple of
 four), one block per sample, the largest supported list (1024 blocks), the
-mask-sweep batches at full size, and two calls in a row on one counter
-buffer (each call leaves it zero)."""
+mask-sweep batches at full size, two calls in a row on one counter
+(each call leaves it zero), subsets of the head classes, and attention on
+the pipeline's lists (the local class stored once)."""
 import numpy as np
 import pytest
 import torch
@@ -23,33 +24,34 @@ def gsa():
     return g
 
 
-def _lists(csr):
-    """(row_ptr, col_ptr, q_order, k_order, per-(sample, class) entries) on the host."""
-    rp, cp = csr.row_ptr.cpu().numpy(), csr.col_ptr.cpu().numpy()
-    ci, ri = csr.col_idx.cpu().numpy(), csr.row_idx.cpu().numpy()
-    ents = []
-    for s in range(rp.shape[0]):
-        for c in range(3):
-            ents.append((ci[s, c, :rp[s, c, -1]].copy(), ri[s, c, :cp[s, c, -1]].copy()))
-    return rp, cp, csr.q_order.cpu().numpy(), csr.k_order.cpu().numpy(), ents
+def _slot_lists(csr, s, c):
+    """Pointers, pairing orders and entries of (sample s, class c) from the slot that holds them."""
+    s = csr.slot(s, c)
+    rp, cp = csr.row_ptr[s, c].cpu().numpy(), csr.col_ptr[s, c].cpu().numpy()
+    return (rp, cp, csr.q_order[s, c].cpu().numpy(), csr.k_order[s, c].cpu().numpy(),
+            csr.col_idx[s, c, :rp[-1]].cpu().numpy(), csr.row_idx[s, c, :cp[-1]].cpu().numpy())
 
 
-def _same(gsa, x: np.ndarray, b: int, w: int, counters=None):
+def _same(gsa, x: np.ndarray, b: int, w: int, counters=None, head_classes=None):
+    """The pipeline against the three calls: lengths and flags bit for bit, and
+    every (sample, class) list of the classes in use equal to the three calls'
+    (the local class read from sample 0's slot, where the pipeline stores it once)."""
     t = torch.from_numpy(np.ascontiguousarray(x)).cuda()
     ln_ref = gsa.gsa_block_lengths(t, b)
     fl_ref = gsa.gsa_literal_flags(ln_ref)
     csr_ref = gsa.gsa_build_block_csr(fl_ref, w)
-    ln, fl, csr = gsa.gsa_mask_pipeline(t, b, w, counters=counters)
+    ln, fl, csr = gsa.gsa_mask_pipeline(t, b, w, counters=counters, head_classes=head_classes)
     torch.cuda.synchronize()
     assert gsa.gsa_device_error() == 0
     assert torch.equal(ln, ln_ref)
     assert torch.equal(fl, fl_ref)
     assert csr.w == csr_ref.w == w
-    a, r = _lists(csr), _lists(csr_ref)
-    for got, want in zip(a[:4], r[:4]):
-        assert np.array_equal(got, want)
-    for (gc, gr), (wc, wr) in zip(a[4], r[4]):
-        assert np.array_equal(gc, wc) and np.array_equal(gr, wr)
+    used = {0, 1, 2} if head_classes is None else set(head_classes)
+    assert csr.classes == sum(1 << c for c in used) | (8 if 0 in used else 0)
+    for s in range(x.shape[0]):
+        for c in sorted(used):
+            for got, want in zip(_slot_lists(csr, s, c), _slot_lists(csr_ref, s, c)):
+                assert np.array_equal(got, want), (s, c)
     return ln.cpu().numpy()
 
 
@@ -77,7 +79,33 @@ def test_pipeline_odd_shapes(gsa, B, nblk, b, w):
 
 def test_pipeline_reuses_its_counters(gsa):
     wl = W.WORKLOADS["b8_4k"]
-    counters = torch.zeros(wl.S, dtype=torch.int32, device="cuda")
+    counters = torch.zeros(1, dtype=torch.int32, device="cuda")
     for seed in (0, 1, 2):
         _same(gsa, W.batch_bytes(wl, seed=seed), wl.b, wl.w, counters=counters)
         assert int(counters.abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("head_classes", [[0], [1, 2], [2, 0, 0], [1]])
+def test_pipeline_classes_in_use(gsa, head_classes):
+    wl = W.WORKLOADS["b8_4k"]
+    _same(gsa, W.batch_bytes(wl, seed=4), wl.b, wl.w, head_classes=head_classes)
+
+
+def test_attention_on_pipeline_lists(gsa):
+    """Forward and backward on the pipeline's lists (local class stored once)
+    give the three-call lists' results bit for bit, at d = 64 and d = 128."""
+    wl = W.WORKLOADS["b8_4k"]
+    hc = [int(c) for c in wl.head_classes()]
+    t = torch.from_numpy(W.batch_bytes(wl, seed=5)).cuda()
+    csr_ref = gsa.gsa_build_block_csr(gsa.gsa_literal_flags(gsa.gsa_block_lengths(t, wl.b)), wl.w)
+    _, _, csr = gsa.gsa_mask_pipeline(t, wl.b, wl.w)
+    for d in (64, 128):
+        q, k, v, do = (x.cuda() for x in W.random_tensors((wl.S, wl.H, wl.L, d), 4, torch.bfloat16, seed=d))
+        outs = []
+        for c in (csr_ref, csr):
+            o, lse = gsa.gsa_attn_fwd(q, k, v, c, hc, wl.b)
+            outs.append([o, lse, *gsa.gsa_attn_bwd(q, k, v, o, lse, do, c, hc, wl.b)])
+        torch.cuda.synchronize()
+        assert gsa.gsa_device_error() == 0
+        for a, b_ in zip(*outs):
+            assert torch.equal(a, b_), d
