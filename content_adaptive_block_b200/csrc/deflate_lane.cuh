@@ -27,7 +27,7 @@
 //    entered before the next one is looked at; after a match of at most 4
 //    bytes that leaves >= 3 bytes, its inner positions are entered too,
 //    after a longer one they are skipped.  The chains here are short bucket
-//    lists (64 buckets on the hash's low bits) filtered by the full hash,
+//    lists (one bucket per position of the largest block, on the hash's low bits) filtered by the full hash,
 //    which visits exactly zlib's chain in the same order.
 //  * trees: the literal/length and distance codes are Huffman codes built
 //    with zlib's heap discipline: leaves in increasing symbol order, a
@@ -54,30 +54,63 @@
 namespace gsa {
 namespace deflate_lane {
 
-constexpr int kBuckets = 64;            // hash-chain buckets per block (low 6 hash bits)
 
-// Per-lane word layout (offsets in words; word i of lane l is at
-// smem[i * 32 + l] of the warp's region).  Phase A (parse) and phase B
-// (trees) overlap: the literal counts survive until their leaves are
-// gathered, which writes only nodes 0 .. leaves-1.
+// Per-lane word layout in shared memory (offsets in words; word i of lane l
+// is at smem[i * 32 + l] of the warp's region).  The literal counts are made
+// after the parse, over the position words it no longer needs; the counts of
+// the length codes (and end of block) and of the distance codes are made
+// during the parse, in words of their own.
 template <int MAXB>
 struct Layout {
-    static constexpr int kMaxLeaves = MAXB + 2;            // symbols of one tree (+ dummies)
+    // Blocks of at most 64 bytes build their (rare) Huffman trees in local
+    // memory and keep only the parse's words here; larger blocks need the
+    // trees often enough that they keep them here too, over words dead by then.
+    static constexpr bool kSharedTrees = MAXB > 64;
+    static constexpr int kMaxLeaves = MAXB + 2;
     static constexpr int kXb = 0;                          // block bytes, 4 per word, zero padded
     static constexpr int kXw = MAXB / 4 + 3;
     static constexpr int kPos = kXb + kXw;                 // per position: hash | previous bucket-mate << 15
+    static constexpr int kBuckets = MAXB;                  // hash buckets (the hash's low bits), one per position
     static constexpr int kHeads = kPos + MAXB;             // bucket heads, 4 positions per word
     static constexpr int kPhaseA = kHeads + kBuckets / 4;
-    static constexpr int kCnt = kPhaseA > kMaxLeaves ? kPhaseA : kMaxLeaves;   // literal/length counts, 4 per word
+    // literal counts (bytes 0..255, 4 per word): over the position words,
+    // made after the parse; with shared trees, in words of their own above
+    // the nodes the leaves take
+    static constexpr int kLcnt = kSharedTrees ? (kPhaseA > kMaxLeaves ? kPhaseA : kMaxLeaves) : kPos;
+    // symbols 256..287 (end of block, length codes), 4 per word, then the distance codes
+    static constexpr int kMcnt = kSharedTrees ? kLcnt + 64 : kPos + (MAXB + kBuckets / 4 > 64 ? MAXB + kBuckets / 4 : 64);
+    // with shared trees the distance counts must outlive the literal/length tree
+    static constexpr int kDcnt = kSharedTrees ? ((kMcnt + 8 > 3 * kMaxLeaves + 1) ? kMcnt + 8 : 3 * kMaxLeaves + 1)
+                                              : kMcnt + 8;
+    static constexpr int kWords = kSharedTrees ? ((kDcnt + 8 > 2 * kMaxLeaves + 64) ? kDcnt + 8 : 2 * kMaxLeaves + 64)
+                                               : kMcnt + 16;
+};
+
+// Words of the Huffman builds: in local memory (blocks <= 64 bytes, whose
+// lower bound below rarely fails) or in the lane's shared words (larger).
+template <int MAXB>
+struct TreeLayout {
+    static constexpr bool kShared = Layout<MAXB>::kSharedTrees;
+    static constexpr int kMaxLeaves = MAXB + 2;            // symbols of one tree (+ dummies)
     static constexpr int kNode = 0;                        // parent | symbol << 9 | freq << 18 | bits << 27
     static constexpr int kHeap = 2 * kMaxLeaves;           // (freq << 8 | depth) << 9 | node, 1-based
-    static constexpr int kDcnt = (kCnt + 72 > kHeap + kMaxLeaves + 1) ? kCnt + 72 : kHeap + kMaxLeaves + 1;
     // code-length tree (<= 19 leaves, 37 nodes, 20 heap entries): its nodes in
-    // heap-exit order, above its heap entries, over words dead by then
-    static constexpr int kOrder = kHeap + 24;
-    static constexpr int kWords = (kDcnt + 8 > kOrder + 40) ? kDcnt + 8 : kOrder + 40;
-    static_assert(kCnt >= kMaxLeaves, "gathering leaves leaves the counts intact");
+    // heap-exit order, above its heap entries (shared: over words dead by then)
+    static constexpr int kOrder = kShared ? kHeap + 24 : kHeap + kMaxLeaves + 1;
+    static constexpr int kWords = kOrder + 40;
+    static_assert(!kShared || kOrder + 40 <= Layout<MAXB>::kWords, "the heap-exit order fits");
+    static_assert(!kShared || kHeap + kMaxLeaves + 1 <= Layout<MAXB>::kDcnt, "distance counts outlive the heap");
+    static_assert(!kShared || Layout<MAXB>::kLcnt >= kMaxLeaves, "leaves gathered below the literal counts");
 };
+
+// Word holding the count of literal/length symbol s (0..287) or, with dist,
+// of distance code s (0..29).
+template <int MAXB>
+__device__ __forceinline__ int cnt_word(int s, bool dist = false) {
+    using Y = Layout<MAXB>;
+    if (dist) return Y::kDcnt + (s >> 2);
+    return s < 256 ? Y::kLcnt + (s >> 2) : Y::kMcnt + ((s - 256) >> 2);
+}
 
 // The 19 code-length symbol counts (each < 512) in three registers, 9 bits
 // apiece: symbol s in word s / 7 at bit 9 (s % 7).
@@ -138,6 +171,13 @@ struct LaneMem {
     __device__ __forceinline__ void st(int i, uint32_t v) const { p[i * 32] = v; }
 };
 
+// One thread's local-memory words.
+struct LocalMem {
+    uint32_t* p;
+    __device__ __forceinline__ uint32_t ld(int i) const { return p[i]; }
+    __device__ __forceinline__ void st(int i, uint32_t v) const { p[i] = v; }
+};
+
 // 4 bytes of the block starting at byte k (little endian; k + 4 within the padded words).
 template <int MAXB>
 __device__ __forceinline__ uint32_t load4(const LaneMem& m, int k) {
@@ -153,9 +193,9 @@ __device__ __forceinline__ int equal_bytes(uint32_t a, uint32_t b) {
 
 // Sift the heap entry at k down (zlib's heap discipline; comparisons on the
 // key bits above the node id).
-template <int MAXB>
-__device__ __forceinline__ void sift_down(const LaneMem& m, int len, int k) {
-    constexpr int H = Layout<MAXB>::kHeap;
+template <int MAXB, typename M>
+__device__ __forceinline__ void sift_down(const M& m, int len, int k) {
+    constexpr int H = TreeLayout<MAXB>::kHeap;
     const uint32_t v = m.ld(H + k);
     const uint32_t kv = v | 511u;
     int j = k << 1;
@@ -181,18 +221,18 @@ __device__ __forceinline__ void sift_down(const LaneMem& m, int len, int k) {
 // its code length (bits 27..31).  track: record the heap-exit order at
 // kOrder (needed for the repair of a length-limited tree).  Returns the
 // number of nodes.
-template <int MAXB>
-__device__ int build_tree(const LaneMem& m, int nleaf, bool track) {
-    using Y = Layout<MAXB>;
+template <int MAXB, typename M>
+__device__ int build_tree(const M& m, int nleaf, bool track) {
+    using Y = TreeLayout<MAXB>;
     for (int i = 0; i < nleaf; ++i) m.st(Y::kHeap + 1 + i, ((m.ld(Y::kNode + i) >> 18 & 511u) << 17) | i);
     int len = nleaf;
-    for (int k = len >> 1; k >= 1; --k) sift_down<MAXB>(m, len, k);
+    for (int k = len >> 1; k >= 1; --k) sift_down<MAXB, M>(m, len, k);
     int next = nleaf, no = 0;
     do {
         const uint32_t a = m.ld(Y::kHeap + 1);
         m.st(Y::kHeap + 1, m.ld(Y::kHeap + len));
         --len;
-        sift_down<MAXB>(m, len, 1);
+        sift_down<MAXB, M>(m, len, 1);
         const uint32_t b = m.ld(Y::kHeap + 1);
         const int na = a & 511u, nb = b & 511u;
         m.st(Y::kNode + na, m.ld(Y::kNode + na) | next);
@@ -208,7 +248,7 @@ __device__ int build_tree(const LaneMem& m, int nleaf, bool track) {
         m.st(Y::kNode + next, 0u);
         m.st(Y::kHeap + 1, (key << 9) | next);
         ++next;
-        sift_down<MAXB>(m, len, 1);
+        sift_down<MAXB, M>(m, len, 1);
     } while (len >= 2);
     if (track) m.st(Y::kOrder + no, m.ld(Y::kHeap + 1) & 511u);
     // lengths, parents before children (a parent's id is above its children's)
@@ -255,6 +295,12 @@ __device__ __forceinline__ int add_run(ClCounts& cl, int v, int R) {
     cl.add(v, nv);
     if (n16) cl.add(16, n16);
     return 2 * n16;
+}
+
+// x (< 2^23) as a float with one integer OR and one subtraction (the
+// float 2^23 + x minus 2^23), leaving the conversion unit alone.
+__device__ __forceinline__ float small_int_float(uint32_t x) {
+    return __uint_as_float(0x4B000000u | x) - 8388608.f;
 }
 
 // Huffman cost (sum of frequency x code length) of at most four symbol
@@ -341,6 +387,181 @@ __device__ __forceinline__ void run_counts(const uint32_t (&um)[NWD], int& z0, i
     if (ones) nz += run <= 3 ? run : 2;
 }
 
+// The exact size, with zlib's trees: the literal/length, distance and
+// code-length Huffman codes built as the header says, their run-length
+// coded lengths, and zlib's choice of block kind.  m: the lane's counts;
+// t: the words of the trees (see TreeLayout).
+template <int MAXB, typename TM>
+__device__ int exact_length(const LaneMem& m, const TM& t, int n, int extra, int stat) {
+    using TY = TreeLayout<MAXB>;
+    // ---- literal/length tree: leaves in symbol order (never fewer than two:
+    // end of block and at least one literal)
+    int nleaf = 0;
+    for (int wd = 0; wd < 72; ++wd) {
+        uint32_t v = m.ld(cnt_word<MAXB>(4 * wd));
+        while (v) {
+            const int j = (__ffs(v) - 1) >> 3;
+            const uint32_t f = (v >> (8 * j)) & 255u;
+            v &= ~(255u << (8 * j));
+            t.st(TY::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
+            ++nleaf;
+        }
+    }
+    ClCounts cl;
+    build_tree<MAXB>(t, nleaf, false);
+    int dyn = extra;
+    int blx = 0;   // extra bits of the code-length symbols
+    {
+        // data bits, and the run-length coding of lengths 0 .. max symbol
+        int prev = -1, rv = -1, rl = 0;
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = t.ld(TY::kNode + i);
+            const int sy = (w >> 9) & 511u, v = w >> 27;
+            dyn += static_cast<int>((w >> 18) & 511u) * v;
+            const int gap = sy - prev - 1;
+            if (gap > 0 || v != rv) {
+                blx += add_run(cl, rv, rl);
+                blx += add_run(cl, 0, gap);
+                rv = v;
+                rl = 1;
+            } else {
+                ++rl;
+            }
+            prev = sy;
+        }
+        blx += add_run(cl, rv, rl);
+    }
+
+    // ---- distance tree (dummies for fewer than two codes)
+    {
+        nleaf = 0;
+        int max_code = -1;
+        for (int wd = 0; wd < 8; ++wd) {
+            uint32_t v = m.ld(cnt_word<MAXB>(4 * wd, true));
+            while (v) {
+                const int j = (__ffs(v) - 1) >> 3;
+                const uint32_t f = (v >> (8 * j)) & 255u;
+                v &= ~(255u << (8 * j));
+                t.st(TY::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
+                max_code = 4 * wd + j;
+                ++nleaf;
+            }
+        }
+        const int nreal = nleaf;
+        while (nleaf < 2) {
+            const int sd = max_code < 2 ? ++max_code : 0;
+            t.st(TY::kNode + nleaf, (static_cast<uint32_t>(sd) << 9) | (1u << 18));
+            ++nleaf;
+        }
+        build_tree<MAXB>(t, nleaf, false);
+        // lengths by code, 4 bits each (codes 0 .. 29), dummies included; data bits of real codes
+        uint64_t dlo = 0, dhi = 0;
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = t.ld(TY::kNode + i);
+            const int sd = (w >> 9) & 511u;
+            const uint64_t v = w >> 27;
+            if (sd < 16) dlo |= v << (4 * sd);
+            else dhi |= v << (4 * (sd - 16));
+            if (i < nreal) dyn += static_cast<int>((w >> 18) & 511u) * static_cast<int>(v);
+        }
+        int rv = -1, rl = 0;
+        for (int sd = 0; sd <= max_code; ++sd) {
+            const int v = static_cast<int>(((sd < 16 ? dlo >> (4 * sd) : dhi >> (4 * (sd - 16)))) & 15u);
+            if (v == rv) {
+                ++rl;
+            } else {
+                blx += add_run(cl, rv, rl);
+                rv = v;
+                rl = 1;
+            }
+        }
+        blx += add_run(cl, rv, rl);
+    }
+
+    // ---- code-length tree (limit 7 bits, with zlib's repair)
+    uint64_t bllen = 0;   // 3 bits per code-length symbol
+    int blbits = blx;
+    {
+        nleaf = 0;
+        int max_code = -1;
+        for (int sy = 0; sy < 19; ++sy) {
+            const int f = cl.get(sy);
+            if (f) {
+                t.st(TY::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (static_cast<uint32_t>(f) << 18));
+                max_code = sy;
+                ++nleaf;
+            }
+        }
+        const int nreal = nleaf;
+        while (nleaf < 2) {
+            const int sy = max_code < 2 ? ++max_code : 0;
+            t.st(TY::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (1u << 18));
+            ++nleaf;
+        }
+        const int nodes = build_tree<MAXB>(t, nleaf, true);
+        // overflow: nodes whose length passed 7 (each clamped in turn from its clamped parent)
+        int overflow = 0;
+        uint64_t count = 0;   // leaves per length 0..7, 8 bits each
+        for (int id = nodes - 1; id >= 0; --id) {
+            const uint32_t w = t.ld(TY::kNode + id);
+            int d = static_cast<int>(w >> 27);
+            if (id < nodes - 1) {
+                const int pdp = static_cast<int>(t.ld(TY::kNode + (w & 511u)) >> 27);
+                d = pdp + 1;
+                if (d > 7) {
+                    d = 7;
+                    ++overflow;
+                }
+                t.st(TY::kNode + id, (w & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
+            }
+            if (id < nleaf) count += uint64_t(1) << (8 * d);
+        }
+        if (overflow > 0) {
+            do {
+                int d = 6;
+                while (((count >> (8 * d)) & 255u) == 0) --d;
+                count -= uint64_t(1) << (8 * d);
+                count += uint64_t(2) << (8 * (d + 1));
+                count -= uint64_t(1) << 56;
+                overflow -= 2;
+            } while (overflow > 0);
+            int r = 0;
+            for (int d = 7; d != 0; --d) {
+                int c = static_cast<int>((count >> (8 * d)) & 255u);
+                while (c != 0) {
+                    const int nd = static_cast<int>(t.ld(TY::kOrder + r));
+                    ++r;
+                    if (nd >= nleaf) continue;
+                    t.st(TY::kNode + nd, (t.ld(TY::kNode + nd) & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
+                    --c;
+                }
+            }
+        }
+        for (int i = 0; i < nleaf; ++i) {
+            const uint32_t w = t.ld(TY::kNode + i);
+            const int sy = (w >> 9) & 511u;
+            bllen |= static_cast<uint64_t>(w >> 27) << (3 * sy);
+            if (i < nreal) blbits += static_cast<int>((w >> 18) & 511u) * static_cast<int>(w >> 27);
+        }
+    }
+    // code-length code lengths sent: RFC order, trailing zeros trimmed, at least 4
+    constexpr uint64_t kOrderNibbles = 0xF1E2D3C4B5A69780ull;   // order positions 3..18: 0 8 7 9 6 10 5 11 4 12 3 13 2 14 1 15
+    int hclen = 4;
+    for (int i = 18; i >= 4; --i) {
+        const int sy = static_cast<int>((kOrderNibbles >> (4 * (i - 3))) & 15u);
+        if ((bllen >> (3 * sy)) & 7u) {
+            hclen = i + 1;
+            break;
+        }
+    }
+    dyn += blbits + 5 + 5 + 4 + 3 * hclen;
+
+    int opt = (dyn + 3 + 7) >> 3;
+    if (stat <= opt) opt = stat;
+    const int raw = (n + 4 <= opt) ? n + 5 : opt;
+    return raw + 18;
+}
+
 // gzip length (18 + raw DEFLATE bytes) of the lane's block of n bytes, whose
 // bytes are already in its words (zero padded).  lanes: the warp's lanes
 // that hold a block (all of them call this together).
@@ -349,11 +570,13 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
     using Y = Layout<MAXB>;
     constexpr int NW = MAXB / 32;   // words of the per-position bitmasks
     // ---- prepass, the same steps on every lane: each position with >= 3
-    // bytes left gets its hash and its previous bucket-mate (64 buckets on the
+    // bytes left gets its hash and its previous bucket-mate (Layout::kBuckets buckets on the
     // hash's low bits; 0 ends a list, as position 0 is never a match source)
-    for (int i = 0; i < kBuckets / 4; ++i) m.st(Y::kHeads + i, 0u);
-    for (int i = 0; i < 72; ++i) m.st(Y::kCnt + i, 0u);
-    for (int i = 0; i < 8; ++i) m.st(Y::kDcnt + i, 0u);
+    for (int i = 0; i < Y::kBuckets / 4; ++i) m.st(Y::kHeads + i, 0u);
+    for (int i = 0; i < 8; ++i) {
+        m.st(Y::kMcnt + i, 0u);
+        m.st(Y::kDcnt + i, 0u);
+    }
     {
         uint32_t h = 0;
         for (int q = 0; q + 2 < n; ++q) {
@@ -365,7 +588,7 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
                 h = (h << 5) ^ x2;
             }
             h &= 0x7fffu;
-            const uint32_t bk = h & (kBuckets - 1);
+            const uint32_t bk = h & (Y::kBuckets - 1);
             const int hw = Y::kHeads + (bk >> 2);
             const uint32_t sh = (bk & 3u) * 8u;
             const uint32_t heads = m.ld(hw);
@@ -444,8 +667,9 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
             length_code(mlen, lc, le);
             dist_code(p - mpos, dc, de);
             const int sym = 257 + lc;
-            m.st(Y::kCnt + (sym >> 2), m.ld(Y::kCnt + (sym >> 2)) + (1u << ((sym & 3) * 8)));
-            m.st(Y::kDcnt + (dc >> 2), m.ld(Y::kDcnt + (dc >> 2)) + (1u << ((dc & 3) * 8)));
+            const int ws = cnt_word<MAXB>(sym), wd = cnt_word<MAXB>(dc, true);
+            m.st(ws, m.ld(ws) + (1u << ((sym & 3) * 8)));
+            m.st(wd, m.ld(wd) + (1u << ((dc & 3) * 8)));
             extra += le + de;
             fix += fixed_len(sym) + 5 + le + de;
             if (mlen <= 4 && rem - mlen >= 3)
@@ -456,16 +680,17 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
             p += 1;
         }
     }
-    // literal counts, the same steps on every lane
+    // literal counts, the same steps on every lane, over the position words
+    for (int i = 0; i < 64; ++i) m.st(Y::kLcnt + i, 0u);
     for (int q = 0; q < n; ++q) {
         if (bit(lit, q)) {
             const uint32_t xq = (m.ld(Y::kXb + (q >> 2)) >> ((q & 3) * 8)) & 255u;
-            m.st(Y::kCnt + (xq >> 2), m.ld(Y::kCnt + (xq >> 2)) + (1u << ((xq & 3) * 8)));
+            m.st(Y::kLcnt + (xq >> 2), m.ld(Y::kLcnt + (xq >> 2)) + (1u << ((xq & 3) * 8)));
             fix += xq < 144 ? 8 : 9;
         }
     }
     // end of block
-    m.st(Y::kCnt + 64, m.ld(Y::kCnt + 64) + 1u);
+    m.st(Y::kMcnt, m.ld(Y::kMcnt) + 1u);
     const int stat = (fix + 3 + 7) >> 3;
 
     // ---- a lower bound on the dynamic block's bits, from the counts alone:
@@ -489,12 +714,15 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
         for (int k = 0; k < 9; ++k) um[k] = 0u;
 #pragma unroll
         for (int wd = 0; wd < 72; ++wd) {
-            const uint32_t v = m.ld(Y::kCnt + wd);
+            const uint32_t v = m.ld(cnt_word<MAXB>(4 * wd));
+            if (v) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int f = static_cast<int>((v >> (8 * j)) & 255u);
-                T += f;
-                slog += static_cast<float>(f) * lg2_approx(static_cast<float>(f > 1 ? f : 1));
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t f = (v >> (8 * j)) & 255u;
+                    T += static_cast<int>(f);
+                    const float ff = small_int_float(f);
+                    slog += ff * lg2_approx(f > 1u ? ff : 1.f);
+                }
             }
             // bytes that are nonzero -> 4 bits (positions 21..24 of the product)
             uint32_t t = v | (v >> 4);
@@ -515,12 +743,13 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
         uint32_t ud[1] = {0u};
 #pragma unroll
         for (int wd = 0; wd < 8; ++wd) {
-            const uint32_t v = m.ld(Y::kDcnt + wd);
+            const uint32_t v = m.ld(cnt_word<MAXB>(4 * wd, true));
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int f = static_cast<int>((v >> (8 * j)) & 255u);
-                Td += f;
-                slogd += static_cast<float>(f) * lg2_approx(static_cast<float>(f > 1 ? f : 1));
+                const uint32_t f = (v >> (8 * j)) & 255u;
+                Td += static_cast<int>(f);
+                const float ff = small_int_float(f);
+                slogd += ff * lg2_approx(f > 1u ? ff : 1.f);
                 if (f) ud[0] |= 1u << (4 * wd + j);
             }
         }
@@ -547,172 +776,12 @@ __device__ int lane_block_length(const LaneMem& m, int n, unsigned lanes) {
     if (__all_sync(lanes, result >= 0)) return result + 18;
     if (result >= 0) return result + 18;   // this lane waits while the others build their trees
 
-    // ---- literal/length tree: leaves in symbol order (never fewer than two:
-    // end of block and at least one literal)
-    int nleaf = 0;
-    for (int wd = 0; wd < 72; ++wd) {
-        uint32_t v = m.ld(Y::kCnt + wd);
-        while (v) {
-            const int j = (__ffs(v) - 1) >> 3;
-            const uint32_t f = (v >> (8 * j)) & 255u;
-            v &= ~(255u << (8 * j));
-            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
-            ++nleaf;
-        }
+    if constexpr (Layout<MAXB>::kSharedTrees) {
+        return exact_length<MAXB>(m, m, n, extra, stat);
+    } else {
+        uint32_t tree_words[TreeLayout<MAXB>::kWords];
+        return exact_length<MAXB>(m, LocalMem{tree_words}, n, extra, stat);
     }
-    ClCounts cl;
-    build_tree<MAXB>(m, nleaf, false);
-    int dyn = extra;
-    int blx = 0;   // extra bits of the code-length symbols
-    {
-        // data bits, and the run-length coding of lengths 0 .. max symbol
-        int prev = -1, rv = -1, rl = 0;
-        for (int i = 0; i < nleaf; ++i) {
-            const uint32_t w = m.ld(Y::kNode + i);
-            const int sy = (w >> 9) & 511u, v = w >> 27;
-            dyn += static_cast<int>((w >> 18) & 511u) * v;
-            const int gap = sy - prev - 1;
-            if (gap > 0 || v != rv) {
-                blx += add_run(cl, rv, rl);
-                blx += add_run(cl, 0, gap);
-                rv = v;
-                rl = 1;
-            } else {
-                ++rl;
-            }
-            prev = sy;
-        }
-        blx += add_run(cl, rv, rl);
-    }
-
-    // ---- distance tree (dummies for fewer than two codes)
-    {
-        nleaf = 0;
-        int max_code = -1;
-        for (int wd = 0; wd < 8; ++wd) {
-            uint32_t v = m.ld(Y::kDcnt + wd);
-            while (v) {
-                const int j = (__ffs(v) - 1) >> 3;
-                const uint32_t f = (v >> (8 * j)) & 255u;
-                v &= ~(255u << (8 * j));
-                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(4 * wd + j) << 9) | (f << 18));
-                max_code = 4 * wd + j;
-                ++nleaf;
-            }
-        }
-        const int nreal = nleaf;
-        while (nleaf < 2) {
-            const int sd = max_code < 2 ? ++max_code : 0;
-            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sd) << 9) | (1u << 18));
-            ++nleaf;
-        }
-        build_tree<MAXB>(m, nleaf, false);
-        // lengths by code, 4 bits each (codes 0 .. 29), dummies included; data bits of real codes
-        uint64_t dlo = 0, dhi = 0;
-        for (int i = 0; i < nleaf; ++i) {
-            const uint32_t w = m.ld(Y::kNode + i);
-            const int sd = (w >> 9) & 511u;
-            const uint64_t v = w >> 27;
-            if (sd < 16) dlo |= v << (4 * sd);
-            else dhi |= v << (4 * (sd - 16));
-            if (i < nreal) dyn += static_cast<int>((w >> 18) & 511u) * static_cast<int>(v);
-        }
-        int rv = -1, rl = 0;
-        for (int sd = 0; sd <= max_code; ++sd) {
-            const int v = static_cast<int>(((sd < 16 ? dlo >> (4 * sd) : dhi >> (4 * (sd - 16)))) & 15u);
-            if (v == rv) {
-                ++rl;
-            } else {
-                blx += add_run(cl, rv, rl);
-                rv = v;
-                rl = 1;
-            }
-        }
-        blx += add_run(cl, rv, rl);
-    }
-
-    // ---- code-length tree (limit 7 bits, with zlib's repair)
-    uint64_t bllen = 0;   // 3 bits per code-length symbol
-    int blbits = blx;
-    {
-        nleaf = 0;
-        int max_code = -1;
-        for (int sy = 0; sy < 19; ++sy) {
-            const int f = cl.get(sy);
-            if (f) {
-                m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (static_cast<uint32_t>(f) << 18));
-                max_code = sy;
-                ++nleaf;
-            }
-        }
-        const int nreal = nleaf;
-        while (nleaf < 2) {
-            const int sy = max_code < 2 ? ++max_code : 0;
-            m.st(Y::kNode + nleaf, (static_cast<uint32_t>(sy) << 9) | (1u << 18));
-            ++nleaf;
-        }
-        const int nodes = build_tree<MAXB>(m, nleaf, true);
-        // overflow: nodes whose length passed 7 (each clamped in turn from its clamped parent)
-        int overflow = 0;
-        uint64_t count = 0;   // leaves per length 0..7, 8 bits each
-        for (int id = nodes - 1; id >= 0; --id) {
-            const uint32_t w = m.ld(Y::kNode + id);
-            int d = static_cast<int>(w >> 27);
-            if (id < nodes - 1) {
-                const int pdp = static_cast<int>(m.ld(Y::kNode + (w & 511u)) >> 27);
-                d = pdp + 1;
-                if (d > 7) {
-                    d = 7;
-                    ++overflow;
-                }
-                m.st(Y::kNode + id, (w & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
-            }
-            if (id < nleaf) count += uint64_t(1) << (8 * d);
-        }
-        if (overflow > 0) {
-            do {
-                int d = 6;
-                while (((count >> (8 * d)) & 255u) == 0) --d;
-                count -= uint64_t(1) << (8 * d);
-                count += uint64_t(2) << (8 * (d + 1));
-                count -= uint64_t(1) << 56;
-                overflow -= 2;
-            } while (overflow > 0);
-            int r = 0;
-            for (int d = 7; d != 0; --d) {
-                int c = static_cast<int>((count >> (8 * d)) & 255u);
-                while (c != 0) {
-                    const int nd = static_cast<int>(m.ld(Y::kOrder + r));
-                    ++r;
-                    if (nd >= nleaf) continue;
-                    m.st(Y::kNode + nd, (m.ld(Y::kNode + nd) & 0x07ffffffu) | (static_cast<uint32_t>(d) << 27));
-                    --c;
-                }
-            }
-        }
-        for (int i = 0; i < nleaf; ++i) {
-            const uint32_t w = m.ld(Y::kNode + i);
-            const int sy = (w >> 9) & 511u;
-            bllen |= static_cast<uint64_t>(w >> 27) << (3 * sy);
-            if (i < nreal) blbits += static_cast<int>((w >> 18) & 511u) * static_cast<int>(w >> 27);
-        }
-    }
-    // code-length code lengths sent: RFC order, trailing zeros trimmed, at least 4
-    constexpr uint64_t kOrderNibbles = 0xF1E2D3C4B5A69780ull;   // order positions 3..18: 0 8 7 9 6 10 5 11 4 12 3 13 2 14 1 15
-    int hclen = 4;
-    for (int i = 18; i >= 4; --i) {
-        const int sy = static_cast<int>((kOrderNibbles >> (4 * (i - 3))) & 15u);
-        if ((bllen >> (3 * sy)) & 7u) {
-            hclen = i + 1;
-            break;
-        }
-    }
-    dyn += blbits + 5 + 5 + 4 + 3 * hclen;
-
-    int opt = (dyn + 3 + 7) >> 3;
-    if (stat <= opt) opt = stat;
-    const int raw = (n + 4 <= opt) ? n + 5 : opt;
-    return raw + 18;
 }
 
 // Per-lane words a warp needs, and warps per CTA, for blocks of at most MAXB bytes.
@@ -721,6 +790,8 @@ struct KernelShape {
     static constexpr int kWarpBytes = Layout<MAXB>::kWords * 32 * 4;
     static constexpr int kWarps = 1;
     static constexpr int kSmemBytes = kWarpBytes * kWarps;
+    // CTAs (warps) resident per SM by shared memory (1 KB reserved per CTA)
+    static constexpr int kResident = 227 * 1024 / (kSmemBytes + 1024) < 32 ? 227 * 1024 / (kSmemBytes + 1024) : 32;
 };
 
 // Lengths of the nb (<= 32) blocks task0 .. task0 + nb - 1 of the batch, one
@@ -752,15 +823,17 @@ __device__ __forceinline__ void warp_block_lengths(uint32_t* region, const uint8
 // warp_block_lengths), one warp per CTA.
 template <int MAXB>
 __global__ void __launch_bounds__(32 * KernelShape<MAXB>::kWarps)
-block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblocks_total,
+block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblocks_total, int bpw,
                           int32_t* __restrict__ lengths) {
     using Y = Layout<MAXB>;
     extern __shared__ __align__(16) uint32_t lsmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t* region = lsmem + static_cast<size_t>(warp) * Y::kWords * 32;
-    const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * 32;
+    // bpw (8, 16 or 32) blocks per warp: fewer when the batch is small, so
+    // that more warps share the blocks and each warp's lanes diverge less
+    const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * bpw;
     if (task0 >= nblocks_total) return;   // warp-uniform
-    const int nb = nblocks_total - task0 < 32 ? static_cast<int>(nblocks_total - task0) : 32;
+    const int nb = nblocks_total - task0 < bpw ? static_cast<int>(nblocks_total - task0) : bpw;
     warp_block_lengths<MAXB>(region, bytes, b, task0, nb, lengths, lane);
 }
 

@@ -89,11 +89,42 @@ struct CsrArgs {
 __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
 __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
 
-// Lists of class c for sample s, by the whole CTA (any multiple of 32
-// threads up to 1024); dsm holds csr_smem_bytes(nblk).  Reads the flags from
-// a.flags (a CTA that wrote them must synchronise first), or, with
-// flags_ready, finds them (0 / 1) already in dsm[0 .. nblk).
-__device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, bool flags_ready = false) {
+// The threads that build one (sample, class)'s lists together: the whole CTA
+// (CtaGroup, any multiple of 32 threads up to 1024) or one warp (WarpGroup).
+struct CtaGroup {
+    __device__ __forceinline__ int rank() const { return threadIdx.x; }
+    __device__ __forceinline__ int size() const { return blockDim.x; }
+    __device__ __forceinline__ int warp() const { return threadIdx.x >> 5; }
+    __device__ __forceinline__ int nwarps() const { return blockDim.x >> 5; }
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+    __device__ __forceinline__ int scan(int v, int* scratch, int* total) const {
+        return block_exclusive_scan(v, scratch, total);
+    }
+};
+struct WarpGroup {
+    __device__ __forceinline__ int rank() const { return threadIdx.x & 31; }
+    __device__ __forceinline__ int size() const { return 32; }
+    __device__ __forceinline__ int warp() const { return 0; }
+    __device__ __forceinline__ int nwarps() const { return 1; }
+    __device__ __forceinline__ void sync() const { __syncwarp(); }
+    __device__ __forceinline__ int scan(int v, int*, int* total) const {
+        const int lane = threadIdx.x & 31;
+        int x = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        *total = __shfl_sync(0xffffffffu, x, 31);
+        return x - v;
+    }
+};
+
+// Lists of class c for sample s, by the group G (every thread of it calls
+// this); dsm holds csr_smem_bytes(nblk).  Reads the flags from a.flags (a
+// group that wrote them must synchronise first), or, with flags_ready,
+// finds them (0 / 1) already in dsm[0 .. nblk).
+template <typename G>
+__device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, bool flags_ready, const G& grp) {
     const int n = a.nblk;
     uint8_t* fl = dsm;                                              // [n]
     int* pre = reinterpret_cast<int*>(dsm + ((n + 15) & ~15));      // [n] inclusive literal count
@@ -105,21 +136,21 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
     const int64_t g = static_cast<int64_t>(s) * 3 + c;
     const int w = a.w;
     if (!flags_ready)
-        for (int i = threadIdx.x; i < n; i += blockDim.x) fl[i] = a.flags[static_cast<int64_t>(s) * n + i] ? 1 : 0;
-    __syncthreads();
+        for (int i = grp.rank(); i < n; i += grp.size()) fl[i] = a.flags[static_cast<int64_t>(s) * n + i] ? 1 : 0;
+    grp.sync();
 
     // literal prefix counts: each thread scans a contiguous chunk
-    const int chunk = (n + blockDim.x - 1) / blockDim.x;
-    const int lo = imin(n, threadIdx.x * chunk), hi = imin(n, lo + chunk);
+    const int chunk = (n + grp.size() - 1) / grp.size();
+    const int lo = imin(n, grp.rank() * chunk), hi = imin(n, lo + chunk);
     int cnt = 0;
     for (int i = lo; i < hi; ++i) cnt += fl[i];
     int nlit;
-    int off = block_exclusive_scan(cnt, scratch, &nlit);
+    int off = grp.scan(cnt, scratch, &nlit);
     for (int i = lo; i < hi; ++i) {
         if (fl[i]) lit[off++] = i;
         pre[i] = off;
     }
-    __syncthreads();
+    grp.sync();
 
     // row and column counts
     auto lit_upto = [&](int i) { return i < 0 ? 0 : pre[i]; };   // literal j <= i
@@ -138,20 +169,20 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
     int rc = 0, cc = 0;
     for (int i = lo; i < hi; ++i) { rc += row_count(i); cc += col_count(i); }
     int rtot, ctot;
-    int roff = block_exclusive_scan(rc, scratch, &rtot);
-    int coff = block_exclusive_scan(cc, scratch, &ctot);
+    int roff = grp.scan(rc, scratch, &rtot);
+    int coff = grp.scan(cc, scratch, &ctot);
     for (int i = lo; i < hi; ++i) {
         rptr[i] = roff;
         roff += row_count(i);
         cptr[i] = coff;
         coff += col_count(i);
     }
-    if (threadIdx.x == 0) {
+    if (grp.rank() == 0) {
         rptr[n] = rtot;
         cptr[n] = ctot;
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+    grp.sync();
+    for (int i = grp.rank(); i <= n; i += grp.size()) {
         a.row_ptr[g * (n + 1) + i] = rptr[i];
         a.col_ptr[g * (n + 1) + i] = cptr[i];
     }
@@ -159,7 +190,7 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
     // tile orders: local classes keep block order; literal and hybrid
     // classes put literal blocks together (descending for query tiles,
     // heaviest first; ascending for key tiles, heaviest first)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = grp.rank(); i < n; i += grp.size()) {
         int qpos, kpos;
         if (c == 0) {
             qpos = i;
@@ -177,7 +208,7 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
     }
 
     // entries: one warp per row / column
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int lane = grp.rank() & 31, warp = grp.warp(), nwarps = grp.nwarps();
     int32_t* cidx = a.col_idx + g * a.cap;
     int32_t* ridx = a.row_idx + g * a.cap;
     for (int i = warp; i < n; i += nwarps) {
@@ -202,6 +233,11 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
             ridx[cptr[i] + e] = q;
         }
     }
+}
+
+__device__ __forceinline__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm,
+                                                 bool flags_ready = false) {
+    build_csr_sample(a, c, s, dsm, flags_ready, CtaGroup{});
 }
 
 __global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {

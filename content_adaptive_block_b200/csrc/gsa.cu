@@ -142,12 +142,16 @@ gsa_status launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtens
 template <int MAXB>
 gsa_status launch_lengths_lane(const uint8_t* bytes, int b, int64_t total, int32_t* lengths, cudaStream_t cs) {
     using K = gsa::deflate_lane::KernelShape<MAXB>;
-    const int64_t per_cta = 32 * K::kWarps;
+    // blocks per warp: the fewest of 8, 16, 32 that still run every block in
+    // one wave of resident warps (fewer blocks per warp diverge less), else 32
+    const int64_t fill = static_cast<int64_t>(gsa::bwd::sm_count()) * K::kResident;
+    const int bpw = total <= 8 * fill ? 8 : (total <= 16 * fill ? 16 : 32);
+    const int64_t per_cta = static_cast<int64_t>(bpw) * K::kWarps;
     const int64_t grid = (total + per_cta - 1) / per_cta;
     if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
     if (!gsa::smem_opt_in(gsa::deflate_lane::block_lengths_lane_kernel<MAXB>, K::kSmemBytes)) return GSA_ERR_CUDA;
     gsa::deflate_lane::block_lengths_lane_kernel<MAXB><<<static_cast<unsigned>(grid), 32 * K::kWarps, K::kSmemBytes,
-                                                         cs>>>(bytes, b, total, lengths);
+                                                         cs>>>(bytes, b, total, bpw, lengths);
     return launch_status();
 }
 
@@ -166,13 +170,21 @@ gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
             cudaSuccess ||
         per_sm < 1)
         return GSA_ERR_CUDA;
-    const int64_t chunks = (P.total + 31) / 32;
+    gsa::pipeline::PipeArgs Q = P;
+    // blocks per warp as in the lengths kernel: the fewest of 8, 16, 32 that fit one wave
+    const int64_t fill = static_cast<int64_t>(per_sm) * sms * S::kWarps;
+    Q.bpw = P.total <= 8 * fill ? 8 : (P.total <= 16 * fill ? 16 : 32);
+    // a list job per warp for short lists (measured faster up to 64 blocks
+    // per sample; longer lists go faster with a CTA's warps on each job)
+    Q.warp_jobs = P.nblk <= 64 && gsa::mask::csr_smem_bytes(P.nblk) <= static_cast<size_t>(S::kWarpBytes) ? 1 : 0;
+    const int64_t chunks = (P.total + Q.bpw - 1) / Q.bpw;
     const int64_t need = (chunks + S::kWarps - 1) / S::kWarps;
-    const int64_t jobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    const int64_t jobs = Q.warp_jobs ? (njobs + S::kWarps - 1) / S::kWarps : njobs;
     int64_t grid = static_cast<int64_t>(per_sm) * sms;
     const int64_t want = need > jobs ? need : jobs;
     if (want < grid) grid = want;
-    void* args[] = {const_cast<gsa::pipeline::PipeArgs*>(&P)};
+    void* args[] = {&Q};
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel),
                                                       dim3(static_cast<unsigned>(grid)),
                                                       dim3(32 * S::kWarps), args, S::kSmemBytes, cs);

@@ -6,9 +6,10 @@
 // each head class.  The flags of a sample need all of its lengths, so the
 // launch is cooperative (every CTA resident at once) with two phases and one
 // grid barrier between them:
-//   1. lengths: every warp takes chunks of 32 consecutive blocks, one block
-//      per lane, exactly as the lengths kernel does (deflate_lane.cuh);
-//   2. lists: jobs (sample, class) spread over all CTAs.  A job sums its
+//   1. lengths: every warp takes chunks of consecutive blocks, one block per
+//      lane, exactly as the lengths kernel does (deflate_lane.cuh);
+//   2. lists: jobs (sample, class) spread over all warps (or, for lists
+//      too long for a warp's words, over all CTAs).  A job sums its
 //      sample's lengths, sets the flags (len_i * nblk > Σ len) in shared
 //      memory — the sample's first job also writes them out — and builds the
 //      class's lists.  The local class's lists depend only on (nblk, w)
@@ -53,6 +54,8 @@ struct PipeArgs {
     int nper;             // classes built per sample (those other than a local class built once)
     int per[3];           // ... and which
     int local_once;       // 1: the local class is in use, built once into sample 0's slot
+    int warp_jobs;        // 1: a list job per warp (its lengths words hold the job's scratch), 0: per CTA
+    int bpw;              // blocks per warp in the lengths phase (8, 16 or 32)
 };
 
 // All CTAs of the grid reach this point (thread 0 of each waits, bounded);
@@ -89,15 +92,15 @@ __global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel
     __shared__ long long part[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- phase 1: lengths, chunks of 32 blocks per warp
+    // ---- phase 1: lengths, chunks of bpw blocks per warp (one per lane)
+    uint32_t* region = reinterpret_cast<uint32_t*>(dsmem) +
+                       static_cast<size_t>(warp) * deflate_lane::Layout<MAXB>::kWords * 32;
     {
-        uint32_t* region = reinterpret_cast<uint32_t*>(dsmem) +
-                           static_cast<size_t>(warp) * deflate_lane::Layout<MAXB>::kWords * 32;
-        const int64_t nchunks = (P.total + 31) / 32;
+        const int64_t nchunks = (P.total + P.bpw - 1) / P.bpw;
         for (int64_t ch = static_cast<int64_t>(blockIdx.x) * kWarps + warp; ch < nchunks;
              ch += static_cast<int64_t>(gridDim.x) * kWarps) {
-            const int64_t task0 = ch * 32;
-            const int nb = P.total - task0 < 32 ? static_cast<int>(P.total - task0) : 32;
+            const int64_t task0 = ch * P.bpw;
+            const int nb = P.total - task0 < P.bpw ? static_cast<int>(P.total - task0) : P.bpw;
             deflate_lane::warp_block_lengths<MAXB>(region, P.bytes, P.b, task0, nb, P.lengths, lane);
         }
     }
@@ -109,6 +112,32 @@ __global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel
     const int n = P.nblk;
     const int jobs_per = P.nper > 0 ? P.nper : 1;
     const int njobs = P.B * jobs_per + P.local_once;
+    if (P.warp_jobs) {
+        // one job per warp at a time, in the warp's own lengths words: all the
+        // jobs run side by side instead of a few per CTA in turn
+        uint8_t* ws = reinterpret_cast<uint8_t*>(region);
+        for (int j = blockIdx.x * kWarps + warp; j < njobs; j += gridDim.x * kWarps) {
+            const bool local = j == P.B * jobs_per;
+            const int s = local ? 0 : j / jobs_per;
+            const int k = local ? 0 : j % jobs_per;
+            const int c = local ? 0 : (P.nper > 0 ? P.per[k] : -1);
+            __syncwarp();
+            const int32_t* row = P.lengths + static_cast<int64_t>(s) * n;
+            long long acc = 0;
+            for (int i = lane; i < n; i += 32) acc += __ldcg(row + i);
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            const bool write = !local && k == 0;
+            for (int i = lane; i < n; i += 32) {
+                const uint8_t f = static_cast<long long>(__ldcg(row + i)) * n > acc ? 1 : 0;
+                ws[i] = f;
+                if (write) P.flags[static_cast<int64_t>(s) * n + i] = f;
+            }
+            if (c >= 0) mask::build_csr_sample(P.a, c, s, ws, true, mask::WarpGroup{});
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && atomicAdd(P.counter, 1) == 2 * static_cast<int>(gridDim.x) - 1) *P.counter = 0;
+        return;
+    }
     uint8_t* fl = dsmem;   // the list builder's flag scratch: dsm[0 .. n)
     for (int j = blockIdx.x; j < njobs; j += gridDim.x) {
         const bool local = j == P.B * jobs_per;
