@@ -25,6 +25,7 @@ __all__ = [
     "gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_build_fixed_csr", "gsa_mask_pipeline",
     "gsa_csr_capacity", "gsa_attn_fwd", "gsa_attn_bwd", "gsa_attn_bwd_workspace", "gsa_attn_bwd_noalloc",
     "gsa_attn_bwd_noalloc_max_rows", "gsa_lm_block_workspace", "gsa_lm_block_fwd", "gsa_lm_block_bwd",
+    "gsa_lm_gemm", "gsa_lm_gemm_workspace",
     "gsa_device_error", "gsa_status_string", "library", "library_path",
 ]
 
@@ -453,7 +454,52 @@ def _lm_fns():
     lib.gsa_lm_block_bwd.argtypes = [vp, ctypes.POINTER(_LmPtrs), ctypes.POINTER(_Csr), ctypes.POINTER(_LmDesc),
                                      vp, ctypes.POINTER(_LmPtrs), vp, ctypes.c_size_t, vp]
     lib.gsa_lm_block_bwd.restype = ctypes.c_int
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    lib.gsa_lm_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i64, vp, i64, ctypes.c_float, vp, i64, vp, i64, i32,
+                                i32, vp, i64, vp, ctypes.c_size_t, vp]
+    lib.gsa_lm_gemm.restype = ctypes.c_int
+    lib.gsa_lm_gemm_workspace.argtypes = [i32, i32, i32, i32]
+    lib.gsa_lm_gemm_workspace.restype = ctypes.c_size_t
     return lib
+
+
+GEMM_EPI_NONE, GEMM_EPI_GELU_AUX, GEMM_EPI_DGELU = 0, 1, 2
+
+
+def gsa_lm_gemm_workspace(M: int, N: int, K: int, out32: bool) -> int:
+    """Scratch bytes gsa_lm_gemm needs for an M x N product over K (0 unless a float32 product splits K)."""
+    return int(_lm_fns().gsa_lm_gemm_workspace(int(M), int(N), int(K), int(out32)))
+
+
+def gsa_lm_gemm(a: torch.Tensor, b: torch.Tensor, ta: bool = False, tb: bool = False, c: torch.Tensor | None = None,
+                beta: float = 0.0, out32: bool = False, epi: int = GEMM_EPI_NONE, aux: torch.Tensor | None = None,
+                d: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-major D = op(A) op(B) (+ beta C, or a GELU epilogue) on the
+    library's tcgen05 GEMM.  ta: a is [K, M] (else [M, K]); tb: b is [N, K]
+    (else [K, N]).  bf16 operands; D bf16, or float32 with out32.  epi
+    GEMM_EPI_GELU_AUX writes GELU(acc) to D and acc to aux; GEMM_EPI_DGELU
+    returns acc * GELU'(aux)."""
+    lib = _lm_fns()
+    _need(a, "a", torch.bfloat16, 2)
+    _need(b, "b", torch.bfloat16, 2)
+    M = a.shape[1] if ta else a.shape[0]
+    K = a.shape[0] if ta else a.shape[1]
+    N = b.shape[0] if tb else b.shape[1]
+    if (b.shape[1] if tb else b.shape[0]) != K:
+        raise ValueError("inner dimensions differ")
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.float32 if out32 else torch.bfloat16, device=a.device)
+    ws_bytes = gsa_lm_gemm_workspace(M, N, K, out32)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=a.device)
+    if epi == GEMM_EPI_GELU_AUX and aux is None:
+        aux = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    _check("gsa_lm_gemm", lib.gsa_lm_gemm(int(ta), int(tb), M, N, K, _ptr(a), a.stride(0), _ptr(b), b.stride(0),
+                                          float(beta), _ptr(c) if c is not None else None,
+                                          c.stride(0) if c is not None else 0, _ptr(d), d.stride(0), int(out32),
+                                          int(epi), _ptr(aux) if aux is not None else None,
+                                          aux.stride(0) if aux is not None else 0, _ptr(ws), ws_bytes,
+                                          _stream(stream)))
+    return d
 
 
 def _lm_desc(B, L, D, H, F, head_classes, b, eps):

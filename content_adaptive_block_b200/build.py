@@ -5,8 +5,8 @@
 Two translation units (csrc/gsa.cu: the mask stage and the attention;
 csrc/lm_block.cu: the ByteLM block around it) compiled by nvcc with
 -gencode arch=compute_100a,code=sm_100a; the CUDA runtime is linked
-statically, cuBLASLt (the block's projections) dynamically from the CUDA
-toolkit, and the driver's tensor-map encoder is looked up at run time.
+statically (no other library is linked: every GEMM is this library's own)
+and the driver's tensor-map encoder is looked up at run time.
 The ptxas resource report is written next to the library.
 """
 from __future__ import annotations
@@ -60,8 +60,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(OUT_DIR, exist_ok=True)
     tmp = LIB + f".tmp{os.getpid()}"
     cuda_lib = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(_nvcc()))), "lib64")
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SRCS, "-L", cuda_lib, "-lcublasLt",
-           "-Xlinker", "-rpath=" + cuda_lib]
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SRCS]
     res = subprocess.run(cmd, capture_output=True, text=True)
     with open(REPORT, "w") as f:
         f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)

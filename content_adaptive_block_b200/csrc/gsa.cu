@@ -22,6 +22,7 @@ static_assert(GSA_MAX_RANDOM_BLOCKS == gsa::fixed::kMaxRandom, "header and kerne
 #include "attn_fwd_f32.cuh"
 #include "attn_fwd_bf16.cuh"
 #include "attn_bwd_bf16.cuh"
+#include "gemm.cuh"
 
 namespace {
 

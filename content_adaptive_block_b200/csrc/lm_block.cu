@@ -15,18 +15,17 @@
 // straight out of the QKV projection's [token][3][head][64] rows and writing
 // O, dQ, dK, dV in the projections' layouts (gsa_attn_layout), so no head
 // transposes run.  The
-// projections are plain bf16 GEMMs with float32 accumulation and go to
-// cuBLASLt, the residual additions folded into them (D = A B + C) and the
-// GELU and its derivative into their epilogues.
-#include <cublasLt.h>
+// projections are bf16 GEMMs with float32 accumulation on this library's
+// tcgen05 GEMM (gemm.cuh), the residual additions folded into them
+// (D = A B + C) and the GELU and its derivative into their epilogues.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
-#include <map>
 #include <mutex>
-#include <tuple>
+#include <utility>
 
+#include "gemm_api.h"
 #include "gsa.h"
 #include "gsa_lm.h"
 #include "host_attr.h"
@@ -261,118 +260,47 @@ __global__ void embed_reduce_kernel(const float* __restrict__ part, int nchunks,
     dE[i] = s;
 }
 
-// ------------------------------------------------------------- cuBLASLt
-// Row-major D[M][N] = op(A)[M][K] op(B)[K][N] + beta C, A / B bf16, float32
-// accumulation; C and D bf16 (residual folded in) or float32 (weight
-// gradients, beta 0).  ta: A is stored [K][M]; tb: B is stored [N][K].  In
-// cuBLASLt's column-major terms this is D^T = op(B)^T op(A)^T.  Epilogues
-// (on the float32 accumulator, cuBLASLt's tanh-form GELU):
+// ------------------------------------------------------------- projections
+// Row-major D[M][N] = op(A)[M][K] op(B)[K][N] + beta C on this library's
+// tcgen05 GEMM (gemm.cuh): bf16 operands, float32 accumulation; C and D bf16
+// (residual folded in) or float32 (weight gradients, beta 0).  ta: A is
+// stored [K][M]; tb: B is stored [N][K].  Epilogues on the float32
+// accumulator (tanh-form GELU):
 //   kEpiGeluAux: D = GELU(A B), aux = A B (bf16, row-major, ld aux_ld);
 //   kEpiDGelu:   D = (A B) * GELU'(aux).
+// ws / ws_bytes: float32 scratch for the K-split weight gradients.
 enum Epi { kEpiNone = 0, kEpiGeluAux = 1, kEpiDGelu = 2 };
 
-struct LtKey {
-    int dev, ta, tb, M, N, K, lda, ldb, ldc, ldd, out32, epi;
-    bool operator<(const LtKey& o) const {
-        return std::tie(dev, ta, tb, M, N, K, lda, ldb, ldc, ldd, out32, epi) <
-               std::tie(o.dev, o.ta, o.tb, o.M, o.N, o.K, o.lda, o.ldb, o.ldc, o.ldd, o.out32, o.epi);
-    }
+struct GemmWs {
+    float* p;
+    size_t bytes;
 };
-
-struct LtPlan {
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr, ld = nullptr;
-    cublasLtMatmulAlgo_t algo;
-};
-
-struct LtState {
-    std::mutex mu;
-    cublasLtHandle_t handle[64] = {};
-    std::map<LtKey, LtPlan> plans;
-};
-
-LtState& lt_state() {
-    static LtState s;
-    return s;
-}
-
-constexpr size_t kLtWorkspace = 32u << 20;
 
 gsa_status gemm_rm(bool ta, bool tb, int M, int N, int K, const bf16* A, int lda, const bf16* B, int ldb,
-                   float beta, const void* C, int ldc, void* Dp, int ldd, bool out32, void* ws, cudaStream_t st,
+                   float beta, const void* C, int ldc, void* Dp, int ldd, bool out32, GemmWs ws, cudaStream_t st,
                    Epi epi = kEpiNone, void* aux = nullptr, int64_t aux_ld = 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GSA_ERR_CUDA;
-    LtState& S = lt_state();
-    const LtKey key{dev, ta, tb, M, N, K, lda, ldb, ldc, ldd, out32, static_cast<int>(epi)};
-    LtPlan plan;
-    cublasLtHandle_t h;
-    // held until the matmul is enqueued: the cached descriptor carries this call's aux pointer
-    std::lock_guard<std::mutex> lock(S.mu);
-    {
-        if (!S.handle[dev] && cublasLtCreate(&S.handle[dev]) != CUBLAS_STATUS_SUCCESS) return GSA_ERR_CUDA;
-        h = S.handle[dev];
-        auto it = S.plans.find(key);
-        if (it != S.plans.end()) {
-            plan = it->second;
-        } else {
-            const cudaDataType_t dt = out32 ? CUDA_R_32F : CUDA_R_16BF;
-            if (cublasLtMatmulDescCreate(&plan.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS)
-                return GSA_ERR_CUDA;
-            // column-major: first operand = B (N x K after its op), second = A (K x M)
-            const cublasOperation_t opa = tb ? CUBLAS_OP_T : CUBLAS_OP_N;
-            const cublasOperation_t opb = ta ? CUBLAS_OP_T : CUBLAS_OP_N;
-            cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_TRANSA, &opa, sizeof(opa));
-            cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_TRANSB, &opb, sizeof(opb));
-            if (epi != kEpiNone) {
-                const cublasLtEpilogue_t e = epi == kEpiGeluAux ? CUBLASLT_EPILOGUE_GELU_AUX : CUBLASLT_EPILOGUE_DGELU;
-                cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_EPILOGUE, &e, sizeof(e));
-                cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_EPILOGUE_AUX_POINTER, &aux, sizeof(aux));
-                cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_EPILOGUE_AUX_LD, &aux_ld, sizeof(aux_ld));
-            }
-            bool ok = cublasLtMatrixLayoutCreate(&plan.la, CUDA_R_16BF, tb ? K : N, tb ? N : K, ldb) ==
-                          CUBLAS_STATUS_SUCCESS &&
-                      cublasLtMatrixLayoutCreate(&plan.lb, CUDA_R_16BF, ta ? M : K, ta ? K : M, lda) ==
-                          CUBLAS_STATUS_SUCCESS &&
-                      cublasLtMatrixLayoutCreate(&plan.lc, dt, N, M, ldc) == CUBLAS_STATUS_SUCCESS &&
-                      cublasLtMatrixLayoutCreate(&plan.ld, dt, N, M, ldd) == CUBLAS_STATUS_SUCCESS;
-            cublasLtMatmulPreference_t pref = nullptr;
-            ok = ok && cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS;
-            size_t wsb = kLtWorkspace;
-            const uint32_t align = 16;   // the calls check 16-byte alignment of every matrix
-            if (ok) {
-                cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &wsb,
-                                                     sizeof(wsb));
-                for (auto a : {CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_A_BYTES, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_B_BYTES,
-                               CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_C_BYTES, CUBLASLT_MATMUL_PREF_MIN_ALIGNMENT_D_BYTES})
-                    cublasLtMatmulPreferenceSetAttribute(pref, a, &align, sizeof(align));
-            }
-            cublasLtMatmulHeuristicResult_t res;
-            int found = 0;
-            ok = ok && cublasLtMatmulAlgoGetHeuristic(h, plan.op, plan.la, plan.lb, plan.lc, plan.ld, pref, 1, &res,
-                                                      &found) == CUBLAS_STATUS_SUCCESS &&
-                 found > 0;
-            if (pref) cublasLtMatmulPreferenceDestroy(pref);
-            if (!ok) return GSA_ERR_UNSUPPORTED;
-            plan.algo = res.algo;
-            S.plans[key] = plan;
-        }
+    const gsa::gemm::Epi e = epi == kEpiGeluAux ? gsa::gemm::kGeluAux : (epi == kEpiDGelu ? gsa::gemm::kDGelu
+                                                                                          : gsa::gemm::kNone);
+    return gsa::gemm::run(ta, tb, M, N, K, A, lda, B, ldb, beta, static_cast<const bf16*>(C), ldc, Dp, ldd, out32, e,
+                          static_cast<bf16*>(aux), aux_ld, ws.p, ws.bytes, st);
+}
+
+// Split scratch of the block's weight-gradient products (K = B L tokens).
+size_t gemm_ws_bytes(const gsa_lm_desc* d) {
+    const int T = d->B * d->L, D = d->D, F = d->F;
+    size_t m = 0;
+    for (const auto& mn : {std::make_pair(D, F), std::make_pair(F, D), std::make_pair(D, D), std::make_pair(3 * D, D)}) {
+        const size_t b = gsa::gemm::split_ws_bytes(mn.first, mn.second, T);
+        if (b > m) m = b;
     }
-    if (epi != kEpiNone &&
-        cublasLtMatmulDescSetAttribute(plan.op, CUBLASLT_MATMUL_DESC_EPILOGUE_AUX_POINTER, &aux, sizeof(aux)) !=
-            CUBLAS_STATUS_SUCCESS)
-        return GSA_ERR_CUDA;
-    const float alpha = 1.f;
-    const cublasStatus_t r = cublasLtMatmul(h, plan.op, &alpha, B, plan.la, A, plan.lb, &beta, C ? C : Dp, plan.lc,
-                                            Dp, plan.ld, &plan.algo, ws, kLtWorkspace, st);
-    return r == CUBLAS_STATUS_SUCCESS ? GSA_OK : GSA_ERR_CUDA;
+    return m;
 }
 
 // ------------------------------------------------------------ workspace
 struct Layout {
     size_t x0, h, st1, qkv, lse, om, x1, h2, st2, pre, act;       // saved by the forward
     size_t dpre, dh2, dx1, dom, dqkv, dh, dx0, part, epart, attn_ws;   // backward scratch
-    size_t lt, total;
+    size_t lt, lt_bytes, total;
     size_t attn_ws_bytes;
 };
 
@@ -410,7 +338,8 @@ Layout layout(const gsa_lm_desc* d, const gsa_attn_desc& ad) {
     l.epart = take((T + kEmbChunk - 1) / kEmbChunk * 256 * d->D * 4);
     l.attn_ws_bytes = gsa_attn_bwd_workspace(&ad);
     l.attn_ws = take(l.attn_ws_bytes);
-    l.lt = take(kLtWorkspace);
+    l.lt_bytes = gemm_ws_bytes(d);
+    l.lt = take(l.lt_bytes);
     l.total = off;
     return l;
 }
@@ -425,7 +354,9 @@ gsa_status check(const gsa_lm_desc* d, gsa_attn_desc* ad) {
     if (!d || d->B < 1 || d->L < 1 || d->H < 1 || d->H > GSA_MAX_HEADS || !d->head_classes || d->b != 64 ||
         d->L % d->b != 0 || d->D != 64 * d->H || d->F < 8 || d->F % 8 != 0 || !(d->ln_eps > 0.f))
         return GSA_ERR_INVALID_ARGUMENT;
-    if (d->D % 256 != 0 || d->D > 2048 || d->L / d->b > GSA_MAX_BLOCKS_BF16) return GSA_ERR_UNSUPPORTED;
+    // the GEMM tiles 256 output columns and 64-wide K slices
+    if (d->D % 256 != 0 || d->D > 2048 || d->F % 256 != 0 || d->L / d->b > GSA_MAX_BLOCKS_BF16)
+        return GSA_ERR_UNSUPPORTED;
     for (int h = 0; h < d->H; ++h)
         if (d->head_classes[h] > 2) return GSA_ERR_INVALID_ARGUMENT;
     ad->B = d->B;
@@ -503,6 +434,23 @@ using namespace gsa::lm;
 
 extern "C" {
 
+gsa_status gsa_lm_gemm(int32_t ta, int32_t tb, int32_t M, int32_t N, int32_t K, const void* A, int64_t lda,
+                       const void* B, int64_t ldb, float beta, const void* C, int64_t ldc, void* D, int64_t ldd,
+                       int32_t out32, int32_t epi, void* aux, int64_t aux_ld, void* workspace, size_t ws_bytes,
+                       void* stream) {
+    const gsa::CallRange nvtx_range("gsa_lm_gemm");
+    if (epi < 0 || epi > 2) return GSA_ERR_INVALID_ARGUMENT;
+    return gsa::gemm::run(ta != 0, tb != 0, M, N, K, static_cast<const bf16*>(A), lda, static_cast<const bf16*>(B),
+                          ldb, beta, static_cast<const bf16*>(C), ldc, D, ldd, out32 != 0,
+                          static_cast<gsa::gemm::Epi>(epi), static_cast<bf16*>(aux), aux_ld,
+                          static_cast<float*>(workspace), ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gsa_lm_gemm_workspace(int32_t M, int32_t N, int32_t K, int32_t out32) {
+    if (M < 1 || N < 1 || K < 1 || !out32) return 0;
+    return gsa::gemm::split_ws_bytes(M, N, K);
+}
+
 size_t gsa_lm_block_workspace(const gsa_lm_desc* desc) {
     gsa_attn_desc ad;
     if (check(desc, &ad) != GSA_OK) return 0;
@@ -535,7 +483,7 @@ gsa_status gsa_lm_block_fwd(const uint8_t* bytes, const gsa_lm_weights* w, const
     const int D = desc->D, F = desc->F, Mi = static_cast<int>(T);
     if (T > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
     const auto* emb = static_cast<const bf16*>(w->emb);
-    void* lt = ws + l.lt;
+    const GemmWs lt{reinterpret_cast<float*>(ws + l.lt), l.lt_bytes};
 
     // x0 = E[bytes], h = LN1(x0)
     ln_fwd(D, true, bytes, emb, w->ln1_g, w->ln1_b, P(l.x0), P(l.h), reinterpret_cast<float2*>(ws + l.st1), T,
@@ -584,7 +532,7 @@ gsa_status gsa_lm_block_bwd(const uint8_t* bytes, const gsa_lm_weights* w, const
     const int D = desc->D, F = desc->F, Mi = static_cast<int>(T);
     if (T > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
     const auto* dyb = static_cast<const bf16*>(dy);
-    void* lt = ws + l.lt;
+    const GemmWs lt{reinterpret_cast<float*>(ws + l.lt), l.lt_bytes};
     float* part = reinterpret_cast<float*>(ws + l.part);
 
     // MLP: dpre = (dy W_2) GELU'(pre) (one GEMM with its epilogue), dW_2 = dy^T act, dW_1 = dpre^T h2,
