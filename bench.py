@@ -1039,7 +1039,7 @@ def lm_block(gsa, dev, steps=10, warmup=3):
             "shape": f"8 x 8192 bytes, D={D}, H={H} x 64, F={F}, gzip mask b=64 w=2, bf16",
             "ms": ms, "mask_ms": float(t[0]), "fwd_ms": float(t[1]), "bwd_ms": float(t[2]),
             "tflops": (3 * gemm_fwd + attn) / (ms * 1e-3) / 1e12, "gemm_gflop": 3 * gemm_fwd / 1e9,
-            "attn_gflop": attn / 1e9, "projections": "cuBLASLt (bf16, fp32 accumulate)"}
+            "attn_gflop": attn / 1e9, "projections": "this library's tcgen05 GEMM (bf16, fp32 accumulate in TMEM)"}
 
 
 def profile_lengths():
