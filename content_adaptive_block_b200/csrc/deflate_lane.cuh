@@ -794,6 +794,18 @@ struct KernelShape {
     static constexpr int kResident = 227 * 1024 / (kSmemBytes + 1024) < 32 ? 227 * 1024 / (kSmemBytes + 1024) : 32;
 };
 
+// Blocks per warp (one per lane) for a batch of total blocks on fill
+// resident warps: the fewest of 1, 2, 4, ..., 32 that still run every block in
+// one wave.  A warp's time is its slowest lane's block plus the steps where
+// its lanes diverge, so when the batch leaves warps to spare, fewer blocks per
+// warp finish sooner (measured at 1024 blocks of 64 bytes: 66 us at one block
+// per warp against 83 us at eight).
+inline int blocks_per_warp(int64_t total, int64_t fill) {
+    int bpw = 1;
+    while (bpw < 32 && total > bpw * fill) bpw *= 2;
+    return bpw;
+}
+
 // Lengths of the nb (<= 32) blocks task0 .. task0 + nb - 1 of the batch, one
 // per lane, into lengths[task0 ..]: the warp stages its blocks (contiguous
 // bytes) into the lanes' words of region with coalesced loads, then each lane
@@ -829,8 +841,8 @@ block_lengths_lane_kernel(const uint8_t* __restrict__ bytes, int b, int64_t nblo
     extern __shared__ __align__(16) uint32_t lsmem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t* region = lsmem + static_cast<size_t>(warp) * Y::kWords * 32;
-    // bpw (8, 16 or 32) blocks per warp: fewer when the batch is small, so
-    // that more warps share the blocks and each warp's lanes diverge less
+    // bpw (1 .. 32) blocks per warp: fewer when the batch is small, so that
+    // more warps share the blocks and each warp's lanes diverge less
     const int64_t task0 = (static_cast<int64_t>(blockIdx.x) * KernelShape<MAXB>::kWarps + warp) * bpw;
     if (task0 >= nblocks_total) return;   // warp-uniform
     const int nb = nblocks_total - task0 < bpw ? static_cast<int>(nblocks_total - task0) : bpw;

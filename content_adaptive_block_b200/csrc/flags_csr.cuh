@@ -207,7 +207,7 @@ __device__ void build_csr_sample(const CsrArgs& a, int c, int s, uint8_t* dsm, b
         a.k_order[g * n + kpos] = i;
     }
 
-    // entries: one warp per row / column
+    // entries: one warp per row / column, so the stores of a row are contiguous
     const int lane = grp.rank() & 31, warp = grp.warp(), nwarps = grp.nwarps();
     int32_t* cidx = a.col_idx + g * a.cap;
     int32_t* ridx = a.row_idx + g * a.cap;
@@ -242,7 +242,10 @@ __device__ __forceinline__ void build_csr_sample(const CsrArgs& a, int c, int s,
 
 __global__ void __launch_bounds__(kThreads) build_csr_kernel(CsrArgs a) {
     extern __shared__ __align__(16) uint8_t dsm[];
-    build_csr_sample(a, a.cls[blockIdx.x], blockIdx.y, dsm);   // grid (classes built, sample)
+    // grid (classes built, sample); a select, not an indexed read, keeps the
+    // parameters out of local memory
+    const int c = blockIdx.x == 0 ? a.cls[0] : (blockIdx.x == 1 ? a.cls[1] : a.cls[2]);
+    build_csr_sample(a, c, blockIdx.y, dsm);
 }
 
 inline size_t csr_smem_bytes(int n) {

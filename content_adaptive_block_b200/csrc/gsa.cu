@@ -143,10 +143,7 @@ gsa_status launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtens
 template <int MAXB>
 gsa_status launch_lengths_lane(const uint8_t* bytes, int b, int64_t total, int32_t* lengths, cudaStream_t cs) {
     using K = gsa::deflate_lane::KernelShape<MAXB>;
-    // blocks per warp: the fewest of 8, 16, 32 that still run every block in
-    // one wave of resident warps (fewer blocks per warp diverge less), else 32
-    const int64_t fill = static_cast<int64_t>(gsa::bwd::sm_count()) * K::kResident;
-    const int bpw = total <= 8 * fill ? 8 : (total <= 16 * fill ? 16 : 32);
+    const int bpw = gsa::deflate_lane::blocks_per_warp(total, static_cast<int64_t>(gsa::bwd::sm_count()) * K::kResident);
     const int64_t per_cta = static_cast<int64_t>(bpw) * K::kWarps;
     const int64_t grid = (total + per_cta - 1) / per_cta;
     if (grid > 0x7fffffff) return GSA_ERR_UNSUPPORTED;
@@ -156,40 +153,51 @@ gsa_status launch_lengths_lane(const uint8_t* bytes, int b, int64_t total, int32
     return launch_status();
 }
 
-// The one-launch mask stage for blocks of at most MAXB bytes: a cooperative
-// launch (every CTA resident: the phases meet at a grid barrier) of as many
-// CTAs as fit on the device at once, at most one per 32-block chunk group.
-template <int MAXB>
-gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
-    using S = gsa::pipeline::Shape<MAXB>;
-    auto kernel = gsa::pipeline::mask_pipeline_kernel<MAXB>;
+// The one-launch mask stage for blocks of at most MAXB bytes on CTAs of T
+// warps (W of them computing lengths): a cooperative launch (every CTA
+// resident: the phases meet at a grid barrier) of as many CTAs as fit on the
+// device at once, or fewer when the batch has fewer chunks and list jobs.
+template <int MAXB, int W, int T>
+gsa_status launch_pipeline_shape(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
+    using S = gsa::pipeline::Shape<MAXB, W, T>;
+    auto kernel = gsa::pipeline::mask_pipeline_kernel<MAXB, W, T>;
     if (!gsa::smem_opt_in(kernel, static_cast<int>(S::kSmemBytes))) return GSA_ERR_CUDA;
-    int dev = 0, per_sm = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * S::kWarps, S::kSmemBytes) !=
-            cudaSuccess ||
-        per_sm < 1)
+    int per_sm = 0;
+    const int sms = gsa::bwd::sm_count();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 32 * T, S::kSmemBytes) != cudaSuccess ||
+        per_sm < 1 || sms < 1)
         return GSA_ERR_CUDA;
     gsa::pipeline::PipeArgs Q = P;
-    // blocks per warp as in the lengths kernel: the fewest of 8, 16, 32 that fit one wave
-    const int64_t fill = static_cast<int64_t>(per_sm) * sms * S::kWarps;
-    Q.bpw = P.total <= 8 * fill ? 8 : (P.total <= 16 * fill ? 16 : 32);
-    // a list job per warp for short lists (measured faster up to 64 blocks
-    // per sample; longer lists go faster with a CTA's warps on each job)
-    Q.warp_jobs = P.nblk <= 64 && gsa::mask::csr_smem_bytes(P.nblk) <= static_cast<size_t>(S::kWarpBytes) ? 1 : 0;
+    Q.bpw = gsa::deflate_lane::blocks_per_warp(P.total, static_cast<int64_t>(per_sm) * sms * W);
     const int64_t chunks = (P.total + Q.bpw - 1) / Q.bpw;
-    const int64_t need = (chunks + S::kWarps - 1) / S::kWarps;
     const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
-    const int64_t jobs = Q.warp_jobs ? (njobs + S::kWarps - 1) / S::kWarps : njobs;
     int64_t grid = static_cast<int64_t>(per_sm) * sms;
-    const int64_t want = need > jobs ? need : jobs;
+    // a list job per warp for short lists when there are more jobs than CTAs
+    // (measured faster up to 64 blocks per sample; longer lists go faster
+    // with a CTA's warps on each job)
+    Q.warp_jobs = P.nblk <= S::kMaxWarpJobBlocks && njobs > grid ? 1 : 0;
+    const int64_t jobs = Q.warp_jobs ? (njobs + T - 1) / T : njobs;
+    const int64_t want = chunks > jobs ? chunks : jobs;   // a chunk per CTA where possible: spread over the SMs
     if (want < grid) grid = want;
     void* args[] = {&Q};
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel),
-                                                      dim3(static_cast<unsigned>(grid)),
-                                                      dim3(32 * S::kWarps), args, S::kSmemBytes, cs);
+                                                      dim3(static_cast<unsigned>(grid)), dim3(32 * T), args,
+                                                      S::kSmemBytes, cs);
     return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+}
+
+// Many short list jobs (more than one per SM, at most 128 blocks a sample)
+// run on the narrow CTAs, one job per CTA side by side; a few jobs, or long
+// lists, run on the wide ones, each job with 16 warps (measured over 256
+// samples: the narrow shape 7-8 % faster at 64 blocks a sample and within 2 %
+// either way at 128, the wide one 6-9 % faster at 256).
+template <int MAXB>
+gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
+    using SS = gsa::pipeline::Shapes<MAXB>;
+    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    if (njobs > gsa::bwd::sm_count() && P.nblk <= 128)
+        return launch_pipeline_shape<MAXB, SS::kNarrowW, SS::kNarrowT>(P, cs);
+    return launch_pipeline_shape<MAXB, SS::kWideW, SS::kWideT>(P, cs);
 }
 
 gsa_status check_attn(const gsa_attn_desc* d, const gsa_block_csr* csr, uint8_t* cls) {

@@ -6,10 +6,12 @@
 // each head class.  The flags of a sample need all of its lengths, so the
 // launch is cooperative (every CTA resident at once) with two phases and one
 // grid barrier between them:
-//   1. lengths: every warp takes chunks of consecutive blocks, one block per
-//      lane, exactly as the lengths kernel does (deflate_lane.cuh);
-//   2. lists: jobs (sample, class) spread over all warps (or, for lists
-//      too long for a warp's words, over all CTAs).  A job sums its
+//   1. lengths: the CTA's lengths warps take chunks of consecutive blocks,
+//      one block per lane, exactly as the lengths kernel does
+//      (deflate_lane.cuh);
+//   2. lists: jobs (sample, class) spread over the CTAs, all of a CTA's
+//      warps on one job (or, for short lists and many jobs, one job per
+//      warp).  A job sums its
 //      sample's lengths, sets the flags (len_i * nblk > Σ len) in shared
 //      memory — the sample's first job also writes them out — and builds the
 //      class's lists.  The local class's lists depend only on (nblk, w)
@@ -30,15 +32,43 @@ namespace pipeline {
 
 constexpr int kMaxBlocks = 1024;   // blocks per sample (the lists' scratch sits in the CTA's shared memory)
 
-template <int MAXB>
+// A CTA of T warps, the first W of which compute lengths in phase 1 (each
+// with its lanes' words in shared memory, which phase 2 reuses as the list
+// jobs' scratch); all T build lists in phase 2.  Phase 1's shared memory caps
+// the lengths warps per SM, phase 2 needs none of it, so the CTA carries
+// more warps than phase 1 can use.
+template <int MAXB, int W, int T>
 struct Shape {
-    // warps per CTA: as many as fit (up to 16) in 220 KB of shared memory; the
-    // list jobs run on all of them
     static constexpr int kWarpBytes = deflate_lane::Layout<MAXB>::kWords * 128;
-    static constexpr int kWarps = 220 * 1024 / kWarpBytes < 16 ? 220 * 1024 / kWarpBytes : 16;
-    static constexpr size_t kLengthsBytes = static_cast<size_t>(kWarps) * kWarpBytes;
+    static constexpr int kLengthsWarps = W;
+    static constexpr int kWarps = T;
+    static constexpr size_t kLengthsBytes = static_cast<size_t>(W) * kWarpBytes;
     static constexpr size_t kListBytes = ((kMaxBlocks + 15) & ~15) + 4 * (2 * kMaxBlocks + 2 * (kMaxBlocks + 1) + 64);
     static constexpr size_t kSmemBytes = kLengthsBytes > kListBytes ? kLengthsBytes : kListBytes;
+    // a warp job's scratch (lists of at most kMaxWarpJobBlocks blocks), one per warp
+    static constexpr int kMaxWarpJobBlocks = 64;
+    static constexpr size_t kWarpJobBytes = (((kMaxWarpJobBlocks + 15) & ~15) + 4 * (2 * kMaxWarpJobBlocks + 2 * (kMaxWarpJobBlocks + 1) + 64) + 15) & ~size_t(15);
+    static_assert(kSmemBytes <= 227 * 1024, "pipeline CTA above the shared-memory limit");
+    static_assert(T * kWarpJobBytes <= kSmemBytes, "warp job scratch does not fit");
+    static_assert(W <= T, "lengths warps are a subset of the CTA");
+    // CTAs per SM that phase 1's shared memory allows: the register cap
+    // below keeps them all resident
+    static constexpr int kPerSm = 232448 / (static_cast<int>(kSmemBytes) + 1024) < 8
+                                      ? 232448 / (static_cast<int>(kSmemBytes) + 1024) : 8;
+};
+
+// The two CTA shapes of each block size.  Wide: as many lengths warps as fit
+// one CTA, and 16 warps in all, so a few list jobs each get many threads.
+// Narrow: the fewest lengths warps that keep an SM's lengths warps at the
+// shared-memory maximum, so many list jobs run side by side (one per CTA),
+// plus list-only warps up to 64 registers a thread over the SM.
+template <int MAXB>
+struct Shapes {
+    static constexpr int kWarpBytes = deflate_lane::Layout<MAXB>::kWords * 128;
+    static constexpr int kWideW = 220 * 1024 / kWarpBytes < 16 ? 220 * 1024 / kWarpBytes : 16;
+    static constexpr int kWideT = 16;
+    static constexpr int kNarrowW = MAXB > 64 ? 1 : 3;
+    static constexpr int kNarrowT = MAXB > 64 ? 8 : 6;
 };
 
 struct PipeArgs {
@@ -55,7 +85,7 @@ struct PipeArgs {
     int per[3];           // ... and which
     int local_once;       // 1: the local class is in use, built once into sample 0's slot
     int warp_jobs;        // 1: a list job per warp (its lengths words hold the job's scratch), 0: per CTA
-    int bpw;              // blocks per warp in the lengths phase (8, 16 or 32)
+    int bpw;              // blocks per warp in the lengths phase (1 .. 32)
 };
 
 // All CTAs of the grid reach this point (thread 0 of each waits, bounded);
@@ -85,20 +115,22 @@ __device__ __forceinline__ bool grid_barrier(int* counter, int target) {
     return ok != 0;
 }
 
-template <int MAXB>
-__global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel(const PipeArgs P) {
-    constexpr int kWarps = Shape<MAXB>::kWarps;
+template <int MAXB, int W, int T>
+__global__ void __launch_bounds__(32 * T, (Shape<MAXB, W, T>::kPerSm)) mask_pipeline_kernel(const PipeArgs P) {
+    using S = Shape<MAXB, W, T>;
     extern __shared__ __align__(16) uint8_t dsmem[];
-    __shared__ long long part[kWarps];
+    __shared__ long long part[T];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- phase 1: lengths, chunks of bpw blocks per warp (one per lane)
-    uint32_t* region = reinterpret_cast<uint32_t*>(dsmem) +
-                       static_cast<size_t>(warp) * deflate_lane::Layout<MAXB>::kWords * 32;
-    {
+    // ---- phase 1: lengths, chunks of bpw blocks per lengths warp (one per
+    // lane); consecutive chunks go to consecutive CTAs, so a small batch
+    // still spreads over the SMs
+    if (warp < W) {
+        uint32_t* region = reinterpret_cast<uint32_t*>(dsmem) +
+                           static_cast<size_t>(warp) * deflate_lane::Layout<MAXB>::kWords * 32;
         const int64_t nchunks = (P.total + P.bpw - 1) / P.bpw;
-        for (int64_t ch = static_cast<int64_t>(blockIdx.x) * kWarps + warp; ch < nchunks;
-             ch += static_cast<int64_t>(gridDim.x) * kWarps) {
+        for (int64_t ch = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; ch < nchunks;
+             ch += static_cast<int64_t>(gridDim.x) * W) {
             const int64_t task0 = ch * P.bpw;
             const int nb = P.total - task0 < P.bpw ? static_cast<int>(P.total - task0) : P.bpw;
             deflate_lane::warp_block_lengths<MAXB>(region, P.bytes, P.b, task0, nb, P.lengths, lane);
@@ -113,10 +145,10 @@ __global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel
     const int jobs_per = P.nper > 0 ? P.nper : 1;
     const int njobs = P.B * jobs_per + P.local_once;
     if (P.warp_jobs) {
-        // one job per warp at a time, in the warp's own lengths words: all the
+        // one job per warp at a time, each warp with its own scratch: all the
         // jobs run side by side instead of a few per CTA in turn
-        uint8_t* ws = reinterpret_cast<uint8_t*>(region);
-        for (int j = blockIdx.x * kWarps + warp; j < njobs; j += gridDim.x * kWarps) {
+        uint8_t* ws = dsmem + static_cast<size_t>(warp) * S::kWarpJobBytes;
+        for (int j = blockIdx.x * T + warp; j < njobs; j += gridDim.x * T) {
             const bool local = j == P.B * jobs_per;
             const int s = local ? 0 : j / jobs_per;
             const int k = local ? 0 : j % jobs_per;
@@ -152,7 +184,7 @@ __global__ void __launch_bounds__(32 * Shape<MAXB>::kWarps) mask_pipeline_kernel
         if (lane == 0) part[warp] = acc;
         __syncthreads();
         long long total = 0;
-        for (int w = 0; w < kWarps; ++w) total += part[w];
+        for (int w = 0; w < T; ++w) total += part[w];
         const bool write = !local && k == 0;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const uint8_t f = static_cast<long long>(__ldcg(row + i)) * n > total ? 1 : 0;
