@@ -1,11 +1,12 @@
-// Forward at d = 64 with persistent CTAs.
+// Forward at d = 64 and d = 128 with persistent CTAs.
 //
-// Same products as attn_fwd_bf16_kernel<64> — S = Q K^T per key block, an
+// Same products as attn_fwd_bf16_kernel<D> — S = Q K^T per key block, an
 // online softmax in exp2 with O rescaled only when a running max grows by
 // more than 8 (log2 units), P packed to bf16 in TMEM as the A operand of
 // O += P V — organised for the short items of the gzip masks (~12 key tiles
 // per 128-row query tile):
-//   persistent CTAs: a fixed grid (two per SM) takes the work items —
+//   persistent CTAs: a fixed grid (two per SM at d = 64, one at d = 128)
+//     takes the work items —
 //     (sample·head, query tile of two blocks from the class's pairing
 //     order), heaviest tile first — one at a time from a device counter, so
 //     set-up, key-list merge, pipeline fill and epilogue overlap the
@@ -42,7 +43,9 @@
 // on a timeout the CTA records an error code, drains its loads and products
 // in flight and every role leaves.
 // TMEM: S[b] at 64 b (P_A packed over its columns 0..15, P_B over 32..47),
-// O_A at 128, O_B at 192.
+// O_A at 128, O_B at 128 + d (256 columns a CTA at d = 64, 512 at d = 128).
+// Shared memory holds d in 64-column atoms of the 128-byte swizzle: a Q
+// buffer is [d / 64][128 rows][64], a K or V stage [d / 64][64 rows][64].
 #pragma once
 
 namespace gsa {
@@ -52,8 +55,11 @@ namespace bf16 {
 #define GSA_FWDP_STAGES 4
 #endif
 
+template <int D_>
 struct FwdPCfg {
-    static constexpr int D = 64;
+    static constexpr int D = D_;
+    static constexpr int kAtoms = D / 64;               // 64-column atoms of a row
+    static constexpr int kCtasPerSm = D == 64 ? 2 : 1;
     static constexpr int kStages = GSA_FWDP_STAGES;
     static constexpr int kQBytes = 128 * D * 2;         // Q tile (two query blocks)
     static constexpr int kKVBytes = kBlk * D * 2;       // one key block of K or V
@@ -72,19 +78,19 @@ struct FwdPCfg {
     static constexpr int kOffMl = kOffBits + 2 * (kListMaxBlocks / 32) * 4;
     static constexpr int kEnd = kOffMl + 2 * 2 * 2 * 128 * 4;
     static constexpr int kSmemBytes = kEnd + 1024;
-    static_assert(kSmemBytes <= 232448 / 2 - 1024, "two CTAs per SM");
+    static_assert(kSmemBytes <= 232448 / kCtasPerSm - 1024, "shared memory per SM");
     static_assert(kQBytes % 1024 == 0 && kStageBytes % 1024 == 0, "1024-byte alignment");
-    static constexpr int kTmemCols = 256;
-    static constexpr uint32_t kTmemS = 0, kTmemO = 128;   // O_h at 128 + 64 h
+    static constexpr int kTmemCols = D == 64 ? 256 : 512;
+    static constexpr uint32_t kTmemS = 0, kTmemO = 128;   // O_h at 128 + D h
     static constexpr int kSoftmax = 256;                  // two warpgroups
     static constexpr int kThreads = 64 + kSoftmax;
 };
 
-template <bool K4>   // strided tensors through 4-D maps (see load_rows)
-__global__ void __launch_bounds__(FwdPCfg::kThreads, 2)
+template <int DH, bool K4>   // head dimension; strided tensors through 4-D maps (see load_rows)
+__global__ void __launch_bounds__(FwdPCfg<DH>::kThreads, FwdPCfg<DH>::kCtasPerSm)
 attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-    using C = FwdPCfg;
+    using C = FwdPCfg<DH>;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -232,8 +238,10 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     for (int half = 0; half < 2; ++half) {
                         const int blk = half ? qb : qa;
                         if (blk < 0) continue;
-                        load_rows<K4>(q_buf(k & 1) + half * (kBlk * 128), &tmQ, &q_full[k & 1], 0, blk * kBlk, h_,
-                                      s_, head_row0);
+#pragma unroll
+                        for (int at = 0; at < C::kAtoms; ++at)
+                            load_rows<K4>(q_buf(k & 1) + at * (128 * 128) + half * (kBlk * 128), &tmQ, &q_full[k & 1],
+                                          64 * at, blk * kBlk, h_, s_, head_row0);
                     }
                     ++loads;
                 }
@@ -256,8 +264,13 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         const uint32_t live = ((ua >> bit) & 1u) | (((ub >> bit) & 1u) << 1);
                         meta[st] = static_cast<uint32_t>(j) | (live << 16) | ((j == last_j ? 1u : 0u) << 18);
                         mbar_arrive_expect_tx(&full[st], C::kStageBytes);
-                        load_rows<K4>(stage_k(st), &tmK, &full[st], 0, j * kBlk, h_, s_, head_row0);
-                        load_rows<K4>(stage_v(st), &tmV, &full[st], 0, j * kBlk, h_, s_, head_row0);
+#pragma unroll
+                        for (int at = 0; at < C::kAtoms; ++at) {
+                            load_rows<K4>(stage_k(st) + at * (kBlk * 128), &tmK, &full[st], 64 * at, j * kBlk, h_, s_,
+                                          head_row0);
+                            load_rows<K4>(stage_v(st) + at * (kBlk * 128), &tmV, &full[st], 64 * at, j * kBlk, h_, s_,
+                                          head_row0);
+                        }
                         ++gt;
                     }
                 }
@@ -298,10 +311,13 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         tc_fence_after();
                         const uint64_t da = sdesc_sw128(smem_u32(q_buf(kq & 1)), 16, 1024);
                         const uint64_t db = sdesc_sw128(smem_u32(stage_k(st)), 16, 1024);
+                        // K step kk: 32 bytes into atom kk / 4 (Q atoms 16 KB apart, K atoms 8 KB)
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)
-                            umma_bf16_w(tmem + C::kTmemS + 64 * sb, sdesc_advance(da, kk * 32),
-                                        sdesc_advance(db, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
+                            umma_bf16_w(tmem + C::kTmemS + 64 * sb,
+                                        sdesc_advance(da, (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                                        sdesc_advance(db, (kk >> 2) * (kBlk * 128) + (kk & 3) * 32), idesc_qk,
+                                        kk > 0 ? 1u : 0u);
                         umma_commit_w(&s_full[sb]);
                         if ((meta[st] >> 18) & 1u) {   // the item's Q is no longer read
                             umma_commit_w(&q_free[kq & 1]);
@@ -323,11 +339,12 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 const bool last = (meta[st] >> 18) & 1u;
                 const uint64_t bv = sdesc_sw128(smem_u32(stage_v(st)), kBlk * 128, 1024);
                 // O_h += P_h V[32 h .. 32 h + 31]: key chunk kk (16 keys) of half kk / 2 sits at
-                // packed column 32 (kk / 2) + 8 (kk % 2) of the S buffer
+                // packed column 32 (kk / 2) + 8 (kk % 2) of the S buffer; V's d spans its atoms
+                // (the descriptor's leading offset: 8 KB apart)
                 const uint32_t ap = tmem + C::kTmemS + 64 * (na & 1);
 #pragma unroll
                 for (int kk = 0; kk < kBlk / 16; ++kk)
-                    umma_bf16_ts_w(tmem + C::kTmemO + 64 * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
+                    umma_bf16_ts_w(tmem + C::kTmemO + D * (kk >> 1), ap + 32 * (kk >> 1) + 8 * (kk & 1),
                                    sdesc_advance(bv, kk * (16 * 128)), idesc_pv, (ta > 0 || (kk & 1)) ? 1u : 0u);
                 umma_commit_w(&empty[st]);
                 ta = last ? 0 : ta + 1;
@@ -351,7 +368,7 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         const int half = r >> 6;
         const int rr = r & 63;
         const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const uint32_t tO = tl + C::kTmemO + 64 * hc;
+        const uint32_t tO = tl + C::kTmemO + D * hc;
         float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
         // the previous item's epilogue, run once its last P V completed: combine the halves'
         // (m, l) through shared memory (double-buffered by item parity: a warp writes a buffer
@@ -377,17 +394,23 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             const float wA = mA == -INFINITY ? 0.f : ex2(mA - mm);
             const float wB = mB == -INFINITY ? 0.f : ex2(mB - mm);
             const float lt = lA * wA + lB * wB;
-            float a[32], b2[32];
-            tmem_ld32(tl + C::kTmemO + c0, a);
-            tmem_ld32(tl + C::kTmemO + 64 + c0, b2);
-            tmem_wait_ld();
+            const float rl = rcp_approx(lt);
+            // this thread's D / 2 output columns, 32 at a time
 #pragma unroll
-            for (int e = 0; e < 32; ++e) a[e] = fmaf(b2[e], wB, a[e] * wA);
-            if (pend.tok >= 0) {
-                __nv_bfloat16* orow = p.o + (K4 ? tok_off(pend.tok, p.L, p.H, p.lo) : pend.tok * D);
-                store_scaled_bf16(orow + c0, a, rcp_approx(lt));
-                if (hc == 0) p.lse[pend.tok] = (mm + lg2_approx(lt)) * 0.69314718055994531f;
+            for (int cb = 0; cb < D / 2; cb += 32) {
+                const int col = hc * (D / 2) + cb;
+                float a[32], b2[32];
+                tmem_ld32(tl + C::kTmemO + col, a);
+                tmem_ld32(tl + C::kTmemO + D + col, b2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) a[e] = fmaf(b2[e], wB, a[e] * wA);
+                if (pend.tok >= 0) {
+                    __nv_bfloat16* orow = p.o + (K4 ? tok_off(pend.tok, p.L, p.H, p.lo) : pend.tok * D);
+                    store_scaled_bf16(orow + col, a, rl);
+                }
             }
+            if (pend.tok >= 0 && hc == 0) p.lse[pend.tok] = (mm + lg2_approx(lt)) * 0.69314718055994531f;
             pend.on = false;
             return true;
         };

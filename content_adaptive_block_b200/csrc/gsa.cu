@@ -129,12 +129,16 @@ gsa_status launch_fwd(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, c
     return launch_status();
 }
 
-template <bool K4>
-gsa_status launch_fwd_persist(unsigned ctas, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+// The persistent forward: as many CTAs as fit on the device at once (two per
+// SM at d = 64, one at d = 128), at most one per work item.
+template <int D, bool K4>
+gsa_status launch_fwd_persist(int64_t items, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const gsa::bf16::FwdParams& p, cudaStream_t cs) {
-    using C = gsa::bf16::FwdPCfg;
-    if (!gsa::smem_opt_in(gsa::bf16::attn_fwd_persist_kernel<K4>, C::kSmemBytes)) return GSA_ERR_CUDA;
-    gsa::bf16::attn_fwd_persist_kernel<K4><<<ctas, C::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
+    using C = gsa::bf16::FwdPCfg<D>;
+    if (!gsa::smem_opt_in(gsa::bf16::attn_fwd_persist_kernel<D, K4>, C::kSmemBytes)) return GSA_ERR_CUDA;
+    const int64_t full = static_cast<int64_t>(C::kCtasPerSm) * gsa::bwd::sm_count();
+    const unsigned ctas = static_cast<unsigned>(items < full ? items : full);
+    gsa::bf16::attn_fwd_persist_kernel<D, K4><<<ctas, C::kThreads, C::kSmemBytes, cs>>>(tq, tk, tv, p);
     return launch_status();
 }
 
@@ -459,13 +463,15 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     std::memcpy(p.cls, cls, desc->H);
     p.local_once = (csr->classes >> 3) & 1;
     dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
-    if (desc->d == 64 && GSA_FWD_PERSIST) {
+    if (GSA_FWD_PERSIST) {
         p.ticket = fwd_ticket_slot();
         if (!p.ticket) return GSA_ERR_CUDA;
         const int64_t items = static_cast<int64_t>(desc->B) * desc->H * ((csr->nblk + 1) / 2);
-        const int64_t ctas = items < 2 * gsa::bwd::sm_count() ? items : 2 * gsa::bwd::sm_count();
-        return k4 ? launch_fwd_persist<true>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs)
-                  : launch_fwd_persist<false>(static_cast<unsigned>(ctas), tq, tk, tv, p, cs);
+        if (desc->d == 64)
+            return k4 ? launch_fwd_persist<64, true>(items, tq, tk, tv, p, cs)
+                      : launch_fwd_persist<64, false>(items, tq, tk, tv, p, cs);
+        return k4 ? launch_fwd_persist<128, true>(items, tq, tk, tv, p, cs)
+                  : launch_fwd_persist<128, false>(items, tq, tk, tv, p, cs);
     }
     if (desc->d == 64)
         return k4 ? launch_fwd<64, true>(grid, tq, tk, tv, p, cs) : launch_fwd<64, false>(grid, tq, tk, tv, p, cs);
