@@ -5,9 +5,10 @@
 A step is one pass of the whole path over one synthetic batch of the 8K-byte
 workload (8 samples x 8192 bytes, 64-byte blocks -> 128 blocks, window 2,
 12 heads split 6 local / 3 literal / 3 hybrid, head dim 64, bf16):
-    gsa_block_lengths -> gsa_literal_flags -> gsa_build_block_csr
+    gsa_mask_pipeline (block lengths -> literal flags -> block lists, one launch)
     -> gsa_attn_fwd -> gsa_attn_bwd
-all through the C ABI (libgsa.so).  The headline value is live-block
+all through the C ABI (libgsa.so); the mask sweep times the three separate
+calls (gsa_block_lengths, gsa_literal_flags, gsa_build_block_csr) beside it.  The headline value is live-block
 attention TFLOP/s (forward 4*d and backward 8*d FLOPs per live
 (query token, key token) pair, the S recompute not counted) of the whole
 step, inputs resident in HBM.  The L2 is flushed between steps (a 256 MiB
@@ -351,7 +352,7 @@ def run_reference(args, rank, world):
 # The kernels behind each timed call, and the sources whose hash ties a
 # recorded traffic figure to the code that produced it.
 _TRAFFIC_CALLS = {
-    "gsa_attn_fwd": (["attn_fwd_persist_kernel<0>"],
+    "gsa_attn_fwd": (["attn_fwd_persist_kernel<64, 0>"],
                      ["content_adaptive_block_b200/csrc/attn_fwd_bf16.cuh",
                       "content_adaptive_block_b200/csrc/attn_fwd_persist.cuh"]),
     "gsa_attn_bwd": (["dot_kernel<64>", "dq_persist_kernel<0>", "dkdv_persist_kernel<0>"],
@@ -491,27 +492,23 @@ def run_ours(args, rank, world, local_rank):
     ws = torch.empty(gsa.gsa_attn_bwd_workspace(q, wl.b, hc), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    names = ("gsa_block_lengths", "gsa_literal_flags", "gsa_build_block_csr", "gsa_attn_fwd", "gsa_attn_bwd")
-    launches_per_step = 1 + 1 + 1 + 1 + 3
+    counters = torch.zeros(1, dtype=torch.int32, device=dev)
+    names = ("gsa_mask_pipeline", "gsa_attn_fwd", "gsa_attn_bwd")
+    launches_per_step = 1 + 1 + 3
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        gsa.gsa_block_lengths(x, wl.b, out=lengths)
+        gsa.gsa_mask_pipeline(x, wl.b, wl.w, csr, lengths=lengths, flags=flags, counters=counters,
+                              head_classes=hc)
         if ev:
             ev[1].record(stream)
-        gsa.gsa_literal_flags(lengths, out=flags)
-        if ev:
-            ev[2].record(stream)
-        gsa.gsa_build_block_csr(flags, wl.w, csr)
-        if ev:
-            ev[3].record(stream)
         gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b, o=o, lse=lse)
         if ev:
-            ev[4].record(stream)
+            ev[2].record(stream)
         gsa.gsa_attn_bwd(q, k, v, o, lse, do, csr, hc, wl.b, dq=dq, dk=dk, dv=dv, workspace=ws)
         if ev:
-            ev[5].record(stream)
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -591,6 +588,7 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
         st["lengths"] = torch.empty((wl.S, wl.N), dtype=torch.int32, device=dev)
         st["flags"] = torch.empty((wl.S, wl.N), dtype=torch.uint8, device=dev)
         st["csr"] = gsa.BlockCsr(wl.S, wl.N, dev)
+        st["counters"] = torch.zeros(1, dtype=torch.int32, device=dev)
         st["o"] = torch.empty_like(q)
         st["lse"] = torch.empty((wl.S, wl.H, wl.L), dtype=torch.float32, device=dev)
         for name in ("dq", "dk", "dv"):
@@ -618,9 +616,8 @@ def e2e_timing(args, gsa, wl, hc, x_host, q, k, v, do, stream, world, dev, step_
         stream.wait_event(ev["up"][j])
         if i >= 2:
             stream.wait_event(ev["down"][j])            # step i - 2's outputs left this set
-        gsa.gsa_block_lengths(st["x"], wl.b, out=st["lengths"])
-        gsa.gsa_literal_flags(st["lengths"], out=st["flags"])
-        gsa.gsa_build_block_csr(st["flags"], wl.w, st["csr"])
+        gsa.gsa_mask_pipeline(st["x"], wl.b, wl.w, st["csr"], lengths=st["lengths"], flags=st["flags"],
+                              counters=st["counters"], head_classes=hc)
         gsa.gsa_attn_fwd(st["q"], st["k"], st["v"], st["csr"], hc, wl.b, o=st["o"], lse=st["lse"])
         gsa.gsa_attn_bwd(st["q"], st["k"], st["v"], st["o"], st["lse"], st["do"], st["csr"], hc, wl.b,
                          dq=st["dq"], dk=st["dk"], dv=st["dv"], workspace=st["ws"])
