@@ -38,7 +38,7 @@ namespace gsa {
 namespace bwd {
 
 #ifndef GSA_DKVP_STAGES
-#define GSA_DKVP_STAGES 5
+#define GSA_DKVP_STAGES 7
 #endif
 
 struct DkvPCfg {

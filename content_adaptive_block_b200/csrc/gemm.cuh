@@ -16,10 +16,11 @@
 //               tcgen05.mma.kind::f16 (M 128, N 256, K 16) into one of two
 //               accumulators, so one tile's epilogue overlaps the next tile's
 //               products;
-//   warps 2-5   epilogue: one output row per thread (its TMEM lane), 64 (or
-//               32 float32) columns at a time: the epilogue arithmetic, then
-//               into a 128-byte swizzled staging box that one thread stores
-//               with TMA.
+//   warps 2-9   epilogue, two warpgroups: one output row per thread (its
+//               TMEM lane), 64 (or 32 float32) columns at a time, each
+//               warpgroup half of them: the epilogue arithmetic (C or the
+//               GELU input of the next chunk already loaded), then into a
+//               128-byte swizzled staging box that one thread stores with TMA.
 // Every wait is bounded: on a timeout the CTA records an error code, drains
 // what it issued and leaves.
 #pragma once
@@ -45,8 +46,8 @@ constexpr int kNumBars = 2 * kStages + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;             // tmem base, abort
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
 
 struct Params {
     int M, N, K;
@@ -77,18 +78,26 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // the four epilogue warps only
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
-// GELU, tanh form, and its derivative.
+// GELU, tanh form, and its derivative, with the hardware tanh approximation
+// (tanh.approx.f32: relative error about 2^-11, below the bf16 rounding of
+// the results).
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ float gelu_tanh(float x) {
     const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-    return 0.5f * x * (1.f + tanhf(k0 * (x + k1 * x * x * x)));
+    return 0.5f * x * (1.f + tanh_fast(k0 * (x + k1 * x * x * x)));
 }
 __device__ __forceinline__ float gelu_tanh_grad(float x) {
     const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-    const float t = tanhf(k0 * (x + k1 * x * x * x));
+    const float t = tanh_fast(k0 * (x + k1 * x * x * x));
     return 0.5f * (1.f + t) + 0.5f * x * (1.f - t * t) * k0 * (1.f + 3.f * k1 * x * x);
 }
 
@@ -214,12 +223,34 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             if (ok) umma_commit_w(&acc_full[buf]);
         }
     } else {
-        // epilogue: thread = output row (TMEM lane quadrant of its warp)
+        // epilogue: thread = output row (TMEM lane quadrant of its warp) and
+        // column half hc of every chunk
         const int quad = warp & 3;
+        const int hc = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
-        const int et = threadIdx.x - 64;   // 0 .. 127
+        const int et = threadIdx.x - 64;   // 0 .. 255
         uint8_t* out_box = smem + kOffOut;
         uint8_t* aux_box = smem + kOffAux;
+        const bool f32 = p.out32 || p.split_out;
+        const int cw = f32 ? 32 : 64;      // columns per staging box (128 bytes a row)
+        const int hw = cw / 2;             // this thread's columns of a chunk: 64 bytes
+        // the chunk's second operand (C for beta C, the GELU input for its
+        // derivative): 32 bf16 of this thread's row, loaded one chunk ahead
+        const __nv_bfloat16* side = (!f32 && p.epi == kNone && p.beta != 0.f) ? p.C
+                                    : ((!f32 && p.epi == kDGelu) ? p.aux_in : nullptr);
+        const int64_t side_ld = p.epi == kDGelu ? p.aux_ld : p.ldc;
+        auto load_side = [&](int row, int col, uint4* dst) {
+            if (side && row < p.M) {
+                const uint4* src = reinterpret_cast<const uint4*>(side + static_cast<int64_t>(row) * side_ld + col);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) dst[x] = src[x];
+            }
+        };
+        // without a GELU output the aux box is free: the chunks alternate
+        // between the two boxes, so a chunk waits only for the store of the
+        // chunk two before
+        const bool dbl = p.epi != kGeluAux;
+        int chunk = 0;
         bool ok = true;
         int local = 0;
         for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
@@ -227,89 +258,88 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             tile_of(t, mb, nb, ks);
             const int m0 = mb * BM, n0 = nb * BN;
             const int buf = local & 1;
+            const int row = m0 + r;
+            uint4 nxt[4];
+            load_side(row, n0 + hc * hw, nxt);   // in flight while the products run
             if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t tacc = tmem + (static_cast<uint32_t>(quad * 32) << 16) + buf * BN;
-            const int row = m0 + r;
-            const bool f32 = p.out32 || p.split_out;
-            const int cw = f32 ? 32 : 64;   // columns per staging box
-            for (int c0 = 0; c0 < BN; c0 += cw) {
-                float v[64];
-                tmem_ld32(tacc + c0, v);
-                if (!f32) tmem_ld32(tacc + c0 + 32, v + 32);
-                tmem_wait_ld();
-                // the staging boxes are free once the previous stores read them
-                if (et == 0) bulk_wait_read0();
-                epi_sync();
-                if (f32) {
-                    // 32 float32 = 8 chunks of 16 bytes, swizzled by row
+            for (int c0 = 0; c0 < BN; c0 += cw, ++chunk) {
+                const int cc = c0 + hc * hw;   // this thread's first column in the tile
+                uint8_t* box = (dbl && (chunk & 1)) ? aux_box : out_box;
+                uint4 cur[4];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) {
+                for (int x = 0; x < 4; ++x) cur[x] = nxt[x];
+                if (c0 + cw < BN) load_side(row, n0 + cc + cw, nxt);
+                float v[32];
+                if (f32) tmem_ld16(tacc + cc, v);
+                else tmem_ld32(tacc + cc, v);
+                tmem_wait_ld();
+                // the staging box is free once the store that last used it read it
+                if (et == 0) {
+                    if (dbl) bulk_wait_read1();
+                    else bulk_wait_read0();
+                }
+                epi_sync();
+                const int xb = hc * 4;   // this thread's four 16-byte pieces of the box row
+                if (f32) {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
                         uint4 q;
                         q.x = __float_as_uint(v[4 * x + 0]);
                         q.y = __float_as_uint(v[4 * x + 1]);
                         q.z = __float_as_uint(v[4 * x + 2]);
                         q.w = __float_as_uint(v[4 * x + 3]);
-                        *reinterpret_cast<uint4*>(out_box + r * 128 + ((x ^ (r & 7)) * 16)) = q;
+                        *reinterpret_cast<uint4*>(box + r * 128 + (((xb + x) ^ (r & 7)) * 16)) = q;
                     }
                 } else {
-                    const int col = n0 + c0;
-                    if (p.epi == kNone && p.beta != 0.f && row < p.M) {
-                        const uint4* cr = reinterpret_cast<const uint4*>(p.C + static_cast<int64_t>(row) * p.ldc + col);
+                    if (side && row < p.M) {
 #pragma unroll
-                        for (int x = 0; x < 8; ++x) {
-                            const uint4 q = cr[x];
-                            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+                        for (int x = 0; x < 4; ++x) {
+                            const uint32_t w[4] = {cur[x].x, cur[x].y, cur[x].z, cur[x].w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                v[8 * x + 2 * e] += p.beta * bf16_lo(w[e]);
-                                v[8 * x + 2 * e + 1] += p.beta * bf16_hi(w[e]);
-                            }
-                        }
-                    } else if (p.epi == kDGelu && row < p.M) {
-                        const uint4* ar = reinterpret_cast<const uint4*>(p.aux_in + static_cast<int64_t>(row) * p.aux_ld + col);
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) {
-                            const uint4 q = ar[x];
-                            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                v[8 * x + 2 * e] *= gelu_tanh_grad(bf16_lo(w[e]));
-                                v[8 * x + 2 * e + 1] *= gelu_tanh_grad(bf16_hi(w[e]));
+                                if (p.epi == kDGelu) {
+                                    v[8 * x + 2 * e] *= gelu_tanh_grad(bf16_lo(w[e]));
+                                    v[8 * x + 2 * e + 1] *= gelu_tanh_grad(bf16_hi(w[e]));
+                                } else {
+                                    v[8 * x + 2 * e] += p.beta * bf16_lo(w[e]);
+                                    v[8 * x + 2 * e + 1] += p.beta * bf16_hi(w[e]);
+                                }
                             }
                         }
                     }
                     if (p.epi == kGeluAux) {
 #pragma unroll
-                        for (int x = 0; x < 8; ++x) {
+                        for (int x = 0; x < 4; ++x) {
                             uint4 q;
                             q.x = pack_bf16x2(v[8 * x + 0], v[8 * x + 1]);
                             q.y = pack_bf16x2(v[8 * x + 2], v[8 * x + 3]);
                             q.z = pack_bf16x2(v[8 * x + 4], v[8 * x + 5]);
                             q.w = pack_bf16x2(v[8 * x + 6], v[8 * x + 7]);
-                            *reinterpret_cast<uint4*>(aux_box + r * 128 + ((x ^ (r & 7)) * 16)) = q;
+                            *reinterpret_cast<uint4*>(aux_box + r * 128 + (((xb + x) ^ (r & 7)) * 16)) = q;
                         }
 #pragma unroll
-                        for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
+                        for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
                     }
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) {
+                    for (int x = 0; x < 4; ++x) {
                         uint4 q;
                         q.x = pack_bf16x2(v[8 * x + 0], v[8 * x + 1]);
                         q.y = pack_bf16x2(v[8 * x + 2], v[8 * x + 3]);
                         q.z = pack_bf16x2(v[8 * x + 4], v[8 * x + 5]);
                         q.w = pack_bf16x2(v[8 * x + 6], v[8 * x + 7]);
-                        *reinterpret_cast<uint4*>(out_box + r * 128 + ((x ^ (r & 7)) * 16)) = q;
+                        *reinterpret_cast<uint4*>(box + r * 128 + (((xb + x) ^ (r & 7)) * 16)) = q;
                     }
                 }
                 fence_proxy_async_smem();
                 epi_sync();
                 if (et == 0) {
                     // split partials: rows of split ks follow the previous splits' M rows
-                    tma_store_2d(&tmD, out_box, n0 + c0, p.split_out ? ks * p.M + m0 : m0);
+                    tma_store_2d(&tmD, box, n0 + c0, p.split_out ? ks * p.M + m0 : m0);
                     if (p.epi == kGeluAux) tma_store_2d(&tmAux, aux_box, n0 + c0, m0);
                     bulk_commit();
                 }
