@@ -37,7 +37,7 @@ def _csv(path, rows):
             w.writerow([str(i), name, rd, wr, "1.0"])
 
 
-FWD = "void bf16::attn_fwd_persist_kernel<0>(CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, bf16::FwdParams)"
+FWD = "void bf16::attn_fwd_persist_kernel<64, 0>(CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, bf16::FwdParams)"
 DOT = "void bwd::dot_kernel<64>(const __nv_bfloat16 *, const __nv_bfloat16 *, gsa::TokLayout, long)"
 DQ = "void bwd::dq_persist_kernel<0>(CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, bwd::Params)"
 DKV = "void bwd::dkdv_persist_kernel<0>(CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, bwd::Params)"
