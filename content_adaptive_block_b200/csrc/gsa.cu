@@ -192,9 +192,9 @@ gsa_status launch_pipeline_shape(const gsa::pipeline::PipeArgs& P, cudaStream_t 
 
 // Many short list jobs (more than one per SM, at most 128 blocks a sample)
 // run on the narrow CTAs, one job per CTA side by side; a few jobs, or long
-// lists, run on the wide ones, each job with 16 warps (measured over 256
-// samples: the narrow shape 7-8 % faster at 64 blocks a sample and within 2 %
-// either way at 128, the wide one 6-9 % faster at 256).
+// lists, run on the wide ones, each job with 32 warps (measured over 256
+// samples: the narrow shape 8-10 % faster at 64 blocks a sample and 0-4 % at
+// 128, the wide one 15-19 % faster at 256).
 template <int MAXB>
 gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
     using SS = gsa::pipeline::Shapes<MAXB>;

@@ -58,7 +58,8 @@ struct Shape {
 };
 
 // The two CTA shapes of each block size.  Wide: as many lengths warps as fit
-// one CTA, and 16 warps in all, so a few list jobs each get many threads.
+// one CTA, and 32 warps in all (64 registers a thread), so a few list jobs,
+// or long lists, each get many threads.
 // Narrow: the fewest lengths warps that keep an SM's lengths warps at the
 // shared-memory maximum, so many list jobs run side by side (one per CTA),
 // plus list-only warps up to 64 registers a thread over the SM.
@@ -66,7 +67,7 @@ template <int MAXB>
 struct Shapes {
     static constexpr int kWarpBytes = deflate_lane::Layout<MAXB>::kWords * 128;
     static constexpr int kWideW = 220 * 1024 / kWarpBytes < 16 ? 220 * 1024 / kWarpBytes : 16;
-    static constexpr int kWideT = 16;
+    static constexpr int kWideT = 32;
     static constexpr int kNarrowW = MAXB > 64 ? 1 : 3;
     static constexpr int kNarrowT = MAXB > 64 ? 8 : 6;
 };
