@@ -63,11 +63,12 @@ def workload_desc(wl):
 
 
 def csr_nnz(csr):
-    """Live block pairs per (sample, class) [S][3] from the lists' pointers
-    (a local class stored once counts for every sample)."""
+    """Live block pairs per (sample, class) [S][3] from the lists' pointers;
+    an implicit local class (not stored) counts its window, min(i, w) + 1
+    key blocks for query block i."""
     nnz = csr.row_ptr[:, :, -1].cpu().numpy().copy()
-    if csr.classes & 8:
-        nnz[:, 0] = nnz[0, 0]
+    if not csr.stored(0):
+        nnz[:, 0] = sum(min(i, csr.w) + 1 for i in range(csr.nblk))
     return nnz
 
 
@@ -747,13 +748,13 @@ def mask_stage(gsa, dev):
         nnz = int(nnz_sc.sum())
         # what the stage writes: lengths (int32) and flags (uint8) per block;
         # CSR and CSC pointers, entries and pairing orders (int32) per (sample,
-        # class) — the three calls for every sample, the pipeline its local
-        # class once
+        # class) — the three calls for every class, the pipeline for the
+        # literal and hybrid classes (the local class's lists are implicit)
         out_bytes = (wl.S * wl.N * (4 + 1)
                      + 4 * (2 * wl.S * 3 * (wl.N + 1) + 2 * nnz + 2 * wl.S * 3 * wl.N))
-        nnz_once = int(nnz_sc[:, 1:].sum()) + int(nnz_sc[0, 0])
+        nnz_pipe = int(nnz_sc[:, 1:].sum())
         out_bytes_pipe = (wl.S * wl.N * (4 + 1)
-                          + 4 * (2 * (2 * wl.S + 1) * (wl.N + 1) + 2 * nnz_once + 2 * (2 * wl.S + 1) * wl.N))
+                          + 4 * (2 * (2 * wl.S) * (wl.N + 1) + 2 * nnz_pipe + 2 * (2 * wl.S) * wl.N))
         best_ms = min(sep_ms, all_ms)
         out["points"][f"b{b}_f{f}"] = {
             "gbs": nbytes / (best_ms * 1e-3) / 1e9, "lengths_gbs": nbytes / (len_ms * 1e-3) / 1e9,

@@ -183,20 +183,23 @@ class BlockCsr:
                     self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_ptr.data_ptr(),
                     self.row_idx.data_ptr(), self.q_order.data_ptr(), self.k_order.data_ptr())
 
-    def slot(self, s: int, c: int) -> int:
-        """The sample whose slot holds (s, c)'s lists: sample 0's for the local
-        class when it is stored once (classes bit 3)."""
-        return 0 if (c == 0 and self.classes & 8) else s
+    def stored(self, c: int) -> bool:
+        """Whether class c's lists are in the buffers: a local class marked
+        implicit (classes bit 3, written by gsa_mask_pipeline) is not stored;
+        the attention kernels derive its lists from (nblk, w)."""
+        return not (c == 0 and self.classes & 8)
 
     def rows(self, s: int, c: int) -> list:
         """Key-block list of every query block of (sample s, class c), on the host."""
-        s = self.slot(s, c)
+        if not self.stored(c):
+            raise ValueError("the local class's lists are implicit (not stored)")
         rp = self.row_ptr[s, c].cpu().tolist()
         ci = self.col_idx[s, c, : rp[-1]].cpu().tolist()
         return [ci[rp[i]: rp[i + 1]] for i in range(self.nblk)]
 
     def cols(self, s: int, c: int) -> list:
-        s = self.slot(s, c)
+        if not self.stored(c):
+            raise ValueError("the local class's lists are implicit (not stored)")
         cp = self.col_ptr[s, c].cpu().tolist()
         ri = self.row_idx[s, c, : cp[-1]].cpu().tolist()
         return [ri[cp[j]: cp[j + 1]] for j in range(self.nblk)]
@@ -251,7 +254,8 @@ def gsa_mask_pipeline(data: torch.Tensor, b: int, w: int, csr: BlockCsr | None =
                       lengths: torch.Tensor | None = None, flags: torch.Tensor | None = None,
                       counters: torch.Tensor | None = None, stream=None, head_classes=None):
     """lengths -> flags -> block lists in one launch; returns (lengths, flags, csr).
-    The local class's lists are stored once (sample 0's slot).  counters (int32,
+    The local class's lists are implicit: not stored (csr.classes bit 3), the
+    attention kernels derive them from (nblk, w).  counters (int32,
     at least one element, zero, left zero by each call) may be passed to avoid
     allocating one per call."""
     _need(data, "data", torch.uint8, 2)

@@ -76,7 +76,8 @@ struct Params {
     float scale_log2;
     int* ticket;            // work counter of the persistent kernel (dot_kernel zeroes both)
     uint8_t cls[kMaxHeads];
-    int local_once;   // the local class's lists are stored once, in sample 0's slot
+    int local_implicit;   // the local class's lists are not stored: derived from (nblk, w)
+    int w;                // the lists' window
 };
 
 // ------------------------------------------------------------ D_t = dO·O
@@ -198,9 +199,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
-    const int qa = p.order[g * nblk + 2 * tile];
-    const int qb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const bool implicit = c == 0 && p.local_implicit;
+    const int32_t* ord = implicit ? nullptr : p.order + g * nblk;
+    const int qa = order_at(ord, 2 * tile);
+    const int qb = (2 * tile + 1 < nblk) ? order_at(ord, 2 * tile + 1) : -1;
     const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (threadIdx.x == 0) {
@@ -235,7 +238,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, qa, qb, nblk);
+    build_tile_list(tl, ListRef{implicit ? nullptr : p.ptr + g * (nblk + 1), p.idx + g * p.cap, p.w, nblk, false}, qa,
+                    qb, nblk);
     if (threadIdx.x == 0) {
         mbar_init(done, *tl.count >= C::G ? C::G : 1);   // one arrival per group that has tiles
         fence_mbar_init();
@@ -519,9 +523,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
-    const int ka = p.order[g * nblk + 2 * tile];
-    const int kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const bool implicit = c == 0 && p.local_implicit;
+    const int32_t* ord = implicit ? nullptr : p.order + g * nblk;
+    const int ka = order_at(ord, 2 * tile);
+    const int kb = (2 * tile + 1 < nblk) ? order_at(ord, 2 * tile + 1) : -1;
     const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;
 
     if (threadIdx.x == 0) {
@@ -558,7 +564,8 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    build_tile_list(tl, p.ptr + g * (nblk + 1), p.idx + g * p.cap, ka, kb, nblk);
+    build_tile_list(tl, ListRef{implicit ? nullptr : p.ptr + g * (nblk + 1), p.idx + g * p.cap, p.w, nblk, true}, ka,
+                    kb, nblk);
     if (threadIdx.x == 0) {
         mbar_init(done, *tl.count >= C::G ? C::G : 1);   // one arrival per group that has tiles
         fence_mbar_init();
@@ -895,7 +902,8 @@ inline gsa_status launch(const void* q, const void* k, const void* v, const void
     base.scale_log2 = scale * kLog2e;
     base.ticket = reinterpret_cast<int*>(work + 2 * ((rows + 63) & ~int64_t(63)));   // after D and LSE2
     for (int h = 0; h < desc->H; ++h) base.cls[h] = cls[h];
-    base.local_once = (csr->classes >> 3) & 1;
+    base.local_implicit = (csr->classes >> 3) & 1;
+    base.w = csr->w;
     Params pq = base, pkv = base;
     pq.ticket = base.ticket + 1;
     pq.ptr = csr->row_ptr;

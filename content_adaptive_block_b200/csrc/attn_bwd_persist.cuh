@@ -120,9 +120,10 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         sh = it % SH;
         const int tile = it / SH;
         const int s = sh / p.H, h = sh % p.H;
-        g = (p.cls[h] == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + p.cls[h];
-        ka = p.order[g * nblk + 2 * tile];
-        kb = (2 * tile + 1 < nblk) ? p.order[g * nblk + 2 * tile + 1] : -1;
+        g = (p.cls[h] == 0 && p.local_implicit) ? -1 : static_cast<int64_t>(s) * 3 + p.cls[h];   // -1: implicit
+        const int32_t* ord = g < 0 ? nullptr : p.order + g * nblk;
+        ka = order_at(ord, 2 * tile);
+        kb = (2 * tile + 1 < nblk) ? order_at(ord, 2 * tile + 1) : -1;
     };
 
     if (threadIdx.x == 0) {
@@ -181,18 +182,10 @@ dkdv_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     bitsB[w] = 0u;
                 }
                 __syncwarp();
-                const int32_t* cp = p.ptr + g * (nblk + 1);
-                const int32_t* ri = p.idx + g * p.cap;
-                for (int e = cp[ka] + lane; e < cp[ka + 1]; e += 32) {
-                    const int i = ri[e];
-                    atomicOr(&bitsA[i >> 5], 1u << (i & 31));
-                }
-                if (kb >= 0) {
-                    for (int e = cp[kb] + lane; e < cp[kb + 1]; e += 32) {
-                        const int i = ri[e];
-                        atomicOr(&bitsB[i >> 5], 1u << (i & 31));
-                    }
-                }
+                const ListRef cols{g < 0 ? nullptr : p.ptr + g * (nblk + 1), p.idx + (g < 0 ? 0 : g) * p.cap, p.w,
+                                   nblk, true};
+                cols.each(ka, lane, 32, [&](int i) { atomicOr(&bitsA[i >> 5], 1u << (i & 31)); });
+                if (kb >= 0) cols.each(kb, lane, 32, [&](int i) { atomicOr(&bitsB[i >> 5], 1u << (i & 31)); });
                 __syncwarp();
             }
             const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;

@@ -109,7 +109,8 @@ struct FwdParams {
     float scale_log2;   // softmax scale * log2(e)
     int* ticket;        // persistent kernel: work counter, CTAs finished (both zero at launch)
     uint8_t cls[kMaxHeads];
-    int local_once;   // the local class's lists are stored once, in sample 0's slot
+    int local_implicit;   // the local class's lists are not stored: derived from (nblk, w)
+    int w;                // the lists' window
 };
 
 template <int D>
@@ -176,9 +177,11 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int tile = blockIdx.y;
     const int c = p.cls[h];
     const int nblk = p.nblk;
-    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
-    const int qa = p.q_order[g * nblk + 2 * tile];
-    const int qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const bool implicit = c == 0 && p.local_implicit;
+    const int32_t* ord = implicit ? nullptr : p.q_order + g * nblk;
+    const int qa = order_at(ord, 2 * tile);
+    const int qb = (2 * tile + 1 < nblk) ? order_at(ord, 2 * tile + 1) : -1;
     const int nwords = (nblk + 31) >> 5;
     const int64_t head_row0 = static_cast<int64_t>(sh) * p.L;   // row of this (s, h)'s first token (LSE index)
 
@@ -222,20 +225,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
     __syncthreads();
     {
-        const int32_t* rp = p.row_ptr + g * (nblk + 1);
-        const int32_t* ci = p.col_idx + g * p.cap;
-        const int a0 = rp[qa], a1 = rp[qa + 1];
-        for (int e = a0 + threadIdx.x; e < a1; e += blockDim.x) {
-            const int j = ci[e];
-            atomicOr(&bitsA[j >> 5], 1u << (j & 31));
-        }
-        if (qb >= 0) {
-            const int b0 = rp[qb], b1 = rp[qb + 1];
-            for (int e = b0 + threadIdx.x; e < b1; e += blockDim.x) {
-                const int j = ci[e];
-                atomicOr(&bitsB[j >> 5], 1u << (j & 31));
-            }
-        }
+        const ListRef rows{implicit ? nullptr : p.row_ptr + g * (nblk + 1), p.col_idx + g * p.cap, p.w, nblk, false};
+        rows.each(qa, threadIdx.x, blockDim.x, [&](int j) { atomicOr(&bitsA[j >> 5], 1u << (j & 31)); });
+        if (qb >= 0) rows.each(qb, threadIdx.x, blockDim.x, [&](int j) { atomicOr(&bitsB[j >> 5], 1u << (j & 31)); });
     }
     __syncthreads();
     if (warp == 0) {

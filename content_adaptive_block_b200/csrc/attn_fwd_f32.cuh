@@ -33,7 +33,8 @@ struct Params {
     int64_t L;
     float scale;
     uint8_t cls[kMaxHeads];
-    int local_once;   // the local class's lists are stored once, in sample 0's slot
+    int local_implicit;   // the local class's lists are not stored: derived from (nblk, w)
+    int w;                // the lists' window
 };
 
 template <int D>
@@ -45,7 +46,8 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(Params p) {
     float* sv = sk + b * D;       // [b][D]
     const int i = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int c = p.cls[h];
-    const int64_t g = (c == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + c;
+    const int64_t g = static_cast<int64_t>(s) * 3 + c;
+    const bool implicit = c == 0 && p.local_implicit;
     const int64_t head_off = (static_cast<int64_t>(s) * p.H + h) * p.L;
     const int r = threadIdx.x;
     const int64_t row0 = head_off + static_cast<int64_t>(i) * b;
@@ -57,11 +59,13 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(Params p) {
     for (int e = 0; e < D; ++e) acc[e] = 0.f;
     float m = -INFINITY, l = 0.f;
 
+    // key blocks of query block i: the stored row, or the implicit local window
     const int32_t* rp = p.row_ptr + g * (p.nblk + 1);
-    const int beg = rp[i], end = rp[i + 1];
     const int32_t* ci = p.col_idx + g * p.cap;
+    const int beg = implicit ? (i - p.w > 0 ? i - p.w : 0) : rp[i];
+    const int end = implicit ? i + 1 : rp[i + 1];
     for (int e = beg; e < end; ++e) {
-        const int j = ci[e];
+        const int j = implicit ? e : ci[e];
         const int64_t krow = head_off + static_cast<int64_t>(j) * b;
         __syncthreads();
         for (int x = threadIdx.x; x < b * D; x += blockDim.x) {

@@ -127,13 +127,15 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const int SH = p.S * p.H;
     const int items = SH * ((nblk + 1) / 2);
     // item it: query tile it / SH (heaviest first), sample-head it % SH
+    // (g < 0: a local class with implicit lists)
     auto item_keys = [&](int it, int& sh, int& qa, int& qb, int64_t& g) {
         sh = it % SH;
         const int tile = it / SH;
         const int s = sh / p.H, h = sh % p.H;
-        g = (p.cls[h] == 0 && p.local_once) ? 0 : static_cast<int64_t>(s) * 3 + p.cls[h];
-        qa = p.q_order[g * nblk + 2 * tile];
-        qb = (2 * tile + 1 < nblk) ? p.q_order[g * nblk + 2 * tile + 1] : -1;
+        g = (p.cls[h] == 0 && p.local_implicit) ? -1 : static_cast<int64_t>(s) * 3 + p.cls[h];
+        const int32_t* ord = g < 0 ? nullptr : p.q_order + g * nblk;
+        qa = order_at(ord, 2 * tile);
+        qb = (2 * tile + 1 < nblk) ? order_at(ord, 2 * tile + 1) : -1;
     };
 
     if (threadIdx.x == 0) {
@@ -189,18 +191,10 @@ attn_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     bitsB[w] = 0u;
                 }
                 __syncwarp();
-                const int32_t* rp = p.row_ptr + g * (nblk + 1);
-                const int32_t* ci = p.col_idx + g * p.cap;
-                for (int e = rp[qa] + lane; e < rp[qa + 1]; e += 32) {
-                    const int j = ci[e];
-                    atomicOr(&bitsA[j >> 5], 1u << (j & 31));
-                }
-                if (qb >= 0) {
-                    for (int e = rp[qb] + lane; e < rp[qb + 1]; e += 32) {
-                        const int j = ci[e];
-                        atomicOr(&bitsB[j >> 5], 1u << (j & 31));
-                    }
-                }
+                const ListRef rows{g < 0 ? nullptr : p.row_ptr + g * (nblk + 1), p.col_idx + (g < 0 ? 0 : g) * p.cap,
+                                   p.w, nblk, false};
+                rows.each(qa, lane, 32, [&](int j) { atomicOr(&bitsA[j >> 5], 1u << (j & 31)); });
+                if (qb >= 0) rows.each(qb, lane, 32, [&](int j) { atomicOr(&bitsB[j >> 5], 1u << (j & 31)); });
                 __syncwarp();
                 uint32_t u = 0u;
                 for (int w = lane; w < nwords; w += 32) u |= bitsA[w] | bitsB[w];

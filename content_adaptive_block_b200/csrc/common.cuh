@@ -543,4 +543,32 @@ inline bool make_tmap_tok(CUtensorMap* map, const void* base, int64_t d, int64_t
     return r == CUDA_SUCCESS;
 }
 
+// One row (or column) of a (sample, class)'s block lists, each entry handed
+// to f by the calling thread's share (entries t, t + step, ...): the stored
+// entries idx[ptr[a] .. ptr[a + 1]), or, for a local class whose lists are
+// implicit (ptr null: the caller's lists mark them so), the window of the
+// mask equation intersected with causality — row i: key blocks
+// max(0, i - w) .. i; column j: query blocks j .. min(nblk - 1, j + w) — in
+// ascending order, as the stored lists hold them.
+struct ListRef {
+    const int32_t* ptr;   // null: implicit local window
+    const int32_t* idx;
+    int w, nblk;
+    bool cols;            // column lists (the query blocks of a key block)
+    template <typename F>
+    __device__ __forceinline__ void each(int a, int t, int step, F&& f) const {
+        if (ptr) {
+            for (int e = ptr[a] + t; e < ptr[a + 1]; e += step) f(idx[e]);
+        } else {
+            const int lo = cols ? a : (a - w > 0 ? a - w : 0);
+            const int hi = cols ? (a + w < nblk - 1 ? a + w : nblk - 1) : a;
+            for (int j = lo + t; j <= hi; j += step) f(j);
+        }
+    }
+};
+
+// Entry k of a (sample, class)'s pairing order; an implicit local class's
+// order is block order (as the list builder writes the local class's).
+__device__ __forceinline__ int order_at(const int32_t* ord, int k) { return ord ? ord[k] : k; }
+
 }  // namespace gsa

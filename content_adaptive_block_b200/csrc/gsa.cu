@@ -174,7 +174,7 @@ gsa_status launch_pipeline_shape(const gsa::pipeline::PipeArgs& P, cudaStream_t 
     gsa::pipeline::PipeArgs Q = P;
     Q.bpw = gsa::deflate_lane::blocks_per_warp(P.total, static_cast<int64_t>(per_sm) * sms * W);
     const int64_t chunks = (P.total + Q.bpw - 1) / Q.bpw;
-    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1);
     int64_t grid = static_cast<int64_t>(per_sm) * sms;
     // a list job per warp for short lists when there are more jobs than CTAs
     // (measured faster up to 64 blocks per sample; longer lists go faster
@@ -198,7 +198,7 @@ gsa_status launch_pipeline_shape(const gsa::pipeline::PipeArgs& P, cudaStream_t 
 template <int MAXB>
 gsa_status launch_pipeline(const gsa::pipeline::PipeArgs& P, cudaStream_t cs) {
     using SS = gsa::pipeline::Shapes<MAXB>;
-    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1) + P.local_once;
+    const int64_t njobs = static_cast<int64_t>(P.B) * (P.nper > 0 ? P.nper : 1);
     if (njobs > gsa::bwd::sm_count() && P.nblk <= 128)
         return launch_pipeline_shape<MAXB, SS::kNarrowW, SS::kNarrowT>(P, cs);
     return launch_pipeline_shape<MAXB, SS::kWideW, SS::kWideT>(P, cs);
@@ -359,7 +359,6 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     P.lengths = lengths;
     P.flags = flags;
     P.counter = counter;
-    P.local_once = classes & 1;
     for (int c = 1; c < 3; ++c)
         if ((classes >> c) & 1) P.per[P.nper++] = c;
     gsa::mask::CsrArgs& a = P.a;
@@ -379,7 +378,8 @@ gsa_status gsa_mask_pipeline(const uint8_t* bytes, int32_t B, int64_t L, int32_t
     else st = launch_pipeline<128>(P, as_stream(stream));
     if (st != GSA_OK) return st;
     csr->w = w;
-    csr->classes = classes | (P.local_once ? 8 : 0);
+    // the local class's lists are implicit: the attention kernels derive them from (nblk, w)
+    csr->classes = classes | ((classes & 1) ? 8 : 0);
     return GSA_OK;
 }
 
@@ -412,7 +412,8 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
         p.L = desc->L;
         p.scale = scale;
         std::memcpy(p.cls, cls, desc->H);
-        p.local_once = (csr->classes >> 3) & 1;
+        p.local_implicit = (csr->classes >> 3) & 1;
+        p.w = csr->w;
         dim3 grid(csr->nblk, desc->H, desc->B);
         const size_t smem = 3u * desc->b * desc->d * sizeof(float);
         bool opted = false;
@@ -461,7 +462,8 @@ gsa_status gsa_attn_fwd(const void* q, const void* k, const void* v, const gsa_b
     p.lse = lse;
     p.scale_log2 = scale * 1.4426950408889634f;
     std::memcpy(p.cls, cls, desc->H);
-    p.local_once = (csr->classes >> 3) & 1;
+    p.local_implicit = (csr->classes >> 3) & 1;
+    p.w = csr->w;
     dim3 grid(desc->B * desc->H, (csr->nblk + 1) / 2);
     if (GSA_FWD_PERSIST) {
         p.ticket = fwd_ticket_slot();

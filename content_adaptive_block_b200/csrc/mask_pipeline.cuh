@@ -11,13 +11,12 @@
 //      (deflate_lane.cuh);
 //   2. lists: jobs (sample, class) spread over the CTAs, all of a CTA's
 //      warps on one job (or, for short lists and many jobs, one job per
-//      warp).  A job sums its
-//      sample's lengths, sets the flags (len_i * nblk > Σ len) in shared
-//      memory — the sample's first job also writes them out — and builds the
-//      class's lists.  The local class's lists depend only on (nblk, w)
-//      (mask equation: |i - j| <= w intersected with causality), so they are
-//      built once, into sample 0's slot, and the attention calls read that
-//      slot for every sample.
+//      warp).  A job sums its sample's lengths, sets the flags
+//      (len_i * nblk > Σ len) in shared memory — the sample's first job also
+//      writes them out — and builds the class's lists.  The local class's
+//      lists depend only on (nblk, w) (mask equation: |i - j| <= w
+//      intersected with causality), so they are not built at all: the
+//      attention kernels derive them.
 // The barrier: each CTA adds one to a counter in caller-owned memory and
 // waits (bounded by a time limit, after which it records an error code and
 // leaves) until all have; each CTA adds one more as it leaves, and the last
@@ -82,9 +81,8 @@ struct PipeArgs {
     uint8_t* flags;       // [B][nblk]
     mask::CsrArgs a;
     int* counter;         // the grid barrier's counter (zero between calls)
-    int nper;             // classes built per sample (those other than a local class built once)
+    int nper;             // classes built per sample (literal, hybrid: the local class is implicit)
     int per[3];           // ... and which
-    int local_once;       // 1: the local class is in use, built once into sample 0's slot
     int warp_jobs;        // 1: a list job per warp (its lengths words hold the job's scratch), 0: per CTA
     int bpw;              // blocks per warp in the lengths phase (1 .. 32)
 };
@@ -140,26 +138,24 @@ __global__ void __launch_bounds__(32 * T, (Shape<MAXB, W, T>::kPerSm)) mask_pipe
     if (!grid_barrier(P.counter, static_cast<int>(gridDim.x))) return;
 
     // ---- phase 2: (sample, class) jobs.  Per sample max(nper, 1) jobs (one
-    // writes the flags even when no per-sample class is built), then the
-    // local class once.
+    // writes the flags even when no list is built).
     const int n = P.nblk;
     const int jobs_per = P.nper > 0 ? P.nper : 1;
-    const int njobs = P.B * jobs_per + P.local_once;
+    const int njobs = P.B * jobs_per;
     if (P.warp_jobs) {
         // one job per warp at a time, each warp with its own scratch: all the
         // jobs run side by side instead of a few per CTA in turn
         uint8_t* ws = dsmem + static_cast<size_t>(warp) * S::kWarpJobBytes;
         for (int j = blockIdx.x * T + warp; j < njobs; j += gridDim.x * T) {
-            const bool local = j == P.B * jobs_per;
-            const int s = local ? 0 : j / jobs_per;
-            const int k = local ? 0 : j % jobs_per;
-            const int c = local ? 0 : (P.nper > 0 ? P.per[k] : -1);
+            const int s = j / jobs_per;
+            const int k = j % jobs_per;
+            const int c = P.nper > 0 ? P.per[k] : -1;
             __syncwarp();
             const int32_t* row = P.lengths + static_cast<int64_t>(s) * n;
             long long acc = 0;
             for (int i = lane; i < n; i += 32) acc += __ldcg(row + i);
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            const bool write = !local && k == 0;
+            const bool write = k == 0;
             for (int i = lane; i < n; i += 32) {
                 const uint8_t f = static_cast<long long>(__ldcg(row + i)) * n > acc ? 1 : 0;
                 ws[i] = f;
@@ -173,10 +169,9 @@ __global__ void __launch_bounds__(32 * T, (Shape<MAXB, W, T>::kPerSm)) mask_pipe
     }
     uint8_t* fl = dsmem;   // the list builder's flag scratch: dsm[0 .. n)
     for (int j = blockIdx.x; j < njobs; j += gridDim.x) {
-        const bool local = j == P.B * jobs_per;
-        const int s = local ? 0 : j / jobs_per;
-        const int k = local ? 0 : j % jobs_per;
-        const int c = local ? 0 : (P.nper > 0 ? P.per[k] : -1);
+        const int s = j / jobs_per;
+        const int k = j % jobs_per;
+        const int c = P.nper > 0 ? P.per[k] : -1;
         __syncthreads();   // the previous job's scratch
         const int32_t* row = P.lengths + static_cast<int64_t>(s) * n;
         long long acc = 0;
@@ -186,7 +181,7 @@ __global__ void __launch_bounds__(32 * T, (Shape<MAXB, W, T>::kPerSm)) mask_pipe
         __syncthreads();
         long long total = 0;
         for (int w = 0; w < T; ++w) total += part[w];
-        const bool write = !local && k == 0;
+        const bool write = k == 0;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const uint8_t f = static_cast<long long>(__ldcg(row + i)) * n > total ? 1 : 0;
             fl[i] = f;

@@ -17,26 +17,17 @@ struct TileList {
     int* count;       // number of entries
 };
 
-// Whole CTA.  ptr/idx: CSR (or CSC) arrays of this (sample, class), a and b:
-// the two rows (b < 0: none).  Ends with __syncthreads().
-__device__ __forceinline__ void build_tile_list(const TileList& t, const int32_t* ptr, const int32_t* idx, int a,
-                                                int b, int nblk) {
+// Whole CTA.  lists: the CSR (or CSC) rows of this (sample, class), stored or
+// implicit; a and b: the two rows (b < 0: none).  Ends with __syncthreads().
+__device__ __forceinline__ void build_tile_list(const TileList& t, const ListRef& lists, int a, int b, int nblk) {
     const int nwords = (nblk + 31) >> 5;
     for (int k = threadIdx.x; k < nwords; k += blockDim.x) {
         t.bitsA[k] = 0u;
         t.bitsB[k] = 0u;
     }
     __syncthreads();
-    for (int e = ptr[a] + threadIdx.x; e < ptr[a + 1]; e += blockDim.x) {
-        const int j = idx[e];
-        atomicOr(&t.bitsA[j >> 5], 1u << (j & 31));
-    }
-    if (b >= 0) {
-        for (int e = ptr[b] + threadIdx.x; e < ptr[b + 1]; e += blockDim.x) {
-            const int j = idx[e];
-            atomicOr(&t.bitsB[j >> 5], 1u << (j & 31));
-        }
-    }
+    lists.each(a, threadIdx.x, blockDim.x, [&](int j) { atomicOr(&t.bitsA[j >> 5], 1u << (j & 31)); });
+    if (b >= 0) lists.each(b, threadIdx.x, blockDim.x, [&](int j) { atomicOr(&t.bitsB[j >> 5], 1u << (j & 31)); });
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;

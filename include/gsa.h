@@ -123,7 +123,9 @@ typedef struct {
     int32_t nblk;
     int32_t w;          /* set by gsa_build_block_csr */
     int32_t classes;    /* bit c set: the lists of head class c were built; bit 3: the local
-                           class's lists are stored once, in sample 0's slot (set by the builders) */
+                           class's lists are implicit — not stored: the attention calls derive
+                           row i = key blocks max(0, i - w) .. i from (nblk, w) (set by the
+                           builders: gsa_mask_pipeline sets it when the local class is in use) */
     int64_t capacity;   /* entries per (sample, class) in col_idx and row_idx */
     int32_t* row_ptr;
     int32_t* col_idx;
@@ -192,10 +194,11 @@ gsa_status gsa_build_block_csr(const uint8_t* flags, int32_t w, const uint8_t* h
  * head class) as one pass: a cooperative launch whose CTAs first compute all
  * lengths, meet at a grid barrier, then share out the (sample, class) list
  * jobs, each of which computes its sample's flags.  The local class's lists
- * depend only on (nblk, w): they are built once, into sample 0's slot, and
- * csr->classes gets bit 3 (value 8) to say so; the attention calls then read
- * that slot for every sample.  Lengths, flags and the other classes' lists
- * are those of the three calls, bit for bit.
+ * depend only on (nblk, w) (the mask equation's window intersected with
+ * causality): they are not written at all, csr->classes gets bit 3
+ * (value 8) to say so, and the attention calls derive them.  Lengths, flags
+ * and the other classes' lists are those of the three calls, bit for bit,
+ * and attention on these lists gives the three calls' results bit for bit.
  *
  *   bytes, B, L, b   as for gsa_block_lengths; L / b = nblk <= GSA_MAX_PIPELINE_BLOCKS
  *   w                local window in blocks, >= 0

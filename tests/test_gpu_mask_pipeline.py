@@ -5,7 +5,8 @@ Cases cover CTAs that straddle samples (blocks per sample not a multiple of
 four), one block per sample, the largest supported list (1024 blocks), the
 mask-sweep batches at full size, two calls in a row on one counter
 (each call leaves it zero), subsets of the head classes, and attention on
-the pipeline's lists (the local class stored once)."""
+the pipeline's lists (the local class implicit: not stored, derived by the
+attention kernels)."""
 import numpy as np
 import pytest
 import torch
@@ -24,9 +25,8 @@ def gsa():
     return g
 
 
-def _slot_lists(csr, s, c):
-    """Pointers, pairing orders and entries of (sample s, class c) from the slot that holds them."""
-    s = csr.slot(s, c)
+def _lists(csr, s, c):
+    """Pointers, pairing orders and entries of (sample s, class c)."""
     rp, cp = csr.row_ptr[s, c].cpu().numpy(), csr.col_ptr[s, c].cpu().numpy()
     return (rp, cp, csr.q_order[s, c].cpu().numpy(), csr.k_order[s, c].cpu().numpy(),
             csr.col_idx[s, c, :rp[-1]].cpu().numpy(), csr.row_idx[s, c, :cp[-1]].cpu().numpy())
@@ -35,7 +35,7 @@ def _slot_lists(csr, s, c):
 def _same(gsa, x: np.ndarray, b: int, w: int, counters=None, head_classes=None):
     """The pipeline against the three calls: lengths and flags bit for bit, and
     every (sample, class) list of the classes in use equal to the three calls'
-    (the local class read from sample 0's slot, where the pipeline stores it once)."""
+    (the local class is implicit: marked, not stored)."""
     t = torch.from_numpy(np.ascontiguousarray(x)).cuda()
     ln_ref = gsa.gsa_block_lengths(t, b)
     fl_ref = gsa.gsa_literal_flags(ln_ref)
@@ -48,9 +48,10 @@ def _same(gsa, x: np.ndarray, b: int, w: int, counters=None, head_classes=None):
     assert csr.w == csr_ref.w == w
     used = {0, 1, 2} if head_classes is None else set(head_classes)
     assert csr.classes == sum(1 << c for c in used) | (8 if 0 in used else 0)
+    assert not csr.stored(0) if 0 in used else True
     for s in range(x.shape[0]):
-        for c in sorted(used):
-            for got, want in zip(_slot_lists(csr, s, c), _slot_lists(csr_ref, s, c)):
+        for c in sorted(used - {0}):
+            for got, want in zip(_lists(csr, s, c), _lists(csr_ref, s, c)):
                 assert np.array_equal(got, want), (s, c)
     return ln.cpu().numpy()
 
@@ -92,8 +93,9 @@ def test_pipeline_classes_in_use(gsa, head_classes):
 
 
 def test_attention_on_pipeline_lists(gsa):
-    """Forward and backward on the pipeline's lists (local class stored once)
-    give the three-call lists' results bit for bit, at d = 64 and d = 128."""
+    """Forward and backward on the pipeline's lists (the local class implicit)
+    give the three-call lists' results bit for bit, at d = 64 and d = 128, and
+    the float32 forward likewise."""
     wl = W.WORKLOADS["b8_4k"]
     hc = [int(c) for c in wl.head_classes()]
     t = torch.from_numpy(W.batch_bytes(wl, seed=5)).cuda()
@@ -109,3 +111,39 @@ def test_attention_on_pipeline_lists(gsa):
         assert gsa.gsa_device_error() == 0
         for a, b_ in zip(*outs):
             assert torch.equal(a, b_), d
+
+    # the float32 path (CUDA cores) on the tiny workload
+    wl = W.WORKLOADS["tiny_fp32"]
+    hc = [int(c) for c in wl.head_classes()]
+    t = torch.from_numpy(W.batch_bytes(wl, seed=6)).cuda()
+    csr_ref = gsa.gsa_build_block_csr(gsa.gsa_literal_flags(gsa.gsa_block_lengths(t, wl.b)), wl.w)
+    _, _, csr = gsa.gsa_mask_pipeline(t, wl.b, wl.w)
+    q, k, v = (x.cuda() for x in W.random_tensors((wl.S, wl.H, wl.L, wl.d), 3, torch.float32, seed=7))
+    o_ref, lse_ref = gsa.gsa_attn_fwd(q, k, v, csr_ref, hc, wl.b)
+    o, lse = gsa.gsa_attn_fwd(q, k, v, csr, hc, wl.b)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+@pytest.mark.parametrize("B,nblk,w", [(2, 17, 0), (2, 9, 20), (1, 33, 3), (3, 1, 2)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_implicit_local_window_edges(gsa, B, nblk, w, d):
+    """The implicit local window at its edges (w = 0, w past the first block,
+    odd block counts, one block) against the stored lists of the three calls:
+    forward and backward bit for bit, local heads only and mixed."""
+    b = 64
+    x = W.custom_bytes(B, nblk * b, ("uniform", 0.2, 0.6), seed=nblk * 10 + w)
+    t = torch.from_numpy(x).cuda()
+    csr_ref = gsa.gsa_build_block_csr(gsa.gsa_literal_flags(gsa.gsa_block_lengths(t, b)), w)
+    for hc in ([0, 0], [0, 1, 2, 0]):
+        _, _, csr = gsa.gsa_mask_pipeline(t, b, w, head_classes=hc)
+        q, k, v, do = (y.cuda() for y in W.random_tensors((B, len(hc), nblk * b, d), 4, torch.bfloat16, seed=d + w))
+        outs = []
+        for c in (csr_ref, csr):
+            o, lse = gsa.gsa_attn_fwd(q, k, v, c, hc, b)
+            outs.append([o, lse, *gsa.gsa_attn_bwd(q, k, v, o, lse, do, c, hc, b)])
+        torch.cuda.synchronize()
+        assert gsa.gsa_device_error() == 0
+        for a, b_ in zip(*outs):
+            assert torch.equal(a, b_), (hc, d)
