@@ -1057,6 +1057,38 @@ def profile_lengths():
     return 0
 
 
+def profile_pipeline():
+    """gsa_mask_pipeline three times on the headline mask point (256 x 8192
+    bytes, b = 64, high-entropy fraction 0.3, all three head classes): a
+    short program for an ncu capture of the one-launch mask stage."""
+    import torch
+    import content_adaptive_block_b200 as gsa
+    from content_adaptive_block_b200 import build
+    build.build()
+    wl = W.mask_sweep(*MASK_POINT)
+    x = torch.from_numpy(W.batch_bytes(wl)).cuda()
+    counters = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csr = gsa.BlockCsr(wl.S, wl.N, x.device)
+    for _ in range(3):
+        gsa.gsa_mask_pipeline(x, wl.b, wl.w, csr, counters=counters)
+    torch.cuda.synchronize()
+    assert gsa.gsa_device_error() == 0
+    print("pipeline ok")
+    return 0
+
+
+def profile_lm():
+    """One ByteLM block forward + backward on the 8x8K batch, twice: a short
+    program for an ncu launch list of the block's kernels."""
+    import torch
+    import content_adaptive_block_b200 as gsa
+    from content_adaptive_block_b200 import build
+    build.build()
+    lm_block(gsa, torch.device("cuda", 0), steps=1, warmup=1)
+    print("lm ok")
+    return 0
+
+
 def profile_attn(name):
     """The mask and the attention calls of one workload, three times (a short
     program for an ncu capture of one attention kernel)."""
@@ -1099,6 +1131,10 @@ def main():
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw-page CSV export and exit")
     ap.add_argument("--capture", default="", help="the ncu command recorded with --record-traffic")
+    ap.add_argument("--profile-pipeline", action="store_true",
+                    help="run gsa_mask_pipeline three times on the headline mask point and exit (for ncu)")
+    ap.add_argument("--profile-lm", action="store_true",
+                    help="run the ByteLM block forward + backward twice and exit (for ncu)")
     ap.add_argument("--profile-lengths", action="store_true",
                     help="run gsa_block_lengths three times on the headline mask point and exit (for ncu)")
     ap.add_argument("--profile-attn", metavar="WORKLOAD", choices=sorted(W.WORKLOADS),
@@ -1106,6 +1142,10 @@ def main():
     args = ap.parse_args()
     if args.profile_lengths:
         return profile_lengths()
+    if args.profile_pipeline:
+        return profile_pipeline()
+    if args.profile_lm:
+        return profile_lm()
     if args.profile_attn:
         return profile_attn(args.profile_attn)
     if args.record_traffic:
