@@ -95,3 +95,32 @@ def test_committed_records_name_existing_sources():
         for r in recs:
             for s in r["sources"]:
                 assert os.path.exists(os.path.join(bench.ROOT, s)), s
+
+
+class _FakeCsr:
+    """The fields csr_nnz reads, on the CPU (no library needed)."""
+
+    def __init__(self, row_ptr, w, classes):
+        import torch
+        self.row_ptr = torch.tensor(row_ptr, dtype=torch.int32)
+        self.nblk = self.row_ptr.shape[2] - 1
+        self.w, self.classes = w, classes
+
+    def stored(self, c):
+        return not (c == 0 and self.classes & 8)
+
+
+def test_csr_nnz_counts_an_implicit_local_window():
+    # two samples, 5 blocks, w = 2: the local window holds min(i, 2) + 1 blocks in row i
+    # (1 + 2 + 3 + 3 + 3 = 12), the closed form N (w + 1) - w (w + 1) / 2 of the mask equation
+    n, w = 5, 2
+    rp = [[[0] * (n + 1), [0, 1, 2, 4, 5, 8], [0, 1, 3, 6, 9, 12]] for _ in range(2)]
+    implicit = bench.csr_nnz(_FakeCsr(rp, w, 7 | 8))
+    assert implicit[:, 0].tolist() == [n * (w + 1) - w * (w + 1) // 2] * 2 == [12, 12]
+    assert implicit[:, 1].tolist() == [8, 8] and implicit[:, 2].tolist() == [12, 12]
+    # stored lists count from their pointers
+    rp[0][0] = [0, 1, 3, 6, 9, 12]
+    rp[1][0] = [0, 1, 3, 6, 9, 12]
+    assert bench.csr_nnz(_FakeCsr(rp, w, 7))[:, 0].tolist() == [12, 12]
+    # a window wider than the sample: the whole causal triangle
+    assert bench.csr_nnz(_FakeCsr(rp, 9, 1 | 8))[:, 0].tolist() == [15, 15]
