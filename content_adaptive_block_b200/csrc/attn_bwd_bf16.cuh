@@ -29,6 +29,8 @@
 // with double-buffered scores): attn_bwd_dq_persist.cuh, attn_bwd_persist.cuh.
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 #include "tiles.cuh"
 
@@ -82,9 +84,14 @@ struct Params {
 
 // ------------------------------------------------------------ D_t = dO·O
 
-// Grid (L / kRowsPerCta, y): CTA (x, y) takes the tokens [x kRowsPerCta,
-// (x + 1) kRowsPerCta) of the (sample, head) pairs sh = y, y + gridDim.y, ...
-// (L is a multiple of 64; consecutive CTAs read consecutive rows).
+// Grid (L / (kRows kRowsPerCta), y): CTA (x, y) takes the tokens
+// [x kRows kRowsPerCta, (x + 1) kRows kRowsPerCta) of the (sample, head)
+// pairs sh = y, y + gridDim.y, ..., kRows rows per thread with their loads in
+// flight together (L is a multiple of 64; consecutive CTAs read consecutive
+// rows).
+#ifndef GSA_DOT_ROWS
+#define GSA_DOT_ROWS 2
+#endif
 template <int D>
 __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                   const __nv_bfloat16* __restrict__ dO, TokLayout lo, int64_t L,
@@ -94,29 +101,37 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) ticket[threadIdx.x] = 0;   // for the persistent kernels
     constexpr int kTpr = D / 8;                  // threads per row, 8 elements (16 bytes) each
     constexpr int kRowsPerCta = 256 / kTpr;
-    const int64_t l = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / kTpr;
+    constexpr int kRows = GSA_DOT_ROWS;
+    const int64_t l0 = static_cast<int64_t>(blockIdx.x) * (kRows * kRowsPerCta) + threadIdx.x / kTpr;
     const int part = threadIdx.x % kTpr;
     for (int sh = blockIdx.y; sh < SH; sh += gridDim.y) {
         const int s = sh / H, h = sh - s * H;
-        const int64_t off = s * lo.s + h * lo.h + l * lo.l + part * 8;
-        const uint4 a = *reinterpret_cast<const uint4*>(o + off);
-        const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
-        const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
-        float acc = 0.f;
+        uint4 a[kRows], b[kRows];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 fa = __bfloat1622float2(ah[e]);
-            const float2 fb = __bfloat1622float2(bh[e]);
-            acc = fmaf(fa.x, fb.x, acc);
-            acc = fmaf(fa.y, fb.y, acc);
+        for (int u = 0; u < kRows; ++u) {
+            const int64_t off = s * lo.s + h * lo.h + (l0 + u * kRowsPerCta) * lo.l + part * 8;
+            a[u] = *reinterpret_cast<const uint4*>(o + off);
+            b[u] = *reinterpret_cast<const uint4*>(dO + off);
         }
 #pragma unroll
-        for (int o2 = kTpr / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
-        if (part == 0) {
-            const int64_t row = static_cast<int64_t>(sh) * L + l;
-            ndvec[row] = -acc;
-            nlse2[row] = -(lse[row] * kLog2e);   // the backward's exponents are in log2 units
+        for (int u = 0; u < kRows; ++u) {
+            const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+            const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fa = __bfloat1622float2(ah[e]);
+                const float2 fb = __bfloat1622float2(bh[e]);
+                acc = fmaf(fa.x, fb.x, acc);
+                acc = fmaf(fa.y, fb.y, acc);
+            }
+#pragma unroll
+            for (int o2 = kTpr / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+            if (part == 0) {
+                const int64_t row = static_cast<int64_t>(sh) * L + l0 + u * kRowsPerCta;
+                ndvec[row] = -acc;
+                nlse2[row] = -(lse[row] * kLog2e);   // the backward's exponents are in log2 units
+            }
         }
     }
 }
@@ -828,15 +843,15 @@ namespace bwd {
 
 // Streaming multiprocessors of the current device (cached per device).
 inline int sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64] = {};   // calls may come from several host threads
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 template <int D, bool K4>
@@ -849,7 +864,8 @@ gsa_status launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
         !(persist_kv ? smem_opt_in(dkdv_persist_kernel<K4>, DkvPCfg::kSmemBytes)
                      : smem_opt_in(dkdv_kernel<D, K4>, DkvCfg<D>::kSmemBytes)))
         return GSA_ERR_CUDA;
-    constexpr int kRowsPerCta = 256 / (D / 8);   // 32 or 16: divides L
+    constexpr int kRowsPerCta = GSA_DOT_ROWS * 256 / (D / 8);   // 32 or 16 rows a thread row group: divides L
+    static_assert(64 % kRowsPerCta == 0, "rows per CTA divide a 64-token block");
     const int sh_grid = S * H < 65535 ? S * H : 65535;
     dot_kernel<D><<<dim3(static_cast<unsigned>(pq.L / kRowsPerCta), static_cast<unsigned>(sh_grid)), 256, 0, st>>>(
         o, dO, lo, pq.L, pq.H, S * H, const_cast<float*>(pq.ndvec), pq.lse, const_cast<float*>(pq.nlse2), pkv.ticket);
