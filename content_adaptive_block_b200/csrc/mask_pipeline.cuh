@@ -83,7 +83,7 @@ struct PipeArgs {
     int* counter;         // the grid barrier's counter (zero between calls)
     int nper;             // classes built per sample (literal, hybrid: the local class is implicit)
     int per[3];           // ... and which
-    int warp_jobs;        // 1: a list job per warp (its lengths words hold the job's scratch), 0: per CTA
+    int warp_jobs;        // 1: a list job per warp (each warp a scratch of its own), 0: a job per CTA
     int bpw;              // blocks per warp in the lengths phase (1 .. 32)
 };
 
