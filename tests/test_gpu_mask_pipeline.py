@@ -78,6 +78,15 @@ def test_pipeline_odd_shapes(gsa, B, nblk, b, w):
     assert np.array_equal(ln, deflate1.block_lengths(x, b, nthreads=8))
 
 
+@pytest.mark.parametrize("B,nblk,b,w", [(1024, 32, 64, 2), (2048, 16, 128, 1)])
+def test_pipeline_list_jobs_per_warp(gsa, B, nblk, b, w):
+    """Many samples of short lists: more list jobs than CTAs, so each warp
+    takes jobs of its own (the warp-job path of phase 2)."""
+    x = W.custom_bytes(B, nblk * b, ("uniform", 0.2, 0.6), seed=B + nblk)
+    ln = _same(gsa, x, b, w)
+    assert np.array_equal(ln, deflate1.block_lengths(x, b, nthreads=8))
+
+
 def test_pipeline_reuses_its_counters(gsa):
     wl = W.WORKLOADS["b8_4k"]
     counters = torch.zeros(1, dtype=torch.int32, device="cuda")
