@@ -94,6 +94,15 @@ def test_lengths_code_length_overflow_fixtures(gsa):
     assert np.array_equal(_gpu_lengths(gsa, x, 128), deflate1.block_lengths(x, 128))
 
 
+@pytest.mark.parametrize("S,b", [(23, 64), (39, 64), (95, 64), (7, 128), (47, 128), (161, 32)])
+def test_lengths_blocks_per_warp(gsa, S, b):
+    """Batch sizes whose blocks fill one wave of resident warps at 2, 4, 8 or
+    16 blocks a warp (the launcher picks the fewest that fit), so every
+    chunk size of the lengths kernel runs, with a ragged last chunk."""
+    x = W.custom_bytes(S, 8192 - b, ("uniform", 0.2, 0.6), seed=S * 7 + b)
+    assert np.array_equal(_gpu_lengths(gsa, x, b), deflate1.block_lengths(x, b, nthreads=8))
+
+
 def test_lengths_several_blocks_per_sample(gsa):
     x = W.custom_bytes(3, 64 * 37, ("fixed", 0.4), seed=5)[:, : 64 * 37]
     for b in (16, 32, 64):
