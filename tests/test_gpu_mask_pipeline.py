@@ -78,13 +78,21 @@ def test_pipeline_odd_shapes(gsa, B, nblk, b, w):
     assert np.array_equal(ln, deflate1.block_lengths(x, b, nthreads=8))
 
 
-@pytest.mark.parametrize("B,nblk,b,w", [(1024, 32, 64, 2), (2048, 16, 128, 1)])
+@pytest.mark.parametrize("B,nblk,b,w", [(1024, 32, 64, 2), (2048, 16, 128, 1), (1024, 16, 16, 1)])
 def test_pipeline_list_jobs_per_warp(gsa, B, nblk, b, w):
     """Many samples of short lists: more list jobs than CTAs, so each warp
     takes jobs of its own (the warp-job path of phase 2)."""
     x = W.custom_bytes(B, nblk * b, ("uniform", 0.2, 0.6), seed=B + nblk)
     ln = _same(gsa, x, b, w)
     assert np.array_equal(ln, deflate1.block_lengths(x, b, nthreads=8))
+
+
+def test_pipeline_narrow_ctas_small_blocks(gsa):
+    """Blocks of at most 32 bytes, more list jobs than SMs and short lists:
+    the narrow CTA shape of the smallest block size, one job per CTA."""
+    x = W.custom_bytes(256, 64 * 32, ("uniform", 0.2, 0.6), seed=31)
+    ln = _same(gsa, x, 32, 2)
+    assert np.array_equal(ln, deflate1.block_lengths(x, 32, nthreads=8))
 
 
 def test_pipeline_reuses_its_counters(gsa):
